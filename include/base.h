@@ -1,0 +1,219 @@
+/*
+ * base.h -- C ABI of libbase, the sm_100a (B200) hot path of a BASE layer.
+ *
+ * A BASE layer ("BASE Layers: Simplifying Training of Large, Sparse Models",
+ * Lewis et al.; the wikillm.com summary's Method section) sends every token
+ * h_t (width D) to exactly one of E experts.  In training the routing is a
+ * balanced linear assignment (eq. 2: maximise sum_t h_t . w_{a_t} with every
+ * expert receiving exactly T/E tokens); at test time each token goes to its
+ * highest-affinity expert ("Test time").  The token leaves the layer as
+ * sigma(h_t . w_{a_t}) f_{a_t}(h_t) + h_t (eq. 1), where f_e is the expert's
+ * position-wise FFN ("Placement and shape").  The fig. 2 listing gives the
+ * order of the steps: affinities -> balanced_assignment -> sort_by_expert ->
+ * gated expert + residual -> inverse_sort.
+ *
+ * Conventions shared by every entry point:
+ *   - Every pointer argument except `stats`' host copy is DEVICE memory owned
+ *     by the caller.  The library never allocates device memory, never
+ *     synchronises the host and enqueues all work on `stream` (may be 0).
+ *   - Tensors are dense row-major.  Base pointers are 16-byte aligned.
+ *     D % 8 == 0 and F % 8 == 0 (16-byte rows); 2 <= E <= 1024; 1 <= T < 2^31.
+ *     Balanced assignment needs T % E == 0 (the page's Pitfalls note that the
+ *     released code silently uses integer division instead).
+ *   - Inputs are const and must not alias outputs.
+ *   - Arguments are checked on the host before anything is launched; a bad
+ *     argument returns BASE_ERR_INVALID_ARG and launches nothing.  A failed
+ *     launch returns BASE_ERR_CUDA.  Failures found while the kernels run
+ *     (round cap reached, a bounded wait that gave up) are written to the
+ *     device-side status word of `base_auction_stats` (auction) or of the
+ *     workspace (GEMMs) and read back by the caller after synchronising.
+ *   - bf16 means IEEE bfloat16 (1-8-7), fp32 IEEE binary32.
+ *   - The library holds no per-call state; calls on different streams with
+ *     disjoint buffers may run concurrently.
+ */
+#ifndef BASE_H
+#define BASE_H
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    BASE_OK = 0,
+    BASE_ERR_INVALID_ARG = 1,   /* bad shape, null or misaligned pointer, small workspace */
+    BASE_ERR_CUDA = 2,          /* a CUDA runtime call or launch failed */
+    BASE_ERR_NOT_CONVERGED = 3, /* auction hit BASE_AUCTION_MAX_ROUNDS (device status) */
+    BASE_ERR_TIMEOUT = 4,       /* a bounded device-side wait gave up (device status) */
+    BASE_ERR_WORKSPACE = 5,     /* workspace smaller than base_workspace_size() */
+    BASE_ERR_UNSUPPORTED = 6    /* shape outside what the kernels implement */
+} base_status;
+
+typedef enum { BASE_F32 = 0, BASE_BF16 = 1 } base_dtype;
+typedef enum { BASE_RELU = 0, BASE_GELU = 1 } base_act;
+typedef enum { BASE_ROUTE_BALANCED = 0, BASE_ROUTE_GREEDY = 1 } base_routing;
+
+/* Quantisation scale of the affinity scores: q = rint(s * 2^16). */
+#define BASE_QSCALE 65536.0f
+/* Hang guard of the auction: total rounds over all phases. */
+#define BASE_AUCTION_MAX_ROUNDS 1000000
+
+/*
+ * Auction statistics, written by base_assign_balanced into DEVICE memory
+ * (48 bytes, 8-byte aligned).  status is a base_status; phases and rounds
+ * count epsilon-scaling phases and Jacobi rounds; final_eps is the last
+ * epsilon (1 on success); objective = sum_t q[t][assign[t]]; bids = total
+ * number of bids over all rounds (sum of the unassigned counts).
+ */
+typedef struct {
+    int64_t status;
+    int64_t phases;
+    int64_t rounds;
+    int64_t final_eps;
+    int64_t objective;
+    int64_t bids;
+} base_auction_stats;
+
+/*
+ * Device buffers of one layer forward, kept for the backward.  All owned by
+ * the caller; sizes in elements.  Pointers marked "fwd-only nullable" may be
+ * NULL when no backward follows.
+ */
+typedef struct {
+    float*   s;        /* T*E   fp32 scores s = h w^T                             */
+    int32_t* q;        /* T*E   int32 quantised scores                            */
+    int32_t* assign;   /* T     expert of every token                             */
+    int64_t* price;    /* E     final auction prices (balanced routing)           */
+    base_auction_stats* stats; /* 1 (device); balanced routing only               */
+    int32_t* perm;     /* T     perm[slot] = token                                */
+    int32_t* inv;      /* T     inv[token] = slot                                 */
+    int32_t* offsets;  /* E+1   first slot of every expert                        */
+    float*   gate;     /* T     s[perm[slot], assign[perm[slot]]], slot order      */
+    void*    x_perm;   /* T*D   bf16 tokens in slot order                          */
+    void*    a1;       /* T*F   bf16 pre-activation (fwd-only nullable)            */
+    void*    h1;       /* T*F   bf16 activation                                    */
+    void*    f;        /* T*D   bf16 expert output f (fwd-only nullable)           */
+    void*    y_perm;   /* T*D   bf16 layer output in slot order                    */
+} base_layer_saved;
+
+/* Human-readable name of a status code (static string). */
+const char* base_status_string(int status);
+
+/* Library version string (static). */
+const char* base_version(void);
+
+/*
+ * Workspace bytes that every call below needs at most for these sizes
+ * (F may be 0 when no FFN runs).  Host only; makes no CUDA call.
+ */
+size_t base_workspace_size(int T, int E, int D, int F);
+
+/*
+ * a1+a2: affinity scores and their quantisation (fig. 2: affinities =
+ * features @ centroids^T; the quantisation scale 2^16 is this library's).
+ *   h: T*D, w: E*D, both of `dtype` (BASE_F32 or BASE_BF16).
+ *   s (nullable): T*E fp32, s[t][e] = sum_d h[t][d] w[e][d], fp32 accumulation.
+ *   q (nullable): T*E int32, q = rint(s * 65536) (round half to even),
+ *     saturated to +-(2^31 - 1).
+ *   bf16 inputs run on the tensor cores (tcgen05); fp32 inputs use fp32 FMA.
+ */
+int base_scores(const void* h, const void* w, int dtype, int T, int D, int E,
+                float* s, int32_t* q, cudaStream_t stream);
+
+/*
+ * a3: greedy test-time routing (Method, "Test time": each token to its
+ * highest-scoring expert).  assign[t] = argmax_e q[t][e], lowest e on ties;
+ * counts (nullable) E int32: number of tokens per expert.
+ */
+int base_assign_greedy(const int32_t* q, int T, int E, int32_t* assign, int32_t* counts,
+                       cudaStream_t stream);
+
+/*
+ * a4: balanced assignment (eq. 2) by a Jacobi token-bidding auction with
+ * epsilon scaling, exact for integer scores.  Values A[t][e] = q[t][e] (T+1);
+ * eps starts at max(1, (max q - min q)(T+1)/50) (the released solver's
+ * range/50 rule, "Paper vs code") and is divided by 8 per phase down to 1.
+ * In every round each unassigned token bids best - second + eps above the
+ * price of its best expert; each expert keeps its C = T/E best bids (larger
+ * bid, then smaller token index) and, once full, sets its price to the
+ * lowest bid it holds.  The result is an exact optimum of eq. 2.
+ *   q: T*E int32 (|q| < 2^31; the scaled range (max-min)(T+1) must be < 2^58).
+ *   assign: T int32 output.  price: E int64 output (final prices).
+ *   stats (nullable): device base_auction_stats.
+ *   ws: workspace of at least base_workspace_size(T, E, 0, 0) bytes.
+ * Runs on one thread-block cluster (up to 16 CTAs) with the experts' held
+ * bids in distributed shared memory.
+ */
+int base_assign_balanced(const int32_t* q, int T, int E, int32_t* assign, int64_t* price,
+                         base_auction_stats* stats, void* ws, size_t ws_bytes,
+                         cudaStream_t stream);
+
+/*
+ * a5: permutation into expert-contiguous slots (fig. 2 sort_by_expert).
+ * Slot order is expert-major and ascending token index inside an expert.
+ *   h: T*D bf16; assign: T int32 in [0, E).
+ *   perm: T (perm[slot] = t); inv: T (inv[t] = slot); offsets: E+1 int32.
+ *   x_perm: T*D bf16, x_perm[slot] = h[perm[slot]].
+ *   s (nullable) T*E fp32 with gate (nullable) T fp32:
+ *     gate[slot] = s[perm[slot]][assign[perm[slot]]].
+ */
+int base_permute(const void* h, const int32_t* assign, int T, int D, int E,
+                 int32_t* perm, int32_t* inv, int32_t* offsets, void* x_perm,
+                 const float* s, float* gate, void* ws, size_t ws_bytes, cudaStream_t stream);
+
+/*
+ * a6+a7: the experts' FFNs on their slot segments with the eq. 1 combine in
+ * the epilogue.  For every expert e and slot r in [offsets[e], offsets[e+1]):
+ *   a1[r] = x_perm[r] W1[e]^T          (W1: E*F*D bf16)
+ *   h1[r] = act(a1[r])                 (ReLU, or GELU 0.5x(1+erf(x/sqrt2)))
+ *   f[r]  = h1[r] W2[e]^T              (W2: E*D*F bf16)
+ *   y_perm[r] = sigmoid(gate[r]) f[r] + x_perm[r]
+ * fp32 accumulation on the tensor cores; h1, a1, f, y_perm stored as bf16.
+ *   h1: T*F bf16 (required: GEMM2 reads it).  a1, f: nullable.
+ */
+int base_expert_ffn(const void* x_perm, const int32_t* offsets, int T, int D, int F, int E,
+                    const void* W1, const void* W2, int act, const float* gate,
+                    void* y_perm, void* h1, void* a1, void* f, void* ws, size_t ws_bytes,
+                    cudaStream_t stream);
+
+/*
+ * a8: combine (fig. 2 inverse_sort): out[perm[slot]] = y_perm[slot], T*D bf16.
+ */
+int base_combine(const void* y_perm, const int32_t* perm, int T, int D, void* out,
+                 cudaStream_t stream);
+
+/*
+ * The whole layer forward on one stream without host synchronisation:
+ * scores -> (balanced auction | greedy) -> permute -> expert FFN + eq. 1 ->
+ * combine.  h: T*D bf16, w: E*D bf16, W1: E*F*D, W2: E*D*F bf16; out: T*D bf16.
+ * sv: host struct of caller-owned device buffers (see base_layer_saved).
+ * Greedy routing fills price/stats untouched and accepts any counts.
+ */
+int base_layer_fwd(const void* h, const void* w, const void* W1, const void* W2, int act,
+                   int routing, int T, int D, int E, int F, void* out,
+                   const base_layer_saved* sv, void* ws, size_t ws_bytes, cudaStream_t stream);
+
+/*
+ * a9: the layer backward with the assignment held fixed (the released code
+ * computes the routing affinities without gradient; the centroids receive
+ * gradient only through the gate, "Paper vs code").  Given dout (T*D bf16):
+ *   dy = dout[perm]; dgate = <dy, f>; ds = dgate sigma (1 - sigma);
+ *   dF = sigma dy; dH1 = dF W2_e; dW2_e = dF^T H1; dA1 = dH1 * act'(A1);
+ *   dW1_e = dA1^T x; dx = dA1 W1_e + dy + ds w_e; dw_e = sum_{t in e} ds h_t;
+ *   dh[t] = dx[inv[t]].
+ * Outputs: dh T*D bf16; dw E*D fp32; dW1 E*F*D fp32; dW2 E*D*F fp32.
+ * sv must hold the forward's a1, h1, f (non-null).
+ */
+int base_layer_bwd(const void* h, const void* w, const void* W1, const void* W2, int act,
+                   int T, int D, int E, int F, const base_layer_saved* sv, const void* dout,
+                   void* dh, float* dw, float* dW1, float* dW2, void* ws, size_t ws_bytes,
+                   cudaStream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BASE_H */
