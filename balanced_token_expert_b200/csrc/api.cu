@@ -1,0 +1,230 @@
+// api.cu -- the C ABI of libbase (declared in include/base.h): host-side
+// argument checks, workspace carving and the order of the launches.
+#include <cstdint>
+#include <cstring>
+
+#include "common.cuh"
+
+namespace base {
+
+int launch_scores_f32(const float* h, const float* w, int T, int D, int E, float* s, int32_t* q,
+                      cudaStream_t stream);
+int launch_scores_bf16(const void* h, const void* w, int T, int D, int E, float* s, int32_t* q,
+                       cudaStream_t stream);
+int launch_greedy(const int32_t* q, int T, int E, int32_t* assign, int32_t* counts,
+                  cudaStream_t stream);
+size_t auction_workspace_bytes(int T, int E);
+int launch_auction(const int32_t* q, int T, int E, int32_t* assign, int64_t* price,
+                   base_auction_stats* stats, void* ws, size_t ws_bytes, long long max_rounds,
+                   cudaStream_t stream);
+size_t permute_workspace_bytes(int T, int E);
+int launch_sort_by_expert(const int32_t* assign, int T, int E, int32_t* perm, int32_t* inv,
+                          int32_t* offsets, const float* s, float* gate, void* ws,
+                          cudaStream_t stream);
+int launch_move_rows(const void* src, const int32_t* idx, int T, int D, void* dst, bool scatter,
+                     cudaStream_t stream);
+size_t ffn_workspace_bytes(int E);
+int launch_expert_ffn(const void* x_perm, const int32_t* offsets, int T, int D, int F, int E,
+                      const void* W1, const void* W2, int act, const float* gate, void* y_perm,
+                      void* h1, void* a1, void* f, void* ws, cudaStream_t stream);
+size_t backward_workspace_bytes(int T, int E, int D, int F);
+int launch_layer_bwd(const void* h, const void* w, const void* W1, const void* W2, int act, int T,
+                     int D, int E, int F, const base_layer_saved* sv, const void* dout, void* dh,
+                     float* dw, float* dW1, float* dW2, void* ws, size_t ws_bytes,
+                     cudaStream_t stream);
+
+static bool aligned(const void* p, size_t a) {
+    return (reinterpret_cast<uintptr_t>(p) % a) == 0;
+}
+
+static bool shapes_ok(int T, int E) { return T >= 1 && E >= 2 && E <= 1024; }
+
+}  // namespace base
+
+using namespace base;
+
+extern "C" {
+
+const char* base_status_string(int status) {
+    switch (status) {
+        case BASE_OK: return "ok";
+        case BASE_ERR_INVALID_ARG: return "invalid argument";
+        case BASE_ERR_CUDA: return "CUDA error";
+        case BASE_ERR_NOT_CONVERGED: return "auction did not converge within the round cap";
+        case BASE_ERR_TIMEOUT: return "a bounded device-side wait gave up";
+        case BASE_ERR_WORKSPACE: return "workspace too small";
+        case BASE_ERR_UNSUPPORTED: return "shape not supported by the kernels";
+        default: return "unknown status";
+    }
+}
+
+const char* base_version(void) { return "libbase 0.1 (sm_100a)"; }
+
+size_t base_workspace_size(int T, int E, int D, int F) {
+    if (!shapes_ok(T, E) || D < 0 || F < 0) return 0;
+    size_t w = auction_workspace_bytes(T, E);
+    const size_t p = permute_workspace_bytes(T, E);
+    if (p > w) w = p;
+    const size_t f = ffn_workspace_bytes(E);
+    if (f > w) w = f;
+    if (F > 0 && D > 0) {
+        const size_t b = backward_workspace_bytes(T, E, D, F);
+        if (b > w) w = b;
+    }
+    return w;
+}
+
+/* Reads (and optionally clears) the sticky device error word.  Synchronous. */
+int base_device_error(int64_t* code, int clear) {
+    int64_t v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_device_error, sizeof(v)) != cudaSuccess) return BASE_ERR_CUDA;
+    if (code) *code = v;
+    if (clear) {
+        const int64_t z = 0;
+        if (cudaMemcpyToSymbol(g_device_error, &z, sizeof(z)) != cudaSuccess) return BASE_ERR_CUDA;
+    }
+    return BASE_OK;
+}
+
+int base_scores(const void* h, const void* w, int dtype, int T, int D, int E, float* s,
+                int32_t* q, cudaStream_t stream) {
+    if (!h || !w || (!s && !q) || !shapes_ok(T, E) || D < 1) return BASE_ERR_INVALID_ARG;
+    if ((s && !aligned(s, 16)) || (q && !aligned(q, 16))) return BASE_ERR_INVALID_ARG;
+    if (dtype == BASE_F32) {
+        if (!aligned(h, 4) || !aligned(w, 4)) return BASE_ERR_INVALID_ARG;
+        return launch_scores_f32(static_cast<const float*>(h), static_cast<const float*>(w), T, D,
+                                 E, s, q, stream);
+    }
+    if (dtype != BASE_BF16) return BASE_ERR_INVALID_ARG;
+    if (D % 8 != 0 || !aligned(h, 16) || !aligned(w, 16)) return BASE_ERR_INVALID_ARG;
+    return launch_scores_bf16(h, w, T, D, E, s, q, stream);
+}
+
+int base_assign_greedy(const int32_t* q, int T, int E, int32_t* assign, int32_t* counts,
+                       cudaStream_t stream) {
+    if (!q || !assign || !shapes_ok(T, E)) return BASE_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(assign, 4) || (counts && !aligned(counts, 4)))
+        return BASE_ERR_INVALID_ARG;
+    return launch_greedy(q, T, E, assign, counts, stream);
+}
+
+int base_assign_balanced(const int32_t* q, int T, int E, int32_t* assign, int64_t* price,
+                         base_auction_stats* stats, void* ws, size_t ws_bytes,
+                         cudaStream_t stream) {
+    if (!q || !assign || !price || !ws || !shapes_ok(T, E) || T % E != 0)
+        return BASE_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(assign, 4) || !aligned(price, 8) || !aligned(ws, 256) ||
+        (stats && !aligned(stats, 8)))
+        return BASE_ERR_INVALID_ARG;
+    if (ws_bytes < auction_workspace_bytes(T, E)) return BASE_ERR_WORKSPACE;
+    return launch_auction(q, T, E, assign, price, stats, ws, ws_bytes, BASE_AUCTION_MAX_ROUNDS,
+                          stream);
+}
+
+/* Same as base_assign_balanced with a smaller round cap (for tests of the
+   not-converged path). */
+int base_assign_balanced_capped(const int32_t* q, int T, int E, int32_t* assign, int64_t* price,
+                                base_auction_stats* stats, void* ws, size_t ws_bytes,
+                                long long max_rounds, cudaStream_t stream) {
+    if (max_rounds < 1 || max_rounds > BASE_AUCTION_MAX_ROUNDS) return BASE_ERR_INVALID_ARG;
+    if (!q || !assign || !price || !ws || !shapes_ok(T, E) || T % E != 0)
+        return BASE_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(assign, 4) || !aligned(price, 8) || !aligned(ws, 256) ||
+        (stats && !aligned(stats, 8)))
+        return BASE_ERR_INVALID_ARG;
+    if (ws_bytes < auction_workspace_bytes(T, E)) return BASE_ERR_WORKSPACE;
+    return launch_auction(q, T, E, assign, price, stats, ws, ws_bytes, max_rounds, stream);
+}
+
+int base_permute(const void* h, const int32_t* assign, int T, int D, int E, int32_t* perm,
+                 int32_t* inv, int32_t* offsets, void* x_perm, const float* s, float* gate,
+                 void* ws, size_t ws_bytes, cudaStream_t stream) {
+    if (!assign || !perm || !inv || !offsets || !ws || !shapes_ok(T, E)) return BASE_ERR_INVALID_ARG;
+    if ((h == nullptr) != (x_perm == nullptr)) return BASE_ERR_INVALID_ARG;
+    if ((s == nullptr) != (gate == nullptr)) return BASE_ERR_INVALID_ARG;
+    if (h && (D < 8 || D % 8 != 0 || !aligned(h, 16) || !aligned(x_perm, 16)))
+        return BASE_ERR_INVALID_ARG;
+    if (!aligned(ws, 256)) return BASE_ERR_INVALID_ARG;
+    if (ws_bytes < permute_workspace_bytes(T, E)) return BASE_ERR_WORKSPACE;
+    int st = launch_sort_by_expert(assign, T, E, perm, inv, offsets, s, gate, ws, stream);
+    if (st != BASE_OK || !h) return st;
+    return launch_move_rows(h, perm, T, D, x_perm, false, stream);
+}
+
+int base_expert_ffn(const void* x_perm, const int32_t* offsets, int T, int D, int F, int E,
+                    const void* W1, const void* W2, int act, const float* gate, void* y_perm,
+                    void* h1, void* a1, void* f, void* ws, size_t ws_bytes, cudaStream_t stream) {
+    if (!x_perm || !offsets || !W1 || !W2 || !gate || !y_perm || !h1 || !ws || !shapes_ok(T, E))
+        return BASE_ERR_INVALID_ARG;
+    if (D < 8 || D % 8 != 0 || F < 8 || F % 8 != 0) return BASE_ERR_INVALID_ARG;
+    if (act != BASE_RELU && act != BASE_GELU) return BASE_ERR_INVALID_ARG;
+    const void* p16[] = {x_perm, W1, W2, y_perm, h1};
+    for (const void* p : p16)
+        if (!aligned(p, 16)) return BASE_ERR_INVALID_ARG;
+    if ((a1 && !aligned(a1, 16)) || (f && !aligned(f, 16)) || !aligned(ws, 256))
+        return BASE_ERR_INVALID_ARG;
+    if (ws_bytes < ffn_workspace_bytes(E)) return BASE_ERR_WORKSPACE;
+    return launch_expert_ffn(x_perm, offsets, T, D, F, E, W1, W2, act, gate, y_perm, h1, a1, f, ws,
+                             stream);
+}
+
+int base_combine(const void* y_perm, const int32_t* perm, int T, int D, void* out,
+                 cudaStream_t stream) {
+    if (!y_perm || !perm || !out || T < 1 || D < 8 || D % 8 != 0) return BASE_ERR_INVALID_ARG;
+    if (!aligned(y_perm, 16) || !aligned(out, 16)) return BASE_ERR_INVALID_ARG;
+    return launch_move_rows(y_perm, perm, T, D, out, true, stream);
+}
+
+int base_layer_fwd(const void* h, const void* w, const void* W1, const void* W2, int act,
+                   int routing, int T, int D, int E, int F, void* out, const base_layer_saved* sv,
+                   void* ws, size_t ws_bytes, cudaStream_t stream) {
+    if (!h || !w || !W1 || !W2 || !out || !sv || !ws || !shapes_ok(T, E))
+        return BASE_ERR_INVALID_ARG;
+    if (!sv->s || !sv->q || !sv->assign || !sv->perm || !sv->inv || !sv->offsets || !sv->gate ||
+        !sv->x_perm || !sv->h1 || !sv->y_perm)
+        return BASE_ERR_INVALID_ARG;
+    if (routing == BASE_ROUTE_BALANCED) {
+        if (!sv->price || T % E != 0) return BASE_ERR_INVALID_ARG;
+    } else if (routing != BASE_ROUTE_GREEDY) {
+        return BASE_ERR_INVALID_ARG;
+    }
+    if (ws_bytes < base_workspace_size(T, E, D, 0)) return BASE_ERR_WORKSPACE;
+    int st = base_scores(h, w, BASE_BF16, T, D, E, sv->s, sv->q, stream);
+    if (st != BASE_OK) return st;
+    if (routing == BASE_ROUTE_BALANCED)
+        st = base_assign_balanced(sv->q, T, E, sv->assign, sv->price, sv->stats, ws, ws_bytes,
+                                  stream);
+    else
+        st = base_assign_greedy(sv->q, T, E, sv->assign, nullptr, stream);
+    if (st != BASE_OK) return st;
+    st = base_permute(h, sv->assign, T, D, E, sv->perm, sv->inv, sv->offsets, sv->x_perm, sv->s,
+                      sv->gate, ws, ws_bytes, stream);
+    if (st != BASE_OK) return st;
+    st = base_expert_ffn(sv->x_perm, sv->offsets, T, D, F, E, W1, W2, act, sv->gate, sv->y_perm,
+                         sv->h1, sv->a1, sv->f, ws, ws_bytes, stream);
+    if (st != BASE_OK) return st;
+    return base_combine(sv->y_perm, sv->perm, T, D, out, stream);
+}
+
+int base_layer_bwd(const void* h, const void* w, const void* W1, const void* W2, int act, int T,
+                   int D, int E, int F, const base_layer_saved* sv, const void* dout, void* dh,
+                   float* dw, float* dW1, float* dW2, void* ws, size_t ws_bytes,
+                   cudaStream_t stream) {
+    if (!h || !w || !W1 || !W2 || !sv || !dout || !dh || !dw || !dW1 || !dW2 || !ws ||
+        !shapes_ok(T, E))
+        return BASE_ERR_INVALID_ARG;
+    if (D < 8 || D % 8 != 0 || F < 8 || F % 8 != 0) return BASE_ERR_INVALID_ARG;
+    if (act != BASE_RELU && act != BASE_GELU) return BASE_ERR_INVALID_ARG;
+    if (!sv->perm || !sv->inv || !sv->offsets || !sv->gate || !sv->x_perm || !sv->a1 || !sv->h1 ||
+        !sv->f || !sv->assign)
+        return BASE_ERR_INVALID_ARG;
+    const void* p16[] = {h, w, W1, W2, dout, dh, dw, dW1, dW2, sv->x_perm, sv->a1, sv->h1, sv->f};
+    for (const void* p : p16)
+        if (!aligned(p, 16)) return BASE_ERR_INVALID_ARG;
+    if (!aligned(ws, 256)) return BASE_ERR_INVALID_ARG;
+    if (ws_bytes < backward_workspace_bytes(T, E, D, F)) return BASE_ERR_WORKSPACE;
+    return launch_layer_bwd(h, w, W1, W2, act, T, D, E, F, sv, dout, dh, dw, dW1, dW2, ws, ws_bytes,
+                            stream);
+}
+
+}  // extern "C"

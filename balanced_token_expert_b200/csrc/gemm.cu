@@ -1,0 +1,716 @@
+// gemm.cu -- persistent, warp-specialised tcgen05 GEMM for sm_100a with the
+// BASE layer's epilogues fused in.
+//
+//   D[m, n] = sum_k A[m, k] B[n, k]     A, B bf16 in global memory, fp32 in TMEM
+//
+// Rows of A may be split into groups (the experts' slot segments,
+// offsets[g] .. offsets[g+1]); group g multiplies with its own block of B
+// rows (the expert's weight matrix).  Tiles are 128 x BN x 64:
+//   warp 0      one lane issues TMA loads of the A and B tiles into a ring of
+//               STAGES shared-memory stages (128-byte swizzle),
+//   warp 1      allocates TMEM (two BN-column fp32 accumulators) and one lane
+//               issues tcgen05.mma (M=128, N=BN, K=16) per 16-wide K slice,
+//   warps 4..7  the epilogue: tcgen05.ld of the accumulator (warp w reads
+//               TMEM lanes 32 (w%4) ..), the fused element-wise work and
+//               16-byte stores; the two accumulators let the epilogue of one
+//               tile overlap the MMAs of the next.
+// Operands may also be MN-major (A stored K x M, B stored K x N, M/N
+// contiguous), read as 64 x 64 TMA boxes and described to the tensor core as
+// MN-major 128-byte-swizzled tiles; the backward uses this to multiply by
+// transposed activations and weights without transposing them in memory.
+// In K-grouped mode (the weight gradients) group g reduces over its own slot
+// range offsets[g] .. offsets[g+1] along K and writes its own M x N block.
+// Every mbarrier wait is bounded; a wait that gives up records an error code
+// in the device error word and the kernel winds down (waiting, bounded, for
+// its own TMA copies and MMAs in flight, then freeing TMEM).
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <mutex>
+
+#include "tc.cuh"
+
+namespace base {
+namespace gemm {
+
+constexpr int BM = 128;
+constexpr int BK = 64;
+constexpr int kThreads = 256;
+
+enum Epi : int {
+    EPI_SCORES = 0,  // s (fp32) and q = rint(s 2^16) (int32)
+    EPI_ACT = 1,     // h1 = act(acc) bf16, a1 = acc bf16 (optional)
+    EPI_GATE = 2,    // y = sigmoid(gate[row]) acc + x[row] bf16, f = acc bf16 (optional)
+    EPI_DACT = 3,    // dA1 = acc * act'(a1[row]) bf16
+    EPI_DX = 4,      // dh[idx[row]] = acc + dy[row] + ds[row] w_g  bf16
+    EPI_F32 = 5,     // out_f32[g][row][col] = acc (K-grouped weight gradients)
+};
+
+struct Args {
+    int M;                       // rows of A
+    int N;                       // columns of D per group (rows of B per group)
+    int K;
+    int groups;                  // 1 when offsets == nullptr
+    const int32_t* offsets;      // [groups+1] row segments of A (nullable)
+    const int32_t* tile_start;   // [groups+1] prefix sums of the groups' 128-row tiles
+    int b_rows_per_group;        // row offset of group g's B block = g * b_rows_per_group
+    int n_tiles;                 // ceil(N / BN)
+    int ld;                      // row stride (elements) of outputs and side inputs
+    int act;                     // base_act
+    float* out_f32;
+    int32_t* out_q;
+    __nv_bfloat16* out0;
+    __nv_bfloat16* out1;
+    const float* gate;
+    const __nv_bfloat16* side;
+    const __nv_bfloat16* side2;  // centroids w (EPI_DX)
+    const int32_t* idx;          // destination rows (EPI_DX)
+    int kgroup;                  // 1: groups split K (weight gradients), M and N fixed
+    int m_tiles;                 // K-grouped mode: tiles along M per group
+};
+
+struct TileInfo {
+    int group, a_row, b_row, n0, m_local0, group_rows;
+    int k0, kblocks;  // first K index and number of 64-wide K blocks
+};
+
+__device__ __forceinline__ TileInfo decode_tile(const Args& a, int tile, int bn) {
+    TileInfo ti;
+    ti.k0 = 0;
+    ti.kblocks = (a.K + BK - 1) / BK;
+    if (a.kgroup) {
+        const int per = a.m_tiles * a.n_tiles;
+        const int g = tile / per, local = tile % per;
+        const int nt = local / a.m_tiles, m = local % a.m_tiles;
+        const int k0 = __ldg(a.offsets + g);
+        ti.group = g;
+        ti.a_row = m * BM;
+        ti.m_local0 = m * BM;
+        ti.group_rows = a.M;
+        ti.n0 = nt * bn;
+        ti.b_row = nt * bn;
+        ti.k0 = k0;
+        ti.kblocks = (__ldg(a.offsets + g + 1) - k0) / BK;
+        return ti;
+    }
+    if (a.offsets == nullptr) {
+        const int mt = (a.M + BM - 1) / BM;
+        const int nt = tile / mt, m = tile % mt;
+        ti.group = 0;
+        ti.a_row = m * BM;
+        ti.m_local0 = m * BM;
+        ti.group_rows = a.M;
+        ti.n0 = nt * bn;
+        ti.b_row = nt * bn;
+        return ti;
+    }
+    // group g holds tiles [tile_start[g] * n_tiles, tile_start[g+1] * n_tiles)
+    int lo = 0, hi = a.groups;  // find the last g with tile_start[g] * n_tiles <= tile
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (__ldg(a.tile_start + mid) * a.n_tiles <= tile) lo = mid; else hi = mid;
+    }
+    const int g = lo;
+    const int ts = __ldg(a.tile_start + g);
+    const int mtg = __ldg(a.tile_start + g + 1) - ts;
+    const int local = tile - ts * a.n_tiles;
+    const int nt = local / mtg, m = local % mtg;
+    const int r0 = __ldg(a.offsets + g);
+    ti.group = g;
+    ti.a_row = r0 + m * BM;
+    ti.m_local0 = m * BM;
+    ti.group_rows = __ldg(a.offsets + g + 1) - r0;
+    ti.n0 = nt * bn;
+    ti.b_row = g * a.b_rows_per_group + nt * bn;
+    return ti;
+}
+
+__device__ __forceinline__ float act_fwd(float x, int act) {
+    if (act == BASE_RELU) return fmaxf(x, 0.f);
+    return 0.5f * x * (1.f + erff(x * 0.70710678118654752f));
+}
+
+__device__ __forceinline__ float act_grad(float x, int act) {
+    if (act == BASE_RELU) return x > 0.f ? 1.f : 0.f;
+    return 0.5f * (1.f + erff(x * 0.70710678118654752f)) +
+           x * expf(-0.5f * x * x) * 0.39894228040143268f;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t*>(&v);
+}
+
+__device__ __forceinline__ void store_bf16x16(__nv_bfloat16* dst, const float (&f)[16]) {
+    uint4 a, b;
+    a.x = pack_bf16x2(f[0], f[1]);
+    a.y = pack_bf16x2(f[2], f[3]);
+    a.z = pack_bf16x2(f[4], f[5]);
+    a.w = pack_bf16x2(f[6], f[7]);
+    b.x = pack_bf16x2(f[8], f[9]);
+    b.y = pack_bf16x2(f[10], f[11]);
+    b.z = pack_bf16x2(f[12], f[13]);
+    b.w = pack_bf16x2(f[14], f[15]);
+    uint4* d = reinterpret_cast<uint4*>(dst);
+    d[0] = a;
+    d[1] = b;
+}
+
+__device__ __forceinline__ void load_bf16x16(const __nv_bfloat16* src, float (&f)[16]) {
+    const uint4* s = reinterpret_cast<const uint4*>(src);
+    const uint4 a = __ldg(s), b = __ldg(s + 1);
+    const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        f[2 * i] = __uint_as_float(w[i] << 16);
+        f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    }
+}
+
+// 16 accumulator columns [col, col+16) of one row.
+template <int EPI>
+__device__ __forceinline__ void epilogue16(const Args& a, const TileInfo& ti, int row, int col,
+                                           const uint32_t (&v)[16]) {
+    float f[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) f[i] = __uint_as_float(v[i]);
+    const size_t base = (size_t)row * a.ld + col;
+    if constexpr (EPI == EPI_SCORES) {
+        if (col + 16 <= a.N && (a.ld & 3) == 0) {
+            if (a.out_f32) {
+                float4* d = reinterpret_cast<float4*>(a.out_f32 + base);
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    d[i] = make_float4(f[4 * i], f[4 * i + 1], f[4 * i + 2], f[4 * i + 3]);
+            }
+            if (a.out_q) {
+                int4* d = reinterpret_cast<int4*>(a.out_q + base);
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    d[i] = make_int4(quantize_score(f[4 * i]), quantize_score(f[4 * i + 1]),
+                                     quantize_score(f[4 * i + 2]), quantize_score(f[4 * i + 3]));
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                if (col + i < a.N) {
+                    if (a.out_f32) a.out_f32[base + i] = f[i];
+                    if (a.out_q) a.out_q[base + i] = quantize_score(f[i]);
+                }
+            }
+        }
+    } else if constexpr (EPI == EPI_ACT) {
+        float h[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) h[i] = act_fwd(f[i], a.act);
+        if (col + 16 <= a.N) {
+            if (a.out1) store_bf16x16(a.out1 + base, f);
+            store_bf16x16(a.out0 + base, h);
+        } else {
+            for (int i = 0; i < a.N - col; ++i) {
+                if (a.out1) a.out1[base + i] = __float2bfloat16_rn(f[i]);
+                a.out0[base + i] = __float2bfloat16_rn(h[i]);
+            }
+        }
+    } else if constexpr (EPI == EPI_GATE) {
+        const float g = __ldg(a.gate + row);
+        const float sg = 1.f / (1.f + expf(-g));
+        if (col + 16 <= a.N) {
+            if (a.out1) store_bf16x16(a.out1 + base, f);
+            float x[16];
+            load_bf16x16(a.side + base, x);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) x[i] = fmaf(sg, f[i], x[i]);
+            store_bf16x16(a.out0 + base, x);
+        } else {
+            for (int i = 0; i < a.N - col; ++i) {
+                if (a.out1) a.out1[base + i] = __float2bfloat16_rn(f[i]);
+                const float x = __bfloat162float(a.side[base + i]);
+                a.out0[base + i] = __float2bfloat16_rn(fmaf(sg, f[i], x));
+            }
+        }
+    } else if constexpr (EPI == EPI_DACT) {
+        const int nv = min(16, a.N - col);
+        if (nv == 16) {
+            float x[16];
+            load_bf16x16(a.side + base, x);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) f[i] *= act_grad(x[i], a.act);
+            store_bf16x16(a.out0 + base, f);
+        } else {
+            for (int i = 0; i < nv; ++i)
+                a.out0[base + i] = __float2bfloat16_rn(
+                    f[i] * act_grad(__bfloat162float(a.side[base + i]), a.act));
+        }
+    } else if constexpr (EPI == EPI_DX) {
+        const float ds = __ldg(a.gate + row);
+        const __nv_bfloat16* wg = a.side2 + (size_t)ti.group * a.N + col;
+        const size_t dst = (size_t)__ldg(a.idx + row) * a.ld + col;
+        const int nv = min(16, a.N - col);
+        if (nv == 16) {
+            float dy[16], wv[16];
+            load_bf16x16(a.side + base, dy);
+            load_bf16x16(wg, wv);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) f[i] = f[i] + dy[i] + ds * wv[i];
+            store_bf16x16(a.out0 + dst, f);
+        } else {
+            for (int i = 0; i < nv; ++i)
+                a.out0[dst + i] = __float2bfloat16_rn(f[i] + __bfloat162float(a.side[base + i]) +
+                                                      ds * __bfloat162float(wg[i]));
+        }
+    } else if constexpr (EPI == EPI_F32) {
+        float* o = a.out_f32 + (size_t)ti.group * a.M * a.N + (size_t)row * a.N + col;
+        const int nv = min(16, a.N - col);
+        if (nv == 16 && (a.N & 3) == 0) {
+            float4* d = reinterpret_cast<float4*>(o);
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                d[i] = make_float4(f[4 * i], f[4 * i + 1], f[4 * i + 2], f[4 * i + 3]);
+        } else {
+            for (int i = 0; i < nv; ++i) o[i] = f[i];
+        }
+    }
+}
+
+template <int BN, int STAGES, int EPI, bool A_MN, bool B_MN>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                const Args args) {
+    constexpr uint32_t A_BYTES = BM * BK * 2;
+    constexpr uint32_t B_BYTES = BN * BK * 2;
+    constexpr uint32_t TMEM_COLS = (2 * BN < 32) ? 32 : 2 * BN;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                               ~uintptr_t(1023));
+    uint8_t* sA = smem;
+    uint8_t* sB = smem + STAGES * A_BYTES;
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * (A_BYTES + B_BYTES));
+    uint64_t* empty = full + STAGES;
+    uint64_t* tfull = empty + STAGES;
+    uint64_t* tempty = tfull + 2;
+    uint64_t* done = tempty + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+
+    const int warp = warp_id(), lane = lane_id();
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            tc::mbar_init(&full[s], 1);
+            tc::mbar_init(&empty[s], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            tc::mbar_init(&tfull[i], 1);
+            tc::mbar_init(&tempty[i], 4);
+        }
+        tc::mbar_init(done, 1);
+        tc::fence_mbar_init();
+    }
+    if (warp == 1) {
+        tc::tmem_alloc(tmem_slot, TMEM_COLS);
+        tc::tmem_relinquish();
+    }
+    if (warp == 0 && lane == 0) {
+        tc::tma_prefetch_desc(&tmA);
+        tc::tma_prefetch_desc(&tmB);
+    }
+    tc::tc_fence_before();
+    __syncthreads();
+    tc::tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    const int mtiles = args.kgroup ? args.m_tiles * args.groups
+                       : args.offsets ? __ldg(args.tile_start + args.groups)
+                                      : (args.M + BM - 1) / BM;
+    const int total = mtiles * args.n_tiles;
+
+    if (warp == 0 && lane == 0) {
+        // ---------------- TMA producer ----------------
+        int stage = 0;
+        uint32_t phase = 0;
+        bool ok = true;
+        uint32_t issued_parity[STAGES];
+        bool issued[STAGES];
+        for (int s = 0; s < STAGES; ++s) issued[s] = false;
+        for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+            const TileInfo ti = decode_tile(args, tile, BN);
+            for (int kb = 0; kb < ti.kblocks; ++kb) {
+                if (!tc::mbar_wait(&empty[stage], phase ^ 1, 3001)) {
+                    ok = false;
+                    break;
+                }
+                tc::mbar_arrive_expect_tx(&full[stage], A_BYTES + B_BYTES);
+                const int kg = ti.k0 + kb * BK;
+                if constexpr (A_MN) {
+                    // A stored K x M: two 64(M) x 64(K) boxes
+#pragma unroll
+                    for (int j = 0; j < BM / 64; ++j)
+                        tc::tma_load_2d(sA + stage * A_BYTES + j * 8192, &tmA, &full[stage],
+                                        ti.a_row + 64 * j, kg);
+                } else {
+                    tc::tma_load_2d(sA + stage * A_BYTES, &tmA, &full[stage], kg, ti.a_row);
+                }
+                if constexpr (B_MN) {
+                    // B stored K x N: BN / 64 boxes; the group's K rows start at b_row_k
+                    const int krow = args.kgroup ? kg : ti.group * args.b_rows_per_group + kb * BK;
+#pragma unroll
+                    for (int j = 0; j < BN / 64; ++j)
+                        tc::tma_load_2d(sB + stage * B_BYTES + j * 8192, &tmB, &full[stage],
+                                        ti.n0 + 64 * j, krow);
+                } else {
+                    tc::tma_load_2d(sB + stage * B_BYTES, &tmB, &full[stage], kg, ti.b_row);
+                }
+                issued[stage] = true;
+                issued_parity[stage] = phase;
+                if (++stage == STAGES) {
+                    stage = 0;
+                    phase ^= 1;
+                }
+            }
+        }
+        if (!ok) {
+            // wind down: let the copies already issued land before the CTA exits
+            for (int s = 0; s < STAGES; ++s) {
+                if (!issued[s]) continue;
+                const uint32_t a = smem_u32(&full[s]);
+                const uint64_t t0 = tc::globaltimer();
+                while (!tc::mbar_try_wait(a, issued_parity[s]) &&
+                       tc::globaltimer() - t0 < 100000000ull) {
+                }
+            }
+        }
+    } else if (warp == 1 && lane == 0) {
+        // ---------------- MMA issuer ----------------
+        constexpr uint32_t idesc = tc::idesc_bf16(BM, BN, A_MN ? 1 : 0, B_MN ? 1 : 0);
+        int stage = 0;
+        uint32_t phase = 0;
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        bool ok = true;
+        for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+            if (!tc::mbar_wait(&tempty[acc], acc_phase ^ 1, 3002)) break;
+            tc::tc_fence_after();
+            const uint32_t d_tmem = tmem_base + acc * BN;
+            const int kblocks = decode_tile(args, tile, BN).kblocks;
+            for (int kb = 0; kb < kblocks; ++kb) {
+                if (!tc::mbar_wait(&full[stage], phase, 3003)) {
+                    ok = false;
+                    break;
+                }
+                tc::tc_fence_after();
+                const uint32_t a_addr = smem_u32(sA + stage * A_BYTES);
+                const uint32_t b_addr = smem_u32(sB + stage * B_BYTES);
+#pragma unroll
+                for (int kk = 0; kk < BK / 16; ++kk) {
+                    // K-major: the 16-wide K slice is 32 bytes into each 128-byte row;
+                    // MN-major: it is 16 rows (2048 bytes) further down the tile
+                    const uint64_t ad = A_MN ? tc::smem_desc_sw128(a_addr + kk * 2048, 8192, 1024)
+                                             : tc::smem_desc_sw128(a_addr + kk * 32, 16, 1024);
+                    const uint64_t bd = B_MN ? tc::smem_desc_sw128(b_addr + kk * 2048, 8192, 1024)
+                                             : tc::smem_desc_sw128(b_addr + kk * 32, 16, 1024);
+                    tc::umma_bf16(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+                }
+                tc::umma_commit(&empty[stage]);
+                if (++stage == STAGES) {
+                    stage = 0;
+                    phase ^= 1;
+                }
+            }
+            if (!ok) break;
+            tc::umma_commit(&tfull[acc]);
+            acc ^= 1;
+            if (acc == 0) acc_phase ^= 1;
+        }
+        // every MMA issued by this thread has finished once `done` flips
+        tc::umma_commit(done);
+        tc::mbar_wait(done, 0, 3004);
+    } else if (warp >= 4) {
+        // ---------------- epilogue ----------------
+        const int ew = warp - 4;
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+            const TileInfo ti = decode_tile(args, tile, BN);
+            const bool ok = tc::mbar_wait(&tfull[acc], acc_phase, 3005);
+            if (!__all_sync(0xffffffffu, ok)) break;  // the whole warp leaves together
+            tc::tc_fence_after();
+            const int r = ew * 32 + lane;
+            const bool valid = ti.m_local0 + r < ti.group_rows;
+            const int row = ti.a_row + r;
+#pragma unroll 1
+            for (int c0 = 0; c0 < BN; c0 += 16) {
+                uint32_t v[16];
+                tc::tmem_ld16(tmem_base + ((uint32_t)(ew * 32) << 16) + acc * BN + c0, v);
+                tc::tmem_wait_ld();
+                if (ti.kblocks == 0) {
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) v[i] = 0u;
+                }
+                if (valid && ti.n0 + c0 < args.N) epilogue16<EPI>(args, ti, row, ti.n0 + c0, v);
+            }
+            tc::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(&tempty[acc]);
+            acc ^= 1;
+            if (acc == 0) acc_phase ^= 1;
+        }
+    }
+    tc::tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc::tc_fence_after();
+        tc::tmem_dealloc(tmem_base, TMEM_COLS);
+    }
+}
+
+__global__ void tile_prefix_kernel(const int32_t* __restrict__ offsets, int G,
+                                   int32_t* __restrict__ tile_start) {
+    __shared__ int32_t s_warp[32];
+    const int g = threadIdx.x;
+    const int lane = lane_id(), w = warp_id();
+    int v = 0;
+    if (g < G) v = (__ldg(offsets + g + 1) - __ldg(offsets + g) + BM - 1) / BM;
+    int incl = v;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int o = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += o;
+    }
+    if (lane == 31) s_warp[w] = incl;
+    __syncthreads();
+    if (w == 0) {
+        const int x = s_warp[lane];
+        int xi = x;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int o = __shfl_up_sync(0xffffffffu, xi, off);
+            if (lane >= off) xi += o;
+        }
+        s_warp[lane] = xi - x;
+    }
+    __syncthreads();
+    const int excl = incl - v + s_warp[w];
+    if (g < G) tile_start[g] = excl;
+    if (g == G - 1) tile_start[G] = excl + v;
+}
+
+// ------------------------------------------------------------------ host side
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// row-major bf16 matrix [rows][cols], box = box_rows x 64 columns, 128 B swizzle
+static bool make_tmap(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
+                      uint32_t box_rows) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols * 2};
+    cuuint32_t box[2] = {(cuuint32_t)BK, box_rows};
+    cuuint32_t es[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+              es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+static int num_sms() {
+    static int n = 0;
+    if (n == 0) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+            n = 148;
+    }
+    return n;
+}
+
+// A: a_rows x a_cols row-major (K-major: a_cols = K; MN-major: a_rows = K)
+// B: b_rows x b_cols row-major (likewise)
+template <int BN, int STAGES, int EPI, bool A_MN = false, bool B_MN = false>
+static int launch(const void* A, uint64_t a_rows, uint64_t a_cols, const void* B, uint64_t b_rows,
+                  uint64_t b_cols, const Args& args, int max_tiles, cudaStream_t stream) {
+    CUtensorMap ta, tb;
+    if (!make_tmap(&ta, A, a_rows, a_cols, A_MN ? 64 : BM)) return BASE_ERR_CUDA;
+    if (!make_tmap(&tb, B, b_rows, b_cols, B_MN ? 64 : BN)) return BASE_ERR_CUDA;
+    constexpr size_t smem = STAGES * (size_t)(BM * BK * 2 + BN * BK * 2) + 1024 + 256;
+    static_assert(smem <= 227 * 1024, "shared memory");
+    static_assert(!B_MN || BN % 64 == 0, "MN-major B needs BN % 64 == 0");
+    auto kern = gemm_kernel<BN, STAGES, EPI, A_MN, B_MN>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+        cudaSuccess)
+        return BASE_ERR_CUDA;
+    int grid = std::min(num_sms(), std::max(1, max_tiles));
+    kern<<<grid, kThreads, smem, stream>>>(ta, tb, args);
+    BASE_RETURN_IF_LAUNCH_FAILED();
+    return BASE_OK;
+}
+
+}  // namespace gemm
+
+// s = h w^T (+ q) for bf16 h (T x D) and w (E x D) on the tensor cores
+int launch_scores_bf16(const void* h, const void* w, int T, int D, int E, float* s, int32_t* q,
+                       cudaStream_t stream) {
+    using namespace gemm;
+    Args a{};
+    a.M = T;
+    a.N = E;
+    a.K = D;
+    a.groups = 1;
+    a.ld = E;
+    a.out_f32 = s;
+    a.out_q = q;
+    const int mt = (T + BM - 1) / BM;
+    if (E <= 16) {
+        a.n_tiles = 1;
+        return launch<16, 8, EPI_SCORES>(h, T, D, w, E, D, a, mt, stream);
+    } else if (E <= 32) {
+        a.n_tiles = 1;
+        return launch<32, 8, EPI_SCORES>(h, T, D, w, E, D, a, mt, stream);
+    } else if (E <= 64) {
+        a.n_tiles = 1;
+        return launch<64, 8, EPI_SCORES>(h, T, D, w, E, D, a, mt, stream);
+    } else if (E <= 128) {
+        a.n_tiles = 1;
+        return launch<128, 6, EPI_SCORES>(h, T, D, w, E, D, a, mt, stream);
+    }
+    a.n_tiles = (E + 255) / 256;
+    return launch<256, 4, EPI_SCORES>(h, T, D, w, E, D, a, mt * a.n_tiles, stream);
+}
+
+size_t ffn_workspace_bytes(int E) { return align_up(sizeof(int32_t) * (E + 1), 256); }
+
+// a6 + a7: h1 = act(x W1_e^T), y = sigmoid(gate) (h1 W2_e^T) + x per expert segment
+int launch_expert_ffn(const void* x_perm, const int32_t* offsets, int T, int D, int F, int E,
+                      const void* W1, const void* W2, int act, const float* gate, void* y_perm,
+                      void* h1, void* a1, void* f, void* ws, cudaStream_t stream) {
+    using namespace gemm;
+    int32_t* tile_start = static_cast<int32_t*>(ws);
+    tile_prefix_kernel<<<1, 1024, 0, stream>>>(offsets, E, tile_start);
+    BASE_RETURN_IF_LAUNCH_FAILED();
+    const int max_mt = (T + BM - 1) / BM + E;
+    Args g1{};
+    g1.M = T;
+    g1.N = F;
+    g1.K = D;
+    g1.groups = E;
+    g1.offsets = offsets;
+    g1.tile_start = tile_start;
+    g1.b_rows_per_group = F;
+    g1.n_tiles = (F + 255) / 256;
+    g1.ld = F;
+    g1.act = act;
+    g1.out0 = static_cast<__nv_bfloat16*>(h1);
+    g1.out1 = static_cast<__nv_bfloat16*>(a1);
+    int st = launch<256, 4, EPI_ACT>(x_perm, T, D, W1, (uint64_t)E * F, D, g1,
+                                     max_mt * g1.n_tiles, stream);
+    if (st != BASE_OK) return st;
+    Args g2{};
+    g2.M = T;
+    g2.N = D;
+    g2.K = F;
+    g2.groups = E;
+    g2.offsets = offsets;
+    g2.tile_start = tile_start;
+    g2.b_rows_per_group = D;
+    g2.n_tiles = (D + 255) / 256;
+    g2.ld = D;
+    g2.out0 = static_cast<__nv_bfloat16*>(y_perm);
+    g2.out1 = static_cast<__nv_bfloat16*>(f);
+    g2.gate = gate;
+    g2.side = static_cast<const __nv_bfloat16*>(x_perm);
+    return launch<256, 4, EPI_GATE>(h1, T, F, W2, (uint64_t)E * D, F, g2, max_mt * g2.n_tiles,
+                                    stream);
+}
+
+}  // namespace base
+
+namespace base {
+
+// the four contractions of the backward (see backward.cu)
+int launch_bwd_gemms(const void* dF, const void* /*unused*/, void* dA1, const void* a1,
+                     const void* h1, const void* x_perm, const void* dy, const float* ds,
+                     const void* w, const int32_t* perm, const int32_t* offsets,
+                     int32_t* tile_start, const void* W1, const void* W2, int act, int T, int D,
+                     int E, int F, void* dh, float* dW1, float* dW2, cudaStream_t stream) {
+    using namespace gemm;
+    tile_prefix_kernel<<<1, 1024, 0, stream>>>(offsets, E, tile_start);
+    BASE_RETURN_IF_LAUNCH_FAILED();
+    const int max_mt = (T + BM - 1) / BM + E;
+    // dH1 = dF W2_e (B = W2_e stored D x F: MN-major), dA1 = dH1 * act'(A1)
+    Args g{};
+    g.M = T;
+    g.N = F;
+    g.K = D;
+    g.groups = E;
+    g.offsets = offsets;
+    g.tile_start = tile_start;
+    g.b_rows_per_group = D;
+    g.n_tiles = (F + 255) / 256;
+    g.ld = F;
+    g.act = act;
+    g.side = static_cast<const __nv_bfloat16*>(a1);
+    g.out0 = static_cast<__nv_bfloat16*>(dA1);
+    int st = launch<256, 4, EPI_DACT, false, true>(dF, T, D, W2, (uint64_t)E * D, F, g,
+                                                   max_mt * g.n_tiles, stream);
+    if (st != BASE_OK) return st;
+    // dx = dA1 W1_e + dy + ds w_e (B = W1_e stored F x D: MN-major) -> dh[perm[r]]
+    Args x{};
+    x.M = T;
+    x.N = D;
+    x.K = F;
+    x.groups = E;
+    x.offsets = offsets;
+    x.tile_start = tile_start;
+    x.b_rows_per_group = F;
+    x.n_tiles = (D + 255) / 256;
+    x.ld = D;
+    x.side = static_cast<const __nv_bfloat16*>(dy);
+    x.gate = ds;
+    x.side2 = static_cast<const __nv_bfloat16*>(w);
+    x.idx = perm;
+    x.out0 = static_cast<__nv_bfloat16*>(dh);
+    st = launch<256, 4, EPI_DX, false, true>(dA1, T, F, W1, (uint64_t)E * F, D, x,
+                                             max_mt * x.n_tiles, stream);
+    if (st != BASE_OK) return st;
+    // dW2_e = dF_e^T H1_e: A = dF (T x D, MN-major, M = D), B = H1 (T x F, MN-major, N = F)
+    Args w2{};
+    w2.M = D;
+    w2.N = F;
+    w2.K = T;
+    w2.groups = E;
+    w2.offsets = offsets;
+    w2.kgroup = 1;
+    w2.m_tiles = (D + BM - 1) / BM;
+    w2.n_tiles = (F + 255) / 256;
+    w2.ld = F;
+    w2.out_f32 = dW2;
+    st = launch<256, 4, EPI_F32, true, true>(dF, T, D, h1, T, F, w2,
+                                             E * w2.m_tiles * w2.n_tiles, stream);
+    if (st != BASE_OK) return st;
+    // dW1_e = dA1_e^T x_e: A = dA1 (T x F, MN-major, M = F), B = x (T x D, MN-major, N = D)
+    Args w1{};
+    w1.M = F;
+    w1.N = D;
+    w1.K = T;
+    w1.groups = E;
+    w1.offsets = offsets;
+    w1.kgroup = 1;
+    w1.m_tiles = (F + BM - 1) / BM;
+    w1.n_tiles = (D + 255) / 256;
+    w1.ld = D;
+    w1.out_f32 = dW1;
+    return launch<256, 4, EPI_F32, true, true>(dA1, T, F, x_perm, T, D, w1,
+                                               E * w1.m_tiles * w1.n_tiles, stream);
+}
+
+}  // namespace base

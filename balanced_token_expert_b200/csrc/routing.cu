@@ -1,0 +1,332 @@
+// routing.cu -- the bandwidth-bound steps of the BASE layer:
+//   * fp32 affinity scores s = h w^T with their quantisation (fig. 2
+//     "affinities"; SIMT fp32 FMA: the tensor cores have no fp32-input mode
+//     accurate to 1e-5),
+//   * greedy test-time routing (argmax over experts, "Test time"),
+//   * the expert-major permutation (fig. 2 sort_by_expert) as a stable
+//     counting sort, and the 16-byte-vector row gather / scatter used by the
+//     permute, the combine (inverse_sort) and the backward.
+#include "common.cuh"
+
+namespace base {
+namespace routing {
+
+// ---------------------------------------------------------------------------
+// fp32 scores: one warp per (token, 32 experts); lanes split D.
+// ---------------------------------------------------------------------------
+__global__ void scores_f32_kernel(const float* __restrict__ h, const float* __restrict__ w,
+                                  int T, int D, int E, float* __restrict__ s,
+                                  int32_t* __restrict__ q) {
+    const int lane = lane_id();
+    const long long gw = (blockIdx.x * (long long)blockDim.x + threadIdx.x) / kWarp;
+    const long long nw = (gridDim.x * (long long)blockDim.x) / kWarp;
+    for (long long item = gw; item < (long long)T * E; item += nw) {
+        const int t = (int)(item / E), e = (int)(item % E);
+        const float* hr = h + (size_t)t * D;
+        const float* wr = w + (size_t)e * D;
+        float acc = 0.f;
+        for (int d = lane; d < D; d += kWarp) acc = fmaf(__ldg(hr + d), __ldg(wr + d), acc);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+        if (lane == 0) {
+            if (s) s[item] = acc;
+            if (q) q[item] = quantize_score(acc);
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// greedy routing: a group of lanes per token row, argmax with lowest index on
+// ties, per-block expert histogram folded into the global counts.
+// ---------------------------------------------------------------------------
+__global__ void greedy_kernel(const int32_t* __restrict__ q, int T, int E,
+                              int32_t* __restrict__ assign, int32_t* __restrict__ counts) {
+    extern __shared__ int32_t s_hist[];
+    for (int e = threadIdx.x; e < E; e += blockDim.x) s_hist[e] = 0;
+    __syncthreads();
+    int G = 1;
+    while (G < E && G < kWarp) G <<= 1;
+    const int lane = lane_id(), sub = lane / G, gl = lane % G;
+    const int per_warp = kWarp / G;
+    const long long gw = (blockIdx.x * (long long)blockDim.x + threadIdx.x) / kWarp;
+    const long long nw = (gridDim.x * (long long)blockDim.x) / kWarp;
+    for (long long base = gw * per_warp; base < T; base += nw * per_warp) {
+        const long long t = base + sub;
+        const bool valid = t < T;
+        int best_v = INT32_MIN, best_e = INT32_MAX;
+        if (valid) {
+            const int32_t* row = q + (size_t)t * E;
+            if ((E & 3) == 0 && G == kWarp) {
+                const int4* r4 = reinterpret_cast<const int4*>(row);
+                for (int j = gl; j < E / 4; j += kWarp) {
+                    const int4 v = __ldg(r4 + j);
+                    const int e0 = 4 * j;
+                    if (v.x > best_v) { best_v = v.x; best_e = e0; }
+                    if (v.y > best_v) { best_v = v.y; best_e = e0 + 1; }
+                    if (v.z > best_v) { best_v = v.z; best_e = e0 + 2; }
+                    if (v.w > best_v) { best_v = v.w; best_e = e0 + 3; }
+                }
+            } else {
+                for (int e = gl; e < E; e += G) {
+                    const int v = __ldg(row + e);
+                    if (v > best_v) { best_v = v; best_e = e; }
+                }
+            }
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            if (off >= G) continue;
+            const int ov = __shfl_xor_sync(0xffffffffu, best_v, off);
+            const int oe = __shfl_xor_sync(0xffffffffu, best_e, off);
+            if (ov > best_v || (ov == best_v && oe < best_e)) { best_v = ov; best_e = oe; }
+        }
+        if (valid && gl == 0) {
+            assign[t] = best_e;
+            if (counts) atomicAdd(&s_hist[best_e], 1);
+        }
+    }
+    if (counts) {
+        __syncthreads();
+        for (int e = threadIdx.x; e < E; e += blockDim.x)
+            if (s_hist[e]) atomicAdd(&counts[e], s_hist[e]);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// stable counting sort of tokens by expert
+//   chunk = kChunk consecutive tokens handled by one warp, in token order.
+//   1) per-chunk expert histogram  2) scan over chunks and experts
+//   3) per-chunk ranks -> perm, inv (and the permuted gate scores)
+// ---------------------------------------------------------------------------
+constexpr int kChunk = 256;
+constexpr int kSortWarps = 4;
+
+__global__ void chunk_hist_kernel(const int32_t* __restrict__ assign, int T, int E,
+                                  int32_t* __restrict__ chunk_counts) {
+    extern __shared__ int32_t s_cnt[];  // [kSortWarps][E]
+    const int w = warp_id(), lane = lane_id();
+    int32_t* my = s_cnt + w * E;
+    const int chunk = blockIdx.x * kSortWarps + w;
+    const int nchunks = (T + kChunk - 1) / kChunk;
+    for (int e = lane; e < E; e += kWarp) my[e] = 0;
+    __syncwarp();
+    if (chunk < nchunks) {
+        const int t0 = chunk * kChunk, t1 = min(T, t0 + kChunk);
+        for (int t = t0 + lane; t < t1; t += kWarp) {
+            const int e = assign[t];
+            if (e < 0 || e >= E) {  // not an expert: recorded, token skipped
+                record_error(2001);
+                continue;
+            }
+            atomicAdd(&my[e], 1);
+        }
+        __syncwarp();
+        for (int e = lane; e < E; e += kWarp) chunk_counts[(size_t)chunk * E + e] = my[e];
+    }
+}
+
+// one thread per expert walks the chunks; then a block scan over experts
+__global__ void chunk_scan_kernel(int32_t* __restrict__ chunk_counts, int nchunks, int E,
+                                  int32_t* __restrict__ offsets) {
+    __shared__ int32_t s_tot[1024];
+    __shared__ int32_t s_warp[32];
+    const int e = threadIdx.x;
+    int run = 0;
+    if (e < E) {
+        for (int c = 0; c < nchunks; ++c) {
+            const int v = chunk_counts[(size_t)c * E + e];
+            chunk_counts[(size_t)c * E + e] = run;
+            run += v;
+        }
+    }
+    // exclusive scan of run over experts (blockDim = 1024)
+    const int lane = lane_id(), w = warp_id();
+    int incl = (e < E) ? run : 0;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int o = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += o;
+    }
+    if (lane == 31) s_warp[w] = incl;
+    __syncthreads();
+    if (w == 0) {
+        int v = s_warp[lane];
+        int vi = v;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int o = __shfl_up_sync(0xffffffffu, vi, off);
+            if (lane >= off) vi += o;
+        }
+        s_warp[lane] = vi - v;
+    }
+    __syncthreads();
+    const int excl = incl - ((e < E) ? run : 0) + s_warp[w];
+    if (e < E) {
+        s_tot[e] = excl;
+        offsets[e] = excl;
+        if (e == E - 1) offsets[E] = excl + run;
+    }
+    __syncthreads();
+    if (e < E) {
+        for (int c = 0; c < nchunks; ++c) chunk_counts[(size_t)c * E + e] += s_tot[e];
+    }
+}
+
+__global__ void chunk_rank_kernel(const int32_t* __restrict__ assign, int T, int E,
+                                  const int32_t* __restrict__ chunk_base,
+                                  int32_t* __restrict__ perm, int32_t* __restrict__ inv,
+                                  const float* __restrict__ s, float* __restrict__ gate) {
+    extern __shared__ int32_t s_run[];  // [kSortWarps][E]
+    const int w = warp_id(), lane = lane_id();
+    int32_t* run = s_run + w * E;
+    const int chunk = blockIdx.x * kSortWarps + w;
+    const int nchunks = (T + kChunk - 1) / kChunk;
+    if (chunk >= nchunks) return;
+    for (int e = lane; e < E; e += kWarp) run[e] = chunk_base[(size_t)chunk * E + e];
+    __syncwarp();
+    const int t0 = chunk * kChunk, t1 = min(T, t0 + kChunk);
+    for (int b = t0; b < t1; b += kWarp) {
+        const int t = b + lane;
+        bool valid = t < t1;
+        int e = valid ? assign[t] : -1;
+        if (e < 0 || e >= E) {
+            e = -1 - lane;  // distinct dummies never match
+            valid = false;
+        }
+        const unsigned peers = __match_any_sync(0xffffffffu, e);
+        const int rank = __popc(peers & ((1u << lane) - 1));
+        int slot = 0;
+        if (valid) slot = run[e] + rank;
+        __syncwarp();
+        if (valid && lane == 31 - __clz(peers)) run[e] += __popc(peers);
+        __syncwarp();
+        if (valid) {
+            perm[slot] = t;
+            inv[t] = slot;
+            if (gate) gate[slot] = s[(size_t)t * E + e];
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// row gather / scatter of bf16 rows with 16-byte vectors:
+//   gather:  dst[r] = src[idx[r]]        scatter: dst[idx[r]] = src[r]
+// ---------------------------------------------------------------------------
+template <bool kScatter>
+__global__ void __launch_bounds__(256) move_rows_kernel(const uint4* __restrict__ src,
+                                                        const int32_t* __restrict__ idx, int T,
+                                                        int vec_per_row, uint4* __restrict__ dst) {
+    constexpr int kUnroll = 4;
+    const long long total = (long long)T * vec_per_row;
+    const long long stride = (long long)gridDim.x * blockDim.x;
+    long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x;
+    for (; i + (kUnroll - 1) * stride < total; i += kUnroll * stride) {
+        uint4 v[kUnroll];
+        long long o[kUnroll];
+        bool bad = false;
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            const long long j = i + u * stride;
+            const int r = (int)(j / vec_per_row), c = (int)(j % vec_per_row);
+            int m = __ldg(idx + r);
+            if ((unsigned)m >= (unsigned)T) {  // not a row: recorded, row 0 used instead
+                bad = true;
+                m = 0;
+            }
+            const long long si = kScatter ? j : (long long)m * vec_per_row + c;
+            o[u] = kScatter ? (long long)m * vec_per_row + c : j;
+            v[u] = __ldcs(src + si);
+        }
+        if (bad) {
+            record_error(2002);
+            continue;
+        }
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) __stcs(dst + o[u], v[u]);
+    }
+    for (; i < total; i += stride) {
+        const int r = (int)(i / vec_per_row), c = (int)(i % vec_per_row);
+        const int m = __ldg(idx + r);
+        if ((unsigned)m >= (unsigned)T) {
+            record_error(2002);
+            continue;
+        }
+        if (kScatter) __stcs(dst + (long long)m * vec_per_row + c, __ldcs(src + i));
+        else __stcs(dst + i, __ldcs(src + (long long)m * vec_per_row + c));
+    }
+}
+
+}  // namespace routing
+
+int launch_scores_f32(const float* h, const float* w, int T, int D, int E, float* s, int32_t* q,
+                      cudaStream_t stream) {
+    const long long items = (long long)T * E;
+    const int threads = 256;
+    long long blocks = (items * kWarp + threads - 1) / threads;
+    if (blocks > 148 * 16) blocks = 148 * 16;
+    routing::scores_f32_kernel<<<(int)blocks, threads, 0, stream>>>(h, w, T, D, E, s, q);
+    BASE_RETURN_IF_LAUNCH_FAILED();
+    return BASE_OK;
+}
+
+int launch_greedy(const int32_t* q, int T, int E, int32_t* assign, int32_t* counts,
+                  cudaStream_t stream) {
+    if (counts && cudaMemsetAsync(counts, 0, sizeof(int32_t) * E, stream) != cudaSuccess)
+        return BASE_ERR_CUDA;
+    const int threads = 256;
+    int G = 1;
+    while (G < E && G < kWarp) G <<= 1;
+    const long long warps_needed = ((long long)T * G + kWarp - 1) / kWarp;
+    long long blocks = (warps_needed * kWarp + threads - 1) / threads;
+    if (blocks > 148 * 8) blocks = 148 * 8;
+    if (blocks < 1) blocks = 1;
+    routing::greedy_kernel<<<(int)blocks, threads, sizeof(int32_t) * E, stream>>>(q, T, E, assign,
+                                                                                   counts);
+    BASE_RETURN_IF_LAUNCH_FAILED();
+    return BASE_OK;
+}
+
+size_t permute_workspace_bytes(int T, int E) {
+    const size_t nchunks = (size_t)(T + routing::kChunk - 1) / routing::kChunk;
+    return align_up(sizeof(int32_t) * nchunks * E, 256) + 256;
+}
+
+// perm / inv / offsets (+ gate) from an assignment.  An expert index out of
+// range is recorded in the device error word and its token is skipped.
+int launch_sort_by_expert(const int32_t* assign, int T, int E, int32_t* perm, int32_t* inv,
+                          int32_t* offsets, const float* s, float* gate, void* ws,
+                          cudaStream_t stream) {
+    using namespace routing;
+    const int nchunks = (T + kChunk - 1) / kChunk;
+    int32_t* chunk_counts = static_cast<int32_t*>(ws);
+    const int blocks = (nchunks + kSortWarps - 1) / kSortWarps;
+    const size_t smem = sizeof(int32_t) * kSortWarps * E;
+    chunk_hist_kernel<<<blocks, kSortWarps * kWarp, smem, stream>>>(assign, T, E, chunk_counts);
+    BASE_RETURN_IF_LAUNCH_FAILED();
+    chunk_scan_kernel<<<1, 1024, 0, stream>>>(chunk_counts, nchunks, E, offsets);
+    BASE_RETURN_IF_LAUNCH_FAILED();
+    chunk_rank_kernel<<<blocks, kSortWarps * kWarp, smem, stream>>>(assign, T, E, chunk_counts, perm,
+                                                                   inv, s, gate);
+    BASE_RETURN_IF_LAUNCH_FAILED();
+    return BASE_OK;
+}
+
+int launch_move_rows(const void* src, const int32_t* idx, int T, int D, void* dst, bool scatter,
+                     cudaStream_t stream) {
+    const int vec = D * 2 / 16;
+    const long long total = (long long)T * vec;
+    const int threads = 256;
+    long long blocks = (total + threads - 1) / threads;
+    if (blocks > 148 * 16) blocks = 148 * 16;
+    if (blocks < 1) blocks = 1;
+    if (scatter)
+        routing::move_rows_kernel<true><<<(int)blocks, threads, 0, stream>>>(
+            static_cast<const uint4*>(src), idx, T, vec, static_cast<uint4*>(dst));
+    else
+        routing::move_rows_kernel<false><<<(int)blocks, threads, 0, stream>>>(
+            static_cast<const uint4*>(src), idx, T, vec, static_cast<uint4*>(dst));
+    BASE_RETURN_IF_LAUNCH_FAILED();
+    return BASE_OK;
+}
+
+}  // namespace base

@@ -1,0 +1,337 @@
+#!/usr/bin/env python
+"""Benchmark of the BASE-layer forward hot path on B200.
+
+One step = one pass of the whole forward path over one batch of synthetic
+tokens: bf16 affinity scores + quantisation (tcgen05) -> balanced Jacobi
+auction -> expert-major permutation -> expert FFNs with the gated residual
+(tcgen05) -> combine.  Default workload: T=8192 tokens, E=16 experts,
+D=1024, FFN 1024 -> 4096 -> 1024 ReLU (bf16, random N(0, 0.02) weights,
+h ~ N(0,1), w ~ N(0, 1/D)).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+With N > 1 (torchrun, one rank per GPU) every rank runs its own independent
+problem (the balanced assignment decomposes per worker, so no collective is
+on the data path); the time is the max over ranks.  Rank 0 prints one JSON
+line.  ``--impl reference`` times the CPU oracle on the host cores instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "tokens routed/s (auction) & BASE-layer fwd tokens/s; % of HBM/TC roofline"
+UNIT = "tokens/s"
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--workload", default="layer_fwd")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--flush-mb", type=int, default=256)
+    return p.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        d = json.load(open(path))
+        return dict(hbm=float(d["hbm_gbs"]), bf16=float(d["bf16_tflops"]),
+                    bf16_sustained=float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                    source="measured")
+    except Exception:
+        return dict(hbm=6650.0, bf16=1590.0, bf16_sustained=1400.0, source="fallback")
+
+
+class Clocks:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+
+    def __init__(self, index: int):
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        try:
+            self.p = subprocess.Popen(["nvidia-smi", "-i", str(index), "--query-gpu=" + q,
+                                       "--format=csv,noheader,nounits", "-lms", "100"],
+                                      stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.p = None
+
+    def stop(self):
+        if self.p is None:
+            return None
+        self.p.terminate()
+        try:
+            self.p.wait(timeout=5)
+        except Exception:
+            self.p.kill()
+        self.f.flush()
+        rows = []
+        for line in open(self.f.name):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) >= 9:
+                rows.append(parts)
+        os.unlink(self.f.name)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i] == "Active"})
+        return dict(sm_mhz=statistics.median(sm) if sm else None,
+                    sm_max_mhz=max(mx) if mx else None, reasons=reasons, samples=len(rows))
+
+
+def cpu_baseline(wl, seed=0):
+    """The oracle as it stands, one full forward of the workload on the host."""
+    import oracle
+    from balanced_token_expert_b200 import synth
+    inp = synth.make_inputs(wl, seed)
+    t0 = time.perf_counter()
+    s = oracle.scores(inp.h, inp.w)
+    a = oracle.auction(oracle.quantize(s))[0]
+    oracle.layer_forward(inp.h, inp.w, inp.W1, inp.W2, wl.act, a)
+    dt = time.perf_counter() - t0
+    return dict(value=wl.T / dt, unit=UNIT, cores=len(os.sched_getaffinity(0)), kind="oracle",
+                sample="one full forward of the workload (T=%d tokens: float64 scores, integer "
+                       "auction, float64 expert FFNs) on the host, %.2f s" % (wl.T, dt))
+
+
+def run_reference(args, wl, rank, world):
+    if rank != 0:
+        return
+    import oracle
+    from balanced_token_expert_b200 import synth
+    oracle.build()
+    inp = synth.make_inputs(wl, 0)
+
+    def step():
+        s = oracle.scores(inp.h, inp.w)
+        a = oracle.auction(oracle.quantize(s))[0]
+        oracle.layer_forward(inp.h, inp.w, inp.W1, inp.W2, wl.act, a)
+
+    for _ in range(args.warmup):
+        step()
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        step()
+        times.append(time.perf_counter() - t0)
+    ms = 1e3 * statistics.mean(times)
+    value = wl.T / (ms / 1e3)
+    cores = len(os.sched_getaffinity(0))
+    print(json.dumps(dict(
+        impl="reference", metric=METRIC, value=value, unit=UNIT, n_gpus=world, steps=args.steps,
+        warmup=args.warmup, ms_per_step=ms, higher_is_better=True, scaling="weak",
+        vs_baseline=None, dtype="f64", data="synthetic",
+        config=_config(wl, args),
+        cpu_baseline=dict(value=value, unit=UNIT, cores=cores, kind="oracle",
+                          sample="every step: one full forward of the workload on the host"),
+        e2e=dict(value=value, unit=UNIT, h2d_bytes_per_step=0, d2h_bytes_per_step=0))))
+
+
+def _config(wl, args):
+    return dict(workload="%s: BASE layer forward, T=%d tokens, E=%d experts, D=%d, FFN %d->%d->%d "
+                         "%s, balanced auction routing, bf16" % (wl.name, wl.T, wl.E, wl.D, wl.D,
+                                                                 wl.F, wl.D, wl.act),
+                T=wl.T, E=wl.E, D=wl.D, F=wl.F, act=wl.act, routing="balanced",
+                l2="flushed between timed steps (%d MiB write)" % args.flush_mb,
+                parallelism="independent replica per GPU")
+
+
+def main():
+    args = parse()
+    from balanced_token_expert_b200 import synth
+    wl = synth.WORKLOADS[args.workload]
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, wl, rank, world)
+        return
+
+    import torch
+    import torch.distributed as dist
+    torch.cuda.set_device(local_rank)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    from balanced_token_expert_b200 import _build
+    from balanced_token_expert_b200 import binding as B
+    from balanced_token_expert_b200 import buffers
+    if rank == 0 or world == 1:
+        _build.build()
+    if world > 1:
+        dist.barrier()
+    B.lib()
+
+    T, E, D, F = wl.T, wl.E, wl.D, wl.F
+    inp = synth.make_inputs(wl, seed=rank)
+    h = inp.h.cuda()
+    w = inp.w.cuda()
+    W1 = inp.W1.cuda()
+    W2 = inp.W2.cuda()
+    act = B.BASE_RELU if wl.act == "relu" else B.BASE_GELU
+    sv = buffers.layer_saved(T, E, D, F, for_backward=False)
+    out = torch.empty(T, D, dtype=torch.bfloat16, device="cuda")
+    ws = buffers.workspace(T, E, D, F)
+    flush = torch.empty(args.flush_mb * (1 << 20), dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    names = ["scores", "auction", "permute", "ffn", "combine"]
+
+    def step(ev):
+        ev[0].record(stream)
+        B.base_scores(h, w, sv["s"], sv["q"])
+        ev[1].record(stream)
+        B.base_assign_balanced(sv["q"], sv["assign"], sv["price"], sv["stats"], ws)
+        ev[2].record(stream)
+        B.base_permute(h, sv["assign"], E, sv["perm"], sv["inv"], sv["offsets"], sv["x_perm"],
+                       sv["s"], sv["gate"], ws)
+        ev[3].record(stream)
+        B.base_expert_ffn(sv["x_perm"], sv["offsets"], W1, W2, act, sv["gate"], sv["y_perm"],
+                          sv["h1"], None, None, ws)
+        ev[4].record(stream)
+        B.base_combine(sv["y_perm"], sv["perm"], out)
+        ev[5].record(stream)
+
+    kernels_per_step = 1 + 3 + 4 + 3 + 1
+    mk = lambda: [torch.cuda.Event(enable_timing=True) for _ in range(6)]  # noqa: E731
+    for _ in range(max(3, args.warmup)):
+        flush.zero_()
+        step(mk())
+    torch.cuda.synchronize()
+    B.base_device_error(clear=True)
+
+    phys = 0
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if vis:
+        try:
+            phys = int(vis.split(",")[local_rank])
+        except ValueError:
+            phys = local_rank
+    else:
+        phys = local_rank
+    clocks = Clocks(phys) if rank == 0 else None
+
+    evs = [mk() for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    wall0 = time.perf_counter()
+    for i in range(args.steps):
+        flush.zero_()
+        step(evs[i])
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    wall = time.perf_counter() - wall0
+    per = {n: [] for n in names}
+    for ev in evs:
+        for j, n in enumerate(names):
+            per[n].append(ev[j].elapsed_time(ev[j + 1]))
+    step_ms = [sum(per[n][i] for n in names) for i in range(args.steps)]
+    ms = statistics.mean(step_ms)
+    st = buffers.stats_dict(sv["stats"])
+    err = B.base_device_error(clear=True)
+    if world > 1:
+        t = torch.tensor([ms], device="cuda", dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    clk = clocks.stop() if clocks else None
+
+    # end to end through the public call: host inputs in, host output back
+    h_host = inp.h.pin_memory()
+    out_host = torch.empty(T, D, dtype=torch.bfloat16).pin_memory()
+    h_dev = torch.empty_like(h)
+    sv2 = buffers.layer_saved(T, E, D, F, for_backward=False)
+
+    def e2e_step():
+        h_dev.copy_(h_host, non_blocking=True)
+        B.base_layer_fwd(h_dev, w, W1, W2, act, B.BASE_ROUTE_BALANCED, out, sv2, ws)
+        out_host.copy_(out, non_blocking=True)
+
+    for _ in range(3):
+        flush.zero_()
+        e2e_step()
+    torch.cuda.synchronize()
+    e2e_ms = []
+    for _ in range(args.steps):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        e2e_step()
+        b.record(stream)
+        b.synchronize()
+        e2e_ms.append(a.elapsed_time(b))
+    e2e = statistics.mean(e2e_ms)
+    if world > 1:
+        t = torch.tensor([e2e], device="cuda", dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e = float(t.item())
+
+    if rank == 0:
+        pk = peaks()
+        comp = {n: statistics.mean(per[n]) for n in names}
+        dom = max(comp, key=comp.get)
+        bids = st["bids"]
+        alg = dict(  # algorithmic work per launch (bytes or flops)
+            scores=("hbm", 2 * T * D + 2 * E * D + 8 * T * E),
+            auction=("hbm", 4 * E * bids + 4 * T + 8 * E),
+            permute=("hbm", 4 * T * D + 12 * T + 8 * T),
+            ffn=("tensor", 4 * T * D * F),
+            combine=("hbm", 4 * T * D + 4 * T))
+
+        def roof(n):
+            bound, work = alg[n]
+            sec = comp[n] / 1e3
+            if bound == "tensor":
+                a_ = work / sec / 1e12
+                return dict(bound="tensor", achieved=a_, peak=pk["bf16"], unit="TFLOP/s",
+                            frac=a_ / pk["bf16"], traffic=None, kernel=n, ms=comp[n],
+                            peak_source=pk["source"] + " burst bf16")
+            a_ = work / sec / 1e9
+            return dict(bound="hbm", achieved=a_, peak=pk["hbm"], unit="GB/s",
+                        frac=a_ / pk["hbm"], traffic=None, kernel=n, ms=comp[n],
+                        peak_source=pk["source"] + " hbm copy")
+
+        res = dict(
+            metric=METRIC, value=T * world / (ms / 1e3), unit=UNIT, n_gpus=world,
+            steps=args.steps, warmup=args.warmup, ms_per_step=ms, higher_is_better=True,
+            scaling="weak", vs_baseline=None, dtype="bf16", data="synthetic",
+            config=_config(wl, args),
+            roofline=roof(dom),
+            per_kernel={n: roof(n) for n in names},
+            auction=dict(tokens_per_s=T * world / (comp["auction"] / 1e3), rounds=st["rounds"],
+                         phases=st["phases"], bids=bids, status=st["status"],
+                         us_per_round=1e3 * comp["auction"] / max(1, st["rounds"])),
+            e2e=dict(value=T * world / (e2e / 1e3), unit=UNIT, h2d_bytes_per_step=T * D * 2,
+                     d2h_bytes_per_step=T * D * 2, ms_per_step=e2e),
+            gpu_launches=kernels_per_step * args.steps,
+            clocks=clk, device_error=err, wall_s=wall,
+        )
+        if world == 1 and not args.no_cpu_baseline:
+            res["cpu_baseline"] = cpu_baseline(wl)
+        print(json.dumps(res))
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

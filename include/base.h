@@ -24,9 +24,10 @@
  *   - Arguments are checked on the host before anything is launched; a bad
  *     argument returns BASE_ERR_INVALID_ARG and launches nothing.  A failed
  *     launch returns BASE_ERR_CUDA.  Failures found while the kernels run
- *     (round cap reached, a bounded wait that gave up) are written to the
- *     device-side status word of `base_auction_stats` (auction) or of the
- *     workspace (GEMMs) and read back by the caller after synchronising.
+ *     are written to device memory and read back by the caller after
+ *     synchronising: the auction's round cap goes to `stats->status`; a
+ *     bounded wait that gave up, or unusable device data, goes to the
+ *     library's sticky device error word (base_device_error).
  *   - bf16 means IEEE bfloat16 (1-8-7), fp32 IEEE binary32.
  *   - The library holds no per-call state; calls on different streams with
  *     disjoint buffers may run concurrently.
@@ -102,6 +103,17 @@ typedef struct {
 /* Human-readable name of a status code (static string). */
 const char* base_status_string(int status);
 
+/*
+ * Reads the library's sticky device error word into *code (0: none) and
+ * clears it when `clear` is non-zero.  A kernel writes it when one of its
+ * bounded waits gives up (codes 3001-3005: tensor-core GEMM pipeline) or when
+ * it meets data it cannot use (1000+e: auction bookkeeping of expert e;
+ * 2001: an assignment entry outside [0, E); 2002: a permutation entry
+ * outside [0, T), its row skipped; 4001: the backward was given a
+ * slot layout that is not the balanced one).  Synchronises the device.
+ */
+int base_device_error(int64_t* code, int clear);
+
 /* Library version string (static). */
 const char* base_version(void);
 
@@ -150,6 +162,15 @@ int base_assign_greedy(const int32_t* q, int T, int E, int32_t* assign, int32_t*
 int base_assign_balanced(const int32_t* q, int T, int E, int32_t* assign, int64_t* price,
                          base_auction_stats* stats, void* ws, size_t ws_bytes,
                          cudaStream_t stream);
+
+/*
+ * base_assign_balanced with the round cap lowered to max_rounds (1 ..
+ * BASE_AUCTION_MAX_ROUNDS): when the cap is reached stats->status becomes
+ * BASE_ERR_NOT_CONVERGED and assign / price hold the unfinished state.
+ */
+int base_assign_balanced_capped(const int32_t* q, int T, int E, int32_t* assign, int64_t* price,
+                                base_auction_stats* stats, void* ws, size_t ws_bytes,
+                                long long max_rounds, cudaStream_t stream);
 
 /*
  * a5: permutation into expert-contiguous slots (fig. 2 sort_by_expert).
@@ -205,7 +226,11 @@ int base_layer_fwd(const void* h, const void* w, const void* W1, const void* W2,
  *   dW1_e = dA1^T x; dx = dA1 W1_e + dy + ds w_e; dw_e = sum_{t in e} ds h_t;
  *   dh[t] = dx[inv[t]].
  * Outputs: dh T*D bf16; dw E*D fp32; dW1 E*F*D fp32; dW2 E*D*F fp32.
- * sv must hold the forward's a1, h1, f (non-null).
+ * sv must hold the forward's a1, h1, f (non-null).  The backward exists for
+ * training, i.e. balanced routing: it needs T % E == 0 with (T/E) % 64 == 0,
+ * D % 64 == 0 and F % 64 == 0 (BASE_ERR_UNSUPPORTED otherwise), and
+ * sv->offsets must be the balanced layout e * T/E (checked on the device,
+ * error word 4001).
  */
 int base_layer_bwd(const void* h, const void* w, const void* W1, const void* W2, int act,
                    int T, int D, int E, int F, const base_layer_saved* sv, const void* dout,

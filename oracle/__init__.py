@@ -260,8 +260,6 @@ def expert_ffn(x_perm, offsets, W1, W2, kind: str, gate_s=None, experts=None):
     ``experts`` limits the work to some experts (rows of the others are NaN).
     Returns dict(a1, h1, f, y)."""
     x = _f64(x_perm)
-    W1 = W1 if isinstance(W1, np.ndarray) and W1.dtype == np.float64 else _f64(W1)
-    W2 = W2 if isinstance(W2, np.ndarray) and W2.dtype == np.float64 else _f64(W2)
     T, D = x.shape
     E, F, _ = W1.shape
     a1 = np.full((T, F), np.nan)
@@ -270,8 +268,8 @@ def expert_ffn(x_perm, offsets, W1, W2, kind: str, gate_s=None, experts=None):
         lo, hi = int(offsets[e]), int(offsets[e + 1])
         if hi == lo:
             continue
-        a1[lo:hi] = x[lo:hi] @ W1[e].T
-        f[lo:hi] = act(a1[lo:hi], kind) @ W2[e].T
+        a1[lo:hi] = x[lo:hi] @ _f64(W1[e]).T
+        f[lo:hi] = act(a1[lo:hi], kind) @ _f64(W2[e]).T
     out = dict(a1=a1, h1=act(a1, kind), f=f)
     if gate_s is not None:
         out["y"] = sigmoid(gate_s)[:, None] * f + x
@@ -295,14 +293,14 @@ def layer_forward(h, w, W1, W2, kind: str, assign: np.ndarray, experts=None):
 
 def layer_backward(fw: dict, h, w, W1, W2, kind: str, dout, experts=None):
     """Gradients of ``L = <out, dout>`` with the assignment held fixed.
+    With ``experts`` given, dW1 / dW2 are dicts {expert: array} of those
+    experts only.
 
     dy = dout[perm]; dgate = <dy, f>; ds = dgate sigma (1 - sigma);
     dF = sigma dy; dH1 = dF W2_e; dW2_e = dF^T H1; dA1 = dH1 * act'(A1);
     dW1_e = dA1^T x; dx = dA1 W1_e + dy + ds w_{a_t}; dw_e = sum ds h_t;
     dh = dx[inv].  Returns dict(dh, dw, dW1, dW2)."""
     h64, w64 = _f64(h), _f64(w)
-    W1 = _f64(W1)
-    W2 = _f64(W2)
     E, F, D = W1.shape
     T = h64.shape[0]
     perm, offsets = fw["perm"], fw["offsets"]
@@ -313,22 +311,24 @@ def layer_backward(fw: dict, h, w, W1, W2, kind: str, dout, experts=None):
     dgate = np.einsum("td,td->t", dy, fw["f"])
     ds = dgate * sg * (1.0 - sg)
     dF = sg[:, None] * dy
-    dW1 = np.full((E, F, D), np.nan)
-    dW2 = np.full((E, D, F), np.nan)
+    dW1, dW2 = {}, {}
     dx = np.full((T, D), np.nan)
     for e in (range(E) if experts is None else experts):
         lo, hi = int(offsets[e]), int(offsets[e + 1])
         a1 = fw["a1"][lo:hi]
         h1 = act(a1, kind)
-        dH1 = dF[lo:hi] @ W2[e]
+        dH1 = dF[lo:hi] @ _f64(W2[e])
         dW2[e] = dF[lo:hi].T @ h1
         dA1 = dH1 * act_grad(a1, kind)
         dW1[e] = dA1.T @ x[lo:hi]
-        dx[lo:hi] = dA1 @ W1[e] + dy[lo:hi] + ds[lo:hi, None] * w64[e][None, :]
+        dx[lo:hi] = dA1 @ _f64(W1[e]) + dy[lo:hi] + ds[lo:hi, None] * w64[e][None, :]
     dw = np.zeros((E, D))
     ex = assign[perm]
     for e in (range(E) if experts is None else experts):
         m = ex == e
         dw[e] = (ds[m][:, None] * x[m]).sum(axis=0)
     dh = dx[fw["inv"]]
+    if experts is None:  # every expert: full (E, F, D) / (E, D, F) arrays
+        dW1 = np.stack([dW1[e] for e in range(E)])
+        dW2 = np.stack([dW2[e] for e in range(E)])
     return dict(dh=dh, dw=dw, dW1=dW1, dW2=dW2, ds=ds, dgate=dgate)

@@ -1,0 +1,215 @@
+"""GPU parity of the routing steps (scores, greedy, balanced auction,
+permute, combine) against the CPU oracle, through the C ABI."""
+import numpy as np
+import pytest
+import torch
+
+from _util import close_scores, dev, to_np
+from balanced_token_expert_b200 import binding as B
+from balanced_token_expert_b200 import buffers, synth
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(autouse=True)
+def no_device_error():
+    B.base_device_error(clear=True)
+    yield
+    torch.cuda.synchronize()
+    assert B.base_device_error(clear=True) == 0
+
+
+def gpu_auction(q_np, max_rounds=None):
+    T, E = q_np.shape
+    q = dev(q_np)
+    assign = torch.full((T,), -1, dtype=torch.int32, device="cuda")
+    price = torch.zeros(E, dtype=torch.int64, device="cuda")
+    st = buffers.stats()
+    ws = buffers.workspace(T, E)
+    if max_rounds is None:
+        B.base_assign_balanced(q, assign, price, st, ws)
+    else:
+        B.base_assign_balanced_capped(q, assign, price, st, ws, max_rounds)
+    torch.cuda.synchronize()
+    return to_np(assign), to_np(price), buffers.stats_dict(st)
+
+
+def oracle_q(orc, wl, seed=0):
+    inp = synth.make_inputs(wl, seed, with_weights=False, with_dout=False)
+    s = orc.scores(inp.h, inp.w)
+    q = orc.quantize(s)
+    if inp.bump_tokens is not None:
+        q[inp.bump_tokens.numpy(), 0] += int(round(inp.bump_value * orc.QSCALE))
+    return inp, s, q
+
+
+# ------------------------------------------------------------------ scores
+def test_scores_fp32_routing_reference(orc):
+    for seed in (0, 1, 2):
+        inp = synth.make_inputs(synth.WORKLOADS["routing_ref"], seed)
+        T, E = 512, 8
+        s = torch.empty(T, E, device="cuda")
+        q = torch.empty(T, E, dtype=torch.int32, device="cuda")
+        B.base_scores(dev(inp.h), dev(inp.w), s, q)
+        torch.cuda.synchronize()
+        so = orc.scores(inp.h, inp.w)
+        ok, worst = close_scores(to_np(s), so, 1e-5)
+        assert ok, worst
+        sg, qg = to_np(s), to_np(q)
+        # q is the kernel's own fp32 s rounded half-to-even after scaling by 2^16
+        assert np.array_equal(qg, np.rint(sg.astype(np.float32) * np.float32(65536)).astype(np.int32))
+        qo = orc.quantize(so)
+        assert np.abs(qg.astype(np.int64) - qo).max() <= 1
+
+
+@pytest.mark.parametrize("T,E,D", [(1000, 16, 200), (333, 40, 64), (256, 8, 128), (640, 300, 96),
+                                   (129, 128, 1024)])
+def test_scores_bf16_shapes(orc, T, E, D):
+    wl = synth.WORKLOADS["layer_fwd"].scaled(T=T, E=E, D=D, F=0)
+    inp = synth.make_inputs(wl, 7)
+    s = torch.empty(T, E, device="cuda")
+    q = torch.empty(T, E, dtype=torch.int32, device="cuda")
+    B.base_scores(dev(inp.h), dev(inp.w), s, q)
+    torch.cuda.synchronize()
+    ok, worst = close_scores(to_np(s), orc.scores(inp.h, inp.w), 1e-5)
+    assert ok, worst
+    sg = to_np(s)
+    assert np.array_equal(to_np(q), np.rint(sg * np.float32(65536)).astype(np.int32))
+
+
+@pytest.mark.parametrize("name", ["layer_fwd", "skewed", "large_routing"])
+def test_scores_bf16_full_workloads(orc, name):
+    wl = synth.WORKLOADS[name]
+    inp = synth.make_inputs(wl, 0, with_weights=False, with_dout=False)
+    s = torch.empty(wl.T, wl.E, device="cuda")
+    q = torch.empty(wl.T, wl.E, dtype=torch.int32, device="cuda")
+    B.base_scores(dev(inp.h), dev(inp.w), s, q)
+    torch.cuda.synchronize()
+    rows = np.random.default_rng(0).choice(wl.T, size=min(wl.T, 4096), replace=False)
+    so = orc.scores(inp.h[rows], inp.w)
+    sg = to_np(s)
+    ok, worst = close_scores(sg[rows], so, 1e-5)
+    assert ok, worst
+    assert np.array_equal(to_np(q), np.rint(sg * np.float32(65536)).astype(np.int32))
+
+
+# ------------------------------------------------------------------ greedy
+@pytest.mark.parametrize("T,E,small", [(512, 8, False), (1000, 5, True), (4096, 16, False),
+                                       (3000, 33, True), (8192, 128, False), (777, 1000, True),
+                                       (64, 2, True)])
+def test_greedy_bit_exact(orc, T, E, small):
+    rng = np.random.default_rng(T + E)
+    q = (rng.integers(0, 3, size=(T, E)) if small else
+         rng.integers(-300000, 300000, size=(T, E))).astype(np.int32)
+    a = torch.empty(T, dtype=torch.int32, device="cuda")
+    c = torch.empty(E, dtype=torch.int32, device="cuda")
+    B.base_assign_greedy(dev(q), a, c)
+    torch.cuda.synchronize()
+    ao, co = orc.greedy(q)
+    assert np.array_equal(to_np(a), ao)
+    assert np.array_equal(to_np(c), co)
+
+
+def test_greedy_large_routing(orc):
+    _, _, q = oracle_q(orc, synth.WORKLOADS["large_routing"])
+    T, E = q.shape
+    a = torch.empty(T, dtype=torch.int32, device="cuda")
+    c = torch.empty(E, dtype=torch.int32, device="cuda")
+    B.base_assign_greedy(dev(q), a, c)
+    torch.cuda.synchronize()
+    ao, co = orc.greedy(q)
+    assert np.array_equal(to_np(a), ao) and np.array_equal(to_np(c), co)
+
+
+# ------------------------------------------------------------------ auction
+def _check_auction(orc, q):
+    a, p, st = gpu_auction(q)
+    ao, po, so = orc.auction(q)
+    assert st == so, (st, so)
+    assert np.array_equal(a, ao)
+    assert np.array_equal(p, po)
+    assert orc.certificate(q, a, p)["ok"]
+    return st
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_auction_routing_reference_is_optimal_and_bit_exact(orc, seed):
+    _, _, q = oracle_q(orc, synth.WORKLOADS["routing_ref"], seed)
+    st = _check_auction(orc, q)
+    assert st["objective"] == orc.hungarian(q)[0]
+
+
+@pytest.mark.parametrize("T,E,small", [(8, 2, False), (12, 3, True), (64, 64, False),
+                                       (100, 4, True), (1000, 8, False), (2048, 2, False),
+                                       (4096, 1024, False), (6000, 3, True), (8192, 16, True),
+                                       (30000, 40, False)])
+def test_auction_shapes_bit_exact(orc, T, E, small):
+    rng = np.random.default_rng(T * 7 + E)
+    q = (rng.integers(0, 4, size=(T, E)) if small else
+         rng.integers(-300000, 300000, size=(T, E))).astype(np.int32)
+    _check_auction(orc, q)
+
+
+def test_auction_many_tiny_problems(orc):
+    rng = np.random.default_rng(99)
+    for i in range(60):
+        T, E = [(8, 2), (12, 3), (12, 4), (16, 8)][i % 4]
+        q = (rng.integers(0, 4, size=(T, E)) if i % 2 else
+             rng.integers(-1000, 1000, size=(T, E))).astype(np.int32)
+        a, p, st = gpu_auction(q)
+        ao, po, so = orc.auction(q)
+        assert st == so and np.array_equal(a, ao) and np.array_equal(p, po)
+        assert st["objective"] == orc.bruteforce(q)[0] if T <= 12 else True
+
+
+@pytest.mark.parametrize("name", ["layer_fwd", "skewed", "large_routing", "layer_fwd_bwd"])
+def test_auction_full_workloads(orc, name):
+    _, _, q = oracle_q(orc, synth.WORKLOADS[name])
+    _check_auction(orc, q)
+
+
+def test_auction_equal_scores_single_phase(orc):
+    q = np.zeros((256, 8), dtype=np.int32)
+    _check_auction(orc, q)
+
+
+def test_auction_round_cap_reports_not_converged(orc):
+    _, _, q = oracle_q(orc, synth.WORKLOADS["routing_ref"], 0)
+    a, p, st = gpu_auction(q, max_rounds=5)
+    assert st["status"] == 3 and st["rounds"] == 5
+    so = orc.auction(q, max_rounds=5)[2]
+    assert so["status"] == 3 and so["rounds"] == 5 and so["bids"] == st["bids"]
+
+
+# ------------------------------------------------------------------ permute / combine
+@pytest.mark.parametrize("T,E,D,kind", [(1536, 4, 64, "balanced"), (1000, 5, 200, "ragged"),
+                                        (4096, 128, 128, "ragged"), (333, 7, 8, "ragged"),
+                                        (2048, 2, 1024, "empty-expert")])
+def test_permute_and_combine_bit_exact(orc, T, E, D, kind):
+    rng = np.random.default_rng(T + D)
+    if kind == "balanced":
+        q = rng.integers(-100000, 100000, size=(T, E)).astype(np.int32)
+        assign = orc.auction(q)[0]
+    elif kind == "empty-expert":
+        assign = np.zeros(T, dtype=np.int32)
+    else:
+        assign = rng.integers(0, E, size=T).astype(np.int32)
+    h = torch.randn(T, D, generator=torch.Generator().manual_seed(3)).to(torch.bfloat16)
+    s = rng.standard_normal((T, E)).astype(np.float32)
+    perm = torch.empty(T, dtype=torch.int32, device="cuda")
+    inv = torch.empty_like(perm)
+    offs = torch.empty(E + 1, dtype=torch.int32, device="cuda")
+    xp = torch.empty(T, D, dtype=torch.bfloat16, device="cuda")
+    gate = torch.empty(T, dtype=torch.float32, device="cuda")
+    ws = buffers.workspace(T, E, D)
+    B.base_permute(dev(h), dev(assign), E, perm, inv, offs, xp, dev(s), gate, ws)
+    out = torch.empty_like(xp)
+    B.base_combine(xp, perm, out)
+    torch.cuda.synchronize()
+    po, io, oo = orc.permutation(assign, E)
+    assert np.array_equal(to_np(perm), po)
+    assert np.array_equal(to_np(inv), io)
+    assert np.array_equal(to_np(offs), oo)
+    assert torch.equal(xp.cpu(), h[torch.from_numpy(po.astype(np.int64))])
+    assert np.array_equal(to_np(gate), s[po, assign[po]])
+    assert torch.equal(out.cpu(), h)  # combine undoes the permutation exactly
