@@ -96,15 +96,27 @@ class Clocks:
                     sm_max_mhz=max(mx) if mx else None, reasons=reasons, samples=len(rows))
 
 
+def _oracle_step(oracle, wl, inp):
+    s = oracle.scores(inp.h, inp.w)
+    q = oracle.quantize(s)
+    if inp.bump_tokens is not None:
+        q[inp.bump_tokens.numpy(), 0] += int(round(inp.bump_value * oracle.QSCALE))
+    a = oracle.auction(q)[0]
+    if wl.F:
+        oracle.layer_forward(inp.h, inp.w, inp.W1, inp.W2, wl.act, a)
+    else:
+        oracle.greedy(q)
+        perm = oracle.permutation(a, wl.E)[0]
+        oracle.gather_rows(inp.h, perm)
+
+
 def cpu_baseline(wl, seed=0):
     """The oracle as it stands, one full forward of the workload on the host."""
     import oracle
     from balanced_token_expert_b200 import synth
     inp = synth.make_inputs(wl, seed)
     t0 = time.perf_counter()
-    s = oracle.scores(inp.h, inp.w)
-    a = oracle.auction(oracle.quantize(s))[0]
-    oracle.layer_forward(inp.h, inp.w, inp.W1, inp.W2, wl.act, a)
+    _oracle_step(oracle, wl, inp)
     dt = time.perf_counter() - t0
     return dict(value=wl.T / dt, unit=UNIT, cores=len(os.sched_getaffinity(0)), kind="oracle",
                 sample="one full forward of the workload (T=%d tokens: float64 scores, integer "
@@ -120,9 +132,7 @@ def run_reference(args, wl, rank, world):
     inp = synth.make_inputs(wl, 0)
 
     def step():
-        s = oracle.scores(inp.h, inp.w)
-        a = oracle.auction(oracle.quantize(s))[0]
-        oracle.layer_forward(inp.h, inp.w, inp.W1, inp.W2, wl.act, a)
+        _oracle_step(oracle, wl, inp)
 
     for _ in range(args.warmup):
         step()
@@ -145,9 +155,16 @@ def run_reference(args, wl, rank, world):
 
 
 def _config(wl, args):
-    return dict(workload="%s: BASE layer forward, T=%d tokens, E=%d experts, D=%d, FFN %d->%d->%d "
-                         "%s, balanced auction routing, bf16" % (wl.name, wl.T, wl.E, wl.D, wl.D,
-                                                                 wl.F, wl.D, wl.act),
+    if wl.F:
+        desc = ("%s: BASE layer forward, T=%d tokens, E=%d experts, D=%d, FFN %d->%d->%d %s, "
+                "balanced auction routing, bf16" % (wl.name, wl.T, wl.E, wl.D, wl.D, wl.F, wl.D,
+                                                     wl.act))
+    else:
+        desc = ("%s: scores + balanced auction + greedy + permute, T=%d tokens, E=%d experts, "
+                "D=%d, bf16%s" % (wl.name, wl.T, wl.E, wl.D,
+                                  ", skewed mixture with +3 affinity on expert 0 for half the "
+                                  "tokens" if wl.kind == "mixture" else ""))
+    return dict(workload=desc,
                 T=wl.T, E=wl.E, D=wl.D, F=wl.F, act=wl.act, routing="balanced",
                 l2="flushed between timed steps (%d MiB write)" % args.flush_mb,
                 parallelism="independent replica per GPU")
@@ -184,34 +201,53 @@ def main():
     inp = synth.make_inputs(wl, seed=rank)
     h = inp.h.cuda()
     w = inp.w.cuda()
-    W1 = inp.W1.cuda()
-    W2 = inp.W2.cuda()
+    W1 = inp.W1.cuda() if F else None
+    W2 = inp.W2.cuda() if F else None
     act = B.BASE_RELU if wl.act == "relu" else B.BASE_GELU
-    sv = buffers.layer_saved(T, E, D, F, for_backward=False)
+    sv = buffers.layer_saved(T, E, D, max(F, 8), for_backward=False)
     out = torch.empty(T, D, dtype=torch.bfloat16, device="cuda")
     ws = buffers.workspace(T, E, D, F)
     flush = torch.empty(args.flush_mb * (1 << 20), dtype=torch.uint8, device="cuda")
     stream = torch.cuda.current_stream()
 
-    names = ["scores", "auction", "permute", "ffn", "combine"]
+    q_bump = None
+    if inp.bump_tokens is not None:  # test data: +bump on expert 0's quantised affinity
+        q_bump = (inp.bump_tokens.cuda(), int(round(inp.bump_value * B.QSCALE)))
+    greedy_assign = torch.empty(T, dtype=torch.int32, device="cuda")
+    greedy_counts = torch.empty(E, dtype=torch.int32, device="cuda")
+
+    comps = [("scores", lambda: B.base_scores(h, w, sv["s"], sv["q"]), 1)]
+    if q_bump is not None:
+        comps.append(("bump", lambda: sv["q"][:, 0].index_add_(
+            0, q_bump[0], torch.full_like(q_bump[0], q_bump[1], dtype=torch.int32)), 0))
+    comps.append(("auction", lambda: B.base_assign_balanced(sv["q"], sv["assign"], sv["price"],
+                                                             sv["stats"], ws), 3))
+    if not F:
+        comps.append(("greedy", lambda: B.base_assign_greedy(sv["q"], greedy_assign,
+                                                              greedy_counts), 1))
+    comps.append(("permute", lambda: B.base_permute(h, sv["assign"], E, sv["perm"], sv["inv"],
+                                                     sv["offsets"], sv["x_perm"], sv["s"],
+                                                     sv["gate"], ws), 4))
+    if F:
+        comps.append(("ffn", lambda: B.base_expert_ffn(sv["x_perm"], sv["offsets"], W1, W2, act,
+                                                       sv["gate"], sv["y_perm"], sv["h1"], None,
+                                                       None, ws), 3))
+        comps.append(("combine", lambda: B.base_combine(sv["y_perm"], sv["perm"], out), 1))
+    names = [n for n, _, _ in comps if n != "bump"]
 
     def step(ev):
-        ev[0].record(stream)
-        B.base_scores(h, w, sv["s"], sv["q"])
-        ev[1].record(stream)
-        B.base_assign_balanced(sv["q"], sv["assign"], sv["price"], sv["stats"], ws)
-        ev[2].record(stream)
-        B.base_permute(h, sv["assign"], E, sv["perm"], sv["inv"], sv["offsets"], sv["x_perm"],
-                       sv["s"], sv["gate"], ws)
-        ev[3].record(stream)
-        B.base_expert_ffn(sv["x_perm"], sv["offsets"], W1, W2, act, sv["gate"], sv["y_perm"],
-                          sv["h1"], None, None, ws)
-        ev[4].record(stream)
-        B.base_combine(sv["y_perm"], sv["perm"], out)
-        ev[5].record(stream)
+        j = 0
+        for n, fn, _ in comps:
+            if n == "bump":
+                fn()
+                continue
+            ev[2 * j].record(stream)
+            fn()
+            ev[2 * j + 1].record(stream)
+            j += 1
 
-    kernels_per_step = 1 + 3 + 4 + 3 + 1
-    mk = lambda: [torch.cuda.Event(enable_timing=True) for _ in range(6)]  # noqa: E731
+    kernels_per_step = sum(k for _, _, k in comps)
+    mk = lambda: [torch.cuda.Event(enable_timing=True) for _ in range(2 * len(names))]  # noqa: E731
     for _ in range(max(3, args.warmup)):
         flush.zero_()
         step(mk())
@@ -244,7 +280,7 @@ def main():
     per = {n: [] for n in names}
     for ev in evs:
         for j, n in enumerate(names):
-            per[n].append(ev[j].elapsed_time(ev[j + 1]))
+            per[n].append(ev[2 * j].elapsed_time(ev[2 * j + 1]))
     step_ms = [sum(per[n][i] for n in names) for i in range(args.steps)]
     ms = statistics.mean(step_ms)
     st = buffers.stats_dict(sv["stats"])
@@ -257,14 +293,29 @@ def main():
 
     # end to end through the public call: host inputs in, host output back
     h_host = inp.h.pin_memory()
-    out_host = torch.empty(T, D, dtype=torch.bfloat16).pin_memory()
     h_dev = torch.empty_like(h)
-    sv2 = buffers.layer_saved(T, E, D, F, for_backward=False)
+    if F:
+        out_host = torch.empty(T, D, dtype=torch.bfloat16).pin_memory()
+        sv2 = buffers.layer_saved(T, E, D, F, for_backward=False)
 
-    def e2e_step():
-        h_dev.copy_(h_host, non_blocking=True)
-        B.base_layer_fwd(h_dev, w, W1, W2, act, B.BASE_ROUTE_BALANCED, out, sv2, ws)
-        out_host.copy_(out, non_blocking=True)
+        def e2e_step():
+            h_dev.copy_(h_host, non_blocking=True)
+            B.base_layer_fwd(h_dev, w, W1, W2, act, B.BASE_ROUTE_BALANCED, out, sv2, ws)
+            out_host.copy_(out, non_blocking=True)
+        d2h = T * D * 2
+    else:
+        out_host = torch.empty(T, dtype=torch.int32).pin_memory()
+
+        def e2e_step():
+            h_dev.copy_(h_host, non_blocking=True)
+            B.base_scores(h_dev, w, sv["s"], sv["q"])
+            if q_bump is not None:
+                comps[1][1]()
+            B.base_assign_balanced(sv["q"], sv["assign"], sv["price"], sv["stats"], ws)
+            B.base_permute(h_dev, sv["assign"], E, sv["perm"], sv["inv"], sv["offsets"],
+                           sv["x_perm"], sv["s"], sv["gate"], ws)
+            out_host.copy_(sv["assign"], non_blocking=True)
+        d2h = T * 4
 
     for _ in range(3):
         flush.zero_()
@@ -295,7 +346,8 @@ def main():
             auction=("hbm", 4 * E * bids + 4 * T + 8 * E),
             permute=("hbm", 4 * T * D + 12 * T + 8 * T),
             ffn=("tensor", 4 * T * D * F),
-            combine=("hbm", 4 * T * D + 4 * T))
+            combine=("hbm", 4 * T * D + 4 * T),
+            greedy=("hbm", 4 * T * E + 4 * T))
 
         def roof(n):
             bound, work = alg[n]
@@ -321,7 +373,7 @@ def main():
                          phases=st["phases"], bids=bids, status=st["status"],
                          us_per_round=1e3 * comp["auction"] / max(1, st["rounds"])),
             e2e=dict(value=T * world / (e2e / 1e3), unit=UNIT, h2d_bytes_per_step=T * D * 2,
-                     d2h_bytes_per_step=T * D * 2, ms_per_step=e2e),
+                     d2h_bytes_per_step=d2h, ms_per_step=e2e),
             gpu_launches=kernels_per_step * args.steps,
             clocks=clk, device_error=err, wall_s=wall,
         )
