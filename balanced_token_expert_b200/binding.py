@@ -20,7 +20,7 @@ __all__ = [
     "BASE_OK", "BASE_F32", "BASE_BF16", "BASE_RELU", "BASE_GELU",
     "BASE_ROUTE_BALANCED", "BASE_ROUTE_GREEDY", "QSCALE",
     "base_status_string", "base_version", "base_workspace_size", "base_device_error",
-    "base_scores", "base_assign_greedy", "base_assign_balanced", "base_assign_balanced_capped",
+    "base_scores", "base_assign_greedy", "base_assign_balanced", "base_assign_balanced_ex",
     "base_permute", "base_expert_ffn", "base_combine", "base_layer_fwd", "base_layer_bwd",
     "EXPORTED",
 ]
@@ -34,7 +34,7 @@ QSCALE = 65536.0
 # every symbol include/base.h declares
 EXPORTED = (
     "base_status_string", "base_device_error", "base_version", "base_workspace_size",
-    "base_scores", "base_assign_greedy", "base_assign_balanced", "base_assign_balanced_capped",
+    "base_scores", "base_assign_greedy", "base_assign_balanced", "base_assign_balanced_ex",
     "base_permute", "base_expert_ffn", "base_combine", "base_layer_fwd", "base_layer_bwd",
 )
 
@@ -74,8 +74,8 @@ _SIGS = {
     "base_scores": (_i, [_vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp]),
     "base_assign_greedy": (_i, [_vp, _i, _i, _vp, _vp, _vp]),
     "base_assign_balanced": (_i, [_vp, _i, _i, _vp, _vp, _vp, _vp, _sz, _vp]),
-    "base_assign_balanced_capped": (_i, [_vp, _i, _i, _vp, _vp, _vp, _vp, _sz, ctypes.c_longlong,
-                                         _vp]),
+    "base_assign_balanced_ex": (_i, [_vp, _i, _i, _vp, _vp, _vp, ctypes.c_longlong, _vp, _vp,
+                                     ctypes.c_longlong, _vp, _sz, _vp]),
     "base_permute": (_i, [_vp, _vp, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "base_expert_ffn": (_i, [_vp, _vp, _i, _i, _i, _i, _vp, _vp, _i, _vp, _vp, _vp, _vp, _vp, _vp,
                              _sz, _vp]),
@@ -166,11 +166,16 @@ def base_assign_balanced(q, assign, price, stats=None, ws=None, stream=None):
         0 if ws is None else ws.numel() * ws.element_size(), _stream(stream)))
 
 
-def base_assign_balanced_capped(q, assign, price, stats, ws, max_rounds: int, stream=None):
+def base_assign_balanced_ex(q, assign, price, stats, ws, max_rounds: int = 1000000,
+                            u_trace=None, t_trace=None, stream=None):
     T, E = q.shape
-    _check("base_assign_balanced_capped", lib().base_assign_balanced_capped(
-        _ptr(q), T, E, _ptr(assign), _ptr(price), _ptr(stats), _ptr(ws),
-        ws.numel() * ws.element_size(), int(max_rounds), _stream(stream)))
+    cap = 0
+    for t in (u_trace, t_trace):
+        if t is not None:
+            cap = t.numel() if cap == 0 else min(cap, t.numel())
+    _check("base_assign_balanced_ex", lib().base_assign_balanced_ex(
+        _ptr(q), T, E, _ptr(assign), _ptr(price), _ptr(stats), int(max_rounds), _ptr(u_trace),
+        _ptr(t_trace), cap, _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)))
 
 
 def base_permute(h, assign, E, perm, inv, offsets, x_perm, s=None, gate=None, ws=None,

@@ -16,7 +16,7 @@ int launch_greedy(const int32_t* q, int T, int E, int32_t* assign, int32_t* coun
 size_t auction_workspace_bytes(int T, int E);
 int launch_auction(const int32_t* q, int T, int E, int32_t* assign, int64_t* price,
                    base_auction_stats* stats, void* ws, size_t ws_bytes, long long max_rounds,
-                   cudaStream_t stream);
+                   int32_t* u_trace, int64_t* t_trace, long long trace_cap, cudaStream_t stream);
 size_t permute_workspace_bytes(int T, int E);
 int launch_sort_by_expert(const int32_t* assign, int T, int E, int32_t* perm, int32_t* inv,
                           int32_t* offsets, const float* s, float* gate, void* ws,
@@ -118,22 +118,25 @@ int base_assign_balanced(const int32_t* q, int T, int E, int32_t* assign, int64_
         return BASE_ERR_INVALID_ARG;
     if (ws_bytes < auction_workspace_bytes(T, E)) return BASE_ERR_WORKSPACE;
     return launch_auction(q, T, E, assign, price, stats, ws, ws_bytes, BASE_AUCTION_MAX_ROUNDS,
-                          stream);
+                          nullptr, nullptr, 0, stream);
 }
 
-/* Same as base_assign_balanced with a smaller round cap (for tests of the
-   not-converged path). */
-int base_assign_balanced_capped(const int32_t* q, int T, int E, int32_t* assign, int64_t* price,
-                                base_auction_stats* stats, void* ws, size_t ws_bytes,
-                                long long max_rounds, cudaStream_t stream) {
-    if (max_rounds < 1 || max_rounds > BASE_AUCTION_MAX_ROUNDS) return BASE_ERR_INVALID_ARG;
+int base_assign_balanced_ex(const int32_t* q, int T, int E, int32_t* assign, int64_t* price,
+                            base_auction_stats* stats, long long max_rounds, int32_t* u_trace,
+                            int64_t* t_trace, long long trace_cap, void* ws, size_t ws_bytes,
+                            cudaStream_t stream) {
+    if (max_rounds < 1 || max_rounds > BASE_AUCTION_MAX_ROUNDS || trace_cap < 0)
+        return BASE_ERR_INVALID_ARG;
+    if ((u_trace || t_trace) && trace_cap == 0) return BASE_ERR_INVALID_ARG;
     if (!q || !assign || !price || !ws || !shapes_ok(T, E) || T % E != 0)
         return BASE_ERR_INVALID_ARG;
     if (!aligned(q, 16) || !aligned(assign, 4) || !aligned(price, 8) || !aligned(ws, 256) ||
-        (stats && !aligned(stats, 8)))
+        (stats && !aligned(stats, 8)) || (u_trace && !aligned(u_trace, 4)) ||
+        (t_trace && !aligned(t_trace, 8)))
         return BASE_ERR_INVALID_ARG;
     if (ws_bytes < auction_workspace_bytes(T, E)) return BASE_ERR_WORKSPACE;
-    return launch_auction(q, T, E, assign, price, stats, ws, ws_bytes, max_rounds, stream);
+    return launch_auction(q, T, E, assign, price, stats, ws, ws_bytes, max_rounds, u_trace, t_trace,
+                          trace_cap, stream);
 }
 
 int base_permute(const void* h, const int32_t* assign, int T, int D, int E, int32_t* perm,

@@ -2,111 +2,83 @@
 // Simplifying Training of Large, Sparse Models", Method / "Training
 // assignment") by a Jacobi token-bidding auction with epsilon scaling.
 //
-// The whole auction runs on ONE thread-block cluster (1..16 CTAs of 1024
-// threads).  Expert e is owned by CTA e % CL; the owner keeps the expert's
-// held bids (at most C = T/E (bid, token) pairs) in its shared memory, so a
-// round never leaves the chip except to read the bidders' score rows.  Most
-// rounds have only a handful of bidders (the tail of every phase), so the
-// cost of a round is its latency: two hardware cluster barriers per round
-// instead of grid-wide barriers through global memory.
-//
-// One round (prices of the round start, identical to the CPU oracle's):
+// One round (prices of the round start; identical to the CPU oracle's):
 //   bid:     every unassigned token t (a group of lanes per token) scans
 //            v_e = q[t][e] (T+1) - price[e], takes the best e* (lowest index
 //            on ties) and the second best v2, and bids
-//            b = q[t][e*] (T+1) - v2 + eps.  The bid goes to e*'s owner:
-//            a DSMEM atomic reserves a place in e*'s bucket (the first 16 in
-//            the owner's shared memory, the rest in a global overflow).
-//   cluster barrier
-//   resolve: one warp per owned expert with new bids keeps the C best of
-//            held + new (larger bid, then smaller token), found as the k-th
-//            worst key (k = held + new - C) by repeated warp minima for small
-//            k or a warp radix select over (bid - min bid, T-1-token) keys;
-//            rejected tokens go to the next round's list; a full expert sets
-//            its price to its smallest held bid and writes it to every CTA.
-//   cluster barrier
-// The phase ends when nobody is unassigned; eps is divided by 8 until 1.
-#include <cooperative_groups.h>
-
+//            b = q[t][e*] (T+1) - v2 + eps to e*.
+//   resolve: every expert keeps the C best of held + new bids (larger bid,
+//            then smaller token); the others become unassigned; a full
+//            expert's price is its smallest held bid.
+// A phase runs rounds until nobody is unassigned; eps is divided by 8 down
+// to 1 (exact optimum for integer scores).
+//
+// The kernel is one persistent cooperative grid (one CTA of 1024 threads per
+// SM) with two modes:
+//   * wide rounds (the start of every phase, where all T tokens bid, and the
+//     next rounds while many tokens are unassigned) use the whole GPU: bids
+//     go to per-expert global buckets, a grid barrier, then one CTA per
+//     expert keeps its C best with a CTA-wide radix select, a grid barrier;
+//   * narrow rounds (the long tail of every phase, mostly a handful of
+//     bidders) run on CTA 0 alone while the other CTAs wait for the phase to
+//     end: prices live in shared memory, and for every full expert CTA 0 keeps
+//     a "fringe" -- its FK worst held bids, sorted -- so a round resolves with
+//     a warp-wide bitonic merge of fringe and new bids instead of a scan of
+//     the expert's C held bids.  Rejected tokens' score rows are prefetched
+//     into L1 for their next bid.
+// Held sets live in global memory (they are touched only when a fringe is
+// rebuilt).  Every wait is bounded; a wait that gives up records an error
+// and all CTAs leave.
 #include <algorithm>
 
 #include "common.cuh"
-
-namespace cg = cooperative_groups;
 
 namespace base {
 namespace auction {
 
 constexpr int kThreads = 1024;
 constexpr int kWarps = kThreads / kWarp;
-constexpr int kSB = 16;          // bids per expert kept in the owner's shared memory
-constexpr int kSmallK = 8;       // rejections up to this count use repeated minima
-constexpr int kHist = 256;       // radix-select bins per warp
+constexpr int kHist = 256;
 constexpr int kEpsDivisor = 50;  // eps0 = (max q - min q)(T+1) / 50
 constexpr int kEpsFactor = 8;    // eps <- eps / 8 per phase
-constexpr size_t kMaxSmem = 200 * 1024;
+constexpr int kNarrowMax = 1024; // rounds with at most this many bidders run on CTA 0
+constexpr uint64_t kWaitNs = 20000000000ull;  // grid-barrier wait limit (20 s)
 
-struct Params {
-    const int32_t* q;
-    int T, E, C;
-    int CL, EL;            // cluster size, experts per CTA
-    int held_in_smem;
-    long long max_rounds;
-    int32_t* assign;
-    int64_t* price_out;
-    base_auction_stats* stats;
-    const int32_t* minmax;  // [min q, max q]
-    int32_t* ulist0;
-    int32_t* ulist1;        // [T] each
-    int64_t* gb_bid;
-    int32_t* gb_tok;        // [E][T] bucket overflow
-    int64_t* gh_bid;
-    int32_t* gh_tok;        // [E][C] held sets when they do not fit on chip
-    int32_t* gfree;         // [E][C] free-slot scratch
-};
-
-struct SmemLayout {
-    size_t price, held_bid, held_tok, hcnt, cnt, sb_bid, sb_tok, hist, ctrl, total;
-};
-
-__host__ __device__ inline SmemLayout smem_layout(int E, int EL, int C, int held_in_smem) {
-    SmemLayout L;
-    size_t o = 0;
-    L.price = o;    o += align_up(sizeof(int64_t) * E, 16);
-    L.held_bid = o; o += held_in_smem ? align_up(sizeof(int64_t) * (size_t)EL * C, 16) : 0;
-    L.held_tok = o; o += held_in_smem ? align_up(sizeof(int32_t) * (size_t)EL * C, 16) : 0;
-    L.hcnt = o;     o += align_up(sizeof(int32_t) * EL, 16);
-    L.cnt = o;      o += align_up(sizeof(int32_t) * EL, 16);
-    L.sb_bid = o;   o += align_up(sizeof(int64_t) * (size_t)EL * kSB, 16);
-    L.sb_tok = o;   o += align_up(sizeof(int32_t) * (size_t)EL * kSB, 16);
-    L.hist = o;     o += sizeof(int32_t) * kWarps * kHist;
-    L.ctrl = o;     o += 64;
-    L.total = o;
-    return L;
-}
-
+// ---------------------------------------------------------------- keys
 struct Key {
     int64_t bid;
     int32_t tok;
+    int32_t slot;  // >= 0: held slot; -1: a new bid; -2: padding
 };
 
-// "worse" order: smaller bid first, then larger token index first.  The C
-// best keys of an expert are the ones it keeps.
+// "worse" order: smaller bid first, then larger token first; an expert keeps
+// the C best keys.
 __device__ __forceinline__ bool worse(const Key& a, const Key& b) {
     return a.bid < b.bid || (a.bid == b.bid && a.tok > b.tok);
 }
 
-__device__ __forceinline__ Key shfl_key(const Key& k, int src_lane_xor) {
+__device__ __forceinline__ Key pad_key() { return Key{INT64_MAX, -1, -2}; }
+
+__device__ __forceinline__ Key shfl_key(const Key& k, int src) {
     Key o;
-    o.bid = __shfl_xor_sync(0xffffffffu, k.bid, src_lane_xor);
-    o.tok = __shfl_xor_sync(0xffffffffu, k.tok, src_lane_xor);
+    o.bid = __shfl_sync(0xffffffffu, k.bid, src);
+    o.tok = __shfl_sync(0xffffffffu, k.tok, src);
+    o.slot = __shfl_sync(0xffffffffu, k.slot, src);
+    return o;
+}
+
+__device__ __forceinline__ Key shfl_xor_key(const Key& k, int m) {
+    Key o;
+    o.bid = __shfl_xor_sync(0xffffffffu, k.bid, m);
+    o.tok = __shfl_xor_sync(0xffffffffu, k.tok, m);
+    o.slot = __shfl_xor_sync(0xffffffffu, k.slot, m);
     return o;
 }
 
 __device__ __forceinline__ Key warp_min_key(Key k) {
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) {
-        Key o = shfl_key(k, off);
+        const Key o = shfl_xor_key(k, off);
         if (worse(o, k)) k = o;
     }
     return k;
@@ -115,10 +87,53 @@ __device__ __forceinline__ Key warp_min_key(Key k) {
 __device__ __forceinline__ Key warp_max_key(Key k) {
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) {
-        Key o = shfl_key(k, off);
+        const Key o = shfl_xor_key(k, off);
         if (worse(k, o)) k = o;
     }
     return k;
+}
+
+// ascending bitonic sort of one key per lane
+__device__ __forceinline__ Key warp_sort(Key x) {
+    const int lane = lane_id();
+#pragma unroll
+    for (int k = 2; k <= 32; k <<= 1) {
+#pragma unroll
+        for (int j = k >> 1; j > 0; j >>= 1) {
+            const Key o = shfl_xor_key(x, j);
+            const bool up = (lane & k) == 0;
+            const bool lower = (lane & j) == 0;
+            if (lower == up ? worse(o, x) : worse(x, o)) x = o;
+        }
+    }
+    return x;
+}
+
+// sorts a bitonic sequence held one key per lane into ascending order
+__device__ __forceinline__ Key warp_bitonic_merge(Key x) {
+    const int lane = lane_id();
+#pragma unroll
+    for (int j = 16; j > 0; j >>= 1) {
+        const Key o = shfl_xor_key(x, j);
+        const bool lower = (lane & j) == 0;
+        if (lower ? worse(o, x) : worse(x, o)) x = o;
+    }
+    return x;
+}
+
+// a, b sorted ascending (one per lane) -> lo, hi: the 64 keys sorted ascending
+// (element i of the result is lo in lane i for i < 32, hi in lane i-32 after)
+__device__ __forceinline__ void warp_merge64(Key a, Key b, Key& lo, Key& hi) {
+    const Key br = shfl_key(b, 31 - lane_id());
+    if (worse(br, a)) {
+        lo = br;
+        hi = a;
+    } else {
+        lo = a;
+        hi = br;
+    }
+    lo = warp_bitonic_merge(lo);
+    hi = warp_bitonic_merge(hi);
 }
 
 __device__ __forceinline__ int64_t warp_min_i64(int64_t v) {
@@ -126,185 +141,658 @@ __device__ __forceinline__ int64_t warp_min_i64(int64_t v) {
     for (int off = 16; off > 0; off >>= 1) v = min(v, __shfl_xor_sync(0xffffffffu, v, off));
     return v;
 }
-
 __device__ __forceinline__ int64_t warp_max_i64(int64_t v) {
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) v = max(v, __shfl_xor_sync(0xffffffffu, v, off));
     return v;
 }
 
-__device__ __forceinline__ void cluster_barrier() {
-    asm volatile("barrier.cluster.arrive.release.aligned;\n"
-                 "barrier.cluster.wait.acquire.aligned;\n" ::: "memory");
+template <typename X>
+__device__ __forceinline__ X vload(const X* p) {
+    return *reinterpret_cast<const volatile X*>(p);
 }
 
 __device__ __forceinline__ int bit_length_u64(uint64_t x) { return x ? 64 - __clzll(x) : 0; }
+__device__ __forceinline__ uint64_t shr64(uint64_t x, int n) { return n >= 64 ? 0ull : (x >> n); }
 
-// Candidates of one expert during a resolve: held slots [0, h) then the new
-// bids [0, n) (the first kSB in the owner's shared memory, the rest in the
-// global overflow bucket).
+// ---------------------------------------------------------------- teams
+// A team is either one warp (TEAM = 32) or the whole CTA (TEAM = 1024).  Its
+// scratch: kHist ints of histogram + 64 bytes.
+template <int TEAM>
+struct Team {
+    int32_t* hist;     // [kHist]
+    int64_t* red;      // [32] (CTA team only)
+    int32_t* cnt;      // [33] (CTA team only)
+    __device__ __forceinline__ int tid() const { return TEAM == 32 ? lane_id() : (int)threadIdx.x; }
+    __device__ __forceinline__ void sync() const {
+        if (TEAM == 32) __syncwarp(); else __syncthreads();
+    }
+    __device__ int64_t min_i64(int64_t v) const {
+        v = warp_min_i64(v);
+        if (TEAM == 32) return v;
+        if (lane_id() == 0) red[warp_id()] = v;
+        __syncthreads();
+        if (warp_id() == 0) {
+            int64_t x = red[lane_id()];
+            x = warp_min_i64(x);
+            if (lane_id() == 0) red[0] = x;
+        }
+        __syncthreads();
+        const int64_t r = red[0];
+        __syncthreads();
+        return r;
+    }
+    __device__ int64_t max_i64(int64_t v) const {
+        v = warp_max_i64(v);
+        if (TEAM == 32) return v;
+        if (lane_id() == 0) red[warp_id()] = v;
+        __syncthreads();
+        if (warp_id() == 0) {
+            int64_t x = red[lane_id()];
+            x = warp_max_i64(x);
+            if (lane_id() == 0) red[0] = x;
+        }
+        __syncthreads();
+        const int64_t r = red[0];
+        __syncthreads();
+        return r;
+    }
+    __device__ Key max_key(Key k) const {
+        k = warp_max_key(k);
+        if (TEAM == 32) return k;
+        Key* sk = reinterpret_cast<Key*>(hist);  // 32 keys fit in the histogram area
+        if (lane_id() == 0) sk[warp_id()] = k;
+        __syncthreads();
+        if (warp_id() == 0) {
+            Key x = warp_max_key(sk[lane_id()]);
+            if (lane_id() == 0) sk[0] = x;
+        }
+        __syncthreads();
+        const Key r = sk[0];
+        __syncthreads();
+        return r;
+    }
+    // rank of this thread among the threads with `flag`, in thread order; total
+    __device__ int rank(bool flag, int& total) const {
+        const unsigned m = __ballot_sync(0xffffffffu, flag);
+        const int in_warp = __popc(m & ((1u << lane_id()) - 1));
+        if (TEAM == 32) {
+            total = __popc(m);
+            return in_warp;
+        }
+        if (lane_id() == 0) cnt[warp_id()] = __popc(m);
+        __syncthreads();
+        if (warp_id() == 0) {
+            const int v = cnt[lane_id()];
+            int incl = v;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const int o = __shfl_up_sync(0xffffffffu, incl, off);
+                if (lane_id() >= off) incl += o;
+            }
+            cnt[lane_id()] = incl - v;
+            if (lane_id() == 31) cnt[32] = incl;
+        }
+        __syncthreads();
+        const int r = cnt[warp_id()] + in_warp;
+        total = cnt[32];
+        __syncthreads();
+        return r;
+    }
+};
+
+// Candidates of one expert: held slots [0, h) then new bids [0, n).
 struct Cands {
     const int64_t* hb;
     const int32_t* ht;
-    const int64_t* sbb;
-    const int32_t* sbt;
-    const int64_t* gbb;
-    const int32_t* gbt;
+    const int64_t* nb;
+    const int32_t* nt;
     int h, n;
     __device__ __forceinline__ Key get(int c) const {
         Key k;
         if (c < h) {
             k.bid = hb[c];
             k.tok = ht[c];
+            k.slot = c;
         } else {
-            const int j = c - h;
-            if (j < kSB) {
-                k.bid = sbb[j];
-                k.tok = sbt[j];
-            } else {
-                k.bid = gbb[j - kSB];
-                k.tok = gbt[j - kSB];
-            }
+            k.bid = nb[c - h];
+            k.tok = nt[c - h];
+            k.slot = -1;
         }
         return k;
     }
 };
 
-// The k-th worst key among the candidates (keys are unique: tokens differ).
-__device__ Key kth_worst(const Cands& cd, int k, int T, int32_t* hist) {
-    const int lane = lane_id();
+// The k-th worst key among the candidates (1 <= k <= h + n; keys are unique).
+// Radix select on the bid (relative to the smallest bid, 8-bit digits from the
+// top), then, among equal bids, on the token.
+template <int TEAM>
+__device__ Key kth_worst(const Team<TEAM>& tm, const Cands& cd, int k, int tm_tmax) {
     const int m = cd.h + cd.n;
-    if (k <= kSmallK) {
-        Key last = {INT64_MIN, INT32_MAX};
+    const int tid = tm.tid();
+    if (TEAM == 32 && k <= 8) {  // a few rejections: repeated minima
+        Key last = Key{INT64_MIN, INT32_MAX, -2};
         for (int it = 0; it < k; ++it) {
-            Key best = {INT64_MAX, -1};
-            for (int c = lane; c < m; c += kWarp) {
-                Key x = cd.get(c);
+            Key best = pad_key();
+            for (int c = tid; c < m; c += TEAM) {
+                const Key x = cd.get(c);
                 if (worse(last, x) && worse(x, best)) best = x;
             }
             last = warp_min_key(best);
         }
         return last;
     }
-    // radix select on the virtual key ((bid - minb) << tb) | (T - 1 - tok)
     int64_t lo = INT64_MAX, hi = INT64_MIN;
-    for (int c = lane; c < m; c += kWarp) {
-        const Key x = cd.get(c);
-        lo = min(lo, x.bid);
-        hi = max(hi, x.bid);
+    for (int c = tid; c < m; c += TEAM) {
+        const int64_t b = cd.get(c).bid;
+        lo = min(lo, b);
+        hi = max(hi, b);
     }
-    lo = warp_min_i64(lo);
-    hi = warp_max_i64(hi);
-    const int tb = bit_length_u64((uint64_t)(T - 1)) > 0 ? bit_length_u64((uint64_t)(T - 1)) : 1;
-    const int NB = bit_length_u64((uint64_t)(hi - lo)) + tb;
-    using u128 = unsigned __int128;
-    auto vkey = [&](const Key& x) -> u128 {
-        return ((u128)(uint64_t)(x.bid - lo) << tb) | (u128)(uint32_t)((T - 1) - x.tok);
-    };
+    lo = tm.min_i64(lo);
+    hi = tm.max_i64(hi);
+    const int nbits = bit_length_u64((uint64_t)(hi - lo));
+    // --- bid digits
     int need = k, pbits = 0;
-    u128 prefix = 0;
-    for (int guard = 0; guard < 16; ++guard) {
-        const int width = min(8, NB - pbits);
-        const int shift = NB - pbits - width;
-        for (int b = lane; b < kHist; b += kWarp) hist[b] = 0;
-        __syncwarp();
-        for (int c = lane; c < m; c += kWarp) {
-            const u128 K = vkey(cd.get(c));
-            if ((K >> (NB - pbits)) == prefix)
-                atomicAdd(&hist[(int)((K >> shift) & (u128)((1u << width) - 1))], 1);
+    uint64_t prefix = 0;
+    bool whole_bucket = false;
+    while (pbits < nbits) {
+        const int width = min(8, nbits - pbits);
+        const int shift = nbits - pbits - width;
+        for (int b = tid; b < kHist; b += TEAM) tm.hist[b] = 0;
+        tm.sync();
+        for (int c = tid; c < m; c += TEAM) {
+            const uint64_t v = (uint64_t)(cd.get(c).bid - lo);
+            if (shr64(v, shift + width) == prefix)
+                atomicAdd(&tm.hist[(int)((v >> shift) & ((1u << width) - 1))], 1);
         }
-        __syncwarp();
-        int cnt8[8];
-        int sum = 0;
-#pragma unroll
-        for (int b = 0; b < 8; ++b) {
-            cnt8[b] = hist[lane * 8 + b];
-            sum += cnt8[b];
-        }
-        int incl = sum;
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-            const int o = __shfl_up_sync(0xffffffffu, incl, off);
-            if (lane >= off) incl += o;
-        }
-        int run = incl - sum;
-        int found_d = -1, found_before = 0, found_cnt = 0;
-#pragma unroll
-        for (int b = 0; b < 8; ++b) {
-            if (found_d < 0 && run < need && run + cnt8[b] >= need) {
-                found_d = lane * 8 + b;
-                found_before = run;
-                found_cnt = cnt8[b];
+        tm.sync();
+        // find the digit whose bucket holds the need-th element
+        int d = 0, before = 0, cnt = 0;
+        {
+            int run = 0;
+            for (int b = 0; b < (1 << width); ++b) {  // every thread scans (<= 256 smem reads)
+                const int c = tm.hist[b];
+                if (run + c >= need) {
+                    d = b;
+                    before = run;
+                    cnt = c;
+                    break;
+                }
+                run += c;
             }
-            run += cnt8[b];
         }
-        const unsigned fm = __ballot_sync(0xffffffffu, found_d >= 0);
-        const int src = __ffs(fm) - 1;
-        const int d = __shfl_sync(0xffffffffu, found_d, src);
-        const int before = __shfl_sync(0xffffffffu, found_before, src);
-        const int cnt = __shfl_sync(0xffffffffu, found_cnt, src);
-        __syncwarp();
-        prefix = (prefix << width) | (u128)d;
+        tm.sync();
+        prefix = (prefix << width) | (uint64_t)d;
         pbits += width;
         need -= before;
-        if (need == cnt || pbits >= NB) break;
+        if (need == cnt) {
+            whole_bucket = true;
+            break;
+        }
     }
-    // the k-th worst is the best key whose top pbits are <= prefix
-    Key best = {INT64_MIN, INT32_MAX};
-    for (int c = lane; c < m; c += kWarp) {
+    if (whole_bucket) {
+        // reject every candidate whose bid's top pbits are <= prefix; the k-th
+        // worst is the best of them
+        Key best = Key{INT64_MIN, INT32_MAX, -2};
+        const int sh = nbits - pbits;
+        for (int c = tid; c < m; c += TEAM) {
+            const Key x = cd.get(c);
+            if (shr64((uint64_t)(x.bid - lo), sh) <= prefix && worse(best, x)) best = x;
+        }
+        return tm.max_key(best);
+    }
+    // every bid digit fixed: B* = lo + prefix; `need` of the candidates with
+    // bid == B* are rejected, the ones with the largest tokens
+    const int64_t bstar = lo + (int64_t)prefix;
+    const uint32_t tmax = (uint32_t)tm_tmax;  // largest token index + 1 bits below
+    const int tbits = bit_length_u64((uint64_t)tmax) > 0 ? bit_length_u64((uint64_t)tmax) : 1;
+    int tneed = need, tp = 0;
+    uint32_t tprefix = 0;
+    // rank by (tmax - tok) ascending: larger tokens first
+    while (tp < tbits) {
+        const int width = min(8, tbits - tp);
+        const int shift = tbits - tp - width;
+        for (int b = tid; b < kHist; b += TEAM) tm.hist[b] = 0;
+        tm.sync();
+        for (int c = tid; c < m; c += TEAM) {
+            const Key x = cd.get(c);
+            if (x.bid != bstar) continue;
+            const uint32_t v = tmax - (uint32_t)x.tok;
+            if ((uint32_t)shr64(v, shift + width) == tprefix)
+                atomicAdd(&tm.hist[(int)((v >> shift) & ((1u << width) - 1))], 1);
+        }
+        tm.sync();
+        int d = 0, before = 0, cnt = 0;
+        {
+            int run = 0;
+            for (int b = 0; b < (1 << width); ++b) {
+                const int c = tm.hist[b];
+                if (run + c >= tneed) {
+                    d = b;
+                    before = run;
+                    cnt = c;
+                    break;
+                }
+                run += c;
+            }
+        }
+        tm.sync();
+        tprefix = (tprefix << width) | (uint32_t)d;
+        tp += width;
+        tneed -= before;
+        if (tneed == cnt) break;
+    }
+    Key best = Key{INT64_MIN, INT32_MAX, -2};
+    const int sh = tbits - tp;
+    for (int c = tid; c < m; c += TEAM) {
         const Key x = cd.get(c);
-        if ((vkey(x) >> (NB - pbits)) <= prefix && worse(best, x)) best = x;
+        bool rej = x.bid < bstar;
+        if (x.bid == bstar) rej = (uint32_t)shr64(tmax - (uint32_t)x.tok, sh) <= tprefix;
+        if (rej && worse(best, x)) best = x;
     }
-    return warp_max_key(best);
+    return tm.max_key(best);
 }
 
-__device__ __forceinline__ int32_t* remote_i32(int32_t* p, int rank) {
-    return cg::this_cluster().map_shared_rank(p, (unsigned)rank);
-}
-__device__ __forceinline__ int64_t* remote_i64(int64_t* p, int rank) {
-    return cg::this_cluster().map_shared_rank(p, (unsigned)rank);
+// ---------------------------------------------------------------- state
+struct Ctrl {
+    unsigned bar_count;
+    unsigned bar_gen;
+    int abort;
+    int ucount[3];
+    int pad[2];
+};
+
+struct Params {
+    const int32_t* q;
+    int T, E, C, FK;
+    long long max_rounds;
+    int narrow_max;
+    int32_t* assign;
+    int64_t* price_out;
+    base_auction_stats* stats;
+    const int32_t* minmax;
+    Ctrl* ctrl;
+    int64_t* gprice;   // [E]
+    int32_t* hcnt;     // [E]
+    int64_t* hb;       // [E][C]
+    int32_t* ht;
+    int32_t* bcnt;     // [E]
+    int64_t* bb;       // [E][T]
+    int32_t* bt;
+    int32_t* ulist0;   // [T]
+    int32_t* ulist1;
+    int32_t* gfree;    // [E][C]
+    unsigned long long* obj;  // [1]
+    int32_t* u_trace;  // nullable: bidders of round r
+    int64_t* t_trace;  // nullable: globaltimer (ns) at the start of round r
+    long long trace_cap;
+};
+
+__device__ __forceinline__ uint64_t globaltimer();
+
+__device__ __forceinline__ void trace_round(const Params& p, long long r, int U) {
+    if (r < p.trace_cap) {
+        if (p.u_trace) p.u_trace[r] = U;
+        if (p.t_trace) p.t_trace[r] = (int64_t)globaltimer();
+    }
 }
 
-// Appends the tokens of the lanes with `rej` set to the next round's list
-// (one DSMEM atomic per warp on CTA 0's counter).
-__device__ __forceinline__ void push_rejected(bool rej, int32_t tok, int32_t* unext,
-                                              int32_t* ucount_remote) {
-    const unsigned m = __ballot_sync(0xffffffffu, rej);
-    if (!m) return;
+// shared memory of every CTA (narrow-mode arrays are used by CTA 0 only)
+struct SmemLayout {
+    size_t price, fr, fsize, hcnt, ncnt, noff, nfill, active, rec_e, rec_b, rec_t, grp_b, grp_t,
+        list0, list1, hist, red, cnt, misc, total;
+};
+
+__host__ __device__ inline SmemLayout smem_layout(int E, int FK, int NM) {
+    SmemLayout L;
+    size_t o = 0;
+    auto take = [&](size_t bytes) { size_t r = o; o += align_up(bytes, 16); return r; };
+    L.price = take(8 * (size_t)E);
+    L.fr = take(sizeof(Key) * (size_t)E * FK);
+    L.fsize = take(4 * (size_t)E);
+    L.hcnt = take(4 * (size_t)E);
+    L.ncnt = take(4 * (size_t)E);
+    L.noff = take(4 * (size_t)E);
+    L.nfill = take(4 * (size_t)E);
+    L.active = take(4 * (size_t)E);
+    L.rec_e = take(4 * (size_t)NM);
+    L.rec_b = take(8 * (size_t)NM);
+    L.rec_t = take(4 * (size_t)NM);
+    L.grp_b = take(8 * (size_t)NM);
+    L.grp_t = take(4 * (size_t)NM);
+    L.list0 = take(4 * (size_t)NM);
+    L.list1 = take(4 * (size_t)NM);
+    L.hist = take(4 * (size_t)kWarps * kHist);
+    L.red = take(8 * 32);
+    L.cnt = take(4 * 64);
+    L.misc = take(64);
+    L.total = o;
+    return L;
+}
+
+__device__ __forceinline__ uint64_t globaltimer() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Grid barrier (all CTAs are co-resident: cooperative launch).  Returns
+// false when the wait gave up or another CTA gave up.
+__device__ bool grid_sync(Ctrl* c, int* s_flag) {
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        volatile unsigned* genp = &c->bar_gen;
+        const unsigned g = *genp;
+        __threadfence();
+        const unsigned arrived = atomicAdd(&c->bar_count, 1u) + 1u;
+        int ok = 1;
+        if (arrived == gridDim.x) {
+            c->bar_count = 0;
+            __threadfence();
+            atomicAdd(&c->bar_gen, 1u);
+        } else {
+            const uint64_t t0 = globaltimer();
+            long long it = 0;
+            while (*genp == g) {
+                if (*reinterpret_cast<volatile int*>(&c->abort)) {
+                    ok = 0;
+                    break;
+                }
+                if (((++it) & 63) == 0 && globaltimer() - t0 > kWaitNs) {
+                    atomicExch(&c->abort, 1);
+                    record_error(5001);
+                    ok = 0;
+                    break;
+                }
+                if (it > (1ll << 34)) {
+                    atomicExch(&c->abort, 1);
+                    record_error(5002);
+                    ok = 0;
+                    break;
+                }
+                __nanosleep(100);
+            }
+        }
+        __threadfence();
+        *s_flag = ok;
+    }
+    __syncthreads();
+    return *s_flag != 0;
+}
+
+// best / second-best scan of one token's row by a group of G lanes
+__device__ __forceinline__ void group_bid(const int32_t* __restrict__ row, const int64_t* price,
+                                          int E, int G, int gl, int64_t scale, int64_t& v1,
+                                          int64_t& v2, int& e1) {
+    v1 = INT64_MIN;
+    v2 = INT64_MIN;
+    e1 = INT32_MAX;
+    for (int e = gl; e < E; e += G) {
+        const int64_t v = (int64_t)__ldg(row + e) * scale - price[e];
+        if (v > v1) {
+            v2 = v1;
+            v1 = v;
+            e1 = e;
+        } else if (v > v2) {
+            v2 = v;
+        }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+        if (off >= G) continue;
+        const int64_t ov1 = __shfl_xor_sync(0xffffffffu, v1, off);
+        const int64_t ov2 = __shfl_xor_sync(0xffffffffu, v2, off);
+        const int oe1 = __shfl_xor_sync(0xffffffffu, e1, off);
+        if (ov1 > v1 || (ov1 == v1 && oe1 < e1)) {
+            v2 = max(v1, ov2);
+            v1 = ov1;
+            e1 = oe1;
+        } else {
+            v2 = max(v2, ov1);
+        }
+    }
+}
+
+__device__ __forceinline__ void prefetch_row_l1(const int32_t* row, int E) {
+    for (int off = 0; off < E * 4; off += 128)
+        asm volatile("prefetch.global.L1 [%0];" ::"l"(reinterpret_cast<const char*>(row) + off));
+}
+
+// Keeps the C best of held + new for expert e (held in global memory), with
+// a team of TEAM threads.  Rejected tokens are appended to `unext` through
+// the counter `ucnt`.  Returns the expert's new held count; `price` is set
+// when the expert is full.
+template <int TEAM>
+__device__ int resolve_general(const Team<TEAM>& tm, const Params& p, int e, const Cands& cd,
+                               int64_t* hb, int32_t* ht, int32_t* unext, int32_t* ucnt,
+                               int64_t& price, bool prefetch) {
+    const int C = p.C, h = cd.h, n = cd.n;
+    const int tid = tm.tid();
+    if (h + n <= C) {
+        for (int j = tid; j < n; j += TEAM) {
+            const Key x = cd.get(h + j);
+            hb[h + j] = x.bid;
+            ht[h + j] = x.tok;
+        }
+        tm.sync();
+        if (h + n == C) {
+            int64_t mn = INT64_MAX;
+            for (int i = tid; i < C; i += TEAM) mn = min(mn, hb[i]);
+            price = tm.min_i64(mn);
+        }
+        return h + n;
+    }
+    const int k = h + n - C;
+    const Key kth = kth_worst<TEAM>(tm, cd, k, p.T - 1);
+    int32_t* gfree = p.gfree + (size_t)e * C;
+    // pass 1: free slots (rejected held, then the empty tail) in slot order
+    int nfree = 0;
+    for (int b0 = 0; b0 < C; b0 += TEAM) {
+        const int i = b0 + tid;
+        bool isfree = false, rej = false;
+        int32_t tok = 0;
+        if (i < C) {
+            if (i < h) {
+                const Key x = cd.get(i);
+                if (!worse(kth, x)) {
+                    isfree = true;
+                    rej = true;
+                    tok = x.tok;
+                }
+            } else {
+                isfree = true;
+            }
+        }
+        int nrej = 0;
+        const int rr = tm.rank(rej, nrej);
+        int base = 0;
+        if (nrej) {
+            if (TEAM == 32) {
+                if (lane_id() == 0) base = atomicAdd(ucnt, nrej);
+                base = __shfl_sync(0xffffffffu, base, 0);
+            } else {
+                if (tid == 0) tm.cnt[33] = atomicAdd(ucnt, nrej);
+                __syncthreads();
+                base = tm.cnt[33];
+                __syncthreads();
+            }
+        }
+        if (rej) {
+            unext[base + rr] = tok;
+            if (prefetch) prefetch_row_l1(p.q + (size_t)tok * p.E, p.E);
+        }
+        int tot = 0;
+        const int r = tm.rank(isfree, tot);
+        if (isfree) gfree[nfree + r] = i;
+        nfree += tot;
+    }
+    tm.sync();
+    __threadfence_block();
+    // pass 2: new bids; accepted ones take the free slots in order
+    int nacc = 0;
+    for (int b0 = 0; b0 < n; b0 += TEAM) {
+        const int j = b0 + tid;
+        bool acc = false, rej = false;
+        Key x = pad_key();
+        if (j < n) {
+            x = cd.get(h + j);
+            if (worse(kth, x)) acc = true; else rej = true;
+        }
+        int nrej = 0;
+        const int rr = tm.rank(rej, nrej);
+        int base = 0;
+        if (nrej) {
+            if (TEAM == 32) {
+                if (lane_id() == 0) base = atomicAdd(ucnt, nrej);
+                base = __shfl_sync(0xffffffffu, base, 0);
+            } else {
+                if (tid == 0) tm.cnt[33] = atomicAdd(ucnt, nrej);
+                __syncthreads();
+                base = tm.cnt[33];
+                __syncthreads();
+            }
+        }
+        if (rej) {
+            unext[base + rr] = x.tok;
+            if (prefetch) prefetch_row_l1(p.q + (size_t)x.tok * p.E, p.E);
+        }
+        int tot = 0;
+        const int r = tm.rank(acc, tot);
+        if (acc) {
+            const int slot = gfree[nacc + r];
+            hb[slot] = x.bid;
+            ht[slot] = x.tok;
+        }
+        nacc += tot;
+    }
+    tm.sync();
+    __threadfence_block();
+    if (nacc != nfree && tid == 0) record_error(1000 + e);
+    int64_t mn = INT64_MAX;
+    for (int i = tid; i < C; i += TEAM) mn = min(mn, hb[i]);
+    price = tm.min_i64(mn);
+    return C;
+}
+
+// Rebuilds the fringe of a full expert: its FK worst held keys, sorted, from
+// a warp-wide scan of the C held bids (chunks of 32 merged into the running
+// 32 lowest).  Returns the fringe size.
+__device__ int rebuild_fringe(const int64_t* hb, const int32_t* ht, int C, int FK, Key* fr) {
     const int lane = lane_id();
+    Key best = pad_key();
+    for (int b0 = 0; b0 < C; b0 += 32) {
+        const int i = b0 + lane;
+        Key x = pad_key();
+        if (i < C) x = Key{hb[i], ht[i], i};
+        x = warp_sort(x);
+        Key lo, hi;
+        warp_merge64(best, x, lo, hi);
+        best = lo;
+    }
+    const int fs = min(FK, C);
+    if (lane < fs) fr[lane] = best;
+    __syncwarp();
+    return fs;
+}
+
+// Fast narrow-mode resolve of a full expert whose fringe is valid and holds
+// at least n + 1 keys (n < 32 new bids, as many rejections): the sorted new
+// bids are merged with the sorted fringe; the n worst of the 64 are rejected,
+// accepted new bids take the slots the rejected fringe keys free, and the
+// survivors not above the old fringe maximum form the new fringe.  Sets fs to
+// the new fringe size (0: the caller rebuilds it) and price to its minimum.
+__device__ __forceinline__ int nth_set_lane(unsigned m, int r) {
+    for (int i = 0; i < r; ++i) m &= m - 1;
+    return m ? __ffs(m) - 1 : 0;
+}
+
+__device__ void resolve_fringe(const Params& p, Key* fr, int& fs, const int64_t* nb,
+                               const int32_t* nt, int n, int64_t* hb, int32_t* ht,
+                               int32_t* next_list, int* next_cnt, int64_t& price) {
+    const int lane = lane_id();
+    const unsigned lt = (1u << lane) - 1;
+    const int k = n;
+    const Key f = lane < fs ? fr[lane] : pad_key();
+    const Key fmax = shfl_key(f, fs - 1);
+    Key x = lane < n ? Key{nb[lane], nt[lane], -1} : pad_key();
+    x = warp_sort(x);
+    Key lo, hi;
+    warp_merge64(f, x, lo, hi);
+    const bool rej = lane < k;  // elements 0 .. k-1 (all in lo since k < 32)
+    const unsigned freed = __ballot_sync(0xffffffffu, rej && lo.slot >= 0);
+    const unsigned acc_lo = __ballot_sync(0xffffffffu, !rej && lo.slot == -1);
+    const unsigned acc_hi = __ballot_sync(0xffffffffu, hi.slot == -1);
+    // the r-th accepted new key takes the slot of the r-th rejected fringe key
+    const int src_lo = nth_set_lane(freed, __popc(acc_lo & lt));
+    const int src_hi = nth_set_lane(freed, __popc(acc_lo) + __popc(acc_hi & lt));
+    const int slot_lo = __shfl_sync(0xffffffffu, lo.slot, src_lo);
+    const int slot_hi = __shfl_sync(0xffffffffu, lo.slot, src_hi);
+    if ((acc_lo >> lane) & 1u) {
+        lo.slot = slot_lo;
+        hb[slot_lo] = lo.bid;
+        ht[slot_lo] = lo.tok;
+    }
+    if ((acc_hi >> lane) & 1u) {
+        hi.slot = slot_hi;
+        hb[slot_hi] = hi.bid;
+        ht[slot_hi] = hi.tok;
+    }
+    // rejected tokens bid next round: append them and fetch their rows into L1
+    const unsigned rm = __ballot_sync(0xffffffffu, rej);
     int base = 0;
-    if (lane == 0) base = atomicAdd(ucount_remote, __popc(m));
+    if (lane == 0) base = atomicAdd(next_cnt, __popc(rm));
     base = __shfl_sync(0xffffffffu, base, 0);
-    if (rej) unext[base + __popc(m & ((1u << lane) - 1))] = tok;
+    if (rej) {
+        next_list[base + __popc(rm & lt)] = lo.tok;
+        prefetch_row_l1(p.q + (size_t)lo.tok * p.E, p.E);
+    }
+    // the new fringe: surviving keys not above the old fringe maximum, in order
+    const bool keep_lo = !rej && !worse(fmax, lo);
+    const bool keep_hi = hi.slot != -2 && !worse(fmax, hi);
+    const unsigned kl = __ballot_sync(0xffffffffu, keep_lo);
+    const unsigned kh = __ballot_sync(0xffffffffu, keep_hi);
+    const int nl = __popc(kl);
+    __syncwarp();
+    if (keep_lo) fr[__popc(kl & lt)] = lo;
+    if (keep_hi) {
+        const int pos = nl + __popc(kh & lt);
+        if (pos < p.FK) fr[pos] = hi;
+    }
+    __syncwarp();
+    fs = min(p.FK, nl + __popc(kh));
+    if (fs > 0) price = fr[0].bid;
 }
 
 __global__ void __launch_bounds__(kThreads, 1) auction_kernel(const __grid_constant__ Params p) {
-    cg::cluster_group cluster = cg::this_cluster();
-    const int rank = (int)cluster.block_rank();
     extern __shared__ __align__(16) unsigned char smem[];
-    const SmemLayout L = smem_layout(p.E, p.EL, p.C, p.held_in_smem);
+    const SmemLayout L = smem_layout(p.E, p.FK, p.narrow_max);
     int64_t* s_price = reinterpret_cast<int64_t*>(smem + L.price);
-    int64_t* s_hb = reinterpret_cast<int64_t*>(smem + L.held_bid);
-    int32_t* s_ht = reinterpret_cast<int32_t*>(smem + L.held_tok);
+    Key* s_fr = reinterpret_cast<Key*>(smem + L.fr);
+    int32_t* s_fsize = reinterpret_cast<int32_t*>(smem + L.fsize);
     int32_t* s_hcnt = reinterpret_cast<int32_t*>(smem + L.hcnt);
-    int32_t* s_cnt = reinterpret_cast<int32_t*>(smem + L.cnt);
-    int64_t* s_sbb = reinterpret_cast<int64_t*>(smem + L.sb_bid);
-    int32_t* s_sbt = reinterpret_cast<int32_t*>(smem + L.sb_tok);
+    int32_t* s_ncnt = reinterpret_cast<int32_t*>(smem + L.ncnt);
+    int32_t* s_noff = reinterpret_cast<int32_t*>(smem + L.noff);
+    int32_t* s_nfill = reinterpret_cast<int32_t*>(smem + L.nfill);
+    int32_t* s_active = reinterpret_cast<int32_t*>(smem + L.active);
+    int32_t* s_rec_e = reinterpret_cast<int32_t*>(smem + L.rec_e);
+    int64_t* s_rec_b = reinterpret_cast<int64_t*>(smem + L.rec_b);
+    int32_t* s_rec_t = reinterpret_cast<int32_t*>(smem + L.rec_t);
+    int64_t* s_grp_b = reinterpret_cast<int64_t*>(smem + L.grp_b);
+    int32_t* s_grp_t = reinterpret_cast<int32_t*>(smem + L.grp_t);
+    int32_t* s_list0 = reinterpret_cast<int32_t*>(smem + L.list0);
+    int32_t* s_list1 = reinterpret_cast<int32_t*>(smem + L.list1);
     int32_t* s_hist = reinterpret_cast<int32_t*>(smem + L.hist);
-    int32_t* s_ucount = reinterpret_cast<int32_t*>(smem + L.ctrl);                  // [4]
-    unsigned long long* s_obj = reinterpret_cast<unsigned long long*>(smem + L.ctrl + 16);
+    int64_t* s_red = reinterpret_cast<int64_t*>(smem + L.red);
+    int32_t* s_cnt = reinterpret_cast<int32_t*>(smem + L.cnt);
+    int32_t* s_misc = reinterpret_cast<int32_t*>(smem + L.misc);
 
-    const int T = p.T, E = p.E, C = p.C, CL = p.CL, EL = p.EL;
+    const int T = p.T, E = p.E, C = p.C, FK = p.FK;
     const int64_t scale = (int64_t)T + 1;
     const int lane = lane_id(), warp = warp_id();
+    const int cta = blockIdx.x, ncta = gridDim.x;
 
-    for (int e = threadIdx.x; e < E; e += kThreads) s_price[e] = 0;
-    for (int i = threadIdx.x; i < EL; i += kThreads) {
-        s_hcnt[i] = 0;
-        s_cnt[i] = 0;
-    }
-    if (threadIdx.x < 4) s_ucount[threadIdx.x] = 0;
-    if (threadIdx.x == 0) *s_obj = 0ull;
+    Team<1024> cta_team{s_hist, s_red, s_cnt};
+    Team<32> warp_team{s_hist + warp * kHist, nullptr, nullptr};
 
     const int64_t qmin = p.minmax[0], qmax = p.minmax[1];
     const int64_t range = qmax - qmin;
@@ -316,215 +804,257 @@ __global__ void __launch_bounds__(kThreads, 1) auction_kernel(const __grid_const
     // lanes per bidding token: the smallest power of two >= E, at most 32
     int G = 1;
     while (G < E && G < kWarp) G <<= 1;
-    const int tok_per_warp = kWarp / G;
+    const int tpw = kWarp / G;
     const int sub = lane / G, gl = lane % G;
 
-    int32_t* ucount0 = remote_i32(s_ucount, 0);
-    cluster_barrier();
-
     long long rounds = 0, phases = 0, bids = 0;
-    int cur = 0;
-    bool stop = (status != BASE_OK);
-    while (!stop) {
+    bool ok = true;
+    int cur = 0;  // which global list holds the bidders
+
+    while (status == BASE_OK && ok) {
         ++phases;
-        for (int i = threadIdx.x; i < EL; i += kThreads) s_hcnt[i] = 0;
+        // ---- phase start: nothing held, prices kept (in p.gprice)
+        for (int e = cta * kThreads + threadIdx.x; e < E; e += ncta * kThreads) {
+            p.hcnt[e] = 0;
+            p.bcnt[e] = 0;
+        }
+        if (cta == 0 && threadIdx.x < 3) p.ctrl->ucount[threadIdx.x] = 0;
+        if (!(ok = grid_sync(p.ctrl, s_misc))) break;
         int U = T;
-        bool phase_start = true;
-        while (U > 0) {
+        bool first = true;
+        bool narrow = false;
+        while (U > 0 && !narrow) {
+            // ================= wide round =================
             if (rounds >= p.max_rounds) {
                 status = BASE_ERR_NOT_CONVERGED;
                 break;
             }
+            if (cta == 0 && threadIdx.x == 0) trace_round(p, rounds, U);
             ++rounds;
             bids += U;
             const int32_t* ulist = cur ? p.ulist1 : p.ulist0;
             int32_t* unext = cur ? p.ulist0 : p.ulist1;
-            int32_t* ucount_w = ucount0 + (int)(rounds % 3);
-
-            // ---------------- bid ----------------
+            int32_t* ucnt = &p.ctrl->ucount[(int)(rounds % 3)];
+            for (int e = threadIdx.x; e < E; e += kThreads) s_price[e] = vload(p.gprice + e);
+            __syncthreads();
             {
-                const int stride = CL * kWarps * tok_per_warp;
-                for (int base = (rank * kWarps + warp) * tok_per_warp; base < U; base += stride) {
-                    const int i = base + sub;
+                const long long gw = (long long)cta * kWarps + warp;
+                const long long stride = (long long)ncta * kWarps * tpw;
+                for (long long base = gw * tpw; base < U; base += stride) {
+                    const long long i = base + sub;
                     const bool valid = i < U;
-                    int t = 0;
-                    if (valid) t = phase_start ? i : ulist[i];
-                    int64_t v1 = INT64_MIN, v2 = INT64_MIN;
-                    int e1 = INT32_MAX;
-                    if (valid) {
-                        const int32_t* row = p.q + (size_t)t * E;
-                        for (int e = gl; e < E; e += G) {
-                            const int64_t v = (int64_t)__ldg(row + e) * scale - s_price[e];
-                            if (v > v1) {
-                                v2 = v1;
-                                v1 = v;
-                                e1 = e;
-                            } else if (v > v2) {
-                                v2 = v;
-                            }
-                        }
-                    }
-#pragma unroll
-                    for (int off = 16; off > 0; off >>= 1) {
-                        if (off >= G) continue;
-                        const int64_t ov1 = __shfl_xor_sync(0xffffffffu, v1, off);
-                        const int64_t ov2 = __shfl_xor_sync(0xffffffffu, v2, off);
-                        const int oe1 = __shfl_xor_sync(0xffffffffu, e1, off);
-                        if (ov1 > v1 || (ov1 == v1 && oe1 < e1)) {
-                            v2 = max(v1, ov2);
-                            v1 = ov1;
-                            e1 = oe1;
-                        } else {
-                            v2 = max(v2, ov1);
-                        }
-                    }
+                    const int t = valid ? (first ? (int)i : vload(ulist + i)) : 0;
+                    int64_t v1, v2;
+                    int e1;
+                    group_bid(p.q + (size_t)t * E, s_price, valid ? E : 0, G, gl, scale, v1, v2,
+                              e1);
                     if (valid && gl == 0) {
-                        const int64_t bid = v1 + s_price[e1] - v2 + eps;
-                        const int owner = e1 % CL, el = e1 / CL;
-                        const int pos = atomicAdd(remote_i32(s_cnt, owner) + el, 1);
-                        if (pos < kSB) {
-                            remote_i64(s_sbb, owner)[el * kSB + pos] = bid;
-                            remote_i32(s_sbt, owner)[el * kSB + pos] = t;
-                        } else {
-                            p.gb_bid[(size_t)e1 * T + (pos - kSB)] = bid;
-                            p.gb_tok[(size_t)e1 * T + (pos - kSB)] = t;
-                        }
+                        const int64_t b = v1 + s_price[e1] - v2 + eps;
+                        const int pos = atomicAdd(&p.bcnt[e1], 1);
+                        p.bb[(size_t)e1 * T + pos] = b;
+                        p.bt[(size_t)e1 * T + pos] = t;
                     }
                 }
             }
-            cluster_barrier();
-
-            // ---------------- resolve ----------------
-            for (int el = warp; el < EL; el += kWarps) {
-                const int e = el * CL + rank;
-                if (e >= E) continue;
-                const int n = s_cnt[el];
+            if (!(ok = grid_sync(p.ctrl, s_misc))) break;
+            for (int e = cta; e < E; e += ncta) {
+                const int n = vload(p.bcnt + e);
                 if (n == 0) continue;
-                __syncwarp();
-                if (lane == 0) s_cnt[el] = 0;
-                const int h = s_hcnt[el];
-                int64_t* hb = p.held_in_smem ? s_hb + (size_t)el * C : p.gh_bid + (size_t)e * C;
-                int32_t* ht = p.held_in_smem ? s_ht + (size_t)el * C : p.gh_tok + (size_t)e * C;
-                Cands cd;
-                cd.hb = hb;
-                cd.ht = ht;
-                cd.sbb = s_sbb + el * kSB;
-                cd.sbt = s_sbt + el * kSB;
-                cd.gbb = p.gb_bid + (size_t)e * T;
-                cd.gbt = p.gb_tok + (size_t)e * T;
-                cd.h = h;
-                cd.n = n;
-                bool full = false;
-                if (h + n <= C) {
-                    for (int j = lane; j < n; j += kWarp) {
-                        const Key x = cd.get(h + j);
-                        hb[h + j] = x.bid;
-                        ht[h + j] = x.tok;
+                __syncthreads();
+                const int h = vload(p.hcnt + e);
+                Cands cd{p.hb + (size_t)e * C, p.ht + (size_t)e * C, p.bb + (size_t)e * T,
+                         p.bt + (size_t)e * T, h, n};
+                int64_t price = INT64_MIN;
+                const int nh = resolve_general<1024>(cta_team, p, e, cd, p.hb + (size_t)e * C,
+                                                     p.ht + (size_t)e * C, unext, ucnt, price,
+                                                     false);
+                if (threadIdx.x == 0) {
+                    p.hcnt[e] = nh;
+                    p.bcnt[e] = 0;
+                    if (nh == C) p.gprice[e] = price;
+                }
+                __syncthreads();
+            }
+            // the counter the next round writes: last read two rounds ago
+            if (cta == 0 && threadIdx.x == 0) p.ctrl->ucount[(int)((rounds + 1) % 3)] = 0;
+            if (!(ok = grid_sync(p.ctrl, s_misc))) break;
+            U = *reinterpret_cast<volatile int*>(ucnt);
+            cur ^= 1;
+            first = false;
+            if (U > 0 && U <= p.narrow_max) narrow = true;
+        }
+        if (!ok || status != BASE_OK) break;
+        if (narrow) {
+            // ================= narrow rounds on CTA 0 =================
+            if (cta == 0) {
+                const int32_t* ulist = cur ? p.ulist1 : p.ulist0;
+                int32_t* lists[2] = {s_list0, s_list1};
+                int lc = 0;
+                for (int i = threadIdx.x; i < U; i += kThreads) s_list0[i] = vload(ulist + i);
+                for (int e = threadIdx.x; e < E; e += kThreads) {
+                    s_price[e] = vload(p.gprice + e);
+                    s_hcnt[e] = vload(p.hcnt + e);
+                    s_fsize[e] = -1;  // fringe not built
+                    s_ncnt[e] = 0;
+                }
+                if (threadIdx.x == 0) s_misc[1] = 0;
+                __syncthreads();
+                while (U > 0) {
+                    if (rounds >= p.max_rounds) {
+                        status = BASE_ERR_NOT_CONVERGED;
+                        break;
                     }
-                    __syncwarp();
-                    if (lane == 0) s_hcnt[el] = h + n;
-                    full = (h + n == C);
-                } else {
-                    const int k = h + n - C;
-                    int32_t* hist = s_hist + warp * kHist;
-                    const Key kth = kth_worst(cd, k, T, hist);
-                    // free slots: rejected held slots and the empty tail, in order
-                    int32_t* gfree = p.gfree + (size_t)e * C;
-                    int nfree = 0;
-                    for (int b0 = 0; b0 < C; b0 += kWarp) {
-                        const int i = b0 + lane;
-                        bool isfree = false, rej = false;
-                        int32_t tok = 0;
-                        if (i < C) {
-                            if (i < h) {
-                                const Key x = cd.get(i);
-                                if (!worse(kth, x)) {
-                                    isfree = true;
-                                    rej = true;
-                                    tok = x.tok;
-                                }
-                            } else {
-                                isfree = true;
+                    if (threadIdx.x == 0) trace_round(p, rounds, U);
+                    ++rounds;
+                    bids += U;
+                    int32_t* list = lists[lc];
+                    int32_t* next = lists[lc ^ 1];
+                    // bid
+                    for (int base = warp * tpw; base < U; base += kWarps * tpw) {
+                        const int i = base + sub;
+                        const bool valid = i < U;
+                        const int t = valid ? list[i] : 0;
+                        int64_t v1, v2;
+                        int e1;
+                        group_bid(p.q + (size_t)t * E, s_price, valid ? E : 0, G, gl, scale, v1,
+                                  v2, e1);
+                        if (valid && gl == 0) {
+                            s_rec_e[i] = e1;
+                            s_rec_b[i] = v1 + s_price[e1] - v2 + eps;
+                            s_rec_t[i] = t;
+                            if (atomicAdd(&s_ncnt[e1], 1) == 0) {
+                                const int a = atomicAdd(&s_misc[1], 1);
+                                s_active[a] = e1;
                             }
                         }
-                        push_rejected(rej, tok, unext, ucount_w);
-                        const unsigned fm = __ballot_sync(0xffffffffu, isfree);
-                        if (isfree) {
-                            const int r = nfree + __popc(fm & ((1u << lane) - 1));
-                            if (r < kHist) hist[r] = i; else gfree[r] = i;
-                        }
-                        nfree += __popc(fm);
                     }
-                    __syncwarp();
-                    // hist was consumed by the selection; it now holds free slots
-                    int nacc = 0;
-                    for (int b0 = 0; b0 < n; b0 += kWarp) {
-                        const int j = b0 + lane;
-                        bool acc = false, rej = false;
-                        Key x = {0, 0};
-                        if (j < n) {
-                            x = cd.get(h + j);
-                            if (worse(kth, x)) acc = true; else rej = true;
+                    __syncthreads();
+                    const int nact = s_misc[1];
+                    // group the records by expert
+                    if (warp == 0) {
+                        int run = 0;
+                        for (int a0 = 0; a0 < nact; a0 += 32) {
+                            const int a = a0 + lane;
+                            const int c = a < nact ? s_ncnt[s_active[a]] : 0;
+                            int incl = c;
+#pragma unroll
+                            for (int off = 1; off < 32; off <<= 1) {
+                                const int o = __shfl_up_sync(0xffffffffu, incl, off);
+                                if (lane >= off) incl += o;
+                            }
+                            if (a < nact) {
+                                s_noff[s_active[a]] = run + incl - c;
+                                s_nfill[s_active[a]] = 0;
+                            }
+                            run += __shfl_sync(0xffffffffu, incl, 31);
                         }
-                        push_rejected(rej, x.tok, unext, ucount_w);
-                        const unsigned am = __ballot_sync(0xffffffffu, acc);
-                        if (acc) {
-                            const int r = nacc + __popc(am & ((1u << lane) - 1));
-                            const int slot = (r < kHist) ? hist[r] : gfree[r];
-                            hb[slot] = x.bid;
-                            ht[slot] = x.tok;
-                        }
-                        nacc += __popc(am);
                     }
-                    __syncwarp();
-                    if (lane == 0) s_hcnt[el] = C;
-                    full = true;
-                    if (nacc != nfree && lane == 0) record_error(1000 + e);
+                    __syncthreads();
+                    for (int i = threadIdx.x; i < U; i += kThreads) {
+                        const int e = s_rec_e[i];
+                        const int pos = s_noff[e] + atomicAdd(&s_nfill[e], 1);
+                        s_grp_b[pos] = s_rec_b[i];
+                        s_grp_t[pos] = s_rec_t[i];
+                    }
+                    if (threadIdx.x == 0) s_misc[2] = 0;  // next list count
+                    __syncthreads();
+                    // resolve: a warp per active expert
+                    for (int a = warp; a < nact; a += kWarps) {
+                        const int e = s_active[a];
+                        const int n = s_ncnt[e];
+                        const int h = s_hcnt[e];
+                        const int64_t* nb = s_grp_b + s_noff[e];
+                        const int32_t* nt = s_grp_t + s_noff[e];
+                        int64_t* hb = p.hb + (size_t)e * C;
+                        int32_t* ht = p.ht + (size_t)e * C;
+                        Key* fr = s_fr + (size_t)e * FK;
+                        int64_t price = s_price[e];
+                        bool done = false;
+                        if (h == C && n < 32) {
+                            int fs = s_fsize[e];
+                            if (fs < n + 1) fs = rebuild_fringe(hb, ht, C, FK, fr);
+                            if (fs >= n + 1) {
+                                resolve_fringe(p, fr, fs, nb, nt, n, hb, ht, next, &s_misc[2],
+                                               price);
+                                if (fs == 0) {
+                                    __syncwarp();
+                                    fs = rebuild_fringe(hb, ht, C, FK, fr);
+                                    price = fr[0].bid;
+                                }
+                                done = true;
+                                if (lane == 0) s_fsize[e] = fs;
+                            }
+                        }
+                        if (!done) {
+                            Cands cd{hb, ht, nb, nt, h, n};
+                            const int nh = resolve_general<32>(warp_team, p, e, cd, hb, ht, next,
+                                                               &s_misc[2], price, true);
+                            if (lane == 0) {
+                                s_hcnt[e] = nh;
+                                s_fsize[e] = -1;
+                            }
+                        }
+                        __syncwarp();
+                        if (lane == 0) {
+                            if (s_hcnt[e] == C) s_price[e] = price;
+                            s_ncnt[e] = 0;
+                        }
+                    }
+                    __syncthreads();
+                    U = s_misc[2];
+                    if (threadIdx.x == 0) s_misc[1] = 0;
+                    lc ^= 1;
+                    __syncthreads();
                 }
-                if (full) {
-                    int64_t mn = INT64_MAX;
-                    for (int i = lane; i < C; i += kWarp) mn = min(mn, hb[i]);
-                    mn = warp_min_i64(mn);
-                    if (lane < CL) remote_i64(s_price, lane)[e] = mn;
+                // hand the prices and counts back to the grid
+                for (int e = threadIdx.x; e < E; e += kThreads) {
+                    p.gprice[e] = s_price[e];
+                    p.hcnt[e] = s_hcnt[e];
                 }
-                __syncwarp();
+                if (threadIdx.x == 0) {
+                    s_misc[3] = status;
+                    reinterpret_cast<volatile long long*>(p.obj)[1] = rounds;
+                    reinterpret_cast<volatile long long*>(p.obj)[2] = bids;
+                    reinterpret_cast<volatile int*>(p.obj)[6] = status;
+                }
             }
-            cluster_barrier();
-            U = *reinterpret_cast<volatile int32_t*>(ucount_w);
-            if (rank == 0 && threadIdx.x == 0) s_ucount[(int)((rounds + 1) % 3)] = 0;
-            cur ^= 1;
-            phase_start = false;
+            if (!(ok = grid_sync(p.ctrl, s_misc))) break;
+            // every CTA takes over CTA 0's counters
+            rounds = reinterpret_cast<volatile long long*>(p.obj)[1];
+            bids = reinterpret_cast<volatile long long*>(p.obj)[2];
+            status = reinterpret_cast<volatile int*>(p.obj)[6];
+            if (!(ok = grid_sync(p.ctrl, s_misc))) break;
         }
         if (status != BASE_OK) break;
         if (eps == 1) break;
         eps /= kEpsFactor;
         if (eps < 1) eps = 1;
     }
+    if (!ok) return;
 
-    // results: every owner writes its experts' tokens and prices
+    // results: every CTA writes its experts' tokens
     unsigned long long part = 0;
-    for (int el = warp; el < EL; el += kWarps) {
-        const int e = el * CL + rank;
-        if (e >= E) continue;
-        const int h = s_hcnt[el];
-        const int32_t* ht = p.held_in_smem ? s_ht + (size_t)el * C : p.gh_tok + (size_t)e * C;
-        for (int j = lane; j < h; j += kWarp) {
-            const int t = ht[j];
+    for (long long i = (long long)cta * kThreads + threadIdx.x; i < (long long)T;
+         i += (long long)ncta * kThreads) {
+        const int e = (int)(i / C);
+        const int t = p.ht[i];
+        if (status == BASE_OK) {
             p.assign[t] = e;
             part += (unsigned long long)(int64_t)p.q[(size_t)t * E + e];
         }
-        if (lane == 0) p.price_out[e] = s_price[e];
     }
+    for (int e = cta * kThreads + threadIdx.x; e < E; e += ncta * kThreads)
+        p.price_out[e] = p.gprice[e];
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
-    if (lane == 0 && part) atomicAdd(cluster.map_shared_rank(s_obj, 0u), part);
-    cluster_barrier();
-    if (rank == 0 && threadIdx.x == 0 && p.stats) {
+    if (lane == 0 && part) atomicAdd(p.obj, part);
+    if (!grid_sync(p.ctrl, s_misc)) return;
+    if (cta == 0 && threadIdx.x == 0 && p.stats) {
         p.stats->status = status;
         p.stats->phases = phases;
         p.stats->rounds = rounds;
         p.stats->final_eps = eps;
-        p.stats->objective = (status == BASE_OK) ? (int64_t)*s_obj : 0;
+        p.stats->objective = (status == BASE_OK) ? (int64_t)*p.obj : 0;
         p.stats->bids = bids;
     }
 }
@@ -570,121 +1100,103 @@ __global__ void minmax_kernel(const int32_t* __restrict__ q, size_t n, int32_t* 
     }
 }
 
-struct Plan {
-    int CL, EL, held_in_smem;
-    size_t smem;
-};
-
-static Plan make_plan(int T, int E) {
-    const int C = T / E;
-    Plan pl{};
-    for (int CL = 1; CL <= 16; CL <<= 1) {
-        if (CL > E) break;
-        const int EL = (E + CL - 1) / CL;
-        const size_t b = smem_layout(E, EL, C, 1).total;
-        if (b <= kMaxSmem) {
-            pl.CL = CL;
-            pl.EL = EL;
-            pl.held_in_smem = 1;
-            pl.smem = b;
-            return pl;
-        }
-    }
-    int CL = 1;
-    while (CL * 2 <= 16 && CL * 2 <= E) CL <<= 1;
-    pl.CL = CL;
-    pl.EL = (E + CL - 1) / CL;
-    pl.held_in_smem = 0;
-    pl.smem = smem_layout(E, pl.EL, C, 0).total;
-    return pl;
+// fringe capacity: as many worst keys per expert as fit next to everything
+// else in 200 KB of shared memory (at most 32, at least 2)
+static int fringe_capacity(int E, int NM) {
+    for (int fk = 32; fk >= 2; fk >>= 1)
+        if (smem_layout(E, fk, NM).total <= 200 * 1024) return fk;
+    return 0;
 }
 
 }  // namespace auction
 
-// Workspace carve-up shared with the API layer.
 size_t auction_workspace_bytes(int T, int E) {
     const int C = T / E;
-    size_t b = 256;                                   // minmax
-    b += 2 * align_up(sizeof(int32_t) * (size_t)T, 256);  // lists
-    b += align_up(sizeof(int64_t) * (size_t)E * T, 256);  // overflow bids
-    b += align_up(sizeof(int32_t) * (size_t)E * T, 256);  // overflow tokens
-    b += align_up(sizeof(int64_t) * (size_t)E * C, 256);  // held (global fallback)
-    b += align_up(sizeof(int32_t) * (size_t)E * C, 256);
-    b += align_up(sizeof(int32_t) * (size_t)E * C, 256);  // free slots
+    size_t b = 256;                                         // minmax
+    b += align_up(sizeof(auction::Ctrl), 256);
+    b += align_up(64, 256);                                 // objective + counters
+    b += align_up(sizeof(int64_t) * (size_t)E, 256);        // prices
+    b += align_up(sizeof(int32_t) * (size_t)E, 256);        // held counts
+    b += align_up(sizeof(int32_t) * (size_t)E, 256);        // bucket counts
+    b += align_up(sizeof(int64_t) * (size_t)E * C, 256);    // held bids
+    b += align_up(sizeof(int32_t) * (size_t)E * C, 256);    // held tokens
+    b += align_up(sizeof(int64_t) * (size_t)E * T, 256);    // bucket bids
+    b += align_up(sizeof(int32_t) * (size_t)E * T, 256);    // bucket tokens
+    b += 2 * align_up(sizeof(int32_t) * (size_t)T, 256);    // lists
+    b += align_up(sizeof(int32_t) * (size_t)E * C, 256);    // free slots
     return b;
 }
 
 int launch_auction(const int32_t* q, int T, int E, int32_t* assign, int64_t* price,
                    base_auction_stats* stats, void* ws, size_t ws_bytes, long long max_rounds,
-                   cudaStream_t stream) {
+                   int32_t* u_trace, int64_t* t_trace, long long trace_cap, cudaStream_t stream) {
     using namespace auction;
     if (ws_bytes < auction_workspace_bytes(T, E)) return BASE_ERR_WORKSPACE;
     const int C = T / E;
-    Plan pl = make_plan(T, E);
+    const int NM = kNarrowMax;
+    const int FK = fringe_capacity(E, NM);
+    if (FK == 0) return BASE_ERR_UNSUPPORTED;
+    const size_t smem = smem_layout(E, FK, NM).total;
 
     unsigned char* w = static_cast<unsigned char*>(ws);
+    size_t o = 0;
+    auto take = [&](size_t bytes) { unsigned char* r = w + o; o += align_up(bytes, 256); return r; };
     Params prm{};
     prm.q = q;
     prm.T = T;
     prm.E = E;
     prm.C = C;
+    prm.FK = FK;
     prm.max_rounds = max_rounds;
+    prm.narrow_max = NM;
     prm.assign = assign;
     prm.price_out = price;
     prm.stats = stats;
-    size_t o = 0;
-    int32_t* mm = reinterpret_cast<int32_t*>(w + o); o += 256;
+    prm.u_trace = u_trace;
+    prm.t_trace = t_trace;
+    prm.trace_cap = (u_trace || t_trace) ? trace_cap : 0;
+    int32_t* mm = reinterpret_cast<int32_t*>(take(256));
     prm.minmax = mm;
-    prm.ulist0 = reinterpret_cast<int32_t*>(w + o); o += align_up(sizeof(int32_t) * (size_t)T, 256);
-    prm.ulist1 = reinterpret_cast<int32_t*>(w + o); o += align_up(sizeof(int32_t) * (size_t)T, 256);
-    prm.gb_bid = reinterpret_cast<int64_t*>(w + o); o += align_up(sizeof(int64_t) * (size_t)E * T, 256);
-    prm.gb_tok = reinterpret_cast<int32_t*>(w + o); o += align_up(sizeof(int32_t) * (size_t)E * T, 256);
-    prm.gh_bid = reinterpret_cast<int64_t*>(w + o); o += align_up(sizeof(int64_t) * (size_t)E * C, 256);
-    prm.gh_tok = reinterpret_cast<int32_t*>(w + o); o += align_up(sizeof(int32_t) * (size_t)E * C, 256);
-    prm.gfree = reinterpret_cast<int32_t*>(w + o); o += align_up(sizeof(int32_t) * (size_t)E * C, 256);
+    unsigned char* zero_begin = w + o;
+    prm.ctrl = reinterpret_cast<Ctrl*>(take(sizeof(Ctrl)));
+    prm.obj = reinterpret_cast<unsigned long long*>(take(64));
+    prm.gprice = reinterpret_cast<int64_t*>(take(sizeof(int64_t) * (size_t)E));
+    prm.hcnt = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * (size_t)E));
+    prm.bcnt = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * (size_t)E));
+    const size_t zero_bytes = (size_t)((w + o) - zero_begin);
+    prm.hb = reinterpret_cast<int64_t*>(take(sizeof(int64_t) * (size_t)E * C));
+    prm.ht = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * (size_t)E * C));
+    prm.bb = reinterpret_cast<int64_t*>(take(sizeof(int64_t) * (size_t)E * T));
+    prm.bt = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * (size_t)E * T));
+    prm.ulist0 = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * (size_t)T));
+    prm.ulist1 = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * (size_t)T));
+    prm.gfree = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * (size_t)E * C));
 
+    // control block, objective, prices (start at 0), counts
+    if (cudaMemsetAsync(zero_begin, 0, zero_bytes, stream) != cudaSuccess) return BASE_ERR_CUDA;
     minmax_init<<<1, 1, 0, stream>>>(mm);
     BASE_RETURN_IF_LAUNCH_FAILED();
     const size_t n = (size_t)T * E;
-    int blocks = (int)std::min<size_t>((n / 4 + 255) / 256 + 1, 148 * 8);
+    const int blocks = (int)std::min<size_t>((n / 4 + 255) / 256 + 1, 148 * 8);
     minmax_kernel<<<blocks, 256, 0, stream>>>(q, n, mm);
     BASE_RETURN_IF_LAUNCH_FAILED();
 
-    cudaLaunchAttribute attr[1];
-    cudaLaunchConfig_t cfg = {};
-    for (int attempt = 0; attempt < 2; ++attempt) {
-        prm.CL = pl.CL;
-        prm.EL = pl.EL;
-        prm.held_in_smem = pl.held_in_smem;
-        if (cudaFuncSetAttribute(auction_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)pl.smem) != cudaSuccess)
-            return BASE_ERR_CUDA;
-        if (pl.CL > 8 && cudaFuncSetAttribute(auction_kernel,
-                                              cudaFuncAttributeNonPortableClusterSizeAllowed,
-                                              1) != cudaSuccess)
-            return BASE_ERR_CUDA;
-        cfg.gridDim = dim3(pl.CL, 1, 1);
-        cfg.blockDim = dim3(kThreads, 1, 1);
-        cfg.dynamicSmemBytes = pl.smem;
-        cfg.stream = stream;
-        attr[0].id = cudaLaunchAttributeClusterDimension;
-        attr[0].val.clusterDim.x = pl.CL;
-        attr[0].val.clusterDim.y = 1;
-        attr[0].val.clusterDim.z = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
-        int nclusters = 0;
-        cudaError_t oe = cudaOccupancyMaxActiveClusters(&nclusters, auction_kernel, &cfg);
-        if (oe == cudaSuccess && nclusters > 0) break;
-        cudaGetLastError();
-        if (attempt == 1 || pl.CL <= 8) return BASE_ERR_UNSUPPORTED;
-        // 16-CTA clusters unavailable: 8 CTAs with the held sets in global memory
-        pl.CL = 8;
-        pl.EL = (E + 7) / 8;
-        pl.held_in_smem = 0;
-        pl.smem = smem_layout(E, pl.EL, C, 0).total;
-    }
-    if (cudaLaunchKernelEx(&cfg, auction_kernel, prm) != cudaSuccess) return BASE_ERR_CUDA;
+    if (cudaFuncSetAttribute(auction_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem) != cudaSuccess)
+        return BASE_ERR_CUDA;
+    int dev = 0, nsm = 0, per_sm = 0;
+    cudaGetDevice(&dev);
+    if (cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return BASE_ERR_CUDA;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, auction_kernel, kThreads, smem) !=
+            cudaSuccess ||
+        per_sm < 1)
+        return BASE_ERR_UNSUPPORTED;
+    const int grid = nsm;  // one CTA per SM, all co-resident
+    void* args[] = {&prm};
+    if (cudaLaunchCooperativeKernel(reinterpret_cast<void*>(auction_kernel), dim3(grid),
+                                    dim3(kThreads), args, smem, stream) != cudaSuccess)
+        return BASE_ERR_CUDA;
     return BASE_OK;
 }
 

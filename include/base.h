@@ -156,21 +156,27 @@ int base_assign_greedy(const int32_t* q, int T, int E, int32_t* assign, int32_t*
  *   assign: T int32 output.  price: E int64 output (final prices).
  *   stats (nullable): device base_auction_stats.
  *   ws: workspace of at least base_workspace_size(T, E, 0, 0) bytes.
- * Runs on one thread-block cluster (up to 16 CTAs) with the experts' held
- * bids in distributed shared memory.
+ * Runs as one cooperative grid of one 1024-thread CTA per SM: rounds with
+ * many bidders use every SM, the tail of each phase runs on one CTA with the
+ * prices and each expert's worst held bids in shared memory.
  */
 int base_assign_balanced(const int32_t* q, int T, int E, int32_t* assign, int64_t* price,
                          base_auction_stats* stats, void* ws, size_t ws_bytes,
                          cudaStream_t stream);
 
 /*
- * base_assign_balanced with the round cap lowered to max_rounds (1 ..
- * BASE_AUCTION_MAX_ROUNDS): when the cap is reached stats->status becomes
- * BASE_ERR_NOT_CONVERGED and assign / price hold the unfinished state.
+ * base_assign_balanced with two extras for tests and profiling:
+ *   max_rounds (1 .. BASE_AUCTION_MAX_ROUNDS) lowers the round cap; when the
+ *     cap is reached stats->status becomes BASE_ERR_NOT_CONVERGED and
+ *     assign / price are not meaningful;
+ *   u_trace (nullable, device int32[trace_cap]) receives the number of
+ *     bidders of round r, and t_trace (nullable, device int64[trace_cap]) the
+ *     GPU global timer (ns) at the start of round r, for r < trace_cap.
  */
-int base_assign_balanced_capped(const int32_t* q, int T, int E, int32_t* assign, int64_t* price,
-                                base_auction_stats* stats, void* ws, size_t ws_bytes,
-                                long long max_rounds, cudaStream_t stream);
+int base_assign_balanced_ex(const int32_t* q, int T, int E, int32_t* assign, int64_t* price,
+                            base_auction_stats* stats, long long max_rounds, int32_t* u_trace,
+                            int64_t* t_trace, long long trace_cap, void* ws, size_t ws_bytes,
+                            cudaStream_t stream);
 
 /*
  * a5: permutation into expert-contiguous slots (fig. 2 sort_by_expert).

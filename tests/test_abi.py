@@ -74,8 +74,9 @@ def test_bad_arguments_are_rejected_on_the_host(L):
     assert L.base_expert_ffn(p, p, 64, 12, 32, 4, p, p, 0, p, p, p, None, None, ws, 1 << 20, None) == 1
     # combine: misaligned output
     assert L.base_combine(p, p, 64, 16, odd, None) == 1
-    # capped auction: cap out of range
-    assert L.base_assign_balanced_capped(p, 64, 8, p, p, None, ws, 1 << 30, 0, None) == 1
+    # extended auction: cap out of range, trace without a capacity
+    assert L.base_assign_balanced_ex(p, 64, 8, p, p, None, 0, None, None, 0, ws, 1 << 30, None) == 1
+    assert L.base_assign_balanced_ex(p, 64, 8, p, p, None, 10, p, None, 0, ws, 1 << 30, None) == 1
 
 
 def test_spec_constants_agree_between_library_and_oracle():

@@ -19,19 +19,23 @@ def no_device_error():
     assert B.base_device_error(clear=True) == 0
 
 
-def gpu_auction(q_np, max_rounds=None):
+def gpu_auction(q_np, max_rounds=None, trace=False):
     T, E = q_np.shape
     q = dev(q_np)
     assign = torch.full((T,), -1, dtype=torch.int32, device="cuda")
     price = torch.zeros(E, dtype=torch.int64, device="cuda")
     st = buffers.stats()
     ws = buffers.workspace(T, E)
-    if max_rounds is None:
+    u = torch.full((200000,), -1, dtype=torch.int32, device="cuda") if trace else None
+    if max_rounds is None and not trace:
         B.base_assign_balanced(q, assign, price, st, ws)
     else:
-        B.base_assign_balanced_capped(q, assign, price, st, ws, max_rounds)
+        B.base_assign_balanced_ex(q, assign, price, st, ws, max_rounds or 1000000, u_trace=u)
     torch.cuda.synchronize()
-    return to_np(assign), to_np(price), buffers.stats_dict(st)
+    out = (to_np(assign), to_np(price), buffers.stats_dict(st))
+    if trace:
+        out = out + (to_np(u)[: out[2]["rounds"]],)
+    return out
 
 
 def oracle_q(orc, wl, seed=0):
@@ -166,6 +170,16 @@ def test_auction_many_tiny_problems(orc):
 def test_auction_full_workloads(orc, name):
     _, _, q = oracle_q(orc, synth.WORKLOADS[name])
     _check_auction(orc, q)
+
+
+@pytest.mark.parametrize("name", ["routing_ref", "layer_fwd", "skewed"])
+def test_auction_trajectory_matches_round_by_round(orc, name):
+    # the number of bidders of every round, not only the totals
+    _, _, q = oracle_q(orc, synth.WORKLOADS[name])
+    a, p, st, u = gpu_auction(q, trace=True)
+    ao, po, so, uo = orc.auction(q, trace=True)
+    assert st == so
+    assert np.array_equal(u, uo)
 
 
 def test_auction_equal_scores_single_phase(orc):
