@@ -24,8 +24,8 @@
 //     end: prices live in shared memory, and for every full expert CTA 0 keeps
 //     a "fringe" -- its FK worst held bids, sorted -- so a round resolves with
 //     a warp-wide bitonic merge of fringe and new bids instead of a scan of
-//     the expert's C held bids.  Rejected tokens' score rows are prefetched
-//     into L1 for their next bid.
+//     the expert's C held bids.  Rejected tokens' score rows are copied into
+//     shared memory (cp.async) for their next bid.
 // Held sets live in global memory (they are touched only when a fringe is
 // rebuilt).  Every wait is bounded; a wait that gives up records an error
 // and all CTAs leave.
@@ -41,7 +41,7 @@ constexpr int kWarps = kThreads / kWarp;
 constexpr int kHist = 256;
 constexpr int kEpsDivisor = 50;  // eps0 = (max q - min q)(T+1) / 50
 constexpr int kEpsFactor = 8;    // eps <- eps / 8 per phase
-constexpr int kNarrowMax = 1024; // rounds with at most this many bidders run on CTA 0
+constexpr int kNarrowMax = 256;  // rounds with at most this many bidders run on CTA 0
 constexpr uint64_t kWaitNs = 20000000000ull;  // grid-barrier wait limit (20 s)
 
 // ---------------------------------------------------------------- keys
@@ -162,7 +162,7 @@ template <int TEAM>
 struct Team {
     int32_t* hist;     // [kHist]
     int64_t* red;      // [32] (CTA team only)
-    int32_t* cnt;      // [33] (CTA team only)
+    int32_t* cnt;      // [64] (CTA team only): warp counts, totals, results
     __device__ __forceinline__ int tid() const { return TEAM == 32 ? lane_id() : (int)threadIdx.x; }
     __device__ __forceinline__ void sync() const {
         if (TEAM == 32) __syncwarp(); else __syncthreads();
@@ -211,6 +211,69 @@ struct Team {
         const Key r = sk[0];
         __syncthreads();
         return r;
+    }
+    // Finds the bin d of the histogram (nbins <= kHist) where the running
+    // count reaches `need`: before = count of bins < d, cnt = count of bin d.
+    __device__ void find_digit(int nbins, int need, int& d, int& before, int& count) const {
+        if (TEAM == 32) {
+            const int lane = lane_id();
+            int c8[8];
+            int sum = 0;
+#pragma unroll
+            for (int b = 0; b < 8; ++b) {
+                const int bin = lane * 8 + b;
+                c8[b] = bin < nbins ? hist[bin] : 0;
+                sum += c8[b];
+            }
+            int incl = sum;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const int o = __shfl_up_sync(0xffffffffu, incl, off);
+                if (lane >= off) incl += o;
+            }
+            int run = incl - sum, fd = -1, fb = 0, fc = 0;
+#pragma unroll
+            for (int b = 0; b < 8; ++b) {
+                if (fd < 0 && run < need && run + c8[b] >= need) {
+                    fd = lane * 8 + b;
+                    fb = run;
+                    fc = c8[b];
+                }
+                run += c8[b];
+            }
+            const unsigned m = __ballot_sync(0xffffffffu, fd >= 0);
+            const int src = __ffs(m) - 1;
+            d = __shfl_sync(0xffffffffu, fd, src);
+            before = __shfl_sync(0xffffffffu, fb, src);
+            count = __shfl_sync(0xffffffffu, fc, src);
+            __syncwarp();
+            return;
+        }
+        // CTA: threads 0..255 own one bin each; block scan over 8 warps
+        const int t = threadIdx.x;
+        const int c = (t < nbins) ? hist[t] : 0;
+        int incl = c;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int o = __shfl_up_sync(0xffffffffu, incl, off);
+            if (lane_id() >= off) incl += o;
+        }
+        if (t < kHist && lane_id() == 31) cnt[34 + warp_id()] = incl;  // 8 warp totals
+        __syncthreads();
+        int wbase = 0;
+        if (t < kHist)
+            for (int w = 0; w < warp_id(); ++w) wbase += cnt[34 + w];
+        const int excl = wbase + incl - c;
+        if (t < nbins && excl < need && excl + c >= need) {
+            cnt[42] = t;
+            cnt[43] = excl;
+            cnt[44] = c;
+        }
+        __syncthreads();
+        d = cnt[42];
+        before = cnt[43];
+        count = cnt[44];
+        __syncthreads();
     }
     // rank of this thread among the threads with `flag`, in thread order; total
     __device__ int rank(bool flag, int& total) const {
@@ -308,20 +371,7 @@ __device__ Key kth_worst(const Team<TEAM>& tm, const Cands& cd, int k, int tm_tm
         tm.sync();
         // find the digit whose bucket holds the need-th element
         int d = 0, before = 0, cnt = 0;
-        {
-            int run = 0;
-            for (int b = 0; b < (1 << width); ++b) {  // every thread scans (<= 256 smem reads)
-                const int c = tm.hist[b];
-                if (run + c >= need) {
-                    d = b;
-                    before = run;
-                    cnt = c;
-                    break;
-                }
-                run += c;
-            }
-        }
-        tm.sync();
+        tm.find_digit(1 << width, need, d, before, cnt);
         prefix = (prefix << width) | (uint64_t)d;
         pbits += width;
         need -= before;
@@ -363,20 +413,7 @@ __device__ Key kth_worst(const Team<TEAM>& tm, const Cands& cd, int k, int tm_tm
         }
         tm.sync();
         int d = 0, before = 0, cnt = 0;
-        {
-            int run = 0;
-            for (int b = 0; b < (1 << width); ++b) {
-                const int c = tm.hist[b];
-                if (run + c >= tneed) {
-                    d = b;
-                    before = run;
-                    cnt = c;
-                    break;
-                }
-                run += c;
-            }
-        }
-        tm.sync();
+        tm.find_digit(1 << width, tneed, d, before, cnt);
         tprefix = (tprefix << width) | (uint32_t)d;
         tp += width;
         tneed -= before;
@@ -404,7 +441,7 @@ struct Ctrl {
 
 struct Params {
     const int32_t* q;
-    int T, E, C, FK;
+    int T, E, C, FK, NB, RC;
     long long max_rounds;
     int narrow_max;
     int32_t* assign;
@@ -422,6 +459,8 @@ struct Params {
     int32_t* ulist0;   // [T]
     int32_t* ulist1;
     int32_t* gfree;    // [E][C]
+    Key* gfr;          // [E][FK] fringes built by the wide rounds
+    int32_t* gfs;      // [E] their sizes (-1: none)
     unsigned long long* obj;  // [1]
     int32_t* u_trace;  // nullable: bidders of round r
     int64_t* t_trace;  // nullable: globaltimer (ns) at the start of round r
@@ -439,11 +478,13 @@ __device__ __forceinline__ void trace_round(const Params& p, long long r, int U)
 
 // shared memory of every CTA (narrow-mode arrays are used by CTA 0 only)
 struct SmemLayout {
-    size_t price, fr, fsize, hcnt, ncnt, noff, nfill, active, rec_e, rec_b, rec_t, grp_b, grp_t,
-        list0, list1, hist, red, cnt, misc, total;
+    size_t price, fr, fsize, hcnt, ncnt, act0, act1, nbk_b, nbk_t, list0, list1, rows, hist, red,
+        cnt, misc, total;
 };
 
-__host__ __device__ inline SmemLayout smem_layout(int E, int FK, int NM) {
+// NB: new bids per expert kept in shared memory (the rest in the global
+// bucket); RC: bidders' score rows staged in shared memory per round parity.
+__host__ __device__ inline SmemLayout smem_layout(int E, int FK, int NM, int NB, int RC) {
     SmemLayout L;
     size_t o = 0;
     auto take = [&](size_t bytes) { size_t r = o; o += align_up(bytes, 16); return r; };
@@ -452,16 +493,13 @@ __host__ __device__ inline SmemLayout smem_layout(int E, int FK, int NM) {
     L.fsize = take(4 * (size_t)E);
     L.hcnt = take(4 * (size_t)E);
     L.ncnt = take(4 * (size_t)E);
-    L.noff = take(4 * (size_t)E);
-    L.nfill = take(4 * (size_t)E);
-    L.active = take(4 * (size_t)E);
-    L.rec_e = take(4 * (size_t)NM);
-    L.rec_b = take(8 * (size_t)NM);
-    L.rec_t = take(4 * (size_t)NM);
-    L.grp_b = take(8 * (size_t)NM);
-    L.grp_t = take(4 * (size_t)NM);
+    L.act0 = take(4 * (size_t)E);
+    L.act1 = take(4 * (size_t)E);
+    L.nbk_b = take(8 * (size_t)E * NB);
+    L.nbk_t = take(4 * (size_t)E * NB);
     L.list0 = take(4 * (size_t)NM);
     L.list1 = take(4 * (size_t)NM);
+    L.rows = take(2 * 4 * (size_t)RC * E);
     L.hist = take(4 * (size_t)kWarps * kHist);
     L.red = take(8 * 32);
     L.cnt = take(4 * 64);
@@ -520,15 +558,16 @@ __device__ bool grid_sync(Ctrl* c, int* s_flag) {
     return *s_flag != 0;
 }
 
-// best / second-best scan of one token's row by a group of G lanes
-__device__ __forceinline__ void group_bid(const int32_t* __restrict__ row, const int64_t* price,
-                                          int E, int G, int gl, int64_t scale, int64_t& v1,
-                                          int64_t& v2, int& e1) {
+// best / second-best scan of one token's row by a group of G lanes (the row
+// may be in global memory or staged in shared memory: generic loads)
+__device__ __forceinline__ void group_bid(const int32_t* row, const int64_t* price, int E, int G,
+                                          int gl, int64_t scale, int64_t& v1, int64_t& v2,
+                                          int& e1) {
     v1 = INT64_MIN;
     v2 = INT64_MIN;
     e1 = INT32_MAX;
     for (int e = gl; e < E; e += G) {
-        const int64_t v = (int64_t)__ldg(row + e) * scale - price[e];
+        const int64_t v = (int64_t)row[e] * scale - price[e];
         if (v > v1) {
             v2 = v1;
             v1 = v;
@@ -553,10 +592,72 @@ __device__ __forceinline__ void group_bid(const int32_t* __restrict__ row, const
     }
 }
 
-__device__ __forceinline__ void prefetch_row_l1(const int32_t* row, int E) {
-    for (int off = 0; off < E * 4; off += 128)
-        asm volatile("prefetch.global.L1 [%0];" ::"l"(reinterpret_cast<const char*>(row) + off));
+// The same for NT tokens at once (their loads in flight together).
+template <int NT>
+__device__ __forceinline__ void group_bid_multi(const int32_t* __restrict__ q, const int (&t)[NT],
+                                                const bool (&valid)[NT], const int64_t* price,
+                                                int E, int G, int gl, int64_t scale,
+                                                int64_t (&v1)[NT], int64_t (&v2)[NT],
+                                                int (&e1)[NT]) {
+#pragma unroll
+    for (int u = 0; u < NT; ++u) {
+        v1[u] = INT64_MIN;
+        v2[u] = INT64_MIN;
+        e1[u] = INT32_MAX;
+    }
+#pragma unroll 2
+    for (int e = gl; e < E; e += G) {
+        int32_t qv[NT];
+#pragma unroll
+        for (int u = 0; u < NT; ++u) qv[u] = valid[u] ? __ldg(q + (size_t)t[u] * E + e) : 0;
+        const int64_t pe = price[e];
+#pragma unroll
+        for (int u = 0; u < NT; ++u) {
+            if (!valid[u]) continue;
+            const int64_t v = (int64_t)qv[u] * scale - pe;
+            if (v > v1[u]) {
+                v2[u] = v1[u];
+                v1[u] = v;
+                e1[u] = e;
+            } else if (v > v2[u]) {
+                v2[u] = v;
+            }
+        }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+        if (off >= G) continue;
+#pragma unroll
+        for (int u = 0; u < NT; ++u) {
+            const int64_t ov1 = __shfl_xor_sync(0xffffffffu, v1[u], off);
+            const int64_t ov2 = __shfl_xor_sync(0xffffffffu, v2[u], off);
+            const int oe1 = __shfl_xor_sync(0xffffffffu, e1[u], off);
+            if (ov1 > v1[u] || (ov1 == v1[u] && oe1 < e1[u])) {
+                v2[u] = max(v1[u], ov2);
+                v1[u] = ov1;
+                e1[u] = oe1;
+            } else {
+                v2[u] = max(v2[u], ov1);
+            }
+        }
+    }
 }
+
+// Where the score rows of the next round's bidders go: list position pos <
+// cap is copied into rows[pos] (E int32, 16-byte chunks, cp.async by the
+// pushing lane); rows == nullptr: no staging (wide rounds).
+struct RowStage {
+    int32_t* rows;
+    int cap;
+    __device__ __forceinline__ void stage(const int32_t* q, int E, int tok, int pos) const {
+        if (rows == nullptr || pos >= cap) return;
+        const char* src = reinterpret_cast<const char*>(q + (size_t)tok * E);
+        const uint32_t dst = smem_u32(rows + (size_t)pos * E);
+        for (int off = 0; off < E * 4; off += 16)
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst + off), "l"(src + off)
+                         : "memory");
+    }
+};
 
 // Keeps the C best of held + new for expert e (held in global memory), with
 // a team of TEAM threads.  Rejected tokens are appended to `unext` through
@@ -565,7 +666,7 @@ __device__ __forceinline__ void prefetch_row_l1(const int32_t* row, int E) {
 template <int TEAM>
 __device__ int resolve_general(const Team<TEAM>& tm, const Params& p, int e, const Cands& cd,
                                int64_t* hb, int32_t* ht, int32_t* unext, int32_t* ucnt,
-                               int64_t& price, bool prefetch) {
+                               int64_t& price, const RowStage& rs) {
     const int C = p.C, h = cd.h, n = cd.n;
     const int tid = tm.tid();
     if (h + n <= C) {
@@ -619,7 +720,7 @@ __device__ int resolve_general(const Team<TEAM>& tm, const Params& p, int e, con
         }
         if (rej) {
             unext[base + rr] = tok;
-            if (prefetch) prefetch_row_l1(p.q + (size_t)tok * p.E, p.E);
+            rs.stage(p.q, p.E, tok, base + rr);
         }
         int tot = 0;
         const int r = tm.rank(isfree, tot);
@@ -654,7 +755,7 @@ __device__ int resolve_general(const Team<TEAM>& tm, const Params& p, int e, con
         }
         if (rej) {
             unext[base + rr] = x.tok;
-            if (prefetch) prefetch_row_l1(p.q + (size_t)x.tok * p.E, p.E);
+            rs.stage(p.q, p.E, x.tok, base + rr);
         }
         int tot = 0;
         const int r = tm.rank(acc, tot);
@@ -674,113 +775,179 @@ __device__ int resolve_general(const Team<TEAM>& tm, const Params& p, int e, con
     return C;
 }
 
-// Rebuilds the fringe of a full expert: its FK worst held keys, sorted, from
-// a warp-wide scan of the C held bids (chunks of 32 merged into the running
-// 32 lowest).  Returns the fringe size.
-__device__ int rebuild_fringe(const int64_t* hb, const int32_t* ht, int C, int FK, Key* fr) {
-    const int lane = lane_id();
-    Key best = pad_key();
-    for (int b0 = 0; b0 < C; b0 += 32) {
-        const int i = b0 + lane;
+// Builds the fringe of an expert holding C keys: its min(FK, C) worst held
+// keys, sorted ascending, found as the FK-th worst key by a radix select,
+// collected with a team-wide ranking and sorted by warp 0.  Returns the
+// fringe size.
+template <int TEAM>
+__device__ int build_fringe(const Team<TEAM>& tm, const int64_t* hb, const int32_t* ht, int C,
+                            int FK, int tmax, Key* fr) {
+    const int k = min(FK, C);
+    if (k == 0) return 0;
+    const Cands cd{hb, ht, nullptr, nullptr, C, 0};
+    const Key kth = kth_worst<TEAM>(tm, cd, k, tmax);
+    Key* stage = reinterpret_cast<Key*>(tm.hist);  // 64 keys fit in the histogram area
+    int got = 0;
+    for (int b0 = 0; b0 < C; b0 += TEAM) {
+        const int i = b0 + tm.tid();
         Key x = pad_key();
-        if (i < C) x = Key{hb[i], ht[i], i};
-        x = warp_sort(x);
-        Key lo, hi;
-        warp_merge64(best, x, lo, hi);
-        best = lo;
+        bool in = false;
+        if (i < C) {
+            x = Key{hb[i], ht[i], i};
+            in = !worse(kth, x);
+        }
+        int tot = 0;
+        const int r = tm.rank(in, tot);
+        if (in) stage[got + r] = x;
+        got += tot;
     }
-    const int fs = min(FK, C);
-    if (lane < fs) fr[lane] = best;
-    __syncwarp();
-    return fs;
+    tm.sync();
+    if (TEAM == 32 || warp_id() == 0) {
+        Key x = lane_id() < k ? stage[lane_id()] : pad_key();
+        x = warp_sort(x);
+        if (lane_id() < k) fr[lane_id()] = x;
+    }
+    tm.sync();
+    return k;
 }
 
-// Fast narrow-mode resolve of a full expert whose fringe is valid and holds
-// at least n + 1 keys (n < 32 new bids, as many rejections): the sorted new
-// bids are merged with the sorted fringe; the n worst of the 64 are rejected,
-// accepted new bids take the slots the rejected fringe keys free, and the
-// survivors not above the old fringe maximum form the new fringe.  Sets fs to
-// the new fringe size (0: the caller rebuilds it) and price to its minimum.
 __device__ __forceinline__ int nth_set_lane(unsigned m, int r) {
     for (int i = 0; i < r; ++i) m &= m - 1;
     return m ? __ffs(m) - 1 : 0;
 }
 
-__device__ void resolve_fringe(const Params& p, Key* fr, int& fs, const int64_t* nb,
-                               const int32_t* nt, int n, int64_t* hb, int32_t* ht,
-                               int32_t* next_list, int* next_cnt, int64_t& price) {
+// Warp-level resolve of one expert from its fringe and n < 32 new bids.
+// The fringe holds the expert's fs worst held keys, sorted ascending; it is
+// "complete" when it holds all h of them.  The k = max(0, h + n - C) worst of
+// held + new are among fringe + new whenever the fringe is complete or k < fs,
+// so the sorted merge of the two lists decides the round: its first k keys
+// are rejected, accepted new keys take the slots of rejected fringe keys and
+// then the empty slots h, h+1, ..; the survivors not above the old fringe
+// maximum (all survivors when complete) form the new fringe.  Returns false
+// (nothing changed) when the fringe cannot decide; sets price when the expert
+// is full and its new fringe is not empty (fs == 0 afterwards: rebuild).
+__device__ bool resolve_warp(const Params& p, Key* fr, int& fs, int& h, const int64_t* nb,
+                             const int32_t* nt, int n, int64_t* hb, int32_t* ht,
+                             int32_t* next_list, int* next_cnt, int64_t& price,
+                             const RowStage& rs) {
+    const int C = p.C, FK = p.FK;
     const int lane = lane_id();
     const unsigned lt = (1u << lane) - 1;
-    const int k = n;
+    const bool complete = (fs == h);
+    const int k = max(0, h + n - C);
+    if (!complete && k >= fs) return false;
+    if (n == 1 && h == C && fs >= 2) {
+        // one bid b to a full expert: b beats the price (the fringe minimum
+        // f0), so f0 is rejected and b takes its slot; the new fringe is
+        // f1.. with b inserted where it belongs (when not above the maximum)
+        const Key b0 = Key{nb[0], nt[0], -1};
+        const Key fi = lane < fs ? fr[lane] : pad_key();
+        const Key fn = lane + 1 < fs ? fr[lane + 1] : pad_key();
+        const Key f0 = shfl_key(fi, 0);
+        const Key b = Key{b0.bid, b0.tok, f0.slot};
+        const bool ins = complete || !worse(shfl_key(fi, fs - 1), b);
+        const int pos = __popc(__ballot_sync(0xffffffffu, lane + 1 < fs && worse(fn, b)));
+        Key out = lane < pos ? fn : (lane == pos ? b : fi);
+        if (!ins) out = fn;
+        const int nfs = ins ? fs : fs - 1;
+        if (lane == 0) {
+            hb[b.slot] = b.bid;
+            ht[b.slot] = b.tok;
+            const int at = atomicAdd(next_cnt, 1);
+            next_list[at] = f0.tok;
+            rs.stage(p.q, p.E, f0.tok, at);
+        }
+        __syncwarp();
+        if (lane < nfs) fr[lane] = out;
+        __syncwarp();
+        fs = nfs;
+        price = shfl_key(out, 0).bid;
+        return true;
+    }
     const Key f = lane < fs ? fr[lane] : pad_key();
-    const Key fmax = shfl_key(f, fs - 1);
-    Key x = lane < n ? Key{nb[lane], nt[lane], -1} : pad_key();
-    x = warp_sort(x);
+    const Key thr = complete ? pad_key() : shfl_key(f, max(fs, 1) - 1);
     Key lo, hi;
-    warp_merge64(f, x, lo, hi);
-    const bool rej = lane < k;  // elements 0 .. k-1 (all in lo since k < 32)
+    if (n == 1) {
+        // one new key: insert it into the sorted fringe
+        const Key b = Key{nb[0], nt[0], -1};
+        const int pos = __popc(__ballot_sync(0xffffffffu, lane < fs && worse(f, b)));
+        const Key prev = shfl_key(f, (lane + 31) & 31);
+        const Key top = shfl_key(f, 31);
+        lo = lane < pos ? f : (lane == pos ? b : prev);
+        hi = pad_key();
+        if (lane == 0 && fs == 32) hi = (pos == 32) ? b : top;
+    } else {
+        Key x = lane < n ? Key{nb[lane], nt[lane], -1} : pad_key();
+        x = warp_sort(x);
+        warp_merge64(f, x, lo, hi);
+    }
+    const bool rej = lane < k;  // the first k elements (k <= n < 32: all in lo)
     const unsigned freed = __ballot_sync(0xffffffffu, rej && lo.slot >= 0);
+    const int nfreed = __popc(freed);
     const unsigned acc_lo = __ballot_sync(0xffffffffu, !rej && lo.slot == -1);
     const unsigned acc_hi = __ballot_sync(0xffffffffu, hi.slot == -1);
-    // the r-th accepted new key takes the slot of the r-th rejected fringe key
-    const int src_lo = nth_set_lane(freed, __popc(acc_lo & lt));
-    const int src_hi = nth_set_lane(freed, __popc(acc_lo) + __popc(acc_hi & lt));
-    const int slot_lo = __shfl_sync(0xffffffffu, lo.slot, src_lo);
-    const int slot_hi = __shfl_sync(0xffffffffu, lo.slot, src_hi);
+    // the r-th accepted new key takes the r-th freed slot, then h + (r - nfreed)
+    const int r_lo = __popc(acc_lo & lt);
+    const int r_hi = __popc(acc_lo) + __popc(acc_hi & lt);
+    const int s_lo = __shfl_sync(0xffffffffu, lo.slot, nth_set_lane(freed, min(r_lo, 31)));
+    const int s_hi = __shfl_sync(0xffffffffu, lo.slot, nth_set_lane(freed, min(r_hi, 31)));
     if ((acc_lo >> lane) & 1u) {
-        lo.slot = slot_lo;
-        hb[slot_lo] = lo.bid;
-        ht[slot_lo] = lo.tok;
+        lo.slot = r_lo < nfreed ? s_lo : h + (r_lo - nfreed);
+        hb[lo.slot] = lo.bid;
+        ht[lo.slot] = lo.tok;
     }
     if ((acc_hi >> lane) & 1u) {
-        hi.slot = slot_hi;
-        hb[slot_hi] = hi.bid;
-        ht[slot_hi] = hi.tok;
+        hi.slot = r_hi < nfreed ? s_hi : h + (r_hi - nfreed);
+        hb[hi.slot] = hi.bid;
+        ht[hi.slot] = hi.tok;
     }
-    // rejected tokens bid next round: append them and fetch their rows into L1
-    const unsigned rm = __ballot_sync(0xffffffffu, rej);
-    int base = 0;
-    if (lane == 0) base = atomicAdd(next_cnt, __popc(rm));
-    base = __shfl_sync(0xffffffffu, base, 0);
-    if (rej) {
-        next_list[base + __popc(rm & lt)] = lo.tok;
-        prefetch_row_l1(p.q + (size_t)lo.tok * p.E, p.E);
+    if (k > 0) {  // rejected tokens bid next round
+        const unsigned rm = __ballot_sync(0xffffffffu, rej);
+        int base = 0;
+        if (lane == 0) base = atomicAdd(next_cnt, k);
+        base = __shfl_sync(0xffffffffu, base, 0);
+        if (rej) {
+            next_list[base + __popc(rm & lt)] = lo.tok;
+            rs.stage(p.q, p.E, lo.tok, base + __popc(rm & lt));
+        }
     }
-    // the new fringe: surviving keys not above the old fringe maximum, in order
-    const bool keep_lo = !rej && !worse(fmax, lo);
-    const bool keep_hi = hi.slot != -2 && !worse(fmax, hi);
+    // the new fringe: survivors not above the threshold, in order, at most FK
+    const bool keep_lo = !rej && lo.slot != -2 && !worse(thr, lo);
+    const bool keep_hi = hi.slot != -2 && !worse(thr, hi);
     const unsigned kl = __ballot_sync(0xffffffffu, keep_lo);
     const unsigned kh = __ballot_sync(0xffffffffu, keep_hi);
     const int nl = __popc(kl);
     __syncwarp();
-    if (keep_lo) fr[__popc(kl & lt)] = lo;
+    if (keep_lo) {
+        const int pos = __popc(kl & lt);
+        if (pos < FK) fr[pos] = lo;
+    }
     if (keep_hi) {
         const int pos = nl + __popc(kh & lt);
-        if (pos < p.FK) fr[pos] = hi;
+        if (pos < FK) fr[pos] = hi;
     }
     __syncwarp();
-    fs = min(p.FK, nl + __popc(kh));
-    if (fs > 0) price = fr[0].bid;
+    fs = min(FK, nl + __popc(kh));
+    h = min(C, h + n);
+    if (h == C && fs > 0) price = fr[0].bid;
+    return true;
 }
 
 __global__ void __launch_bounds__(kThreads, 1) auction_kernel(const __grid_constant__ Params p) {
     extern __shared__ __align__(16) unsigned char smem[];
-    const SmemLayout L = smem_layout(p.E, p.FK, p.narrow_max);
+    const SmemLayout L = smem_layout(p.E, p.FK, p.narrow_max, p.NB, p.RC);
     int64_t* s_price = reinterpret_cast<int64_t*>(smem + L.price);
     Key* s_fr = reinterpret_cast<Key*>(smem + L.fr);
     int32_t* s_fsize = reinterpret_cast<int32_t*>(smem + L.fsize);
     int32_t* s_hcnt = reinterpret_cast<int32_t*>(smem + L.hcnt);
     int32_t* s_ncnt = reinterpret_cast<int32_t*>(smem + L.ncnt);
-    int32_t* s_noff = reinterpret_cast<int32_t*>(smem + L.noff);
-    int32_t* s_nfill = reinterpret_cast<int32_t*>(smem + L.nfill);
-    int32_t* s_active = reinterpret_cast<int32_t*>(smem + L.active);
-    int32_t* s_rec_e = reinterpret_cast<int32_t*>(smem + L.rec_e);
-    int64_t* s_rec_b = reinterpret_cast<int64_t*>(smem + L.rec_b);
-    int32_t* s_rec_t = reinterpret_cast<int32_t*>(smem + L.rec_t);
-    int64_t* s_grp_b = reinterpret_cast<int64_t*>(smem + L.grp_b);
-    int32_t* s_grp_t = reinterpret_cast<int32_t*>(smem + L.grp_t);
+    int32_t* s_act0 = reinterpret_cast<int32_t*>(smem + L.act0);
+    int32_t* s_act1 = reinterpret_cast<int32_t*>(smem + L.act1);
+    int64_t* s_nbk_b = reinterpret_cast<int64_t*>(smem + L.nbk_b);
+    int32_t* s_nbk_t = reinterpret_cast<int32_t*>(smem + L.nbk_t);
     int32_t* s_list0 = reinterpret_cast<int32_t*>(smem + L.list0);
     int32_t* s_list1 = reinterpret_cast<int32_t*>(smem + L.list1);
+    int32_t* s_rows = reinterpret_cast<int32_t*>(smem + L.rows);
     int32_t* s_hist = reinterpret_cast<int32_t*>(smem + L.hist);
     int64_t* s_red = reinterpret_cast<int64_t*>(smem + L.red);
     int32_t* s_cnt = reinterpret_cast<int32_t*>(smem + L.cnt);
@@ -817,6 +984,7 @@ __global__ void __launch_bounds__(kThreads, 1) auction_kernel(const __grid_const
         for (int e = cta * kThreads + threadIdx.x; e < E; e += ncta * kThreads) {
             p.hcnt[e] = 0;
             p.bcnt[e] = 0;
+            p.gfs[e] = 0;  // empty held set: an empty, complete fringe
         }
         if (cta == 0 && threadIdx.x < 3) p.ctrl->ucount[threadIdx.x] = 0;
         if (!(ok = grid_sync(p.ctrl, s_misc))) break;
@@ -838,21 +1006,33 @@ __global__ void __launch_bounds__(kThreads, 1) auction_kernel(const __grid_const
             for (int e = threadIdx.x; e < E; e += kThreads) s_price[e] = vload(p.gprice + e);
             __syncthreads();
             {
+                // 4 tokens per lane group per step: a group handles tokens
+                // base + sub + k * tpw * nwarps_total, k = 0..3
+                constexpr int NT = 4;
+                const long long nw = (long long)ncta * kWarps;
                 const long long gw = (long long)cta * kWarps + warp;
-                const long long stride = (long long)ncta * kWarps * tpw;
+                const long long stride = nw * tpw * NT;
                 for (long long base = gw * tpw; base < U; base += stride) {
-                    const long long i = base + sub;
-                    const bool valid = i < U;
-                    const int t = valid ? (first ? (int)i : vload(ulist + i)) : 0;
-                    int64_t v1, v2;
-                    int e1;
-                    group_bid(p.q + (size_t)t * E, s_price, valid ? E : 0, G, gl, scale, v1, v2,
-                              e1);
-                    if (valid && gl == 0) {
-                        const int64_t b = v1 + s_price[e1] - v2 + eps;
-                        const int pos = atomicAdd(&p.bcnt[e1], 1);
-                        p.bb[(size_t)e1 * T + pos] = b;
-                        p.bt[(size_t)e1 * T + pos] = t;
+                    int t[NT];
+                    bool valid[NT];
+#pragma unroll
+                    for (int u = 0; u < NT; ++u) {
+                        const long long i = base + sub + (long long)u * nw * tpw;
+                        valid[u] = i < U;
+                        t[u] = valid[u] ? (first ? (int)i : vload(ulist + i)) : 0;
+                    }
+                    int64_t v1[NT], v2[NT];
+                    int e1[NT];
+                    group_bid_multi<NT>(p.q, t, valid, s_price, E, G, gl, scale, v1, v2, e1);
+                    if (gl == 0) {
+#pragma unroll
+                        for (int u = 0; u < NT; ++u) {
+                            if (!valid[u]) continue;
+                            const int64_t b = v1[u] + s_price[e1[u]] - v2[u] + eps;
+                            const int pos = atomicAdd(&p.bcnt[e1[u]], 1);
+                            p.bb[(size_t)e1[u] * T + pos] = b;
+                            p.bt[(size_t)e1[u] * T + pos] = t[u];
+                        }
                     }
                 }
             }
@@ -861,16 +1041,42 @@ __global__ void __launch_bounds__(kThreads, 1) auction_kernel(const __grid_const
                 const int n = vload(p.bcnt + e);
                 if (n == 0) continue;
                 __syncthreads();
-                const int h = vload(p.hcnt + e);
-                Cands cd{p.hb + (size_t)e * C, p.ht + (size_t)e * C, p.bb + (size_t)e * T,
-                         p.bt + (size_t)e * T, h, n};
+                const int h0 = vload(p.hcnt + e);
+                int64_t* hb = p.hb + (size_t)e * C;
+                int32_t* ht = p.ht + (size_t)e * C;
+                Key* gfr = p.gfr + (size_t)e * FK;
+                const int fs0 = vload(p.gfs + e);
+                const bool warp_ok = n < 32 && (fs0 == h0 || max(0, h0 + n - C) < fs0);
+                if (warp_ok) {
+                    // a few bids: merge them with the expert's fringe (warp 0)
+                    if (warp == 0) {
+                        int fs = fs0, h = h0;
+                        int64_t price = INT64_MIN;
+                        resolve_warp(p, gfr, fs, h, p.bb + (size_t)e * T, p.bt + (size_t)e * T, n,
+                                     hb, ht, unext, ucnt, price, RowStage{nullptr, 0});
+                        if (h == C && fs == 0) {
+                            fs = build_fringe<32>(warp_team, hb, ht, C, FK, T - 1, gfr);
+                            price = gfr[0].bid;
+                        }
+                        if (lane == 0) {
+                            p.gfs[e] = fs;
+                            p.hcnt[e] = h;
+                            p.bcnt[e] = 0;
+                            if (h == C) p.gprice[e] = price;
+                        }
+                    }
+                    __syncthreads();
+                    continue;
+                }
+                Cands cd{hb, ht, p.bb + (size_t)e * T, p.bt + (size_t)e * T, h0, n};
                 int64_t price = INT64_MIN;
-                const int nh = resolve_general<1024>(cta_team, p, e, cd, p.hb + (size_t)e * C,
-                                                     p.ht + (size_t)e * C, unext, ucnt, price,
-                                                     false);
+                const int nh = resolve_general<1024>(cta_team, p, e, cd, hb, ht, unext, ucnt,
+                                                     price, RowStage{nullptr, 0});
+                const int fs = build_fringe<1024>(cta_team, hb, ht, nh, FK, T - 1, gfr);
                 if (threadIdx.x == 0) {
                     p.hcnt[e] = nh;
                     p.bcnt[e] = 0;
+                    p.gfs[e] = fs;
                     if (nh == C) p.gprice[e] = price;
                 }
                 __syncthreads();
@@ -886,18 +1092,34 @@ __global__ void __launch_bounds__(kThreads, 1) auction_kernel(const __grid_const
         if (!ok || status != BASE_OK) break;
         if (narrow) {
             // ================= narrow rounds on CTA 0 =================
+            // Two block barriers per round.  A bid goes straight into its
+            // expert's shared-memory bucket (the first NB; the rest to the
+            // global bucket); after the barrier each warp resolves active
+            // experts.  A rejected token's score row is copied into shared
+            // memory (cp.async) for its bid in the next round.  Counters used
+            // across a barrier are double / triple buffered by round parity.
             if (cta == 0) {
                 const int32_t* ulist = cur ? p.ulist1 : p.ulist0;
                 int32_t* lists[2] = {s_list0, s_list1};
+                int32_t* s_act[2] = {s_act0, s_act1};
+                int32_t* s_nact = s_misc + 4;  // [2]
+                int32_t* s_next = s_misc + 8;  // [3]
+                const int NB = p.NB, RC = p.RC;
+                const bool stage_rows = RC > 0 && (E % 4) == 0;
                 int lc = 0;
+                bool staged = false;  // the current list's first RC rows are in s_rows[lc]
                 for (int i = threadIdx.x; i < U; i += kThreads) s_list0[i] = vload(ulist + i);
                 for (int e = threadIdx.x; e < E; e += kThreads) {
                     s_price[e] = vload(p.gprice + e);
                     s_hcnt[e] = vload(p.hcnt + e);
-                    s_fsize[e] = -1;  // fringe not built
+                    s_fsize[e] = vload(p.gfs + e);
                     s_ncnt[e] = 0;
                 }
-                if (threadIdx.x == 0) s_misc[1] = 0;
+                for (int i = threadIdx.x; i < E * FK; i += kThreads) {
+                    const Key* g = p.gfr + i;
+                    s_fr[i] = Key{vload(&g->bid), vload(&g->tok), vload(&g->slot)};
+                }
+                if (threadIdx.x < 5) s_misc[4 + (threadIdx.x < 2 ? threadIdx.x : threadIdx.x + 2)] = 0;
                 __syncthreads();
                 while (U > 0) {
                     if (rounds >= p.max_rounds) {
@@ -907,91 +1129,91 @@ __global__ void __launch_bounds__(kThreads, 1) auction_kernel(const __grid_const
                     if (threadIdx.x == 0) trace_round(p, rounds, U);
                     ++rounds;
                     bids += U;
+                    const int ra = (int)(rounds & 1);
                     int32_t* list = lists[lc];
                     int32_t* next = lists[lc ^ 1];
-                    // bid
+                    int32_t* act = s_act[ra];
+                    const int32_t* rows_cur = s_rows + (size_t)lc * RC * E;
+                    int32_t* rows_next = s_rows + (size_t)(lc ^ 1) * RC * E;
+                    // the counter the next round's resolve writes was last read
+                    // two barriers ago
+                    if (threadIdx.x == 0) s_next[(int)((rounds + 1) % 3)] = 0;
+                    // ---- bid
                     for (int base = warp * tpw; base < U; base += kWarps * tpw) {
                         const int i = base + sub;
                         const bool valid = i < U;
                         const int t = valid ? list[i] : 0;
+                        const int32_t* row = (staged && i < RC) ? rows_cur + (size_t)i * E
+                                                                : p.q + (size_t)t * E;
                         int64_t v1, v2;
                         int e1;
-                        group_bid(p.q + (size_t)t * E, s_price, valid ? E : 0, G, gl, scale, v1,
-                                  v2, e1);
+                        group_bid(row, s_price, valid ? E : 0, G, gl, scale, v1, v2, e1);
                         if (valid && gl == 0) {
-                            s_rec_e[i] = e1;
-                            s_rec_b[i] = v1 + s_price[e1] - v2 + eps;
-                            s_rec_t[i] = t;
-                            if (atomicAdd(&s_ncnt[e1], 1) == 0) {
-                                const int a = atomicAdd(&s_misc[1], 1);
-                                s_active[a] = e1;
+                            const int64_t b = v1 + s_price[e1] - v2 + eps;
+                            const int pos = atomicAdd(&s_ncnt[e1], 1);
+                            if (pos == 0) act[atomicAdd(&s_nact[ra], 1)] = e1;
+                            if (pos < NB) {
+                                s_nbk_b[(size_t)e1 * NB + pos] = b;
+                                s_nbk_t[(size_t)e1 * NB + pos] = t;
+                            } else {
+                                p.bb[(size_t)e1 * T + pos] = b;
+                                p.bt[(size_t)e1 * T + pos] = t;
                             }
                         }
                     }
                     __syncthreads();
-                    const int nact = s_misc[1];
-                    // group the records by expert
-                    if (warp == 0) {
-                        int run = 0;
-                        for (int a0 = 0; a0 < nact; a0 += 32) {
-                            const int a = a0 + lane;
-                            const int c = a < nact ? s_ncnt[s_active[a]] : 0;
-                            int incl = c;
-#pragma unroll
-                            for (int off = 1; off < 32; off <<= 1) {
-                                const int o = __shfl_up_sync(0xffffffffu, incl, off);
-                                if (lane >= off) incl += o;
-                            }
-                            if (a < nact) {
-                                s_noff[s_active[a]] = run + incl - c;
-                                s_nfill[s_active[a]] = 0;
-                            }
-                            run += __shfl_sync(0xffffffffu, incl, 31);
-                        }
-                    }
-                    __syncthreads();
-                    for (int i = threadIdx.x; i < U; i += kThreads) {
-                        const int e = s_rec_e[i];
-                        const int pos = s_noff[e] + atomicAdd(&s_nfill[e], 1);
-                        s_grp_b[pos] = s_rec_b[i];
-                        s_grp_t[pos] = s_rec_t[i];
-                    }
-                    if (threadIdx.x == 0) s_misc[2] = 0;  // next list count
-                    __syncthreads();
-                    // resolve: a warp per active expert
+                    // ---- resolve: a warp per active expert
+                    const int nact = s_nact[ra];
+                    int32_t* ncnt_next = &s_next[(int)(rounds % 3)];
+                    RowStage rs{stage_rows ? rows_next : nullptr, RC};
                     for (int a = warp; a < nact; a += kWarps) {
-                        const int e = s_active[a];
+                        const int e = act[a];
                         const int n = s_ncnt[e];
                         const int h = s_hcnt[e];
-                        const int64_t* nb = s_grp_b + s_noff[e];
-                        const int32_t* nt = s_grp_t + s_noff[e];
                         int64_t* hb = p.hb + (size_t)e * C;
                         int32_t* ht = p.ht + (size_t)e * C;
                         Key* fr = s_fr + (size_t)e * FK;
+                        const int64_t* nb = s_nbk_b + (size_t)e * NB;
+                        const int32_t* nt = s_nbk_t + (size_t)e * NB;
+                        if (n > NB) {
+                            // spilled: move the shared part next to the rest
+                            int64_t* gb = p.bb + (size_t)e * T;
+                            int32_t* gt = p.bt + (size_t)e * T;
+                            for (int j = lane; j < NB; j += 32) {
+                                gb[j] = nb[j];
+                                gt[j] = nt[j];
+                            }
+                            __syncwarp();
+                            nb = gb;
+                            nt = gt;
+                        }
                         int64_t price = s_price[e];
                         bool done = false;
-                        if (h == C && n < 32) {
-                            int fs = s_fsize[e];
-                            if (fs < n + 1) fs = rebuild_fringe(hb, ht, C, FK, fr);
-                            if (fs >= n + 1) {
-                                resolve_fringe(p, fr, fs, nb, nt, n, hb, ht, next, &s_misc[2],
-                                               price);
-                                if (fs == 0) {
-                                    __syncwarp();
-                                    fs = rebuild_fringe(hb, ht, C, FK, fr);
+                        if (n < 32) {
+                            int fs = s_fsize[e], hh = h;
+                            if (fs != hh && max(0, hh + n - C) >= fs)  // depleted: rebuild
+                                fs = build_fringe<32>(warp_team, hb, ht, hh, FK, T - 1, fr);
+                            done = resolve_warp(p, fr, fs, hh, nb, nt, n, hb, ht, next, ncnt_next,
+                                                price, rs);
+                            if (done) {
+                                if (hh == C && fs == 0) {
+                                    fs = build_fringe<32>(warp_team, hb, ht, hh, FK, T - 1, fr);
                                     price = fr[0].bid;
                                 }
-                                done = true;
-                                if (lane == 0) s_fsize[e] = fs;
+                                if (lane == 0) {
+                                    s_fsize[e] = fs;
+                                    s_hcnt[e] = hh;
+                                }
                             }
                         }
                         if (!done) {
                             Cands cd{hb, ht, nb, nt, h, n};
                             const int nh = resolve_general<32>(warp_team, p, e, cd, hb, ht, next,
-                                                               &s_misc[2], price, true);
+                                                               ncnt_next, price, rs);
+                            const int fs = build_fringe<32>(warp_team, hb, ht, nh, FK, T - 1, fr);
                             if (lane == 0) {
                                 s_hcnt[e] = nh;
-                                s_fsize[e] = -1;
+                                s_fsize[e] = fs;
                             }
                         }
                         __syncwarp();
@@ -1000,11 +1222,14 @@ __global__ void __launch_bounds__(kThreads, 1) auction_kernel(const __grid_const
                             s_ncnt[e] = 0;
                         }
                     }
+                    // the row copies this warp issued land before the barrier
+                    asm volatile("cp.async.wait_all;" ::: "memory");
+                    // the other parity's active count: read in the previous round
+                    if (threadIdx.x == 0) s_nact[ra ^ 1] = 0;
                     __syncthreads();
-                    U = s_misc[2];
-                    if (threadIdx.x == 0) s_misc[1] = 0;
+                    U = s_next[(int)(rounds % 3)];
                     lc ^= 1;
-                    __syncthreads();
+                    staged = stage_rows;
                 }
                 // hand the prices and counts back to the grid
                 for (int e = threadIdx.x; e < E; e += kThreads) {
@@ -1012,7 +1237,6 @@ __global__ void __launch_bounds__(kThreads, 1) auction_kernel(const __grid_const
                     p.hcnt[e] = s_hcnt[e];
                 }
                 if (threadIdx.x == 0) {
-                    s_misc[3] = status;
                     reinterpret_cast<volatile long long*>(p.obj)[1] = rounds;
                     reinterpret_cast<volatile long long*>(p.obj)[2] = bids;
                     reinterpret_cast<volatile int*>(p.obj)[6] = status;
@@ -1100,12 +1324,27 @@ __global__ void minmax_kernel(const int32_t* __restrict__ q, size_t n, int32_t* 
     }
 }
 
-// fringe capacity: as many worst keys per expert as fit next to everything
-// else in 200 KB of shared memory (at most 32, at least 2)
-static int fringe_capacity(int E, int NM) {
-    for (int fk = 32; fk >= 2; fk >>= 1)
-        if (smem_layout(E, fk, NM).total <= 200 * 1024) return fk;
-    return 0;
+// Shared-memory plan: the fringe capacity FK (<= 32), the per-expert bid
+// bucket NB (<= 32) and the staged rows RC (<= 32) as large as 200 KB allows,
+// the fringe first.
+struct SmemPlan {
+    int FK, NB, RC;
+    size_t bytes;
+};
+
+static SmemPlan smem_plan(int E, int NM) {
+    constexpr size_t kBudget = 200 * 1024;
+    SmemPlan pl{0, 0, 0, 0};
+    for (int fk = 32; fk >= 2; fk >>= 1) {
+        if (smem_layout(E, fk, NM, 1, 0).total > kBudget) continue;
+        int nb = 32;
+        while (nb > 1 && smem_layout(E, fk, NM, nb, 0).total > kBudget) nb >>= 1;
+        int rc = 32;
+        while (rc > 0 && smem_layout(E, fk, NM, nb, rc).total > kBudget) rc >>= 1;
+        pl = SmemPlan{fk, nb, rc, smem_layout(E, fk, NM, nb, rc).total};
+        return pl;
+    }
+    return pl;
 }
 
 }  // namespace auction
@@ -1124,6 +1363,8 @@ size_t auction_workspace_bytes(int T, int E) {
     b += align_up(sizeof(int32_t) * (size_t)E * T, 256);    // bucket tokens
     b += 2 * align_up(sizeof(int32_t) * (size_t)T, 256);    // lists
     b += align_up(sizeof(int32_t) * (size_t)E * C, 256);    // free slots
+    b += align_up(sizeof(auction::Key) * (size_t)E * 32, 256);  // fringes
+    b += align_up(sizeof(int32_t) * (size_t)E, 256);        // fringe sizes
     return b;
 }
 
@@ -1134,9 +1375,10 @@ int launch_auction(const int32_t* q, int T, int E, int32_t* assign, int64_t* pri
     if (ws_bytes < auction_workspace_bytes(T, E)) return BASE_ERR_WORKSPACE;
     const int C = T / E;
     const int NM = kNarrowMax;
-    const int FK = fringe_capacity(E, NM);
-    if (FK == 0) return BASE_ERR_UNSUPPORTED;
-    const size_t smem = smem_layout(E, FK, NM).total;
+    const SmemPlan sp = smem_plan(E, NM);
+    if (sp.FK == 0) return BASE_ERR_UNSUPPORTED;
+    const int FK = sp.FK;
+    const size_t smem = sp.bytes;
 
     unsigned char* w = static_cast<unsigned char*>(ws);
     size_t o = 0;
@@ -1147,6 +1389,8 @@ int launch_auction(const int32_t* q, int T, int E, int32_t* assign, int64_t* pri
     prm.E = E;
     prm.C = C;
     prm.FK = FK;
+    prm.NB = sp.NB;
+    prm.RC = sp.RC;
     prm.max_rounds = max_rounds;
     prm.narrow_max = NM;
     prm.assign = assign;
@@ -1171,6 +1415,8 @@ int launch_auction(const int32_t* q, int T, int E, int32_t* assign, int64_t* pri
     prm.ulist0 = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * (size_t)T));
     prm.ulist1 = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * (size_t)T));
     prm.gfree = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * (size_t)E * C));
+    prm.gfr = reinterpret_cast<Key*>(take(sizeof(Key) * (size_t)E * 32));
+    prm.gfs = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * (size_t)E));
 
     // control block, objective, prices (start at 0), counts
     if (cudaMemsetAsync(zero_begin, 0, zero_bytes, stream) != cudaSuccess) return BASE_ERR_CUDA;

@@ -57,41 +57,64 @@ def peaks():
 
 
 class Clocks:
-    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+    """nvidia-smi sampling of SM clocks and throttle reasons.  Sampling runs
+    from before the warm-up to after the timed region; the summary keeps the
+    samples taken inside [t0 - 0.1 s, t1 + 0.1 s] of the timed region."""
+
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
     def __init__(self, index: int):
         self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
-        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        self.t0 = self.t1 = None
         try:
-            self.p = subprocess.Popen(["nvidia-smi", "-i", str(index), "--query-gpu=" + q,
-                                       "--format=csv,noheader,nounits", "-lms", "100"],
+            self.p = subprocess.Popen(["nvidia-smi", "-i", str(index), "--query-gpu=" + self.FIELDS,
+                                       "--format=csv,noheader,nounits", "-lms", "20"],
                                       stdout=self.f, stderr=subprocess.DEVNULL)
         except Exception:
             self.p = None
 
+    def mark_start(self):
+        self.t0 = time.time()
+
+    def mark_end(self):
+        self.t1 = time.time()
+
     def stop(self):
         if self.p is None:
             return None
+        time.sleep(0.15)
         self.p.terminate()
         try:
             self.p.wait(timeout=5)
         except Exception:
             self.p.kill()
         self.f.flush()
+        import datetime
         rows = []
         for line in open(self.f.name):
             parts = [x.strip() for x in line.split(",")]
-            if len(parts) >= 9:
-                rows.append(parts)
+            if len(parts) < 10:
+                continue
+            try:
+                ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+            except ValueError:
+                continue
+            rows.append((ts, parts))
         os.unlink(self.f.name)
+        if self.t0 is not None and self.t1 is not None:
+            inside = [r for ts, r in rows if self.t0 - 0.1 <= ts <= self.t1 + 0.1]
+            if inside:
+                rows = [(0, r) for r in inside]
+        rows = [r for _, r in rows]
         if not rows:
             return None
-        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
-        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        num = lambda x: float(x) if x.replace(".", "", 1).isdigit() else None  # noqa: E731
+        sm = [num(r[2]) for r in rows if num(r[2]) is not None]
+        mx = [num(r[3]) for r in rows if num(r[3]) is not None]
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i] == "Active"})
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[6 + i] == "Active"})
         return dict(sm_mhz=statistics.median(sm) if sm else None,
                     sm_max_mhz=max(mx) if mx else None, reasons=reasons, samples=len(rows))
 
@@ -246,14 +269,6 @@ def main():
             ev[2 * j + 1].record(stream)
             j += 1
 
-    kernels_per_step = sum(k for _, _, k in comps)
-    mk = lambda: [torch.cuda.Event(enable_timing=True) for _ in range(2 * len(names))]  # noqa: E731
-    for _ in range(max(3, args.warmup)):
-        flush.zero_()
-        step(mk())
-    torch.cuda.synchronize()
-    B.base_device_error(clear=True)
-
     phys = 0
     vis = os.environ.get("CUDA_VISIBLE_DEVICES")
     if vis:
@@ -264,16 +279,27 @@ def main():
     else:
         phys = local_rank
     clocks = Clocks(phys) if rank == 0 else None
+    kernels_per_step = sum(k for _, _, k in comps)
+    mk = lambda: [torch.cuda.Event(enable_timing=True) for _ in range(2 * len(names))]  # noqa: E731
+    for _ in range(max(3, args.warmup)):
+        flush.zero_()
+        step(mk())
+    torch.cuda.synchronize()
+    B.base_device_error(clear=True)
 
     evs = [mk() for _ in range(args.steps)]
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
+    if clocks:
+        clocks.mark_start()
     wall0 = time.perf_counter()
     for i in range(args.steps):
         flush.zero_()
         step(evs[i])
     torch.cuda.synchronize()
+    if clocks:
+        clocks.mark_end()
     if world > 1:
         dist.barrier()
     wall = time.perf_counter() - wall0
