@@ -21,8 +21,8 @@ __all__ = [
     "BASE_ROUTE_BALANCED", "BASE_ROUTE_GREEDY", "QSCALE",
     "base_status_string", "base_version", "base_workspace_size", "base_device_error",
     "base_scores", "base_assign_greedy", "base_assign_balanced", "base_assign_balanced_ex",
-    "base_permute", "base_expert_ffn", "base_combine", "base_layer_fwd", "base_layer_bwd",
-    "EXPORTED",
+    "base_permute", "base_permute_noalloc", "base_expert_ffn", "base_combine", "base_layer_fwd",
+    "base_layer_bwd", "EXPORTED",
 ]
 
 BASE_OK = 0
@@ -35,7 +35,8 @@ QSCALE = 65536.0
 EXPORTED = (
     "base_status_string", "base_device_error", "base_version", "base_workspace_size",
     "base_scores", "base_assign_greedy", "base_assign_balanced", "base_assign_balanced_ex",
-    "base_permute", "base_expert_ffn", "base_combine", "base_layer_fwd", "base_layer_bwd",
+    "base_permute", "base_permute_noalloc", "base_expert_ffn", "base_combine", "base_layer_fwd",
+    "base_layer_bwd",
 )
 
 
@@ -77,6 +78,7 @@ _SIGS = {
     "base_assign_balanced_ex": (_i, [_vp, _i, _i, _vp, _vp, _vp, ctypes.c_longlong, _vp, _vp,
                                      ctypes.c_longlong, _vp, _sz, _vp]),
     "base_permute": (_i, [_vp, _vp, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "base_permute_noalloc": (_i, [_vp, _vp, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
     "base_expert_ffn": (_i, [_vp, _vp, _i, _i, _i, _i, _vp, _vp, _i, _vp, _vp, _vp, _vp, _vp, _vp,
                              _sz, _vp]),
     "base_combine": (_i, [_vp, _vp, _i, _i, _vp, _vp]),
@@ -186,6 +188,16 @@ def base_permute(h, assign, E, perm, inv, offsets, x_perm, s=None, gate=None, ws
         _ptr(h), _ptr(assign), T, D, E, _ptr(perm), _ptr(inv), _ptr(offsets), _ptr(x_perm),
         _ptr(s), _ptr(gate), _ptr(ws), 0 if ws is None else ws.numel() * ws.element_size(),
         _stream(stream)))
+
+
+def base_permute_noalloc(h, assign, E, perm, inv, offsets, x_perm, s=None, gate=None,
+                         stream=None):
+    """base_permute without a workspace (the library's own fixed scratch)."""
+    T = assign.shape[0]
+    D = 0 if h is None else h.shape[1]
+    _check("base_permute_noalloc", lib().base_permute_noalloc(
+        _ptr(h), _ptr(assign), T, D, E, _ptr(perm), _ptr(inv), _ptr(offsets), _ptr(x_perm),
+        _ptr(s), _ptr(gate), _stream(stream)))
 
 
 def base_expert_ffn(x_perm, offsets, W1, W2, act: int, gate, y_perm, h1, a1=None, f=None, ws=None,

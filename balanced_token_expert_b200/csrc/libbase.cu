@@ -5,3 +5,4 @@
 #include "gemm.cu"
 #include "backward.cu"
 #include "api.cu"
+#include "noalloc.cu"

@@ -192,6 +192,27 @@ int base_permute(const void* h, const int32_t* assign, int T, int D, int E,
                  const float* s, float* gate, void* ws, size_t ws_bytes, cudaStream_t stream);
 
 /*
+ * base_permute for callers that cannot allocate device memory.  The paper has
+ * no counterpart: this is a deployment variant.  A caller that only holds its
+ * inputs, outputs and a stream -- a plugin inside another runtime that owns
+ * all device memory, or a serving loop that must not call cudaMalloc -- has
+ * no workspace to give base_permute.  This entry point takes the same
+ * arguments minus the workspace and keeps the scratch (the per-chunk expert
+ * counts, ceil(T/256) * E int32) in a 4 MiB array that the library reserves
+ * in every GPU that loads it, for the life of the process.
+ *   Limit: ceil(T/256) * E <= 1048576, else BASE_ERR_WORKSPACE and nothing
+ *   is launched.  Allocates nothing.
+ *   The first call on a device looks up the array's device address (a CUDA
+ *   runtime query); make that first call before any stream capture.
+ *   All calls share the one array, whose contents the next call overwrites
+ *   before reading; calls that overlap on the GPU race on it, so the caller
+ *   must order them (one stream, or events).
+ */
+int base_permute_noalloc(const void* h, const int32_t* assign, int T, int D, int E,
+                         int32_t* perm, int32_t* inv, int32_t* offsets, void* x_perm,
+                         const float* s, float* gate, cudaStream_t stream);
+
+/*
  * a6+a7: the experts' FFNs on their slot segments with the eq. 1 combine in
  * the epilogue.  For every expert e and slot r in [offsets[e], offsets[e+1]):
  *   a1[r] = x_perm[r] W1[e]^T          (W1: E*F*D bf16)
