@@ -13,7 +13,7 @@
 // A phase runs rounds until nobody is unassigned; eps is divided by 8 down
 // to 1 (exact optimum for integer scores).
 //
-// The kernel is one persistent cooperative grid (one CTA of 1024 threads per
+// The kernel is one persistent cooperative grid (one CTA of 512 threads per
 // SM) with two modes:
 //   * wide rounds (the start of every phase, where all T tokens bid, and the
 //     next rounds while many tokens are unassigned) use the whole GPU: bids
@@ -36,7 +36,7 @@
 namespace base {
 namespace auction {
 
-constexpr int kThreads = 1024;
+constexpr int kThreads = 512;  // 16 warps: 128 registers per thread, no spills
 constexpr int kWarps = kThreads / kWarp;
 constexpr int kHist = 256;
 constexpr int kEpsDivisor = 50;  // eps0 = (max q - min q)(T+1) / 50
@@ -156,8 +156,8 @@ __device__ __forceinline__ int bit_length_u64(uint64_t x) { return x ? 64 - __cl
 __device__ __forceinline__ uint64_t shr64(uint64_t x, int n) { return n >= 64 ? 0ull : (x >> n); }
 
 // ---------------------------------------------------------------- teams
-// A team is either one warp (TEAM = 32) or the whole CTA (TEAM = 1024).  Its
-// scratch: kHist ints of histogram + 64 bytes.
+// A team is either one warp (TEAM = 32) or the whole CTA (TEAM = kThreads,
+// at least 256).  Its scratch: kHist ints of histogram, 32 int64, 64 ints.
 template <int TEAM>
 struct Team {
     int32_t* hist;     // [kHist]
@@ -173,7 +173,7 @@ struct Team {
         if (lane_id() == 0) red[warp_id()] = v;
         __syncthreads();
         if (warp_id() == 0) {
-            int64_t x = red[lane_id()];
+            int64_t x = lane_id() < TEAM / 32 ? red[lane_id()] : INT64_MAX;
             x = warp_min_i64(x);
             if (lane_id() == 0) red[0] = x;
         }
@@ -188,7 +188,7 @@ struct Team {
         if (lane_id() == 0) red[warp_id()] = v;
         __syncthreads();
         if (warp_id() == 0) {
-            int64_t x = red[lane_id()];
+            int64_t x = lane_id() < TEAM / 32 ? red[lane_id()] : INT64_MIN;
             x = warp_max_i64(x);
             if (lane_id() == 0) red[0] = x;
         }
@@ -204,7 +204,7 @@ struct Team {
         if (lane_id() == 0) sk[warp_id()] = k;
         __syncthreads();
         if (warp_id() == 0) {
-            Key x = warp_max_key(sk[lane_id()]);
+            Key x = warp_max_key(lane_id() < TEAM / 32 ? sk[lane_id()] : Key{INT64_MIN, INT32_MAX, -2});
             if (lane_id() == 0) sk[0] = x;
         }
         __syncthreads();
@@ -286,7 +286,7 @@ struct Team {
         if (lane_id() == 0) cnt[warp_id()] = __popc(m);
         __syncthreads();
         if (warp_id() == 0) {
-            const int v = cnt[lane_id()];
+            const int v = lane_id() < TEAM / 32 ? cnt[lane_id()] : 0;
             int incl = v;
 #pragma unroll
             for (int off = 1; off < 32; off <<= 1) {
@@ -326,34 +326,21 @@ struct Cands {
     }
 };
 
-// The k-th worst key among the candidates (1 <= k <= h + n; keys are unique).
-// Radix select on the bid (relative to the smallest bid, 8-bit digits from the
-// top), then, among equal bids, on the token.
-template <int TEAM>
-__device__ Key kth_worst(const Team<TEAM>& tm, const Cands& cd, int k, int tm_tmax) {
-    const int m = cd.h + cd.n;
-    const int tid = tm.tid();
-    if (TEAM == 32 && k <= 8) {  // a few rejections: repeated minima
-        Key last = Key{INT64_MIN, INT32_MAX, -2};
-        for (int it = 0; it < k; ++it) {
-            Key best = pad_key();
-            for (int c = tid; c < m; c += TEAM) {
-                const Key x = cd.get(c);
-                if (worse(last, x) && worse(x, best)) best = x;
-            }
-            last = warp_min_key(best);
-        }
-        return last;
-    }
+// The k-th worst key among a team's candidates (1 <= k <= m; keys are
+// unique).  `visit(f)` calls f(key) for each candidate this thread owns.
+// Radix select on the bid (relative to the smallest bid, 8-bit digits from
+// the top), then, among equal bids, on the token.
+template <int TEAM, class Visit>
+__device__ Key kth_worst_v(const Team<TEAM>& tm, Visit visit, int k, int tmax) {
     int64_t lo = INT64_MAX, hi = INT64_MIN;
-    for (int c = tid; c < m; c += TEAM) {
-        const int64_t b = cd.get(c).bid;
-        lo = min(lo, b);
-        hi = max(hi, b);
-    }
+    visit([&](const Key& x) {
+        lo = min(lo, x.bid);
+        hi = max(hi, x.bid);
+    });
     lo = tm.min_i64(lo);
     hi = tm.max_i64(hi);
     const int nbits = bit_length_u64((uint64_t)(hi - lo));
+    const int tid = tm.tid();
     // --- bid digits
     int need = k, pbits = 0;
     uint64_t prefix = 0;
@@ -363,13 +350,12 @@ __device__ Key kth_worst(const Team<TEAM>& tm, const Cands& cd, int k, int tm_tm
         const int shift = nbits - pbits - width;
         for (int b = tid; b < kHist; b += TEAM) tm.hist[b] = 0;
         tm.sync();
-        for (int c = tid; c < m; c += TEAM) {
-            const uint64_t v = (uint64_t)(cd.get(c).bid - lo);
+        visit([&](const Key& x) {
+            const uint64_t v = (uint64_t)(x.bid - lo);
             if (shr64(v, shift + width) == prefix)
                 atomicAdd(&tm.hist[(int)((v >> shift) & ((1u << width) - 1))], 1);
-        }
+        });
         tm.sync();
-        // find the digit whose bucket holds the need-th element
         int d = 0, before = 0, cnt = 0;
         tm.find_digit(1 << width, need, d, before, cnt);
         prefix = (prefix << width) | (uint64_t)d;
@@ -385,17 +371,16 @@ __device__ Key kth_worst(const Team<TEAM>& tm, const Cands& cd, int k, int tm_tm
         // worst is the best of them
         Key best = Key{INT64_MIN, INT32_MAX, -2};
         const int sh = nbits - pbits;
-        for (int c = tid; c < m; c += TEAM) {
-            const Key x = cd.get(c);
+        visit([&](const Key& x) {
             if (shr64((uint64_t)(x.bid - lo), sh) <= prefix && worse(best, x)) best = x;
-        }
+        });
         return tm.max_key(best);
     }
     // every bid digit fixed: B* = lo + prefix; `need` of the candidates with
     // bid == B* are rejected, the ones with the largest tokens
     const int64_t bstar = lo + (int64_t)prefix;
-    const uint32_t tmax = (uint32_t)tm_tmax;  // largest token index + 1 bits below
-    const int tbits = bit_length_u64((uint64_t)tmax) > 0 ? bit_length_u64((uint64_t)tmax) : 1;
+    const uint32_t tm_max = (uint32_t)tmax;
+    const int tbits = bit_length_u64((uint64_t)tm_max) > 0 ? bit_length_u64((uint64_t)tm_max) : 1;
     int tneed = need, tp = 0;
     uint32_t tprefix = 0;
     // rank by (tmax - tok) ascending: larger tokens first
@@ -404,13 +389,12 @@ __device__ Key kth_worst(const Team<TEAM>& tm, const Cands& cd, int k, int tm_tm
         const int shift = tbits - tp - width;
         for (int b = tid; b < kHist; b += TEAM) tm.hist[b] = 0;
         tm.sync();
-        for (int c = tid; c < m; c += TEAM) {
-            const Key x = cd.get(c);
-            if (x.bid != bstar) continue;
-            const uint32_t v = tmax - (uint32_t)x.tok;
+        visit([&](const Key& x) {
+            if (x.bid != bstar) return;
+            const uint32_t v = tm_max - (uint32_t)x.tok;
             if ((uint32_t)shr64(v, shift + width) == tprefix)
                 atomicAdd(&tm.hist[(int)((v >> shift) & ((1u << width) - 1))], 1);
-        }
+        });
         tm.sync();
         int d = 0, before = 0, cnt = 0;
         tm.find_digit(1 << width, tneed, d, before, cnt);
@@ -421,13 +405,46 @@ __device__ Key kth_worst(const Team<TEAM>& tm, const Cands& cd, int k, int tm_tm
     }
     Key best = Key{INT64_MIN, INT32_MAX, -2};
     const int sh = tbits - tp;
-    for (int c = tid; c < m; c += TEAM) {
-        const Key x = cd.get(c);
+    visit([&](const Key& x) {
         bool rej = x.bid < bstar;
-        if (x.bid == bstar) rej = (uint32_t)shr64(tmax - (uint32_t)x.tok, sh) <= tprefix;
+        if (x.bid == bstar) rej = (uint32_t)shr64(tm_max - (uint32_t)x.tok, sh) <= tprefix;
         if (rej && worse(best, x)) best = x;
-    }
+    });
     return tm.max_key(best);
+}
+
+// Candidates read from memory on every pass; a warp with few rejections
+// uses repeated minima instead of the radix select.
+template <int TEAM>
+__device__ Key kth_worst(const Team<TEAM>& tm, const Cands& cd, int k, int tmax) {
+    const int m = cd.h + cd.n;
+    const int tid = tm.tid();
+    if (TEAM == 32 && k <= 8) {
+        Key last = Key{INT64_MIN, INT32_MAX, -2};
+        for (int it = 0; it < k; ++it) {
+            Key best = pad_key();
+            for (int c = tid; c < m; c += TEAM) {
+                const Key x = cd.get(c);
+                if (worse(last, x) && worse(x, best)) best = x;
+            }
+            last = warp_min_key(best);
+        }
+        return last;
+    }
+    if (TEAM > 32 && m <= 2 * TEAM) {
+        // the whole candidate set fits in registers: two keys per thread
+        const Key k0 = tid < m ? cd.get(tid) : pad_key();
+        const Key k1 = tid + TEAM < m ? cd.get(tid + TEAM) : pad_key();
+        auto visit = [&](auto f) {
+            if (tid < m) f(k0);
+            if (tid + TEAM < m) f(k1);
+        };
+        return kth_worst_v<TEAM>(tm, visit, k, tmax);
+    }
+    auto visit = [&](auto f) {
+        for (int c = tid; c < m; c += TEAM) f(cd.get(c));
+    };
+    return kth_worst_v<TEAM>(tm, visit, k, tmax);
 }
 
 // ---------------------------------------------------------------- state
@@ -478,9 +495,11 @@ __device__ __forceinline__ void trace_round(const Params& p, long long r, int U)
 
 // shared memory of every CTA (narrow-mode arrays are used by CTA 0 only)
 struct SmemLayout {
-    size_t price, fr, fsize, hcnt, ncnt, act0, act1, nbk_b, nbk_t, list0, list1, rows, hist, red,
-        cnt, misc, total;
+    size_t price, fr, fsize, hcnt, ncnt, act0, act1, nbk_b, nbk_t, list0, list1, rows, wb, wt, we,
+        wp, hist, red, cnt, misc, total;
 };
+
+constexpr int kWideChunk = 1024;  // bids a CTA stages before reserving bucket space
 
 // NB: new bids per expert kept in shared memory (the rest in the global
 // bucket); RC: bidders' score rows staged in shared memory per round parity.
@@ -500,6 +519,10 @@ __host__ __device__ inline SmemLayout smem_layout(int E, int FK, int NM, int NB,
     L.list0 = take(4 * (size_t)NM);
     L.list1 = take(4 * (size_t)NM);
     L.rows = take(2 * 4 * (size_t)RC * E);
+    L.wb = take(8 * (size_t)kWideChunk);
+    L.wt = take(4 * (size_t)kWideChunk);
+    L.we = take(4 * (size_t)kWideChunk);
+    L.wp = take(4 * (size_t)kWideChunk);
     L.hist = take(4 * (size_t)kWarps * kHist);
     L.red = take(8 * 32);
     L.cnt = take(4 * 64);
@@ -657,6 +680,15 @@ struct RowStage {
             asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst + off), "l"(src + off)
                          : "memory");
     }
+    // the same copy spread over the 32 lanes of a warp (all lanes call it)
+    __device__ __forceinline__ void stage_warp(const int32_t* q, int E, int tok, int pos) const {
+        if (rows == nullptr || pos >= cap) return;
+        const char* src = reinterpret_cast<const char*>(q + (size_t)tok * E);
+        const uint32_t dst = smem_u32(rows + (size_t)pos * E);
+        for (int off = lane_id() * 16; off < E * 4; off += 32 * 16)
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst + off), "l"(src + off)
+                         : "memory");
+    }
 };
 
 // Keeps the C best of held + new for expert e (held in global memory), with
@@ -780,8 +812,8 @@ __device__ int resolve_general(const Team<TEAM>& tm, const Params& p, int e, con
 // collected with a team-wide ranking and sorted by warp 0.  Returns the
 // fringe size.
 template <int TEAM>
-__device__ int build_fringe(const Team<TEAM>& tm, const int64_t* hb, const int32_t* ht, int C,
-                            int FK, int tmax, Key* fr) {
+__device__ int build_fringe_radix(const Team<TEAM>& tm, const int64_t* hb, const int32_t* ht,
+                                  int C, int FK, int tmax, Key* fr) {
     const int k = min(FK, C);
     if (k == 0) return 0;
     const Cands cd{hb, ht, nullptr, nullptr, C, 0};
@@ -809,6 +841,66 @@ __device__ int build_fringe(const Team<TEAM>& tm, const int64_t* hb, const int32
     }
     tm.sync();
     return k;
+}
+
+// Warp version: a sampled threshold first.  Each lane keeps the two worst
+// keys of its stripe; the 32nd worst of those 64 keys, theta, has at least 32
+// held keys at or below it, and usually not many more: they are collected
+// (at most 64, else the radix build runs) and sorted.  Two passes over the
+// held keys instead of one per radix digit.
+__device__ int build_fringe_warp(const Team<32>& tm, const int64_t* hb, const int32_t* ht, int C,
+                                 int FK, int tmax, Key* fr) {
+    const int k = min(FK, C);
+    if (k == 0) return 0;
+    const int lane = lane_id();
+    Key* stage = reinterpret_cast<Key*>(tm.hist);  // 64 keys
+    Key lo, hi;
+    if (C <= 64) {
+        Key a = lane < C ? Key{hb[lane], ht[lane], lane} : pad_key();
+        Key b = lane + 32 < C ? Key{hb[lane + 32], ht[lane + 32], lane + 32} : pad_key();
+        warp_merge64(warp_sort(a), warp_sort(b), lo, hi);
+    } else {
+        Key a = pad_key(), b = pad_key();
+#pragma unroll 4
+        for (int i = lane; i < C; i += 32) {
+            const Key x = Key{hb[i], ht[i], i};
+            if (worse(x, a)) {
+                b = a;
+                a = x;
+            } else if (worse(x, b)) {
+                b = x;
+            }
+        }
+        warp_merge64(warp_sort(a), warp_sort(b), lo, hi);
+        const Key theta = shfl_key(lo, 31);
+        int got = 0;
+#pragma unroll 4
+        for (int i0 = 0; i0 < C; i0 += 32) {  // uniform trip count: the ballot needs all lanes
+            const int i = i0 + lane;
+            const Key x = i < C ? Key{hb[i], ht[i], i} : pad_key();
+            const bool in = i < C && !worse(theta, x);
+            const unsigned m = __ballot_sync(0xffffffffu, in);
+            const int pos = got + __popc(m & ((1u << lane) - 1));
+            if (in && pos < 64) stage[pos] = x;
+            got += __popc(m);
+        }
+        __syncwarp();
+        if (got > 64) return build_fringe_radix<32>(tm, hb, ht, C, FK, tmax, fr);
+        const Key sa = lane < got ? stage[lane] : pad_key();
+        const Key sb = lane + 32 < got ? stage[lane + 32] : pad_key();
+        __syncwarp();
+        warp_merge64(warp_sort(sa), warp_sort(sb), lo, hi);
+    }
+    if (lane < k) fr[lane] = lo;
+    __syncwarp();
+    return k;
+}
+
+template <int TEAM>
+__device__ int build_fringe(const Team<TEAM>& tm, const int64_t* hb, const int32_t* ht, int C,
+                            int FK, int tmax, Key* fr) {
+    if constexpr (TEAM == 32) return build_fringe_warp(tm, hb, ht, C, FK, tmax, fr);
+    else return build_fringe_radix<TEAM>(tm, hb, ht, C, FK, tmax, fr);
 }
 
 __device__ __forceinline__ int nth_set_lane(unsigned m, int r) {
@@ -850,13 +942,15 @@ __device__ bool resolve_warp(const Params& p, Key* fr, int& fs, int& h, const in
         Key out = lane < pos ? fn : (lane == pos ? b : fi);
         if (!ins) out = fn;
         const int nfs = ins ? fs : fs - 1;
+        int at = 0;
         if (lane == 0) {
             hb[b.slot] = b.bid;
             ht[b.slot] = b.tok;
-            const int at = atomicAdd(next_cnt, 1);
+            at = atomicAdd(next_cnt, 1);
             next_list[at] = f0.tok;
-            rs.stage(p.q, p.E, f0.tok, at);
         }
+        at = __shfl_sync(0xffffffffu, at, 0);
+        rs.stage_warp(p.q, p.E, f0.tok, at);
         __syncwarp();
         if (lane < nfs) fr[lane] = out;
         __syncwarp();
@@ -948,6 +1042,10 @@ __global__ void __launch_bounds__(kThreads, 1) auction_kernel(const __grid_const
     int32_t* s_list0 = reinterpret_cast<int32_t*>(smem + L.list0);
     int32_t* s_list1 = reinterpret_cast<int32_t*>(smem + L.list1);
     int32_t* s_rows = reinterpret_cast<int32_t*>(smem + L.rows);
+    int64_t* s_wb = reinterpret_cast<int64_t*>(smem + L.wb);
+    int32_t* s_wt = reinterpret_cast<int32_t*>(smem + L.wt);
+    int32_t* s_we = reinterpret_cast<int32_t*>(smem + L.we);
+    int32_t* s_wp = reinterpret_cast<int32_t*>(smem + L.wp);
     int32_t* s_hist = reinterpret_cast<int32_t*>(smem + L.hist);
     int64_t* s_red = reinterpret_cast<int64_t*>(smem + L.red);
     int32_t* s_cnt = reinterpret_cast<int32_t*>(smem + L.cnt);
@@ -958,7 +1056,7 @@ __global__ void __launch_bounds__(kThreads, 1) auction_kernel(const __grid_const
     const int lane = lane_id(), warp = warp_id();
     const int cta = blockIdx.x, ncta = gridDim.x;
 
-    Team<1024> cta_team{s_hist, s_red, s_cnt};
+    Team<kThreads> cta_team{s_hist, s_red, s_cnt};
     Team<32> warp_team{s_hist + warp * kHist, nullptr, nullptr};
 
     const int64_t qmin = p.minmax[0], qmax = p.minmax[1];
@@ -976,18 +1074,23 @@ __global__ void __launch_bounds__(kThreads, 1) auction_kernel(const __grid_const
 
     long long rounds = 0, phases = 0, bids = 0;
     bool ok = true;
+    bool reset_done = false;
     int cur = 0;  // which global list holds the bidders
 
     while (status == BASE_OK && ok) {
         ++phases;
-        // ---- phase start: nothing held, prices kept (in p.gprice)
-        for (int e = cta * kThreads + threadIdx.x; e < E; e += ncta * kThreads) {
-            p.hcnt[e] = 0;
-            p.bcnt[e] = 0;
-            p.gfs[e] = 0;  // empty held set: an empty, complete fringe
+        // ---- phase start: nothing held, prices kept (in p.gprice); after a
+        // narrow phase CTA 0 has done this already, before the grid barrier
+        if (!reset_done) {
+            for (int e = cta * kThreads + threadIdx.x; e < E; e += ncta * kThreads) {
+                p.hcnt[e] = 0;
+                p.bcnt[e] = 0;
+                p.gfs[e] = 0;  // empty held set: an empty, complete fringe
+            }
+            if (cta == 0 && threadIdx.x < 3) p.ctrl->ucount[threadIdx.x] = 0;
+            if (!(ok = grid_sync(p.ctrl, s_misc))) break;
         }
-        if (cta == 0 && threadIdx.x < 3) p.ctrl->ucount[threadIdx.x] = 0;
-        if (!(ok = grid_sync(p.ctrl, s_misc))) break;
+        reset_done = false;
         int U = T;
         bool first = true;
         bool narrow = false;
@@ -1006,34 +1109,59 @@ __global__ void __launch_bounds__(kThreads, 1) auction_kernel(const __grid_const
             for (int e = threadIdx.x; e < E; e += kThreads) s_price[e] = vload(p.gprice + e);
             __syncthreads();
             {
-                // 4 tokens per lane group per step: a group handles tokens
-                // base + sub + k * tpw * nwarps_total, k = 0..3
+                // The CTA takes chunks of up to kWideChunk bidders; each bid is
+                // staged in shared memory with its rank among the chunk's bids
+                // to the same expert, then one global atomic per (chunk,
+                // expert) reserves bucket space and the bids are written out.
                 constexpr int NT = 4;
-                const long long nw = (long long)ncta * kWarps;
-                const long long gw = (long long)cta * kWarps + warp;
-                const long long stride = nw * tpw * NT;
-                for (long long base = gw * tpw; base < U; base += stride) {
-                    int t[NT];
-                    bool valid[NT];
-#pragma unroll
-                    for (int u = 0; u < NT; ++u) {
-                        const long long i = base + sub + (long long)u * nw * tpw;
-                        valid[u] = i < U;
-                        t[u] = valid[u] ? (first ? (int)i : vload(ulist + i)) : 0;
-                    }
-                    int64_t v1[NT], v2[NT];
-                    int e1[NT];
-                    group_bid_multi<NT>(p.q, t, valid, s_price, E, G, gl, scale, v1, v2, e1);
-                    if (gl == 0) {
+                const int per_cta = (U + ncta - 1) / ncta;
+                const int CH = min(kWideChunk, max(32, per_cta));
+                const int groups = kWarps * tpw;  // lane groups in the CTA
+                for (long long c0 = (long long)cta * CH; c0 < U; c0 += (long long)ncta * CH) {
+                    const int cn = (int)min((long long)CH, (long long)U - c0);
+                    for (int e = threadIdx.x; e < E; e += kThreads) s_ncnt[e] = 0;
+                    __syncthreads();
+                    // warp-uniform trip count: the lane groups of a warp shuffle
+                    // together, so the loop runs on the warp's first group index
+                    for (int jw = warp * tpw; jw < cn; jw += groups * NT) {
+                        const int j0 = jw + sub;
+                        int t[NT];
+                        bool valid[NT];
 #pragma unroll
                         for (int u = 0; u < NT; ++u) {
-                            if (!valid[u]) continue;
-                            const int64_t b = v1[u] + s_price[e1[u]] - v2[u] + eps;
-                            const int pos = atomicAdd(&p.bcnt[e1[u]], 1);
-                            p.bb[(size_t)e1[u] * T + pos] = b;
-                            p.bt[(size_t)e1[u] * T + pos] = t[u];
+                            const int j = j0 + u * groups;
+                            valid[u] = j < cn;
+                            const long long i = c0 + j;
+                            t[u] = valid[u] ? (first ? (int)i : vload(ulist + i)) : 0;
+                        }
+                        int64_t v1[NT], v2[NT];
+                        int e1[NT];
+                        group_bid_multi<NT>(p.q, t, valid, s_price, E, G, gl, scale, v1, v2, e1);
+                        if (gl == 0) {
+#pragma unroll
+                            for (int u = 0; u < NT; ++u) {
+                                if (!valid[u]) continue;
+                                const int j = j0 + u * groups;
+                                s_wb[j] = v1[u] + s_price[e1[u]] - v2[u] + eps;
+                                s_wt[j] = t[u];
+                                s_we[j] = e1[u];
+                                s_wp[j] = atomicAdd(&s_ncnt[e1[u]], 1);
+                            }
                         }
                     }
+                    __syncthreads();
+                    for (int e = threadIdx.x; e < E; e += kThreads) {
+                        const int c = s_ncnt[e];
+                        if (c) s_act0[e] = atomicAdd(&p.bcnt[e], c);
+                    }
+                    __syncthreads();
+                    for (int j = threadIdx.x; j < cn; j += kThreads) {
+                        const int e = s_we[j];
+                        const size_t at = (size_t)e * T + s_act0[e] + s_wp[j];
+                        p.bb[at] = s_wb[j];
+                        p.bt[at] = s_wt[j];
+                    }
+                    __syncthreads();
                 }
             }
             if (!(ok = grid_sync(p.ctrl, s_misc))) break;
@@ -1070,9 +1198,9 @@ __global__ void __launch_bounds__(kThreads, 1) auction_kernel(const __grid_const
                 }
                 Cands cd{hb, ht, p.bb + (size_t)e * T, p.bt + (size_t)e * T, h0, n};
                 int64_t price = INT64_MIN;
-                const int nh = resolve_general<1024>(cta_team, p, e, cd, hb, ht, unext, ucnt,
+                const int nh = resolve_general<kThreads>(cta_team, p, e, cd, hb, ht, unext, ucnt,
                                                      price, RowStage{nullptr, 0});
-                const int fs = build_fringe<1024>(cta_team, hb, ht, nh, FK, T - 1, gfr);
+                const int fs = build_fringe<kThreads>(cta_team, hb, ht, nh, FK, T - 1, gfr);
                 if (threadIdx.x == 0) {
                     p.hcnt[e] = nh;
                     p.bcnt[e] = 0;
@@ -1231,11 +1359,18 @@ __global__ void __launch_bounds__(kThreads, 1) auction_kernel(const __grid_const
                     lc ^= 1;
                     staged = stage_rows;
                 }
-                // hand the prices and counts back to the grid
+                // hand the prices back to the grid; when another phase follows,
+                // reset its state now (the phase start then needs no barrier)
+                const bool again = status == BASE_OK && eps != 1;
                 for (int e = threadIdx.x; e < E; e += kThreads) {
                     p.gprice[e] = s_price[e];
-                    p.hcnt[e] = s_hcnt[e];
+                    p.hcnt[e] = again ? 0 : s_hcnt[e];
+                    if (again) {
+                        p.bcnt[e] = 0;
+                        p.gfs[e] = 0;
+                    }
                 }
+                if (again && threadIdx.x < 3) p.ctrl->ucount[threadIdx.x] = 0;
                 if (threadIdx.x == 0) {
                     reinterpret_cast<volatile long long*>(p.obj)[1] = rounds;
                     reinterpret_cast<volatile long long*>(p.obj)[2] = bids;
@@ -1243,11 +1378,12 @@ __global__ void __launch_bounds__(kThreads, 1) auction_kernel(const __grid_const
                 }
             }
             if (!(ok = grid_sync(p.ctrl, s_misc))) break;
-            // every CTA takes over CTA 0's counters
+            // every CTA takes over CTA 0's counters (rewritten no earlier than
+            // the next narrow phase, several grid barriers later)
             rounds = reinterpret_cast<volatile long long*>(p.obj)[1];
             bids = reinterpret_cast<volatile long long*>(p.obj)[2];
             status = reinterpret_cast<volatile int*>(p.obj)[6];
-            if (!(ok = grid_sync(p.ctrl, s_misc))) break;
+            reset_done = status == BASE_OK && eps != 1;
         }
         if (status != BASE_OK) break;
         if (eps == 1) break;

@@ -156,7 +156,7 @@ int base_assign_greedy(const int32_t* q, int T, int E, int32_t* assign, int32_t*
  *   assign: T int32 output.  price: E int64 output (final prices).
  *   stats (nullable): device base_auction_stats.
  *   ws: workspace of at least base_workspace_size(T, E, 0, 0) bytes.
- * Runs as one cooperative grid of one 1024-thread CTA per SM: rounds with
+ * Runs as one cooperative grid of one 512-thread CTA per SM: rounds with
  * many bidders use every SM, the tail of each phase runs on one CTA with the
  * prices and each expert's worst held bids in shared memory.
  */
