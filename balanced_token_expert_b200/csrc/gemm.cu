@@ -74,7 +74,8 @@ struct TileInfo {
     int k0, kblocks;  // first K index and number of 64-wide K blocks
 };
 
-__device__ __forceinline__ TileInfo decode_tile(const Args& a, int tile, int bn) {
+// bm: rows of A per tile (128, or 256 for a CTA pair)
+__device__ __forceinline__ TileInfo decode_tile(const Args& a, int tile, int bn, int bm = BM) {
     TileInfo ti;
     ti.k0 = 0;
     ti.kblocks = (a.K + BK - 1) / BK;
@@ -84,8 +85,8 @@ __device__ __forceinline__ TileInfo decode_tile(const Args& a, int tile, int bn)
         const int nt = local / a.m_tiles, m = local % a.m_tiles;
         const int k0 = __ldg(a.offsets + g);
         ti.group = g;
-        ti.a_row = m * BM;
-        ti.m_local0 = m * BM;
+        ti.a_row = m * bm;
+        ti.m_local0 = m * bm;
         ti.group_rows = a.M;
         ti.n0 = nt * bn;
         ti.b_row = nt * bn;
@@ -94,11 +95,11 @@ __device__ __forceinline__ TileInfo decode_tile(const Args& a, int tile, int bn)
         return ti;
     }
     if (a.offsets == nullptr) {
-        const int mt = (a.M + BM - 1) / BM;
+        const int mt = (a.M + bm - 1) / bm;
         const int nt = tile / mt, m = tile % mt;
         ti.group = 0;
-        ti.a_row = m * BM;
-        ti.m_local0 = m * BM;
+        ti.a_row = m * bm;
+        ti.m_local0 = m * bm;
         ti.group_rows = a.M;
         ti.n0 = nt * bn;
         ti.b_row = nt * bn;
@@ -117,8 +118,8 @@ __device__ __forceinline__ TileInfo decode_tile(const Args& a, int tile, int bn)
     const int nt = local / mtg, m = local % mtg;
     const int r0 = __ldg(a.offsets + g);
     ti.group = g;
-    ti.a_row = r0 + m * BM;
-    ti.m_local0 = m * BM;
+    ti.a_row = r0 + m * bm;
+    ti.m_local0 = m * bm;
     ti.group_rows = __ldg(a.offsets + g + 1) - r0;
     ti.n0 = nt * bn;
     ti.b_row = g * a.b_rows_per_group + nt * bn;
@@ -273,12 +274,20 @@ __device__ __forceinline__ void epilogue16(const Args& a, const TileInfo& ti, in
     }
 }
 
-template <int BN, int STAGES, int EPI, bool A_MN, bool B_MN>
+// CG = 2: a CTA pair of a cluster computes a (2 x 128) x BN tile with
+// tcgen05.mma.cta_group::2: each CTA loads its own 128 rows of A and BN/2 rows
+// of B (the TMA completions of both land on the leader's barrier), the leader
+// issues the MMAs, each CTA's TMEM holds its 128 rows x BN accumulator and its
+// epilogue writes them.
+template <int BN, int STAGES, int EPI, bool A_MN, bool B_MN, int CG = 1>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const Args args) {
+    static_assert(CG == 1 || CG == 2, "one CTA or a CTA pair");
+    constexpr int BNC = BN / CG;  // rows of B loaded by one CTA
+    constexpr int BMP = BM * CG;  // rows of A per tile
     constexpr uint32_t A_BYTES = BM * BK * 2;
-    constexpr uint32_t B_BYTES = BN * BK * 2;
+    constexpr uint32_t B_BYTES = BNC * BK * 2;
     constexpr uint32_t TMEM_COLS = (2 * BN < 32) ? 32 : 2 * BN;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -293,6 +302,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
 
     const int warp = warp_id(), lane = lane_id();
+    const uint32_t rank = (CG == 2) ? tc::cluster_ctarank() : 0u;
+    const bool leader = rank == 0;
+    const int unit = (CG == 2) ? (int)(blockIdx.x / 2) : (int)blockIdx.x;
+    const int nunits = (CG == 2) ? (int)(gridDim.x / 2) : (int)gridDim.x;
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
             tc::mbar_init(&full[s], 1);
@@ -300,14 +313,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int i = 0; i < 2; ++i) {
             tc::mbar_init(&tfull[i], 1);
-            tc::mbar_init(&tempty[i], 4);
+            tc::mbar_init(&tempty[i], 4 * CG);
         }
         tc::mbar_init(done, 1);
         tc::fence_mbar_init();
     }
     if (warp == 1) {
-        tc::tmem_alloc(tmem_slot, TMEM_COLS);
-        tc::tmem_relinquish();
+        if constexpr (CG == 2) {
+            tc::tmem_alloc_cg2(tmem_slot, TMEM_COLS);
+            tc::tmem_relinquish_cg2();
+        } else {
+            tc::tmem_alloc(tmem_slot, TMEM_COLS);
+            tc::tmem_relinquish();
+        }
     }
     if (warp == 0 && lane == 0) {
         tc::tma_prefetch_desc(&tmA);
@@ -315,49 +333,61 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     tc::tc_fence_before();
     __syncthreads();
+    if constexpr (CG == 2) tc::cluster_sync_all();  // both CTAs' barriers and TMEM are ready
     tc::tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
 
     const int mtiles = args.kgroup ? args.m_tiles * args.groups
                        : args.offsets ? __ldg(args.tile_start + args.groups)
-                                      : (args.M + BM - 1) / BM;
+                                      : (args.M + BMP - 1) / BMP;
     const int total = mtiles * args.n_tiles;
 
     if (warp == 0 && lane == 0) {
-        // ---------------- TMA producer ----------------
+        // ---------------- TMA producer (both CTAs of a pair) ----------------
         int stage = 0;
         uint32_t phase = 0;
         bool ok = true;
         uint32_t issued_parity[STAGES];
         bool issued[STAGES];
         for (int s = 0; s < STAGES; ++s) issued[s] = false;
-        for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
-            const TileInfo ti = decode_tile(args, tile, BN);
+        for (int tile = unit; tile < total && ok; tile += nunits) {
+            const TileInfo ti = decode_tile(args, tile, BN, BMP);
+            const int a_row = ti.a_row + BM * (int)rank;
             for (int kb = 0; kb < ti.kblocks; ++kb) {
                 if (!tc::mbar_wait(&empty[stage], phase ^ 1, 3001)) {
                     ok = false;
                     break;
                 }
-                tc::mbar_arrive_expect_tx(&full[stage], A_BYTES + B_BYTES);
+                uint32_t fbar;
+                if constexpr (CG == 2) {
+                    if (leader) tc::mbar_arrive_expect_tx(&full[stage], CG * (A_BYTES + B_BYTES));
+                    fbar = tc::map_to_rank(&full[stage], 0);
+                } else {
+                    tc::mbar_arrive_expect_tx(&full[stage], A_BYTES + B_BYTES);
+                    fbar = smem_u32(&full[stage]);
+                }
+                auto load = [&](void* dst, const CUtensorMap* tm, int c0, int c1) {
+                    if constexpr (CG == 2) tc::tma_load_2d_cg2(dst, tm, fbar, c0, c1);
+                    else tc::tma_load_2d(dst, tm, &full[stage], c0, c1);
+                };
                 const int kg = ti.k0 + kb * BK;
                 if constexpr (A_MN) {
                     // A stored K x M: two 64(M) x 64(K) boxes
 #pragma unroll
                     for (int j = 0; j < BM / 64; ++j)
-                        tc::tma_load_2d(sA + stage * A_BYTES + j * 8192, &tmA, &full[stage],
-                                        ti.a_row + 64 * j, kg);
+                        load(sA + stage * A_BYTES + j * 8192, &tmA, a_row + 64 * j, kg);
                 } else {
-                    tc::tma_load_2d(sA + stage * A_BYTES, &tmA, &full[stage], kg, ti.a_row);
+                    load(sA + stage * A_BYTES, &tmA, kg, a_row);
                 }
                 if constexpr (B_MN) {
-                    // B stored K x N: BN / 64 boxes; the group's K rows start at b_row_k
+                    // B stored K x N: BNC / 64 boxes; the group's K rows start at krow
                     const int krow = args.kgroup ? kg : ti.group * args.b_rows_per_group + kb * BK;
 #pragma unroll
-                    for (int j = 0; j < BN / 64; ++j)
-                        tc::tma_load_2d(sB + stage * B_BYTES + j * 8192, &tmB, &full[stage],
-                                        ti.n0 + 64 * j, krow);
+                    for (int j = 0; j < BNC / 64; ++j)
+                        load(sB + stage * B_BYTES + j * 8192, &tmB,
+                             ti.n0 + BNC * (int)rank + 64 * j, krow);
                 } else {
-                    tc::tma_load_2d(sB + stage * B_BYTES, &tmB, &full[stage], kg, ti.b_row);
+                    load(sB + stage * B_BYTES, &tmB, kg, ti.b_row + BNC * (int)rank);
                 }
                 issued[stage] = true;
                 issued_parity[stage] = phase;
@@ -369,28 +399,35 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (!ok) {
             // wind down: let the copies already issued land before the CTA exits
-            for (int s = 0; s < STAGES; ++s) {
-                if (!issued[s]) continue;
-                const uint32_t a = smem_u32(&full[s]);
-                const uint64_t t0 = tc::globaltimer();
-                while (!tc::mbar_try_wait(a, issued_parity[s]) &&
-                       tc::globaltimer() - t0 < 100000000ull) {
+            // (a pair's copies complete on the leader's barrier: the peer waits
+            // a fixed time instead)
+            const uint64_t t0 = tc::globaltimer();
+            if (CG == 1 || leader) {
+                for (int s = 0; s < STAGES; ++s) {
+                    if (!issued[s]) continue;
+                    const uint32_t a = smem_u32(&full[s]);
+                    while (!tc::mbar_try_wait(a, issued_parity[s]) &&
+                           tc::globaltimer() - t0 < 100000000ull) {
+                    }
+                }
+            } else {
+                while (tc::globaltimer() - t0 < 10000000ull) {
                 }
             }
         }
-    } else if (warp == 1 && lane == 0) {
-        // ---------------- MMA issuer ----------------
-        constexpr uint32_t idesc = tc::idesc_bf16(BM, BN, A_MN ? 1 : 0, B_MN ? 1 : 0);
+    } else if (warp == 1 && lane == 0 && leader) {
+        // ---------------- MMA issuer (the leader of a pair) ----------------
+        constexpr uint32_t idesc = tc::idesc_bf16(BMP, BN, A_MN ? 1 : 0, B_MN ? 1 : 0);
         int stage = 0;
         uint32_t phase = 0;
         int acc = 0;
         uint32_t acc_phase = 0;
         bool ok = true;
-        for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+        for (int tile = unit; tile < total && ok; tile += nunits) {
             if (!tc::mbar_wait(&tempty[acc], acc_phase ^ 1, 3002)) break;
             tc::tc_fence_after();
             const uint32_t d_tmem = tmem_base + acc * BN;
-            const int kblocks = decode_tile(args, tile, BN).kblocks;
+            const int kblocks = decode_tile(args, tile, BN, BMP).kblocks;
             for (int kb = 0; kb < kblocks; ++kb) {
                 if (!tc::mbar_wait(&full[stage], phase, 3003)) {
                     ok = false;
@@ -407,33 +444,41 @@ __global__ void __launch_bounds__(kThreads, 1)
                                              : tc::smem_desc_sw128(a_addr + kk * 32, 16, 1024);
                     const uint64_t bd = B_MN ? tc::smem_desc_sw128(b_addr + kk * 2048, 8192, 1024)
                                              : tc::smem_desc_sw128(b_addr + kk * 32, 16, 1024);
-                    tc::umma_bf16(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+                    if constexpr (CG == 2)
+                        tc::umma_bf16_cg2(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+                    else
+                        tc::umma_bf16(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
                 }
-                tc::umma_commit(&empty[stage]);
+                if constexpr (CG == 2) tc::umma_commit_cg2_mc(&empty[stage], 0x3);
+                else tc::umma_commit(&empty[stage]);
                 if (++stage == STAGES) {
                     stage = 0;
                     phase ^= 1;
                 }
             }
             if (!ok) break;
-            tc::umma_commit(&tfull[acc]);
+            if constexpr (CG == 2) tc::umma_commit_cg2_mc(&tfull[acc], 0x3);
+            else tc::umma_commit(&tfull[acc]);
             acc ^= 1;
             if (acc == 0) acc_phase ^= 1;
         }
         // every MMA issued by this thread has finished once `done` flips
-        tc::umma_commit(done);
+        if constexpr (CG == 2) tc::umma_commit_cg2_mc(done, 0x1);
+        else tc::umma_commit(done);
         tc::mbar_wait(done, 0, 3004);
     } else if (warp >= 4) {
         // ---------------- epilogue ----------------
         const int ew = warp - 4;
         int acc = 0;
         uint32_t acc_phase = 0;
-        for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
-            const TileInfo ti = decode_tile(args, tile, BN);
+        const uint32_t tempty_leader0 = (CG == 2) ? tc::map_to_rank(&tempty[0], 0) : 0u;
+        const uint32_t tempty_leader1 = (CG == 2) ? tc::map_to_rank(&tempty[1], 0) : 0u;
+        for (int tile = unit; tile < total; tile += nunits) {
+            const TileInfo ti = decode_tile(args, tile, BN, BMP);
             const bool ok = tc::mbar_wait(&tfull[acc], acc_phase, 3005);
             if (!__all_sync(0xffffffffu, ok)) break;  // the whole warp leaves together
             tc::tc_fence_after();
-            const int r = ew * 32 + lane;
+            const int r = BM * (int)rank + ew * 32 + lane;
             const bool valid = ti.m_local0 + r < ti.group_rows;
             const int row = ti.a_row + r;
 #pragma unroll 1
@@ -449,26 +494,31 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             tc::tc_fence_before();
             __syncwarp();
-            if (lane == 0) tc::mbar_arrive(&tempty[acc]);
+            if (lane == 0) {
+                if constexpr (CG == 2) tc::mbar_arrive_remote(acc ? tempty_leader1 : tempty_leader0);
+                else tc::mbar_arrive(&tempty[acc]);
+            }
             acc ^= 1;
             if (acc == 0) acc_phase ^= 1;
         }
     }
     tc::tc_fence_before();
     __syncthreads();
+    if constexpr (CG == 2) tc::cluster_sync_all();  // the pair is done with TMEM
     if (warp == 1) {
         tc::tc_fence_after();
-        tc::tmem_dealloc(tmem_base, TMEM_COLS);
+        if constexpr (CG == 2) tc::tmem_dealloc_cg2(tmem_base, TMEM_COLS);
+        else tc::tmem_dealloc(tmem_base, TMEM_COLS);
     }
 }
 
-__global__ void tile_prefix_kernel(const int32_t* __restrict__ offsets, int G,
+__global__ void tile_prefix_kernel(const int32_t* __restrict__ offsets, int G, int bm,
                                    int32_t* __restrict__ tile_start) {
     __shared__ int32_t s_warp[32];
     const int g = threadIdx.x;
     const int lane = lane_id(), w = warp_id();
     int v = 0;
-    if (g < G) v = (__ldg(offsets + g + 1) - __ldg(offsets + g) + BM - 1) / BM;
+    if (g < G) v = (__ldg(offsets + g + 1) - __ldg(offsets + g) + bm - 1) / bm;
     int incl = v;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
@@ -535,24 +585,43 @@ static int num_sms() {
 }
 
 // A: a_rows x a_cols row-major (K-major: a_cols = K; MN-major: a_rows = K)
-// B: b_rows x b_cols row-major (likewise)
-template <int BN, int STAGES, int EPI, bool A_MN = false, bool B_MN = false>
+// B: b_rows x b_cols row-major (likewise).  CG = 2 launches clusters of two
+// CTAs (pair tiles of 256 rows).
+template <int BN, int STAGES, int EPI, bool A_MN = false, bool B_MN = false, int CG = 1>
 static int launch(const void* A, uint64_t a_rows, uint64_t a_cols, const void* B, uint64_t b_rows,
                   uint64_t b_cols, const Args& args, int max_tiles, cudaStream_t stream) {
     CUtensorMap ta, tb;
     if (!make_tmap(&ta, A, a_rows, a_cols, A_MN ? 64 : BM)) return BASE_ERR_CUDA;
-    if (!make_tmap(&tb, B, b_rows, b_cols, B_MN ? 64 : BN)) return BASE_ERR_CUDA;
-    constexpr size_t smem = STAGES * (size_t)(BM * BK * 2 + BN * BK * 2) + 1024 + 256;
+    if (!make_tmap(&tb, B, b_rows, b_cols, B_MN ? 64 : BN / CG)) return BASE_ERR_CUDA;
+    constexpr size_t smem = STAGES * (size_t)(BM * BK * 2 + (BN / CG) * BK * 2) + 1024 + 256;
     static_assert(smem <= 227 * 1024, "shared memory");
-    static_assert(!B_MN || BN % 64 == 0, "MN-major B needs BN % 64 == 0");
-    auto kern = gemm_kernel<BN, STAGES, EPI, A_MN, B_MN>;
+    static_assert(!B_MN || (BN / CG) % 64 == 0, "MN-major B needs 64-wide blocks");
+    auto kern = gemm_kernel<BN, STAGES, EPI, A_MN, B_MN, CG>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
         cudaSuccess)
         return BASE_ERR_CUDA;
-    int grid = std::min(num_sms(), std::max(1, max_tiles));
-    kern<<<grid, kThreads, smem, stream>>>(ta, tb, args);
-    BASE_RETURN_IF_LAUNCH_FAILED();
-    return BASE_OK;
+    if constexpr (CG == 1) {
+        const int grid = std::min(num_sms(), std::max(1, max_tiles));
+        kern<<<grid, kThreads, smem, stream>>>(ta, tb, args);
+        BASE_RETURN_IF_LAUNCH_FAILED();
+        return BASE_OK;
+    } else {
+        const int grid = 2 * std::min(num_sms() / 2, std::max(1, max_tiles));
+        cudaLaunchConfig_t cfg = {};
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.gridDim = dim3(grid, 1, 1);
+        cfg.blockDim = dim3(kThreads, 1, 1);
+        cfg.dynamicSmemBytes = smem;
+        cfg.stream = stream;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        if (cudaLaunchKernelEx(&cfg, kern, ta, tb, args) != cudaSuccess) return BASE_ERR_CUDA;
+        return BASE_OK;
+    }
 }
 
 }  // namespace gemm
@@ -594,10 +663,11 @@ int launch_expert_ffn(const void* x_perm, const int32_t* offsets, int T, int D, 
                       const void* W1, const void* W2, int act, const float* gate, void* y_perm,
                       void* h1, void* a1, void* f, void* ws, cudaStream_t stream) {
     using namespace gemm;
+    constexpr int BMP = 2 * BM;  // CTA-pair tiles
     int32_t* tile_start = static_cast<int32_t*>(ws);
-    tile_prefix_kernel<<<1, 1024, 0, stream>>>(offsets, E, tile_start);
+    tile_prefix_kernel<<<1, 1024, 0, stream>>>(offsets, E, BMP, tile_start);
     BASE_RETURN_IF_LAUNCH_FAILED();
-    const int max_mt = (T + BM - 1) / BM + E;
+    const int max_mt = (T + BMP - 1) / BMP + E;
     Args g1{};
     g1.M = T;
     g1.N = F;
@@ -611,8 +681,8 @@ int launch_expert_ffn(const void* x_perm, const int32_t* offsets, int T, int D, 
     g1.act = act;
     g1.out0 = static_cast<__nv_bfloat16*>(h1);
     g1.out1 = static_cast<__nv_bfloat16*>(a1);
-    int st = launch<256, 4, EPI_ACT>(x_perm, T, D, W1, (uint64_t)E * F, D, g1,
-                                     max_mt * g1.n_tiles, stream);
+    int st = launch<256, 6, EPI_ACT, false, false, 2>(x_perm, T, D, W1, (uint64_t)E * F, D, g1,
+                                                      max_mt * g1.n_tiles, stream);
     if (st != BASE_OK) return st;
     Args g2{};
     g2.M = T;
@@ -628,24 +698,25 @@ int launch_expert_ffn(const void* x_perm, const int32_t* offsets, int T, int D, 
     g2.out1 = static_cast<__nv_bfloat16*>(f);
     g2.gate = gate;
     g2.side = static_cast<const __nv_bfloat16*>(x_perm);
-    return launch<256, 4, EPI_GATE>(h1, T, F, W2, (uint64_t)E * D, F, g2, max_mt * g2.n_tiles,
-                                    stream);
+    return launch<256, 6, EPI_GATE, false, false, 2>(h1, T, F, W2, (uint64_t)E * D, F, g2,
+                                                     max_mt * g2.n_tiles, stream);
 }
 
 }  // namespace base
 
 namespace base {
 
-// the four contractions of the backward (see backward.cu)
+// the four contractions of the backward (see backward.cu), on CTA pairs
 int launch_bwd_gemms(const void* dF, const void* /*unused*/, void* dA1, const void* a1,
                      const void* h1, const void* x_perm, const void* dy, const float* ds,
                      const void* w, const int32_t* perm, const int32_t* offsets,
                      int32_t* tile_start, const void* W1, const void* W2, int act, int T, int D,
                      int E, int F, void* dh, float* dW1, float* dW2, cudaStream_t stream) {
     using namespace gemm;
-    tile_prefix_kernel<<<1, 1024, 0, stream>>>(offsets, E, tile_start);
+    constexpr int BMP = 2 * BM;
+    tile_prefix_kernel<<<1, 1024, 0, stream>>>(offsets, E, BMP, tile_start);
     BASE_RETURN_IF_LAUNCH_FAILED();
-    const int max_mt = (T + BM - 1) / BM + E;
+    const int max_mt = (T + BMP - 1) / BMP + E;
     // dH1 = dF W2_e (B = W2_e stored D x F: MN-major), dA1 = dH1 * act'(A1)
     Args g{};
     g.M = T;
@@ -660,8 +731,8 @@ int launch_bwd_gemms(const void* dF, const void* /*unused*/, void* dA1, const vo
     g.act = act;
     g.side = static_cast<const __nv_bfloat16*>(a1);
     g.out0 = static_cast<__nv_bfloat16*>(dA1);
-    int st = launch<256, 4, EPI_DACT, false, true>(dF, T, D, W2, (uint64_t)E * D, F, g,
-                                                   max_mt * g.n_tiles, stream);
+    int st = launch<256, 6, EPI_DACT, false, true, 2>(dF, T, D, W2, (uint64_t)E * D, F, g,
+                                                      max_mt * g.n_tiles, stream);
     if (st != BASE_OK) return st;
     // dx = dA1 W1_e + dy + ds w_e (B = W1_e stored F x D: MN-major) -> dh[perm[r]]
     Args x{};
@@ -679,8 +750,8 @@ int launch_bwd_gemms(const void* dF, const void* /*unused*/, void* dA1, const vo
     x.side2 = static_cast<const __nv_bfloat16*>(w);
     x.idx = perm;
     x.out0 = static_cast<__nv_bfloat16*>(dh);
-    st = launch<256, 4, EPI_DX, false, true>(dA1, T, F, W1, (uint64_t)E * F, D, x,
-                                             max_mt * x.n_tiles, stream);
+    st = launch<256, 6, EPI_DX, false, true, 2>(dA1, T, F, W1, (uint64_t)E * F, D, x,
+                                                max_mt * x.n_tiles, stream);
     if (st != BASE_OK) return st;
     // dW2_e = dF_e^T H1_e: A = dF (T x D, MN-major, M = D), B = H1 (T x F, MN-major, N = F)
     Args w2{};
@@ -690,12 +761,12 @@ int launch_bwd_gemms(const void* dF, const void* /*unused*/, void* dA1, const vo
     w2.groups = E;
     w2.offsets = offsets;
     w2.kgroup = 1;
-    w2.m_tiles = (D + BM - 1) / BM;
+    w2.m_tiles = (D + BMP - 1) / BMP;
     w2.n_tiles = (F + 255) / 256;
     w2.ld = F;
     w2.out_f32 = dW2;
-    st = launch<256, 4, EPI_F32, true, true>(dF, T, D, h1, T, F, w2,
-                                             E * w2.m_tiles * w2.n_tiles, stream);
+    st = launch<256, 6, EPI_F32, true, true, 2>(dF, T, D, h1, T, F, w2,
+                                                E * w2.m_tiles * w2.n_tiles, stream);
     if (st != BASE_OK) return st;
     // dW1_e = dA1_e^T x_e: A = dA1 (T x F, MN-major, M = F), B = x (T x D, MN-major, N = D)
     Args w1{};
@@ -705,12 +776,12 @@ int launch_bwd_gemms(const void* dF, const void* /*unused*/, void* dA1, const vo
     w1.groups = E;
     w1.offsets = offsets;
     w1.kgroup = 1;
-    w1.m_tiles = (F + BM - 1) / BM;
+    w1.m_tiles = (F + BMP - 1) / BMP;
     w1.n_tiles = (D + 255) / 256;
     w1.ld = D;
     w1.out_f32 = dW1;
-    return launch<256, 4, EPI_F32, true, true>(dA1, T, F, x_perm, T, D, w1,
-                                               E * w1.m_tiles * w1.n_tiles, stream);
+    return launch<256, 6, EPI_F32, true, true, 2>(dA1, T, F, x_perm, T, D, w1,
+                                                  E * w1.m_tiles * w1.n_tiles, stream);
 }
 
 }  // namespace base

@@ -42,6 +42,8 @@ def parse():
     p.add_argument("--workload", default="layer_fwd")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--flush-mb", type=int, default=256)
+    p.add_argument("--tokens", type=int, default=0,
+                   help="run the workload with this many tokens instead (profiling a small case)")
     return p.parse_args()
 
 
@@ -179,9 +181,10 @@ def run_reference(args, wl, rank, world):
 
 def _config(wl, args):
     if wl.F:
-        desc = ("%s: BASE layer forward, T=%d tokens, E=%d experts, D=%d, FFN %d->%d->%d %s, "
-                "balanced auction routing, bf16" % (wl.name, wl.T, wl.E, wl.D, wl.D, wl.F, wl.D,
-                                                     wl.act))
+        desc = ("%s: BASE layer %s, T=%d tokens, E=%d experts, D=%d, FFN %d->%d->%d %s, "
+                "balanced auction routing, bf16" % (wl.name, "forward+backward" if wl.backward
+                                                     else "forward", wl.T, wl.E, wl.D, wl.D, wl.F,
+                                                     wl.D, wl.act))
     else:
         desc = ("%s: scores + balanced auction + greedy + permute, T=%d tokens, E=%d experts, "
                 "D=%d, bf16%s" % (wl.name, wl.T, wl.E, wl.D,
@@ -197,6 +200,8 @@ def main():
     args = parse()
     from balanced_token_expert_b200 import synth
     wl = synth.WORKLOADS[args.workload]
+    if args.tokens:
+        wl = wl.scaled(T=args.tokens)
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
@@ -227,7 +232,7 @@ def main():
     W1 = inp.W1.cuda() if F else None
     W2 = inp.W2.cuda() if F else None
     act = B.BASE_RELU if wl.act == "relu" else B.BASE_GELU
-    sv = buffers.layer_saved(T, E, D, max(F, 8), for_backward=False)
+    sv = buffers.layer_saved(T, E, D, max(F, 8), for_backward=wl.backward)
     out = torch.empty(T, D, dtype=torch.bfloat16, device="cuda")
     ws = buffers.workspace(T, E, D, F)
     flush = torch.empty(args.flush_mb * (1 << 20), dtype=torch.uint8, device="cuda")
@@ -253,9 +258,17 @@ def main():
                                                      sv["gate"], ws), 4))
     if F:
         comps.append(("ffn", lambda: B.base_expert_ffn(sv["x_perm"], sv["offsets"], W1, W2, act,
-                                                       sv["gate"], sv["y_perm"], sv["h1"], None,
-                                                       None, ws), 3))
+                                                       sv["gate"], sv["y_perm"], sv["h1"],
+                                                       sv.get("a1"), sv.get("f"), ws), 3))
         comps.append(("combine", lambda: B.base_combine(sv["y_perm"], sv["perm"], out), 1))
+    if wl.backward:
+        dout = inp.dout.cuda()
+        dh = torch.empty(T, D, dtype=torch.bfloat16, device="cuda")
+        dw = torch.empty(E, D, device="cuda")
+        dW1 = torch.empty(E, F, D, device="cuda")
+        dW2 = torch.empty(E, D, F, device="cuda")
+        comps.append(("backward", lambda: B.base_layer_bwd(h, w, W1, W2, act, sv, dout, dh, dw,
+                                                           dW1, dW2, ws), 8))
     names = [n for n, _, _ in comps if n != "bump"]
 
     def step(ev):
@@ -373,7 +386,8 @@ def main():
             permute=("hbm", 4 * T * D + 12 * T + 8 * T),
             ffn=("tensor", 4 * T * D * F),
             combine=("hbm", 4 * T * D + 4 * T),
-            greedy=("hbm", 4 * T * E + 4 * T))
+            greedy=("hbm", 4 * T * E + 4 * T),
+            backward=("tensor", 8 * T * D * F))
 
         def roof(n):
             bound, work = alg[n]
