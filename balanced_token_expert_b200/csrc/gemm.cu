@@ -10,10 +10,11 @@
 //               STAGES shared-memory stages (128-byte swizzle),
 //   warp 1      allocates TMEM (two BN-column fp32 accumulators) and one lane
 //               issues tcgen05.mma (M=128, N=BN, K=16) per 16-wide K slice,
-//   warps 4..7  the epilogue: tcgen05.ld of the accumulator (warp w reads
-//               TMEM lanes 32 (w%4) ..), the fused element-wise work and
-//               16-byte stores; the two accumulators let the epilogue of one
-//               tile overlap the MMAs of the next.
+//   warps 4..11 the epilogue: tcgen05.ld of the accumulator (warp w reads
+//               TMEM lanes 32 (w%4) .., two warps per lane quadrant split the
+//               columns), the fused element-wise work and 16-byte stores; the
+//               two accumulators let the epilogue of one tile overlap the MMAs
+//               of the next.
 // Operands may also be MN-major (A stored K x M, B stored K x N, M/N
 // contiguous), read as 64 x 64 TMA boxes and described to the tensor core as
 // MN-major 128-byte-swizzled tiles; the backward uses this to multiply by
@@ -35,7 +36,10 @@ namespace gemm {
 
 constexpr int BM = 128;
 constexpr int BK = 64;
-constexpr int kThreads = 256;
+// warp 0: TMA, warp 1: MMA, warps 2-3: idle, warps 4..: epilogue, two per
+// TMEM lane quadrant (warp w reads lanes 32 (w % 4) ..), each half the columns
+constexpr int kEpiWarps = 8;
+constexpr int kThreads = 128 + 32 * kEpiWarps;
 
 enum Epi : int {
     EPI_SCORES = 0,  // s (fp32) and q = rint(s 2^16) (int32)
@@ -284,6 +288,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const Args args) {
     static_assert(CG == 1 || CG == 2, "one CTA or a CTA pair");
+    static_assert(BN % 16 == 0 && kEpiWarps == 8, "16-column chunks over two column halves");
     constexpr int BNC = BN / CG;  // rows of B loaded by one CTA
     constexpr int BMP = BM * CG;  // rows of A per tile
     constexpr uint32_t A_BYTES = BM * BK * 2;
@@ -313,7 +318,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int i = 0; i < 2; ++i) {
             tc::mbar_init(&tfull[i], 1);
-            tc::mbar_init(&tempty[i], 4 * CG);
+            tc::mbar_init(&tempty[i], kEpiWarps * CG);
         }
         tc::mbar_init(done, 1);
         tc::fence_mbar_init();
@@ -468,7 +473,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc::mbar_wait(done, 0, 3004);
     } else if (warp >= 4) {
         // ---------------- epilogue ----------------
-        const int ew = warp - 4;
+        const int ew = (warp - 4) & 3;                   // lane quadrant
+        const int half = (warp - 4) >> 2;                // column half
+        constexpr int kChunks = BN / 16;                 // 16-column chunks per row
+        constexpr int kPerHalf = (kChunks + 1) / 2;      // the second half may be empty
+        const int c_begin = 16 * min(kChunks, half * kPerHalf);
+        const int c_end = 16 * min(kChunks, (half + 1) * kPerHalf);
         int acc = 0;
         uint32_t acc_phase = 0;
         const uint32_t tempty_leader0 = (CG == 2) ? tc::map_to_rank(&tempty[0], 0) : 0u;
@@ -482,7 +492,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const bool valid = ti.m_local0 + r < ti.group_rows;
             const int row = ti.a_row + r;
 #pragma unroll 1
-            for (int c0 = 0; c0 < BN; c0 += 16) {
+            for (int c0 = c_begin; c0 < c_end; c0 += 16) {
                 uint32_t v[16];
                 tc::tmem_ld16(tmem_base + ((uint32_t)(ew * 32) << 16) + acc * BN + c0, v);
                 tc::tmem_wait_ld();
