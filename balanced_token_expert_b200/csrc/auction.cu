@@ -1027,6 +1027,152 @@ __device__ bool resolve_warp(const Params& p, Key* fr, int& fs, int& h, const in
     return true;
 }
 
+// The end of a phase.  Once a round has a single bidder, so has every
+// following round: its one bid either goes to an expert with room (the phase
+// ends) or to a full expert, which then rejects exactly its worst held key
+// (every bid is above the expert's price, the smallest held bid).  One warp
+// runs these rounds back to back with no block barrier: lanes take experts
+// (lane + 32 j, j < NJ) for the bid, the expert's fringe decides the round,
+// and the rejected token's score row is loaded into registers while the
+// resolve is written back.  The rounds are the same as in the other modes.
+struct ChainScratch {
+    int64_t* one_b;   // [1] the bid, for resolve_warp
+    int32_t* one_t;   // [1]
+    int32_t* next;    // [1] a rejected token
+    int32_t* cnt;     // [1]
+};
+
+template <int NJ>
+__device__ __forceinline__ void chain_rounds(const Params& p, int t, int64_t eps, int64_t scale,
+                                          int64_t* s_price, Key* s_fr, int32_t* s_fsize,
+                                          int32_t* s_hcnt, const ChainScratch cs,
+                                          const Team<32>& wt, long long& rounds,
+                                          long long& bids, int& status) {
+    const int E = p.E, C = p.C, FK = p.FK, T = p.T;
+    const int lane = lane_id();
+    int32_t rv[NJ];
+#pragma unroll
+    for (int j = 0; j < NJ; ++j) {
+        const int e = lane + 32 * j;
+        rv[j] = e < E ? __ldg(p.q + (size_t)t * E + e) : 0;
+    }
+    while (true) {
+        if (rounds >= p.max_rounds) {
+            status = BASE_ERR_NOT_CONVERGED;
+            return;
+        }
+        if (lane == 0) trace_round(p, rounds, 1);
+        ++rounds;
+        ++bids;
+        // ---- bid: best and second-best value over the experts, lowest e on ties
+        int64_t v1 = INT64_MIN, v2 = INT64_MIN;
+        int e1 = INT32_MAX;
+#pragma unroll
+        for (int j = 0; j < NJ; ++j) {
+            const int e = lane + 32 * j;
+            if (e < E) {
+                const int64_t v = (int64_t)rv[j] * scale - s_price[e];
+                if (v > v1) {
+                    v2 = v1;
+                    v1 = v;
+                    e1 = e;
+                } else if (v > v2) {
+                    v2 = v;
+                }
+            }
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            const int64_t ov1 = __shfl_xor_sync(0xffffffffu, v1, off);
+            const int64_t ov2 = __shfl_xor_sync(0xffffffffu, v2, off);
+            const int oe1 = __shfl_xor_sync(0xffffffffu, e1, off);
+            if (ov1 > v1 || (ov1 == v1 && oe1 < e1)) {
+                v2 = max(v1, ov2);
+                v1 = ov1;
+                e1 = oe1;
+            } else {
+                v2 = max(v2, ov1);
+            }
+        }
+        const int e = e1;
+        // bid = q[t][e] (T+1) - v2 + eps = price[e] + (v1 - v2) + eps
+        const int64_t bid = v1 + s_price[e] - v2 + eps;
+        const int h = s_hcnt[e];
+        const int fs = s_fsize[e];
+        Key* fr = s_fr + (size_t)e * FK;
+        int64_t* hb = p.hb + (size_t)e * C;
+        int32_t* ht = p.ht + (size_t)e * C;
+        int tn = -1;
+        if (h == C && fs >= 2) {
+            // the fringe minimum f0 is rejected, the bid takes its slot
+            const Key f0 = fr[0];
+            tn = f0.tok;
+#pragma unroll
+            for (int j = 0; j < NJ; ++j) {
+                const int ee = lane + 32 * j;
+                rv[j] = ee < E ? __ldg(p.q + (size_t)tn * E + ee) : 0;
+            }
+            const Key f1 = fr[1];
+            const Key fl = fr[fs - 1];
+            const Key fi = lane < fs ? fr[lane] : pad_key();
+            const Key fn = lane + 1 < fs ? fr[lane + 1] : pad_key();
+            const Key b = Key{bid, t, f0.slot};
+            const bool ins = fs == h || !worse(fl, b);
+            const int pos = __popc(__ballot_sync(0xffffffffu, lane + 1 < fs && worse(fn, b)));
+            Key out = lane < pos ? fn : (lane == pos ? b : fi);
+            if (!ins) out = fn;
+            const int nfs = ins ? fs : fs - 1;
+            const int64_t price = (ins && pos == 0) ? bid : f1.bid;
+            __syncwarp();
+            if (lane < nfs) fr[lane] = out;
+            if (lane == 0) {
+                hb[b.slot] = bid;
+                ht[b.slot] = t;
+                s_fsize[e] = nfs;
+                s_price[e] = price;
+            }
+            __syncwarp();
+        } else {
+            // the general merge (a fringe that must be rebuilt first, an
+            // expert with room, a fringe of one key)
+            if (lane == 0) {
+                cs.one_b[0] = bid;
+                cs.one_t[0] = t;
+                cs.cnt[0] = 0;
+            }
+            __syncwarp();
+            int fs2 = fs, hh = h;
+            int64_t price = s_price[e];
+            if (fs2 != hh && max(0, hh + 1 - C) >= fs2)
+                fs2 = build_fringe<32>(wt, hb, ht, hh, FK, T - 1, fr);
+            resolve_warp(p, fr, fs2, hh, cs.one_b, cs.one_t, 1, hb, ht, cs.next, cs.cnt, price,
+                         RowStage{nullptr, 0});
+            if (hh == C && fs2 == 0) {
+                fs2 = build_fringe<32>(wt, hb, ht, hh, FK, T - 1, fr);
+                price = fr[0].bid;
+            }
+            __syncwarp();
+            if (lane == 0) {
+                s_fsize[e] = fs2;
+                s_hcnt[e] = hh;
+                if (hh == C) s_price[e] = price;
+            }
+            const int n = cs.cnt[0];
+            if (n > 0) {
+                tn = cs.next[0];
+#pragma unroll
+                for (int j = 0; j < NJ; ++j) {
+                    const int ee = lane + 32 * j;
+                    rv[j] = ee < E ? __ldg(p.q + (size_t)tn * E + ee) : 0;
+                }
+            }
+            __syncwarp();
+        }
+        if (tn < 0) return;  // the bid found room: the phase is over
+        t = tn;
+    }
+}
+
 __global__ void __launch_bounds__(kThreads, 1) auction_kernel(const __grid_constant__ Params p) {
     extern __shared__ __align__(16) unsigned char smem[];
     const SmemLayout L = smem_layout(p.E, p.FK, p.narrow_max, p.NB, p.RC);
@@ -1250,6 +1396,35 @@ __global__ void __launch_bounds__(kThreads, 1) auction_kernel(const __grid_const
                 if (threadIdx.x < 5) s_misc[4 + (threadIdx.x < 2 ? threadIdx.x : threadIdx.x + 2)] = 0;
                 __syncthreads();
                 while (U > 0) {
+                    if (U == 1 && E <= 128) {
+                        // one bidder: warp 0 ends the phase alone
+                        long long* s_ll = reinterpret_cast<long long*>(s_misc + 12);
+                        if (warp == 0) {
+                            const int t0 = (lc ? s_list1 : s_list0)[0];
+                            // scratch: the bid buckets are free between rounds
+                            const ChainScratch cs{s_nbk_b, s_nbk_t, s_nbk_t + 1, s_misc + 2};
+                            if (E <= 32)
+                                chain_rounds<1>(p, t0, eps, scale, s_price, s_fr, s_fsize, s_hcnt,
+                                                cs, warp_team, rounds, bids, status);
+                            else if (E <= 64)
+                                chain_rounds<2>(p, t0, eps, scale, s_price, s_fr, s_fsize, s_hcnt,
+                                                cs, warp_team, rounds, bids, status);
+                            else
+                                chain_rounds<4>(p, t0, eps, scale, s_price, s_fr, s_fsize, s_hcnt,
+                                                cs, warp_team, rounds, bids, status);
+                            if (lane == 0) {
+                                s_ll[0] = rounds;
+                                s_ll[1] = bids;
+                                s_misc[1] = status;
+                            }
+                        }
+                        __syncthreads();
+                        rounds = s_ll[0];
+                        bids = s_ll[1];
+                        status = s_misc[1];
+                        U = 0;
+                        break;
+                    }
                     if (rounds >= p.max_rounds) {
                         status = BASE_ERR_NOT_CONVERGED;
                         break;
