@@ -27,6 +27,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <cstring>
 #include <mutex>
 
 #include "tc.cuh"
@@ -71,6 +72,7 @@ struct Args {
     const int32_t* idx;          // destination rows (EPI_DX)
     int kgroup;                  // 1: groups split K (weight gradients), M and N fixed
     int m_tiles;                 // K-grouped mode: tiles along M per group
+    int staged;                  // set by the launcher: output tensor maps are valid
 };
 
 struct TileInfo {
@@ -278,6 +280,64 @@ __device__ __forceinline__ void epilogue16(const Args& a, const TileInfo& ti, in
     }
 }
 
+// The epilogues whose output rows are contiguous (h1 / a1, y / f, dA1, dW)
+// stage each warp's 32 rows x 128 bytes of output in shared memory and write
+// them with one TMA store: 128-byte line writes instead of 16-byte pieces of
+// 32 different rows per instruction.
+template <int EPI>
+constexpr bool kStagedEpi = EPI == EPI_ACT || EPI == EPI_GATE || EPI == EPI_DACT || EPI == EPI_F32;
+constexpr uint32_t kStageBuf = 32 * 128;  // one warp's 32 rows x 128 bytes
+constexpr int kStageSlots = 2;            // per epilogue warp
+
+// the 16 output values of pass 0 (out0 / out_f32) or pass 1 (out1: the raw
+// accumulator) for columns [col, col + 16) of one row
+template <int EPI>
+__device__ __forceinline__ void epi_values16(const Args& a, int row, int col, int pass,
+                                             const uint32_t (&v)[16], float (&o)[16]) {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) o[i] = __uint_as_float(v[i]);
+    if (pass == 1) return;
+    const size_t base = (size_t)row * a.ld + col;
+    if constexpr (EPI == EPI_ACT) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) o[i] = act_fwd(o[i], a.act);
+    } else if constexpr (EPI == EPI_GATE) {
+        const float g = __ldg(a.gate + row);
+        const float sg = 1.f / (1.f + expf(-g));
+        float x[16];
+        load_bf16x16(a.side + base, x);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) o[i] = fmaf(sg, o[i], x[i]);
+    } else if constexpr (EPI == EPI_DACT) {
+        float x[16];
+        load_bf16x16(a.side + base, x);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) o[i] *= act_grad(x[i], a.act);
+    }
+}
+
+// row `lane` of a 32 x 128-byte staging buffer in the TMA 128-byte swizzle
+// (16-byte unit u of row r sits at unit u ^ (r % 8)); c = first column
+template <bool F32OUT>
+__device__ __forceinline__ void stage16(uint8_t* buf, int lane, int c, const float (&o)[16]) {
+    uint4* rowp = reinterpret_cast<uint4*>(buf + lane * 128);
+    const int sw = lane & 7;
+    if constexpr (F32OUT) {
+        const int u0 = c >> 2;
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            rowp[(u0 + i) ^ sw] = make_uint4(__float_as_uint(o[4 * i]), __float_as_uint(o[4 * i + 1]),
+                                             __float_as_uint(o[4 * i + 2]),
+                                             __float_as_uint(o[4 * i + 3]));
+    } else {
+        const int u0 = c >> 3;
+        rowp[u0 ^ sw] = make_uint4(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]),
+                                   pack_bf16x2(o[4], o[5]), pack_bf16x2(o[6], o[7]));
+        rowp[(u0 + 1) ^ sw] = make_uint4(pack_bf16x2(o[8], o[9]), pack_bf16x2(o[10], o[11]),
+                                         pack_bf16x2(o[12], o[13]), pack_bf16x2(o[14], o[15]));
+    }
+}
+
 // CG = 2: a CTA pair of a cluster computes a (2 x 128) x BN tile with
 // tcgen05.mma.cta_group::2: each CTA loads its own 128 rows of A and BN/2 rows
 // of B (the TMA completions of both land on the leader's barrier), the leader
@@ -286,6 +346,7 @@ __device__ __forceinline__ void epilogue16(const Args& a, const TileInfo& ti, in
 template <int BN, int STAGES, int EPI, bool A_MN, bool B_MN, int CG = 1>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                const __grid_constant__ CUtensorMap tmO0, const __grid_constant__ CUtensorMap tmO1,
                 const Args args) {
     static_assert(CG == 1 || CG == 2, "one CTA or a CTA pair");
     static_assert(BN % 16 == 0 && kEpiWarps == 8, "16-column chunks over two column halves");
@@ -297,9 +358,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~uintptr_t(1023));
+    constexpr bool kStaged = kStagedEpi<EPI>;
+    constexpr uint32_t STAGE_AREA = kStaged ? kEpiWarps * kStageSlots * kStageBuf : 0;
     uint8_t* sA = smem;
     uint8_t* sB = smem + STAGES * A_BYTES;
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * (A_BYTES + B_BYTES));
+    uint8_t* sOut = smem + STAGES * (A_BYTES + B_BYTES);  // 1024-byte aligned
+    uint64_t* full = reinterpret_cast<uint64_t*>(sOut + STAGE_AREA);
     uint64_t* empty = full + STAGES;
     uint64_t* tfull = empty + STAGES;
     uint64_t* tempty = tfull + 2;
@@ -481,6 +545,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int c_end = 16 * min(kChunks, (half + 1) * kPerHalf);
         int acc = 0;
         uint32_t acc_phase = 0;
+        int slot = 0;
         const uint32_t tempty_leader0 = (CG == 2) ? tc::map_to_rank(&tempty[0], 0) : 0u;
         const uint32_t tempty_leader1 = (CG == 2) ? tc::map_to_rank(&tempty[1], 0) : 0u;
         for (int tile = unit; tile < total; tile += nunits) {
@@ -491,16 +556,56 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int r = BM * (int)rank + ew * 32 + lane;
             const bool valid = ti.m_local0 + r < ti.group_rows;
             const int row = ti.a_row + r;
+            const uint32_t tbase = tmem_base + ((uint32_t)(ew * 32) << 16) + acc * BN;
+            // staged when the warp's 32 rows all belong to the tile's group
+            if (kStaged && args.staged && __all_sync(0xffffffffu, valid)) {
+                constexpr int GC = (EPI == EPI_F32) ? 32 : 64;  // columns per 128-byte row piece
+                // the warp's first row in the output tensor (dW: group blocks stacked)
+                const int orow = (EPI == EPI_F32 ? ti.group * args.M : 0) + ti.a_row +
+                                 BM * (int)rank + ew * 32;
+                const int npass = (EPI != EPI_F32 && EPI != EPI_DACT && args.out1) ? 2 : 1;
 #pragma unroll 1
-            for (int c0 = c_begin; c0 < c_end; c0 += 16) {
-                uint32_t v[16];
-                tc::tmem_ld16(tmem_base + ((uint32_t)(ew * 32) << 16) + acc * BN + c0, v);
-                tc::tmem_wait_ld();
-                if (ti.kblocks == 0) {
+                for (int gc = c_begin; gc < c_end && ti.n0 + gc < args.N; gc += GC) {
+#pragma unroll 1
+                    for (int pass = 0; pass < npass; ++pass) {
+                        uint8_t* buf = sOut + ((warp - 4) * kStageSlots + slot) * kStageBuf;
+                        // the store issued from this slot two pieces ago has read it
+                        if (lane == 0) tc::bulk_wait_read<kStageSlots - 1>();
+                        __syncwarp();
+#pragma unroll 1
+                        for (int c = 0; c < GC; c += 16) {
+                            uint32_t v[16];
+                            tc::tmem_ld16(tbase + gc + c, v);
+                            tc::tmem_wait_ld();
+                            if (ti.kblocks == 0) {
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) v[i] = 0u;
+                                for (int i = 0; i < 16; ++i) v[i] = 0u;
+                            }
+                            float o[16];
+                            epi_values16<EPI>(args, row, ti.n0 + gc + c, pass, v, o);
+                            stage16<EPI == EPI_F32>(buf, lane, c, o);
+                        }
+                        tc::fence_proxy_async_smem();
+                        __syncwarp();
+                        if (lane == 0) {
+                            tc::tma_store_2d(pass ? &tmO1 : &tmO0, buf, ti.n0 + gc, orow);
+                            tc::bulk_commit();
+                        }
+                        slot = (slot + 1) % kStageSlots;
+                    }
                 }
-                if (valid && ti.n0 + c0 < args.N) epilogue16<EPI>(args, ti, row, ti.n0 + c0, v);
+            } else {
+#pragma unroll 1
+                for (int c0 = c_begin; c0 < c_end; c0 += 16) {
+                    uint32_t v[16];
+                    tc::tmem_ld16(tbase + c0, v);
+                    tc::tmem_wait_ld();
+                    if (ti.kblocks == 0) {
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) v[i] = 0u;
+                    }
+                    if (valid && ti.n0 + c0 < args.N) epilogue16<EPI>(args, ti, row, ti.n0 + c0, v);
+                }
             }
             tc::tc_fence_before();
             __syncwarp();
@@ -511,6 +616,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             acc ^= 1;
             if (acc == 0) acc_phase ^= 1;
         }
+        // the staged stores have landed before the CTA (and its shared memory) goes
+        if (kStaged && lane == 0) tc::bulk_wait_all();
     }
     tc::tc_fence_before();
     __syncthreads();
@@ -583,6 +690,23 @@ static bool make_tmap(CUtensorMap* m, const void* base, uint64_t rows, uint64_t 
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// output tensor [rows][cols] with row stride ld elements (bf16 or fp32), box =
+// 32 rows x 128 bytes, 128 B swizzle: one epilogue warp's staged piece
+static bool make_tmap_out(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
+                          uint64_t ld, bool f32) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    const uint64_t es = f32 ? 4 : 2;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {ld * es};
+    cuuint32_t box[2] = {(cuuint32_t)(128 / es), 32};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+              const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 static int num_sms() {
     static int n = 0;
     if (n == 0) {
@@ -600,10 +724,30 @@ static int num_sms() {
 template <int BN, int STAGES, int EPI, bool A_MN = false, bool B_MN = false, int CG = 1>
 static int launch(const void* A, uint64_t a_rows, uint64_t a_cols, const void* B, uint64_t b_rows,
                   uint64_t b_cols, const Args& args, int max_tiles, cudaStream_t stream) {
-    CUtensorMap ta, tb;
+    CUtensorMap ta, tb, to0, to1;
     if (!make_tmap(&ta, A, a_rows, a_cols, A_MN ? 64 : BM)) return BASE_ERR_CUDA;
     if (!make_tmap(&tb, B, b_rows, b_cols, B_MN ? 64 : BN / CG)) return BASE_ERR_CUDA;
-    constexpr size_t smem = STAGES * (size_t)(BM * BK * 2 + (BN / CG) * BK * 2) + 1024 + 256;
+    memset(&to0, 0, sizeof(to0));
+    memset(&to1, 0, sizeof(to1));
+    Args a = args;
+    a.staged = 0;
+    // whole 128-byte row pieces and 16-byte aligned rows
+    const bool stageable = EPI == EPI_F32 ? (args.N % 32 == 0) : (args.N % 64 == 0 && args.ld % 8 == 0);
+    if (kStagedEpi<EPI> && stageable) {
+        a.staged = 1;
+        // dW: the groups' M x N blocks stacked; otherwise M x N with row stride ld
+        if (EPI == EPI_F32) {
+            if (!make_tmap_out(&to0, args.out_f32, (uint64_t)args.groups * args.M, args.N, args.N,
+                               true))
+                return BASE_ERR_CUDA;
+        } else {
+            if (!make_tmap_out(&to0, args.out0, args.M, args.N, args.ld, false)) return BASE_ERR_CUDA;
+            if (args.out1 && !make_tmap_out(&to1, args.out1, args.M, args.N, args.ld, false))
+                return BASE_ERR_CUDA;
+        }
+    }
+    constexpr size_t smem = STAGES * (size_t)(BM * BK * 2 + (BN / CG) * BK * 2) +
+                            (kStagedEpi<EPI> ? kEpiWarps * kStageSlots * kStageBuf : 0) + 1024 + 256;
     static_assert(smem <= 227 * 1024, "shared memory");
     static_assert(!B_MN || (BN / CG) % 64 == 0, "MN-major B needs 64-wide blocks");
     auto kern = gemm_kernel<BN, STAGES, EPI, A_MN, B_MN, CG>;
@@ -612,7 +756,7 @@ static int launch(const void* A, uint64_t a_rows, uint64_t a_cols, const void* B
         return BASE_ERR_CUDA;
     if constexpr (CG == 1) {
         const int grid = std::min(num_sms(), std::max(1, max_tiles));
-        kern<<<grid, kThreads, smem, stream>>>(ta, tb, args);
+        kern<<<grid, kThreads, smem, stream>>>(ta, tb, to0, to1, a);
         BASE_RETURN_IF_LAUNCH_FAILED();
         return BASE_OK;
     } else {
@@ -629,7 +773,8 @@ static int launch(const void* A, uint64_t a_rows, uint64_t a_cols, const void* B
         cfg.stream = stream;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
-        if (cudaLaunchKernelEx(&cfg, kern, ta, tb, args) != cudaSuccess) return BASE_ERR_CUDA;
+        if (cudaLaunchKernelEx(&cfg, kern, ta, tb, to0, to1, a) != cudaSuccess)
+            return BASE_ERR_CUDA;
         return BASE_OK;
     }
 }
@@ -691,7 +836,7 @@ int launch_expert_ffn(const void* x_perm, const int32_t* offsets, int T, int D, 
     g1.act = act;
     g1.out0 = static_cast<__nv_bfloat16*>(h1);
     g1.out1 = static_cast<__nv_bfloat16*>(a1);
-    int st = launch<256, 6, EPI_ACT, false, false, 2>(x_perm, T, D, W1, (uint64_t)E * F, D, g1,
+    int st = launch<256, 5, EPI_ACT, false, false, 2>(x_perm, T, D, W1, (uint64_t)E * F, D, g1,
                                                       max_mt * g1.n_tiles, stream);
     if (st != BASE_OK) return st;
     Args g2{};
@@ -708,7 +853,7 @@ int launch_expert_ffn(const void* x_perm, const int32_t* offsets, int T, int D, 
     g2.out1 = static_cast<__nv_bfloat16*>(f);
     g2.gate = gate;
     g2.side = static_cast<const __nv_bfloat16*>(x_perm);
-    return launch<256, 6, EPI_GATE, false, false, 2>(h1, T, F, W2, (uint64_t)E * D, F, g2,
+    return launch<256, 5, EPI_GATE, false, false, 2>(h1, T, F, W2, (uint64_t)E * D, F, g2,
                                                      max_mt * g2.n_tiles, stream);
 }
 
@@ -741,7 +886,7 @@ int launch_bwd_gemms(const void* dF, const void* /*unused*/, void* dA1, const vo
     g.act = act;
     g.side = static_cast<const __nv_bfloat16*>(a1);
     g.out0 = static_cast<__nv_bfloat16*>(dA1);
-    int st = launch<256, 6, EPI_DACT, false, true, 2>(dF, T, D, W2, (uint64_t)E * D, F, g,
+    int st = launch<256, 5, EPI_DACT, false, true, 2>(dF, T, D, W2, (uint64_t)E * D, F, g,
                                                       max_mt * g.n_tiles, stream);
     if (st != BASE_OK) return st;
     // dx = dA1 W1_e + dy + ds w_e (B = W1_e stored F x D: MN-major) -> dh[perm[r]]
@@ -775,7 +920,7 @@ int launch_bwd_gemms(const void* dF, const void* /*unused*/, void* dA1, const vo
     w2.n_tiles = (F + 255) / 256;
     w2.ld = F;
     w2.out_f32 = dW2;
-    st = launch<256, 6, EPI_F32, true, true, 2>(dF, T, D, h1, T, F, w2,
+    st = launch<256, 5, EPI_F32, true, true, 2>(dF, T, D, h1, T, F, w2,
                                                 E * w2.m_tiles * w2.n_tiles, stream);
     if (st != BASE_OK) return st;
     // dW1_e = dA1_e^T x_e: A = dA1 (T x F, MN-major, M = F), B = x (T x D, MN-major, N = D)
@@ -790,7 +935,7 @@ int launch_bwd_gemms(const void* dF, const void* /*unused*/, void* dA1, const vo
     w1.n_tiles = (D + 255) / 256;
     w1.ld = D;
     w1.out_f32 = dW1;
-    return launch<256, 6, EPI_F32, true, true, 2>(dA1, T, F, x_perm, T, D, w1,
+    return launch<256, 5, EPI_F32, true, true, 2>(dA1, T, F, x_perm, T, D, w1,
                                                   E * w1.m_tiles * w1.n_tiles, stream);
 }
 
