@@ -41,7 +41,11 @@ constexpr int kWarps = kThreads / kWarp;
 constexpr int kHist = 256;
 constexpr int kEpsDivisor = 50;  // eps0 = (max q - min q)(T+1) / 50
 constexpr int kEpsFactor = 8;    // eps <- eps / 8 per phase
-constexpr int kNarrowMax = 256;  // rounds with at most this many bidders run on CTA 0
+// Rounds with at most this many bidders run on CTA 0: with few experts a
+// narrow round stays cheaper than a grid-wide one up to a few hundred
+// bidders; with 32 or more experts its resolves (several bids per expert,
+// fringe rebuilds) outgrow a wide round beyond about 32 bidders.
+__host__ __device__ constexpr int narrow_max_for(int E) { return E <= 16 ? 256 : 32; }
 constexpr uint64_t kWaitNs = 20000000000ull;  // grid-barrier wait limit (20 s)
 
 // ---------------------------------------------------------------- keys
@@ -449,8 +453,6 @@ __device__ Key kth_worst(const Team<TEAM>& tm, const Cands& cd, int k, int tmax)
 
 // ---------------------------------------------------------------- state
 struct Ctrl {
-    unsigned bar_count;
-    unsigned bar_gen;
     int abort;
     int ucount[3];
     int pad[2];
@@ -459,6 +461,7 @@ struct Ctrl {
 struct Params {
     const int32_t* q;
     int T, E, C, FK, NB, RC;
+    int HS;  // 1: CTA 0 keeps the held sets in shared memory during narrow rounds
     long long max_rounds;
     int narrow_max;
     int32_t* assign;
@@ -466,6 +469,7 @@ struct Params {
     base_auction_stats* stats;
     const int32_t* minmax;
     Ctrl* ctrl;
+    unsigned* bar_flags;  // [gridDim.x] grid-barrier counts
     int64_t* gprice;   // [E]
     int32_t* hcnt;     // [E]
     int64_t* hb;       // [E][C]
@@ -496,29 +500,24 @@ __device__ __forceinline__ void trace_round(const Params& p, long long r, int U)
 // shared memory of every CTA (narrow-mode arrays are used by CTA 0 only)
 struct SmemLayout {
     size_t price, fr, fsize, hcnt, ncnt, act0, act1, nbk_b, nbk_t, list0, list1, rows, wb, wt, we,
-        wp, hist, red, cnt, misc, total;
+        wp, hist, red, cnt, misc, hb, ht, scratch, total;
 };
 
 constexpr int kWideChunk = 1024;  // bids a CTA stages before reserving bucket space
+constexpr int kMaxGrid = 1024;    // CTAs of the cooperative grid (one per SM)
 
 // NB: new bids per expert kept in shared memory (the rest in the global
 // bucket); RC: bidders' score rows staged in shared memory per round parity.
-__host__ __device__ inline SmemLayout smem_layout(int E, int FK, int NM, int NB, int RC) {
+// HS: the held sets (E x C = T keys) in shared memory too.
+__host__ __device__ inline SmemLayout smem_layout(int E, int FK, int NM, int NB, int RC, int T = 0,
+                                                  int HS = 0) {
     SmemLayout L;
     size_t o = 0;
     auto take = [&](size_t bytes) { size_t r = o; o += align_up(bytes, 16); return r; };
+    // used by every CTA in wide rounds
     L.price = take(8 * (size_t)E);
-    L.fr = take(sizeof(Key) * (size_t)E * FK);
-    L.fsize = take(4 * (size_t)E);
-    L.hcnt = take(4 * (size_t)E);
     L.ncnt = take(4 * (size_t)E);
     L.act0 = take(4 * (size_t)E);
-    L.act1 = take(4 * (size_t)E);
-    L.nbk_b = take(8 * (size_t)E * NB);
-    L.nbk_t = take(4 * (size_t)E * NB);
-    L.list0 = take(4 * (size_t)NM);
-    L.list1 = take(4 * (size_t)NM);
-    L.rows = take(2 * 4 * (size_t)RC * E);
     L.wb = take(8 * (size_t)kWideChunk);
     L.wt = take(4 * (size_t)kWideChunk);
     L.we = take(4 * (size_t)kWideChunk);
@@ -527,6 +526,19 @@ __host__ __device__ inline SmemLayout smem_layout(int E, int FK, int NM, int NB,
     L.red = take(8 * 32);
     L.cnt = take(4 * 64);
     L.misc = take(64);
+    // narrow rounds (CTA 0) only; in wide rounds the scratch of the resolve
+    L.scratch = o;
+    L.fr = take(sizeof(Key) * (size_t)E * FK);
+    L.fsize = take(4 * (size_t)E);
+    L.hcnt = take(4 * (size_t)E);
+    L.act1 = take(4 * (size_t)E);
+    L.nbk_b = take(8 * (size_t)E * NB);
+    L.nbk_t = take(4 * (size_t)E * NB);
+    L.list0 = take(4 * (size_t)NM);
+    L.list1 = take(4 * (size_t)NM);
+    L.rows = take(2 * 4 * (size_t)RC * E);
+    L.hb = take(HS ? 8 * (size_t)T : 0);
+    L.ht = take(HS ? 4 * (size_t)T : 0);
     L.total = o;
     return L;
 }
@@ -537,45 +549,49 @@ __device__ __forceinline__ uint64_t globaltimer() {
     return t;
 }
 
-// Grid barrier (all CTAs are co-resident: cooperative launch).  Returns
-// false when the wait gave up or another CTA gave up.
-__device__ bool grid_sync(Ctrl* c, int* s_flag) {
+// Grid barrier (all CTAs are co-resident: cooperative launch).  Every CTA
+// publishes its barrier count in its own flag (no serialised atomics) and
+// warp 0 polls all flags.  Every CTA calls it the same number of times, so
+// the counts agree.  Returns false when the wait gave up or another CTA gave
+// up.
+__device__ bool grid_sync(const Params& p, unsigned& gen, int* s_flag) {
     __syncthreads();
-    if (threadIdx.x == 0) {
-        volatile unsigned* genp = &c->bar_gen;
-        const unsigned g = *genp;
-        __threadfence();
-        const unsigned arrived = atomicAdd(&c->bar_count, 1u) + 1u;
-        int ok = 1;
-        if (arrived == gridDim.x) {
-            c->bar_count = 0;
+    ++gen;
+    if (warp_id() == 0) {
+        const int lane = lane_id();
+        if (lane == 0) {
             __threadfence();
-            atomicAdd(&c->bar_gen, 1u);
-        } else {
-            const uint64_t t0 = globaltimer();
-            long long it = 0;
-            while (*genp == g) {
-                if (*reinterpret_cast<volatile int*>(&c->abort)) {
+            *reinterpret_cast<volatile unsigned*>(p.bar_flags + blockIdx.x) = gen;
+        }
+        int ok = 1;
+        const uint64_t t0 = globaltimer();
+        for (long long it = 1;; ++it) {
+            bool mine = true;
+            for (int c = lane; c < (int)gridDim.x; c += 32)
+                mine &= (int)(vload(p.bar_flags + c) - gen) >= 0;
+            if (__all_sync(0xffffffffu, mine)) break;
+            // short naps while the barrier is young, longer ones in a long
+            // wait (the narrow rounds of CTA 0) to spare the L2
+            __nanosleep(it < 64 ? 20 : 200);
+            if ((it & 31) == 0) {
+                int stop = 0;
+                if (lane == 0) {
+                    if (*reinterpret_cast<volatile int*>(&p.ctrl->abort)) {
+                        stop = 1;
+                    } else if (globaltimer() - t0 > kWaitNs || it > (1ll << 30)) {
+                        atomicExch(&p.ctrl->abort, 1);
+                        record_error(5001);
+                        stop = 1;
+                    }
+                }
+                if (__shfl_sync(0xffffffffu, stop, 0)) {
                     ok = 0;
                     break;
                 }
-                if (((++it) & 63) == 0 && globaltimer() - t0 > kWaitNs) {
-                    atomicExch(&c->abort, 1);
-                    record_error(5001);
-                    ok = 0;
-                    break;
-                }
-                if (it > (1ll << 34)) {
-                    atomicExch(&c->abort, 1);
-                    record_error(5002);
-                    ok = 0;
-                    break;
-                }
-                __nanosleep(100);
             }
         }
         __threadfence();
-        *s_flag = ok;
+        if (lane == 0) *s_flag = ok;
     }
     __syncthreads();
     return *s_flag != 0;
@@ -652,6 +668,56 @@ __device__ __forceinline__ void group_bid_multi(const int32_t* __restrict__ q, c
         if (off >= G) continue;
 #pragma unroll
         for (int u = 0; u < NT; ++u) {
+            const int64_t ov1 = __shfl_xor_sync(0xffffffffu, v1[u], off);
+            const int64_t ov2 = __shfl_xor_sync(0xffffffffu, v2[u], off);
+            const int oe1 = __shfl_xor_sync(0xffffffffu, e1[u], off);
+            if (ov1 > v1[u] || (ov1 == v1[u] && oe1 < e1[u])) {
+                v2[u] = max(v1[u], ov2);
+                v1[u] = ov1;
+                e1[u] = oe1;
+            } else {
+                v2[u] = max(v2[u], ov1);
+            }
+        }
+    }
+}
+
+// Two tokens' scans interleaved (their loads in flight together); the rows
+// may be in global or shared memory (generic loads).
+__device__ __forceinline__ void group_bid2(const int32_t* r0, const int32_t* r1, bool ok0, bool ok1,
+                                           const int64_t* price, int E, int G, int gl,
+                                           int64_t scale, int64_t (&v1)[2], int64_t (&v2)[2],
+                                           int (&e1)[2]) {
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+        v1[u] = INT64_MIN;
+        v2[u] = INT64_MIN;
+        e1[u] = INT32_MAX;
+    }
+    for (int e = gl; e < E; e += G) {
+        const int32_t a0 = ok0 ? r0[e] : 0;
+        const int32_t a1 = ok1 ? r1[e] : 0;
+        const int64_t pe = price[e];
+        const int32_t qa[2] = {a0, a1};
+        const bool ok[2] = {ok0, ok1};
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            if (!ok[u]) continue;
+            const int64_t v = (int64_t)qa[u] * scale - pe;
+            if (v > v1[u]) {
+                v2[u] = v1[u];
+                v1[u] = v;
+                e1[u] = e;
+            } else if (v > v2[u]) {
+                v2[u] = v;
+            }
+        }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+        if (off >= G) continue;
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
             const int64_t ov1 = __shfl_xor_sync(0xffffffffu, v1[u], off);
             const int64_t ov2 = __shfl_xor_sync(0xffffffffu, v2[u], off);
             const int oe1 = __shfl_xor_sync(0xffffffffu, e1[u], off);
@@ -811,6 +877,126 @@ __device__ int resolve_general(const Team<TEAM>& tm, const Params& p, int e, con
 // keys, sorted ascending, found as the FK-th worst key by a radix select,
 // collected with a team-wide ranking and sorted by warp 0.  Returns the
 // fringe size.
+// Ascending sort (in "worse" order) of P keys in shared memory, P a power of
+// two <= 2 kThreads; the whole CTA takes part (bitonic network; one warp
+// in registers when P <= 64).
+__device__ void cta_sort_keys(Key* a, int P) {
+    if (P <= 64) {
+        if (warp_id() == 0) {
+            const int lane = lane_id();
+            Key x0 = lane < P ? a[lane] : pad_key();
+            Key x1 = lane + 32 < P ? a[lane + 32] : pad_key();
+            Key lo, hi;
+            warp_merge64(warp_sort(x0), warp_sort(x1), lo, hi);
+            if (lane < P) a[lane] = lo;
+            if (lane + 32 < P) a[lane + 32] = hi;
+        }
+        __syncthreads();
+        return;
+    }
+    for (int size = 2; size <= P; size <<= 1) {
+        for (int stride = size >> 1; stride > 0; stride >>= 1) {
+            for (int t = threadIdx.x; t < P / 2; t += kThreads) {
+                const int lo = 2 * t - (t & (stride - 1));
+                const int hi = lo + stride;
+                const bool up = (lo & size) == 0;
+                const Key x = a[lo], y = a[hi];
+                if (up ? worse(y, x) : worse(x, y)) {
+                    a[lo] = y;
+                    a[hi] = x;
+                }
+            }
+            __syncthreads();
+        }
+    }
+}
+
+constexpr int kSortMax = kWarps * kHist * 4 / (int)sizeof(Key);  // keys the histogram area holds
+
+// CTA-wide resolve of one expert in a wide round with every candidate (held
+// keys, then new bids) copied into shared memory once.  With k rejections
+// and f keys in the new fringe, the (k + f)-th worst key is found by a radix
+// select over the copy and the k + f keys up to it are sorted: the first k
+// are rejected, the next f are the new fringe (exact), and the price is the
+// smallest kept bid.  Accepted bids take the freed slots (rejected held keys'
+// slots, then the empty ones).  Returns false, having done nothing, when the
+// candidates do not fit the scratch or k + f keys do not fit the sort.
+__device__ bool resolve_cta_cached(const Team<kThreads>& tm, const Params& p, const Cands& cd,
+                                   Key* sk, int cap, int64_t* hb, int32_t* ht, int32_t* unext,
+                                   int32_t* ucnt, Key* gfr, int& h_out, int& fs_out,
+                                   int64_t& price) {
+    const int C = p.C, h = cd.h, n = cd.n, m = h + n;
+    const int tid = threadIdx.x;
+    const int k = max(0, m - C);
+    const int nh = m - k;          // held after the round: min(m, C)
+    const int f = min(p.FK, nh);   // the new fringe (complete when nh <= FK)
+    const int S = k + f;
+    // the copy (m keys) and the freed-slot list (C ints) share the scratch
+    if (m == 0 || m + (C + 3) / 4 > cap || S > kSortMax) return false;
+    for (int c = tid; c < m; c += kThreads) sk[c] = cd.get(c);  // slot: c (held) or -1 (new)
+    __syncthreads();
+    auto visit = [&](auto fn) {
+        for (int c = tid; c < m; c += kThreads) fn(sk[c]);
+    };
+    const Key Y = kth_worst_v<kThreads>(tm, visit, S, p.T - 1);
+    // the S keys up to Y, with their candidate index in .slot
+    Key* srt = reinterpret_cast<Key*>(tm.hist);
+    if (tid == 0) tm.cnt[45] = 0;
+    __syncthreads();
+    for (int c = tid; c < m; c += kThreads) {
+        const Key x = sk[c];
+        if (!worse(Y, x)) srt[atomicAdd(&tm.cnt[45], 1)] = Key{x.bid, x.tok, c};
+    }
+    __syncthreads();
+    int P = 1;
+    while (P < S) P <<= 1;
+    for (int i = S + tid; i < P; i += kThreads) srt[i] = pad_key();
+    __syncthreads();
+    cta_sort_keys(srt, P);
+    // rejected: srt[0, k) -> the next round's bidders; held ones free their slot
+    int32_t* fslot = reinterpret_cast<int32_t*>(sk + m);  // freed slots
+    if (tid == 0) {
+        tm.cnt[46] = k > 0 ? atomicAdd(ucnt, k) : 0;
+        tm.cnt[47] = 0;
+    }
+    __syncthreads();
+    const int base = tm.cnt[46];
+    for (int i = tid; i < k; i += kThreads) {
+        const Key x = srt[i];
+        unext[base + i] = x.tok;
+        if (x.slot < h) fslot[atomicAdd(&tm.cnt[47], 1)] = x.slot;
+    }
+    __syncthreads();
+    const int kh = tm.cnt[47];
+    for (int j = tid; j < C - h; j += kThreads) fslot[kh + j] = h + j;
+    if (tid == 0) tm.cnt[45] = 0;
+    __syncthreads();
+    // accepted new bids (above the k-th worst) take the freed slots
+    const bool any_rej = k > 0;
+    const Key Xk = any_rej ? srt[k - 1] : Key{INT64_MIN, INT32_MAX, -2};
+    for (int c = h + tid; c < m; c += kThreads) {
+        const Key x = sk[c];
+        if (!any_rej || worse(Xk, x)) {
+            const int slot = fslot[atomicAdd(&tm.cnt[45], 1)];
+            hb[slot] = x.bid;
+            ht[slot] = x.tok;
+            sk[c].slot = slot;
+        }
+    }
+    __syncthreads();
+    if (tm.cnt[45] != (h + n - k) - (h - kh) && tid == 0) record_error(1100);
+    // the new fringe: srt[k, k + f) with their final slots
+    for (int i = tid; i < f; i += kThreads) {
+        const Key x = srt[k + i];
+        gfr[i] = Key{x.bid, x.tok, sk[x.slot].slot};
+    }
+    if (nh == C) price = srt[k].bid;
+    h_out = nh;
+    fs_out = f;
+    __syncthreads();
+    return true;
+}
+
 template <int TEAM>
 __device__ int build_fringe_radix(const Team<TEAM>& tm, const int64_t* hb, const int32_t* ht,
                                   int C, int FK, int tmax, Key* fr) {
@@ -906,6 +1092,38 @@ __device__ int build_fringe(const Team<TEAM>& tm, const int64_t* hb, const int32
 __device__ __forceinline__ int nth_set_lane(unsigned m, int r) {
     for (int i = 0; i < r; ++i) m &= m - 1;
     return m ? __ffs(m) - 1 : 0;
+}
+
+// One bid to a full expert whose fringe holds at least two keys (the usual
+// case in the last rounds of a phase): the bid is above the price, the
+// fringe minimum f0, so f0 is rejected and the bid takes its slot; the new
+// fringe is f1.. with the bid inserted where it belongs (when not above the
+// fringe maximum of an incomplete fringe).  Every load is issued up front.
+// Returns the rejected token; sets fs and the new price (the new minimum).
+__device__ __forceinline__ int fringe_take_one(Key* fr, int& fs, int h, int64_t bid, int tok,
+                                               int64_t* hb, int32_t* ht, int64_t& price) {
+    const int lane = lane_id();
+    const Key f0 = fr[0];
+    const Key f1 = fr[1];
+    const Key fl = fr[fs - 1];
+    const Key fi = lane < fs ? fr[lane] : pad_key();
+    const Key fn = lane + 1 < fs ? fr[lane + 1] : pad_key();
+    const Key b = Key{bid, tok, f0.slot};
+    const bool ins = fs == h || !worse(fl, b);
+    const int pos = __popc(__ballot_sync(0xffffffffu, lane + 1 < fs && worse(fn, b)));
+    Key out = lane < pos ? fn : (lane == pos ? b : fi);
+    if (!ins) out = fn;
+    const int nfs = ins ? fs : fs - 1;
+    price = (ins && pos == 0) ? bid : f1.bid;
+    __syncwarp();
+    if (lane < nfs) fr[lane] = out;
+    if (lane == 0) {
+        hb[b.slot] = bid;
+        ht[b.slot] = tok;
+    }
+    __syncwarp();
+    fs = nfs;
+    return f0.tok;
 }
 
 // Warp-level resolve of one expert from its fringe and n < 32 new bids.
@@ -1045,7 +1263,8 @@ struct ChainScratch {
 template <int NJ>
 __device__ __forceinline__ void chain_rounds(const Params& p, int t, int64_t eps, int64_t scale,
                                           int64_t* s_price, Key* s_fr, int32_t* s_fsize,
-                                          int32_t* s_hcnt, const ChainScratch cs,
+                                          int32_t* s_hcnt, int64_t* hbase, int32_t* htbase,
+                                          const ChainScratch cs,
                                           const Team<32>& wt, long long& rounds,
                                           long long& bids, int& status) {
     const int E = p.E, C = p.C, FK = p.FK, T = p.T;
@@ -1100,34 +1319,21 @@ __device__ __forceinline__ void chain_rounds(const Params& p, int t, int64_t eps
         const int h = s_hcnt[e];
         const int fs = s_fsize[e];
         Key* fr = s_fr + (size_t)e * FK;
-        int64_t* hb = p.hb + (size_t)e * C;
-        int32_t* ht = p.ht + (size_t)e * C;
+        int64_t* hb = hbase + (size_t)e * C;
+        int32_t* ht = htbase + (size_t)e * C;
         int tn = -1;
         if (h == C && fs >= 2) {
-            // the fringe minimum f0 is rejected, the bid takes its slot
-            const Key f0 = fr[0];
-            tn = f0.tok;
+            // the fringe minimum f0 is rejected (its row loaded right away)
+            tn = fr[0].tok;
 #pragma unroll
             for (int j = 0; j < NJ; ++j) {
                 const int ee = lane + 32 * j;
                 rv[j] = ee < E ? __ldg(p.q + (size_t)tn * E + ee) : 0;
             }
-            const Key f1 = fr[1];
-            const Key fl = fr[fs - 1];
-            const Key fi = lane < fs ? fr[lane] : pad_key();
-            const Key fn = lane + 1 < fs ? fr[lane + 1] : pad_key();
-            const Key b = Key{bid, t, f0.slot};
-            const bool ins = fs == h || !worse(fl, b);
-            const int pos = __popc(__ballot_sync(0xffffffffu, lane + 1 < fs && worse(fn, b)));
-            Key out = lane < pos ? fn : (lane == pos ? b : fi);
-            if (!ins) out = fn;
-            const int nfs = ins ? fs : fs - 1;
-            const int64_t price = (ins && pos == 0) ? bid : f1.bid;
-            __syncwarp();
-            if (lane < nfs) fr[lane] = out;
+            int nfs = fs;
+            int64_t price;
+            fringe_take_one(fr, nfs, h, bid, t, hb, ht, price);
             if (lane == 0) {
-                hb[b.slot] = bid;
-                ht[b.slot] = t;
                 s_fsize[e] = nfs;
                 s_price[e] = price;
             }
@@ -1175,7 +1381,7 @@ __device__ __forceinline__ void chain_rounds(const Params& p, int t, int64_t eps
 
 __global__ void __launch_bounds__(kThreads, 1) auction_kernel(const __grid_constant__ Params p) {
     extern __shared__ __align__(16) unsigned char smem[];
-    const SmemLayout L = smem_layout(p.E, p.FK, p.narrow_max, p.NB, p.RC);
+    const SmemLayout L = smem_layout(p.E, p.FK, p.narrow_max, p.NB, p.RC, p.T, p.HS);
     int64_t* s_price = reinterpret_cast<int64_t*>(smem + L.price);
     Key* s_fr = reinterpret_cast<Key*>(smem + L.fr);
     int32_t* s_fsize = reinterpret_cast<int32_t*>(smem + L.fsize);
@@ -1196,6 +1402,8 @@ __global__ void __launch_bounds__(kThreads, 1) auction_kernel(const __grid_const
     int64_t* s_red = reinterpret_cast<int64_t*>(smem + L.red);
     int32_t* s_cnt = reinterpret_cast<int32_t*>(smem + L.cnt);
     int32_t* s_misc = reinterpret_cast<int32_t*>(smem + L.misc);
+    Key* s_scratch = reinterpret_cast<Key*>(smem + L.scratch);  // wide rounds only
+    const int scratch_cap = (int)((L.total - L.scratch) / sizeof(Key));
 
     const int T = p.T, E = p.E, C = p.C, FK = p.FK;
     const int64_t scale = (int64_t)T + 1;
@@ -1208,6 +1416,7 @@ __global__ void __launch_bounds__(kThreads, 1) auction_kernel(const __grid_const
     const int64_t qmin = p.minmax[0], qmax = p.minmax[1];
     const int64_t range = qmax - qmin;
     int status = BASE_OK;
+    unsigned bar_gen = 0;  // grid barriers passed (the same in every CTA)
     if (range > 0 && range > ((int64_t)1 << 58) / scale) status = BASE_ERR_INVALID_ARG;
     int64_t eps = range * scale / kEpsDivisor;
     if (eps < 1) eps = 1;
@@ -1234,7 +1443,7 @@ __global__ void __launch_bounds__(kThreads, 1) auction_kernel(const __grid_const
                 p.gfs[e] = 0;  // empty held set: an empty, complete fringe
             }
             if (cta == 0 && threadIdx.x < 3) p.ctrl->ucount[threadIdx.x] = 0;
-            if (!(ok = grid_sync(p.ctrl, s_misc))) break;
+            if (!(ok = grid_sync(p, bar_gen, s_misc))) break;
         }
         reset_done = false;
         int U = T;
@@ -1310,7 +1519,7 @@ __global__ void __launch_bounds__(kThreads, 1) auction_kernel(const __grid_const
                     __syncthreads();
                 }
             }
-            if (!(ok = grid_sync(p.ctrl, s_misc))) break;
+            if (!(ok = grid_sync(p, bar_gen, s_misc))) break;
             for (int e = cta; e < E; e += ncta) {
                 const int n = vload(p.bcnt + e);
                 if (n == 0) continue;
@@ -1343,6 +1552,21 @@ __global__ void __launch_bounds__(kThreads, 1) auction_kernel(const __grid_const
                     continue;
                 }
                 Cands cd{hb, ht, p.bb + (size_t)e * T, p.bt + (size_t)e * T, h0, n};
+                {
+                    int nh = 0, fs = 0;
+                    int64_t price = INT64_MIN;
+                    if (resolve_cta_cached(cta_team, p, cd, s_scratch, scratch_cap, hb, ht, unext,
+                                           ucnt, gfr, nh, fs, price)) {
+                        if (threadIdx.x == 0) {
+                            p.hcnt[e] = nh;
+                            p.bcnt[e] = 0;
+                            p.gfs[e] = fs;
+                            if (nh == C) p.gprice[e] = price;
+                        }
+                        __syncthreads();
+                        continue;
+                    }
+                }
                 int64_t price = INT64_MIN;
                 const int nh = resolve_general<kThreads>(cta_team, p, e, cd, hb, ht, unext, ucnt,
                                                      price, RowStage{nullptr, 0});
@@ -1357,7 +1581,7 @@ __global__ void __launch_bounds__(kThreads, 1) auction_kernel(const __grid_const
             }
             // the counter the next round writes: last read two rounds ago
             if (cta == 0 && threadIdx.x == 0) p.ctrl->ucount[(int)((rounds + 1) % 3)] = 0;
-            if (!(ok = grid_sync(p.ctrl, s_misc))) break;
+            if (!(ok = grid_sync(p, bar_gen, s_misc))) break;
             U = *reinterpret_cast<volatile int*>(ucnt);
             cur ^= 1;
             first = false;
@@ -1374,13 +1598,12 @@ __global__ void __launch_bounds__(kThreads, 1) auction_kernel(const __grid_const
             // across a barrier are double / triple buffered by round parity.
             if (cta == 0) {
                 const int32_t* ulist = cur ? p.ulist1 : p.ulist0;
-                int32_t* lists[2] = {s_list0, s_list1};
-                int32_t* s_act[2] = {s_act0, s_act1};
                 int32_t* s_nact = s_misc + 4;  // [2]
                 int32_t* s_next = s_misc + 8;  // [3]
                 const int NB = p.NB, RC = p.RC;
                 const bool stage_rows = RC > 0 && (E % 4) == 0;
                 int lc = 0;
+                int r3_prev = (int)(rounds % 3);  // the counter of the round before
                 bool staged = false;  // the current list's first RC rows are in s_rows[lc]
                 for (int i = threadIdx.x; i < U; i += kThreads) s_list0[i] = vload(ulist + i);
                 for (int e = threadIdx.x; e < E; e += kThreads) {
@@ -1393,6 +1616,18 @@ __global__ void __launch_bounds__(kThreads, 1) auction_kernel(const __grid_const
                     const Key* g = p.gfr + i;
                     s_fr[i] = Key{vload(&g->bid), vload(&g->tok), vload(&g->slot)};
                 }
+                // the held sets: in shared memory when they fit (written by
+                // the wide rounds of other CTAs: read past L1)
+                int64_t* hbase = p.hb;
+                int32_t* htbase = p.ht;
+                if (p.HS) {
+                    hbase = reinterpret_cast<int64_t*>(smem + L.hb);
+                    htbase = reinterpret_cast<int32_t*>(smem + L.ht);
+                    for (int i = threadIdx.x; i < T; i += kThreads) {
+                        hbase[i] = __ldcg(p.hb + i);
+                        htbase[i] = __ldcg(p.ht + i);
+                    }
+                }
                 if (threadIdx.x < 5) s_misc[4 + (threadIdx.x < 2 ? threadIdx.x : threadIdx.x + 2)] = 0;
                 __syncthreads();
                 while (U > 0) {
@@ -1400,18 +1635,23 @@ __global__ void __launch_bounds__(kThreads, 1) auction_kernel(const __grid_const
                         // one bidder: warp 0 ends the phase alone
                         long long* s_ll = reinterpret_cast<long long*>(s_misc + 12);
                         if (warp == 0) {
-                            const int t0 = (lc ? s_list1 : s_list0)[0];
-                            // scratch: the bid buckets are free between rounds
-                            const ChainScratch cs{s_nbk_b, s_nbk_t, s_nbk_t + 1, s_misc + 2};
-                            if (E <= 32)
-                                chain_rounds<1>(p, t0, eps, scale, s_price, s_fr, s_fsize, s_hcnt,
-                                                cs, warp_team, rounds, bids, status);
-                            else if (E <= 64)
-                                chain_rounds<2>(p, t0, eps, scale, s_price, s_fr, s_fsize, s_hcnt,
-                                                cs, warp_team, rounds, bids, status);
-                            else
-                                chain_rounds<4>(p, t0, eps, scale, s_price, s_fr, s_fsize, s_hcnt,
-                                                cs, warp_team, rounds, bids, status);
+                            if (U == 1 && status == BASE_OK) {
+                                const int t0 = (lc ? s_list1 : s_list0)[0];
+                                // scratch: the bid buckets are free between rounds
+                                const ChainScratch cs{s_nbk_b, s_nbk_t, s_nbk_t + 1, s_misc + 2};
+                                if (E <= 32)
+                                    chain_rounds<1>(p, t0, eps, scale, s_price, s_fr, s_fsize,
+                                                    s_hcnt, hbase, htbase, cs, warp_team, rounds,
+                                                    bids, status);
+                                else if (E <= 64)
+                                    chain_rounds<2>(p, t0, eps, scale, s_price, s_fr, s_fsize,
+                                                    s_hcnt, hbase, htbase, cs, warp_team, rounds,
+                                                    bids, status);
+                                else
+                                    chain_rounds<4>(p, t0, eps, scale, s_price, s_fr, s_fsize,
+                                                    s_hcnt, hbase, htbase, cs, warp_team, rounds,
+                                                    bids, status);
+                            }
                             if (lane == 0) {
                                 s_ll[0] = rounds;
                                 s_ll[1] = bids;
@@ -1433,48 +1673,71 @@ __global__ void __launch_bounds__(kThreads, 1) auction_kernel(const __grid_const
                     ++rounds;
                     bids += U;
                     const int ra = (int)(rounds & 1);
-                    int32_t* list = lists[lc];
-                    int32_t* next = lists[lc ^ 1];
-                    int32_t* act = s_act[ra];
+                    int32_t* list = lc ? s_list1 : s_list0;
+                    int32_t* next = lc ? s_list0 : s_list1;
+                    int32_t* act = ra ? s_act1 : s_act0;
+                    // round r uses counter r % 3; r3 = rounds % 3 after the increment
+                    const int r3 = r3_prev == 2 ? 0 : r3_prev + 1;
+                    r3_prev = r3;
                     const int32_t* rows_cur = s_rows + (size_t)lc * RC * E;
                     int32_t* rows_next = s_rows + (size_t)(lc ^ 1) * RC * E;
                     // the counter the next round's resolve writes was last read
                     // two barriers ago
-                    if (threadIdx.x == 0) s_next[(int)((rounds + 1) % 3)] = 0;
-                    // ---- bid
-                    for (int base = warp * tpw; base < U; base += kWarps * tpw) {
-                        const int i = base + sub;
-                        const bool valid = i < U;
-                        const int t = valid ? list[i] : 0;
-                        const int32_t* row = (staged && i < RC) ? rows_cur + (size_t)i * E
-                                                                : p.q + (size_t)t * E;
-                        int64_t v1, v2;
-                        int e1;
-                        group_bid(row, s_price, valid ? E : 0, G, gl, scale, v1, v2, e1);
-                        if (valid && gl == 0) {
-                            const int64_t b = v1 + s_price[e1] - v2 + eps;
-                            const int pos = atomicAdd(&s_ncnt[e1], 1);
-                            if (pos == 0) act[atomicAdd(&s_nact[ra], 1)] = e1;
-                            if (pos < NB) {
-                                s_nbk_b[(size_t)e1 * NB + pos] = b;
-                                s_nbk_t[(size_t)e1 * NB + pos] = t;
-                            } else {
-                                p.bb[(size_t)e1 * T + pos] = b;
-                                p.bt[(size_t)e1 * T + pos] = t;
+                    if (threadIdx.x == 0) s_next[r3 == 2 ? 0 : r3 + 1] = 0;
+                    // ---- bid (two tokens per lane group and pass when there are as many)
+                    auto place = [&](int t, int e, int64_t v1, int64_t v2) {
+                        const int64_t b = v1 + s_price[e] - v2 + eps;
+                        const int pos = atomicAdd(&s_ncnt[e], 1);
+                        if (pos == 0) act[atomicAdd(&s_nact[ra], 1)] = e;
+                        if (pos < NB) {
+                            s_nbk_b[(size_t)e * NB + pos] = b;
+                            s_nbk_t[(size_t)e * NB + pos] = t;
+                        } else {
+                            p.bb[(size_t)e * T + pos] = b;
+                            p.bt[(size_t)e * T + pos] = t;
+                        }
+                    };
+                    if (U > kWarps * tpw) {
+                        for (int base = warp * tpw; base < U; base += kWarps * tpw * 2) {
+                            const int i0 = base + sub, i1 = base + kWarps * tpw + sub;
+                            const bool ok0 = i0 < U, ok1 = i1 < U;
+                            const int t0 = ok0 ? list[i0] : 0, t1 = ok1 ? list[i1] : 0;
+                            const int32_t* r0 = (staged && i0 < RC) ? rows_cur + (size_t)i0 * E
+                                                                    : p.q + (size_t)t0 * E;
+                            const int32_t* r1 = (staged && i1 < RC) ? rows_cur + (size_t)i1 * E
+                                                                    : p.q + (size_t)t1 * E;
+                            int64_t v1[2], v2[2];
+                            int e1[2];
+                            group_bid2(r0, r1, ok0, ok1, s_price, E, G, gl, scale, v1, v2, e1);
+                            if (gl == 0) {
+                                if (ok0) place(t0, e1[0], v1[0], v2[0]);
+                                if (ok1) place(t1, e1[1], v1[1], v2[1]);
                             }
+                        }
+                    } else {
+                        const int i = warp * tpw + sub;  // at most one token per lane group
+                        if (warp * tpw < U) {
+                            const bool valid = i < U;
+                            const int t = valid ? list[i] : 0;
+                            const int32_t* row = (staged && i < RC) ? rows_cur + (size_t)i * E
+                                                                    : p.q + (size_t)t * E;
+                            int64_t v1, v2;
+                            int e1;
+                            group_bid(row, s_price, valid ? E : 0, G, gl, scale, v1, v2, e1);
+                            if (valid && gl == 0) place(t, e1, v1, v2);
                         }
                     }
                     __syncthreads();
                     // ---- resolve: a warp per active expert
                     const int nact = s_nact[ra];
-                    int32_t* ncnt_next = &s_next[(int)(rounds % 3)];
+                    int32_t* ncnt_next = &s_next[r3];
                     RowStage rs{stage_rows ? rows_next : nullptr, RC};
                     for (int a = warp; a < nact; a += kWarps) {
                         const int e = act[a];
                         const int n = s_ncnt[e];
                         const int h = s_hcnt[e];
-                        int64_t* hb = p.hb + (size_t)e * C;
-                        int32_t* ht = p.ht + (size_t)e * C;
+                        int64_t* hb = hbase + (size_t)e * C;
+                        int32_t* ht = htbase + (size_t)e * C;
                         Key* fr = s_fr + (size_t)e * FK;
                         const int64_t* nb = s_nbk_b + (size_t)e * NB;
                         const int32_t* nt = s_nbk_t + (size_t)e * NB;
@@ -1492,7 +1755,20 @@ __global__ void __launch_bounds__(kThreads, 1) auction_kernel(const __grid_const
                         }
                         int64_t price = s_price[e];
                         bool done = false;
-                        if (n < 32) {
+                        if (n == 1 && h == C && s_fsize[e] >= 2) {
+                            int fs = s_fsize[e];
+                            const int rej = fringe_take_one(fr, fs, h, nb[0], nt[0], hb, ht, price);
+                            int at = 0;
+                            if (lane == 0) {
+                                at = atomicAdd(ncnt_next, 1);
+                                next[at] = rej;
+                                s_fsize[e] = fs;
+                            }
+                            at = __shfl_sync(0xffffffffu, at, 0);
+                            rs.stage_warp(p.q, E, rej, at);
+                            done = true;
+                        }
+                        if (!done && n < 32) {
                             int fs = s_fsize[e], hh = h;
                             if (fs != hh && max(0, hh + n - C) >= fs)  // depleted: rebuild
                                 fs = build_fringe<32>(warp_team, hb, ht, hh, FK, T - 1, fr);
@@ -1530,13 +1806,15 @@ __global__ void __launch_bounds__(kThreads, 1) auction_kernel(const __grid_const
                     // the other parity's active count: read in the previous round
                     if (threadIdx.x == 0) s_nact[ra ^ 1] = 0;
                     __syncthreads();
-                    U = s_next[(int)(rounds % 3)];
+                    U = s_next[r3];
                     lc ^= 1;
                     staged = stage_rows;
                 }
                 // hand the prices back to the grid; when another phase follows,
                 // reset its state now (the phase start then needs no barrier)
                 const bool again = status == BASE_OK && eps != 1;
+                if (p.HS && !again)  // the last phase: the assignment is read from p.ht
+                    for (int i = threadIdx.x; i < T; i += kThreads) p.ht[i] = htbase[i];
                 for (int e = threadIdx.x; e < E; e += kThreads) {
                     p.gprice[e] = s_price[e];
                     p.hcnt[e] = again ? 0 : s_hcnt[e];
@@ -1552,7 +1830,7 @@ __global__ void __launch_bounds__(kThreads, 1) auction_kernel(const __grid_const
                     reinterpret_cast<volatile int*>(p.obj)[6] = status;
                 }
             }
-            if (!(ok = grid_sync(p.ctrl, s_misc))) break;
+            if (!(ok = grid_sync(p, bar_gen, s_misc))) break;
             // every CTA takes over CTA 0's counters (rewritten no earlier than
             // the next narrow phase, several grid barriers later)
             rounds = reinterpret_cast<volatile long long*>(p.obj)[1];
@@ -1583,7 +1861,7 @@ __global__ void __launch_bounds__(kThreads, 1) auction_kernel(const __grid_const
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
     if (lane == 0 && part) atomicAdd(p.obj, part);
-    if (!grid_sync(p.ctrl, s_misc)) return;
+    if (!grid_sync(p, bar_gen, s_misc)) return;
     if (cta == 0 && threadIdx.x == 0 && p.stats) {
         p.stats->status = status;
         p.stats->phases = phases;
@@ -1639,20 +1917,26 @@ __global__ void minmax_kernel(const int32_t* __restrict__ q, size_t n, int32_t* 
 // bucket NB (<= 32) and the staged rows RC (<= 32) as large as 200 KB allows,
 // the fringe first.
 struct SmemPlan {
-    int FK, NB, RC;
+    int FK, NB, RC, HS;
     size_t bytes;
 };
 
-static SmemPlan smem_plan(int E, int NM) {
+static SmemPlan smem_plan(int E, int NM, int T) {
     constexpr size_t kBudget = 200 * 1024;
-    SmemPlan pl{0, 0, 0, 0};
+    SmemPlan pl{0, 0, 0, 0, 0};
     for (int fk = 32; fk >= 2; fk >>= 1) {
         if (smem_layout(E, fk, NM, 1, 0).total > kBudget) continue;
         int nb = 32;
         while (nb > 1 && smem_layout(E, fk, NM, nb, 0).total > kBudget) nb >>= 1;
         int rc = 32;
         while (rc > 0 && smem_layout(E, fk, NM, nb, rc).total > kBudget) rc >>= 1;
-        pl = SmemPlan{fk, nb, rc, smem_layout(E, fk, NM, nb, rc).total};
+        pl = SmemPlan{fk, nb, rc, 0, smem_layout(E, fk, NM, nb, rc).total};
+        // the held sets too, when they fit (small T)
+        const size_t with_held = smem_layout(E, fk, NM, nb, rc, T, 1).total;
+        if (with_held <= kBudget) {
+            pl.HS = 1;
+            pl.bytes = with_held;
+        }
         return pl;
     }
     return pl;
@@ -1664,6 +1948,7 @@ size_t auction_workspace_bytes(int T, int E) {
     const int C = T / E;
     size_t b = 256;                                         // minmax
     b += align_up(sizeof(auction::Ctrl), 256);
+    b += align_up(sizeof(unsigned) * auction::kMaxGrid, 256);  // grid-barrier flags
     b += align_up(64, 256);                                 // objective + counters
     b += align_up(sizeof(int64_t) * (size_t)E, 256);        // prices
     b += align_up(sizeof(int32_t) * (size_t)E, 256);        // held counts
@@ -1685,8 +1970,8 @@ int launch_auction(const int32_t* q, int T, int E, int32_t* assign, int64_t* pri
     using namespace auction;
     if (ws_bytes < auction_workspace_bytes(T, E)) return BASE_ERR_WORKSPACE;
     const int C = T / E;
-    const int NM = kNarrowMax;
-    const SmemPlan sp = smem_plan(E, NM);
+    const int NM = narrow_max_for(E);
+    const SmemPlan sp = smem_plan(E, NM, T);
     if (sp.FK == 0) return BASE_ERR_UNSUPPORTED;
     const int FK = sp.FK;
     const size_t smem = sp.bytes;
@@ -1702,6 +1987,7 @@ int launch_auction(const int32_t* q, int T, int E, int32_t* assign, int64_t* pri
     prm.FK = FK;
     prm.NB = sp.NB;
     prm.RC = sp.RC;
+    prm.HS = sp.HS;
     prm.max_rounds = max_rounds;
     prm.narrow_max = NM;
     prm.assign = assign;
@@ -1714,6 +2000,7 @@ int launch_auction(const int32_t* q, int T, int E, int32_t* assign, int64_t* pri
     prm.minmax = mm;
     unsigned char* zero_begin = w + o;
     prm.ctrl = reinterpret_cast<Ctrl*>(take(sizeof(Ctrl)));
+    prm.bar_flags = reinterpret_cast<unsigned*>(take(sizeof(unsigned) * kMaxGrid));
     prm.obj = reinterpret_cast<unsigned long long*>(take(64));
     prm.gprice = reinterpret_cast<int64_t*>(take(sizeof(int64_t) * (size_t)E));
     prm.hcnt = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * (size_t)E));
@@ -1750,6 +2037,7 @@ int launch_auction(const int32_t* q, int T, int E, int32_t* assign, int64_t* pri
         per_sm < 1)
         return BASE_ERR_UNSUPPORTED;
     const int grid = nsm;  // one CTA per SM, all co-resident
+    if (grid > kMaxGrid) return BASE_ERR_UNSUPPORTED;
     void* args[] = {&prm};
     if (cudaLaunchCooperativeKernel(reinterpret_cast<void*>(auction_kernel), dim3(grid),
                                     dim3(kThreads), args, smem, stream) != cudaSuccess)

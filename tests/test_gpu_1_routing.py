@@ -195,6 +195,18 @@ def test_auction_round_cap_reports_not_converged(orc):
     assert so["status"] == 3 and so["rounds"] == 5 and so["bids"] == st["bids"]
 
 
+@pytest.mark.parametrize("name", ["layer_fwd", "skewed"])
+def test_auction_round_cap_in_the_last_rounds_of_a_phase(orc, name):
+    # caps that fall in the tails of phases (few bidders, one warp) and in
+    # the middle of the run: the same stopping point as the oracle
+    _, _, q = oracle_q(orc, synth.WORKLOADS[name])
+    R = orc.auction(q)[2]["rounds"]
+    for cap in sorted({R - 1, R - 2, R - 3, R - 6, R - 11, R // 2, R // 3 + 1}):
+        a, p, st = gpu_auction(q, max_rounds=cap)
+        so = orc.auction(q, max_rounds=cap)[2]
+        assert st == so, (cap, st, so)
+
+
 # ------------------------------------------------------------------ permute / combine
 @pytest.mark.parametrize("T,E,D,kind", [(1536, 4, 64, "balanced"), (1000, 5, 200, "ragged"),
                                         (4096, 128, 128, "ragged"), (333, 7, 8, "ragged"),
