@@ -496,7 +496,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!tc::mbar_wait(&tempty[acc], acc_phase ^ 1, 3002)) break;
             tc::tc_fence_after();
             const uint32_t d_tmem = tmem_base + acc * BN;
-            const int kblocks = decode_tile(args, tile, BN, BMP).kblocks;
+            // only K-grouped tiles differ in depth (and need the tile's group)
+            const int kblocks = args.kgroup ? decode_tile(args, tile, BN, BMP).kblocks
+                                            : (args.K + BK - 1) / BK;
             for (int kb = 0; kb < kblocks; ++kb) {
                 if (!tc::mbar_wait(&full[stage], phase, 3003)) {
                     ok = false;
