@@ -1126,6 +1126,18 @@ __device__ __forceinline__ int fringe_take_one(Key* fr, int& fs, int h, int64_t 
     return f0.tok;
 }
 
+// One step of a sequential resolve: key b enters a full expert and the worst
+// key leaves.  When b is worse than the fringe minimum f0, b itself leaves;
+// otherwise f0 leaves and b takes its slot (inserted into the fringe as in
+// fringe_take_one).  Needs fs >= 2.  Returns the token that left.
+__device__ __forceinline__ int fringe_push_pop(Key* fr, int& fs, int h, int64_t bid, int tok,
+                                               int64_t* hb, int32_t* ht) {
+    const Key f0 = fr[0];
+    if (worse(Key{bid, tok, -1}, f0)) return tok;
+    int64_t price;
+    return fringe_take_one(fr, fs, h, bid, tok, hb, ht, price);
+}
+
 // Warp-level resolve of one expert from its fringe and n < 32 new bids.
 // The fringe holds the expert's fs worst held keys, sorted ascending; it is
 // "complete" when it holds all h of them.  The k = max(0, h + n - C) worst of
@@ -1146,6 +1158,26 @@ __device__ bool resolve_warp(const Params& p, Key* fr, int& fs, int& h, const in
     const bool complete = (fs == h);
     const int k = max(0, h + n - C);
     if (!complete && k >= fs) return false;
+    if (h == C && n >= 2 && n <= 8 && fs >= 2 && (complete || fs >= n + 1)) {
+        // a few bids to a full expert: "one in, the worst out" n times keeps
+        // the C best of held + new, the same set as the merge below, and
+        // rejects the n worst; each step is one pass over the fringe
+        int rej = -1;
+        for (int i = 0; i < n; ++i) {
+            const int t = fringe_push_pop(fr, fs, h, nb[i], nt[i], hb, ht);
+            if (lane == i) rej = t;
+        }
+        int base = 0;
+        if (lane == 0) base = atomicAdd(next_cnt, n);
+        base = __shfl_sync(0xffffffffu, base, 0);
+        if (lane < n) {
+            next_list[base + lane] = rej;
+            rs.stage(p.q, p.E, rej, base + lane);
+        }
+        __syncwarp();
+        price = fr[0].bid;
+        return true;
+    }
     if (n == 1 && h == C && fs >= 2) {
         // one bid b to a full expert: b beats the price (the fringe minimum
         // f0), so f0 is rejected and b takes its slot; the new fringe is
