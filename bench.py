@@ -202,9 +202,8 @@ def main():
     wl = synth.WORKLOADS[args.workload]
     if args.tokens:
         wl = wl.scaled(T=args.tokens)
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    from balanced_token_expert_b200 import replicas
+    rank, world, local_rank = replicas.rank_env()
     if args.impl == "reference":
         run_reference(args, wl, rank, world)
         return
@@ -226,7 +225,7 @@ def main():
     B.lib()
 
     T, E, D, F = wl.T, wl.E, wl.D, wl.F
-    inp = synth.make_inputs(wl, seed=rank)
+    inp = synth.make_inputs(wl, seed=replicas.rank_seed(rank))
     h = inp.h.cuda()
     w = inp.w.cuda()
     W1 = inp.W1.cuda() if F else None
@@ -324,10 +323,7 @@ def main():
     ms = statistics.mean(step_ms)
     st = buffers.stats_dict(sv["stats"])
     err = B.base_device_error(clear=True)
-    if world > 1:
-        t = torch.tensor([ms], device="cuda", dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = replicas.max_over_ranks(ms, device=torch.device("cuda"))
     clk = clocks.stop() if clocks else None
 
     # end to end through the public call: host inputs in, host output back
@@ -370,10 +366,7 @@ def main():
         b.synchronize()
         e2e_ms.append(a.elapsed_time(b))
     e2e = statistics.mean(e2e_ms)
-    if world > 1:
-        t = torch.tensor([e2e], device="cuda", dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e = float(t.item())
+    e2e = replicas.max_over_ranks(e2e, device=torch.device("cuda"))
 
     if rank == 0:
         pk = peaks()
@@ -403,16 +396,18 @@ def main():
                         peak_source=pk["source"] + " hbm copy")
 
         res = dict(
-            metric=METRIC, value=T * world / (ms / 1e3), unit=UNIT, n_gpus=world,
+            metric=METRIC, value=replicas.job_tokens_per_s(T, world, ms), unit=UNIT, n_gpus=world,
             steps=args.steps, warmup=args.warmup, ms_per_step=ms, higher_is_better=True,
             scaling="weak", vs_baseline=None, dtype="bf16", data="synthetic",
             config=_config(wl, args),
             roofline=roof(dom),
             per_kernel={n: roof(n) for n in names},
-            auction=dict(tokens_per_s=T * world / (comp["auction"] / 1e3), rounds=st["rounds"],
+            auction=dict(tokens_per_s=replicas.job_tokens_per_s(T, world, comp["auction"]),
+                         rounds=st["rounds"],
                          phases=st["phases"], bids=bids, status=st["status"],
                          us_per_round=1e3 * comp["auction"] / max(1, st["rounds"])),
-            e2e=dict(value=T * world / (e2e / 1e3), unit=UNIT, h2d_bytes_per_step=T * D * 2,
+            e2e=dict(value=replicas.job_tokens_per_s(T, world, e2e), unit=UNIT,
+                     h2d_bytes_per_step=T * D * 2,
                      d2h_bytes_per_step=d2h, ms_per_step=e2e),
             gpu_launches=kernels_per_step * args.steps,
             clocks=clk, device_error=err, wall_s=wall,
