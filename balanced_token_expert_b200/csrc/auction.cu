@@ -38,6 +38,7 @@ namespace auction {
 
 constexpr int kThreads = 512;  // 16 warps: 128 registers per thread, no spills
 constexpr int kWarps = kThreads / kWarp;
+static_assert(kWarps <= 16, "the team reductions keep 16 warp minima and 16 maxima");
 constexpr int kHist = 256;
 constexpr int kEpsDivisor = 50;  // eps0 = (max q - min q)(T+1) / 50
 constexpr int kEpsFactor = 8;    // eps <- eps / 8 per phase
@@ -201,6 +202,32 @@ struct Team {
         __syncthreads();
         return r;
     }
+    // (min, max) of v over the team in one reduction
+    __device__ void minmax_i64(int64_t& lo, int64_t& hi) const {
+        lo = warp_min_i64(lo);
+        hi = warp_max_i64(hi);
+        if (TEAM == 32) return;
+        if (lane_id() == 0) {
+            red[warp_id()] = lo;
+            red[16 + warp_id()] = hi;
+        }
+        __syncthreads();
+        if (warp_id() == 0) {
+            int64_t x = lane_id() < TEAM / 32 ? red[lane_id()] : INT64_MAX;
+            int64_t y = lane_id() < TEAM / 32 ? red[16 + lane_id()] : INT64_MIN;
+            x = warp_min_i64(x);
+            y = warp_max_i64(y);
+            __syncwarp();
+            if (lane_id() == 0) {
+                red[0] = x;
+                red[16] = y;
+            }
+        }
+        __syncthreads();
+        lo = red[0];
+        hi = red[16];
+        __syncthreads();
+    }
     __device__ Key max_key(Key k) const {
         k = warp_max_key(k);
         if (TEAM == 32) return k;
@@ -334,32 +361,183 @@ struct Cands {
 // unique).  `visit(f)` calls f(key) for each candidate this thread owns.
 // Radix select on the bid (relative to the smallest bid, 8-bit digits from
 // the top), then, among equal bids, on the token.
-template <int TEAM, class Visit>
-__device__ Key kth_worst_v(const Team<TEAM>& tm, Visit visit, int k, int tmax) {
+// Digit pass helper of the CTA select: warp 0 scans the 256-bin histogram
+// (eight bins per lane), finds the bin where the running count reaches
+// `need`, publishes (bin, count before it, its count) in out[0..2] and zeroes
+// the histogram for the next pass.  The caller's barrier publishes both.
+__device__ __forceinline__ void cta_find_digit(int32_t* hist, int nbins, int need, int32_t* out) {
+    const int lane = lane_id();
+    int c8[8];
+    const int4* h4 = reinterpret_cast<const int4*>(hist + lane * 8);
+    const int4 a = h4[0], b = h4[1];
+    c8[0] = a.x; c8[1] = a.y; c8[2] = a.z; c8[3] = a.w;
+    c8[4] = b.x; c8[5] = b.y; c8[6] = b.z; c8[7] = b.w;
+    int sum = 0;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+        if (lane * 8 + q >= nbins) c8[q] = 0;
+        sum += c8[q];
+    }
+    int incl = sum;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int o = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += o;
+    }
+    int run = incl - sum;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+        if (run < need && run + c8[q] >= need) {
+            out[0] = lane * 8 + q;
+            out[1] = run;
+            out[2] = c8[q];
+        }
+        run += c8[q];
+    }
+    int4* w4 = reinterpret_cast<int4*>(hist + lane * 8);
+    w4[0] = make_int4(0, 0, 0, 0);
+    w4[1] = make_int4(0, 0, 0, 0);
+}
+
+// The k-th worst key among a CTA's candidates (1 <= k <= m; keys unique):
+// radix select on the bid (relative to the smallest, 8-bit digits from the
+// top), then among equal bids on the token; two barriers per digit.
+// `visit(f)` calls f(key) for each candidate this thread owns.
+template <class Visit>
+__device__ Key kth_worst_cta(const Team<kThreads>& tm, Visit visit, int k, int tmax) {
+    const int lane = lane_id(), warp = warp_id();
+    int32_t* hist = tm.hist;     // 256 bins, zero between passes
+    int32_t* res = tm.cnt + 50;  // [3] a pass's result
+    __syncthreads();  // the caller may still be reading the histogram area
+    if (warp == 0) {
+        int4* w4 = reinterpret_cast<int4*>(hist + lane * 8);
+        w4[0] = make_int4(0, 0, 0, 0);
+        w4[1] = make_int4(0, 0, 0, 0);
+    }
     int64_t lo = INT64_MAX, hi = INT64_MIN;
     visit([&](const Key& x) {
         lo = min(lo, x.bid);
         hi = max(hi, x.bid);
     });
-    lo = tm.min_i64(lo);
-    hi = tm.max_i64(hi);
+    lo = warp_min_i64(lo);
+    hi = warp_max_i64(hi);
+    if (lane == 0) {
+        tm.red[warp] = lo;
+        tm.red[16 + warp] = hi;
+    }
+    __syncthreads();
+    {
+        int64_t x = lane < kWarps ? tm.red[lane] : INT64_MAX;
+        int64_t y = lane < kWarps ? tm.red[16 + lane] : INT64_MIN;
+        lo = warp_min_i64(x);  // every warp reduces the 16 partials itself
+        hi = warp_max_i64(y);
+    }
     const int nbits = bit_length_u64((uint64_t)(hi - lo));
-    const int tid = tm.tid();
-    // --- bid digits
     int need = k, pbits = 0;
     uint64_t prefix = 0;
     bool whole_bucket = false;
     while (pbits < nbits) {
         const int width = min(8, nbits - pbits);
         const int shift = nbits - pbits - width;
-        for (int b = tid; b < kHist; b += TEAM) tm.hist[b] = 0;
-        tm.sync();
         visit([&](const Key& x) {
             const uint64_t v = (uint64_t)(x.bid - lo);
             if (shr64(v, shift + width) == prefix)
-                atomicAdd(&tm.hist[(int)((v >> shift) & ((1u << width) - 1))], 1);
+                atomicAdd(&hist[(int)((v >> shift) & ((1u << width) - 1))], 1);
         });
+        __syncthreads();
+        if (warp == 0) cta_find_digit(hist, 1 << width, need, res);
+        __syncthreads();
+        const int d = res[0], before = res[1], cnt = res[2];
+        prefix = (prefix << width) | (uint64_t)d;
+        pbits += width;
+        need -= before;
+        if (need == cnt) {
+            whole_bucket = true;
+            break;
+        }
+    }
+    Key best = Key{INT64_MIN, INT32_MAX, -2};
+    if (whole_bucket) {
+        // the k-th worst is the best of the candidates whose bid's top pbits
+        // are <= prefix
+        const int sh = nbits - pbits;
+        visit([&](const Key& x) {
+            if (shr64((uint64_t)(x.bid - lo), sh) <= prefix && worse(best, x)) best = x;
+        });
+    } else {
+        // every bid digit fixed: B* = lo + prefix; `need` of the candidates
+        // with bid == B* are rejected, those with the largest tokens
+        const int64_t bstar = lo + (int64_t)prefix;
+        const uint32_t tm_max = (uint32_t)tmax;
+        const int tbits = bit_length_u64((uint64_t)tm_max) > 0 ? bit_length_u64((uint64_t)tm_max) : 1;
+        int tneed = need, tp = 0;
+        uint32_t tprefix = 0;
+        while (tp < tbits) {
+            const int width = min(8, tbits - tp);
+            const int shift = tbits - tp - width;
+            visit([&](const Key& x) {
+                if (x.bid != bstar) return;
+                const uint32_t v = tm_max - (uint32_t)x.tok;
+                if ((uint32_t)shr64(v, shift + width) == tprefix)
+                    atomicAdd(&hist[(int)((v >> shift) & ((1u << width) - 1))], 1);
+            });
+            __syncthreads();
+            if (warp == 0) cta_find_digit(hist, 1 << width, tneed, res);
+            __syncthreads();
+            const int d = res[0], before = res[1], cnt = res[2];
+            tprefix = (tprefix << width) | (uint32_t)d;
+            tp += width;
+            tneed -= before;
+            if (tneed == cnt) break;
+        }
+        const int sh = tbits - tp;
+        visit([&](const Key& x) {
+            bool rej = x.bid < bstar;
+            if (x.bid == bstar) rej = (uint32_t)shr64(tm_max - (uint32_t)x.tok, sh) <= tprefix;
+            if (rej && worse(best, x)) best = x;
+        });
+    }
+    // the best over the CTA: warp maxima, then every warp reduces them
+    best = warp_max_key(best);
+    Key* wk = reinterpret_cast<Key*>(tm.hist + kHist);  // past the histogram: 16 keys
+    if (lane == 0) wk[warp] = best;
+    __syncthreads();
+    const Key r = warp_max_key(lane < kWarps ? wk[lane] : Key{INT64_MIN, INT32_MAX, -2});
+    __syncthreads();  // wk and red are free again once every warp has read them
+    return r;
+}
+
+template <int TEAM, class Visit>
+__device__ Key kth_worst_v(const Team<TEAM>& tm, Visit visit, int k, int tmax) {
+    if constexpr (TEAM > 32) return kth_worst_cta(tm, visit, k, tmax);
+    int64_t lo = INT64_MAX, hi = INT64_MIN;
+    visit([&](const Key& x) {
+        lo = min(lo, x.bid);
+        hi = max(hi, x.bid);
+    });
+    tm.minmax_i64(lo, hi);
+    const int nbits = bit_length_u64((uint64_t)(hi - lo));
+    const int tid = tm.tid();
+    // --- bid digits
+    int need = k, pbits = 0;
+    uint64_t prefix = 0;
+    bool whole_bucket = false;
+    int32_t* hist = tm.hist;
+    auto clear_hist = [&]() {
+        for (int b = tid; b < kHist; b += TEAM) tm.hist[b] = 0;
         tm.sync();
+    };
+    auto sum_hist = [&]() { tm.sync(); };
+    while (pbits < nbits) {
+        const int width = min(8, nbits - pbits);
+        const int shift = nbits - pbits - width;
+        clear_hist();
+        visit([&](const Key& x) {
+            const uint64_t v = (uint64_t)(x.bid - lo);
+            if (shr64(v, shift + width) == prefix)
+                atomicAdd(&hist[(int)((v >> shift) & ((1u << width) - 1))], 1);
+        });
+        sum_hist();
         int d = 0, before = 0, cnt = 0;
         tm.find_digit(1 << width, need, d, before, cnt);
         prefix = (prefix << width) | (uint64_t)d;
@@ -391,15 +569,14 @@ __device__ Key kth_worst_v(const Team<TEAM>& tm, Visit visit, int k, int tmax) {
     while (tp < tbits) {
         const int width = min(8, tbits - tp);
         const int shift = tbits - tp - width;
-        for (int b = tid; b < kHist; b += TEAM) tm.hist[b] = 0;
-        tm.sync();
+        clear_hist();
         visit([&](const Key& x) {
             if (x.bid != bstar) return;
             const uint32_t v = tm_max - (uint32_t)x.tok;
             if ((uint32_t)shr64(v, shift + width) == tprefix)
-                atomicAdd(&tm.hist[(int)((v >> shift) & ((1u << width) - 1))], 1);
+                atomicAdd(&hist[(int)((v >> shift) & ((1u << width) - 1))], 1);
         });
-        tm.sync();
+        sum_hist();
         int d = 0, before = 0, cnt = 0;
         tm.find_digit(1 << width, tneed, d, before, cnt);
         tprefix = (tprefix << width) | (uint32_t)d;
@@ -913,14 +1090,68 @@ __device__ void cta_sort_keys(Key* a, int P) {
 
 constexpr int kSortMax = kWarps * kHist * 4 / (int)sizeof(Key);  // keys the histogram area holds
 
+// The end of a CTA-wide resolve: the k rejected keys rejs[0, k) (any order)
+// and the f new fringe keys frs[0, f) (sorted), each with its candidate
+// index in .slot; Xk = the k-th worst (k > 0).  Rejected tokens go to the
+// next round's list, accepted bids take the freed slots (rejected held
+// keys' slots, then the empty ones), the fringe gets the final slots.
+__device__ void finish_cta_resolve(const Team<kThreads>& tm, const Params& p, const Cands& cd,
+                                   Key* sk, int64_t* hb, int32_t* ht, int32_t* unext,
+                                   int32_t* ucnt, Key* gfr, const Key* rejs, int k,
+                                   const Key* frs, int f, const Key& Xk, int& h_out, int& fs_out,
+                                   int64_t& price) {
+    const int C = p.C, h = cd.h, n = cd.n, m = h + n;
+    const int tid = threadIdx.x;
+    int32_t* fslot = reinterpret_cast<int32_t*>(sk + m);  // freed slots
+    if (tid == 0) {
+        tm.cnt[46] = k > 0 ? atomicAdd(ucnt, k) : 0;
+        tm.cnt[47] = 0;
+    }
+    __syncthreads();
+    const int base = tm.cnt[46];
+    for (int i = tid; i < k; i += kThreads) {
+        const Key x = rejs[i];
+        unext[base + i] = x.tok;
+        if (x.slot < h) fslot[atomicAdd(&tm.cnt[47], 1)] = x.slot;
+    }
+    __syncthreads();
+    const int kh = tm.cnt[47];
+    for (int j = tid; j < C - h; j += kThreads) fslot[kh + j] = h + j;
+    if (tid == 0) tm.cnt[45] = 0;
+    __syncthreads();
+    // accepted new bids (above the k-th worst) take the freed slots
+    for (int c = h + tid; c < m; c += kThreads) {
+        const Key x = sk[c];
+        if (k == 0 || worse(Xk, x)) {
+            const int slot = fslot[atomicAdd(&tm.cnt[45], 1)];
+            hb[slot] = x.bid;
+            ht[slot] = x.tok;
+            sk[c].slot = slot;
+        }
+    }
+    __syncthreads();
+    if (tm.cnt[45] != n - k + kh && tid == 0) record_error(1100);
+    // the new fringe with the final slots
+    for (int i = tid; i < f; i += kThreads) {
+        const Key x = frs[i];
+        gfr[i] = Key{x.bid, x.tok, sk[x.slot].slot};
+    }
+    const int nh = m - k;
+    if (nh == C) price = frs[0].bid;
+    h_out = nh;
+    fs_out = f;
+    __syncthreads();
+}
+
 // CTA-wide resolve of one expert in a wide round with every candidate (held
 // keys, then new bids) copied into shared memory once.  With k rejections
 // and f keys in the new fringe, the (k + f)-th worst key is found by a radix
-// select over the copy and the k + f keys up to it are sorted: the first k
-// are rejected, the next f are the new fringe (exact), and the price is the
-// smallest kept bid.  Accepted bids take the freed slots (rejected held keys'
-// slots, then the empty ones).  Returns false, having done nothing, when the
-// candidates do not fit the scratch or k + f keys do not fit the sort.
+// select over the copy and the k + f keys up to it are collected; a second
+// select over those splits off the k rejected (or, for at most 64 keys, a
+// sort orders them); the f others, sorted, are the new fringe (exact), and
+// the price is the smallest kept bid.  Returns false, having done nothing,
+// when the candidates do not fit the scratch or k + f keys do not fit the
+// collection area.
 __device__ bool resolve_cta_cached(const Team<kThreads>& tm, const Params& p, const Cands& cd,
                                    Key* sk, int cap, int64_t* hb, int32_t* ht, int32_t* unext,
                                    int32_t* ucnt, Key* gfr, int& h_out, int& fs_out,
@@ -932,7 +1163,7 @@ __device__ bool resolve_cta_cached(const Team<kThreads>& tm, const Params& p, co
     const int f = min(p.FK, nh);   // the new fringe (complete when nh <= FK)
     const int S = k + f;
     // the copy (m keys) and the freed-slot list (C ints) share the scratch
-    if (m == 0 || m + (C + 3) / 4 > cap || S > kSortMax) return false;
+    if (m == 0 || m + (C + 3) / 4 > cap || S > kSortMax || S > 2 * kThreads) return false;
     for (int c = tid; c < m; c += kThreads) sk[c] = cd.get(c);  // slot: c (held) or -1 (new)
     __syncthreads();
     auto visit = [&](auto fn) {
@@ -948,52 +1179,50 @@ __device__ bool resolve_cta_cached(const Team<kThreads>& tm, const Params& p, co
         if (!worse(Y, x)) srt[atomicAdd(&tm.cnt[45], 1)] = Key{x.bid, x.tok, c};
     }
     __syncthreads();
-    int P = 1;
-    while (P < S) P <<= 1;
-    for (int i = S + tid; i < P; i += kThreads) srt[i] = pad_key();
-    __syncthreads();
-    cta_sort_keys(srt, P);
-    // rejected: srt[0, k) -> the next round's bidders; held ones free their slot
-    int32_t* fslot = reinterpret_cast<int32_t*>(sk + m);  // freed slots
+    if (S <= 64) {
+        // one warp sorts them (padded): rejected srt[0, k), fringe srt[k, S)
+        for (int i = S + tid; i < 64; i += kThreads) srt[i] = pad_key();
+        __syncthreads();
+        cta_sort_keys(srt, 64);
+        const Key Xk = k > 0 ? srt[k - 1] : pad_key();
+        finish_cta_resolve(tm, p, cd, sk, hb, ht, unext, ucnt, gfr, srt, k, srt + k, f, Xk, h_out,
+                           fs_out, price);
+        return true;
+    }
+    // k > 0 here (S > 64 > f): the k worst of the S collected keys by a
+    // second select over them (two per thread, in registers); then the f
+    // others are moved to the front and sorted, the rejected ones follow
+    const Key k0 = tid < S ? srt[tid] : pad_key();
+    const Key k1 = tid + kThreads < S ? srt[tid + kThreads] : pad_key();
+    auto visit2 = [&](auto fn) {
+        if (tid < S) fn(k0);
+        if (tid + kThreads < S) fn(k1);
+    };
+    const Key Xk = kth_worst_v<kThreads>(tm, visit2, k, p.T - 1);
     if (tid == 0) {
-        tm.cnt[46] = k > 0 ? atomicAdd(ucnt, k) : 0;
-        tm.cnt[47] = 0;
+        tm.cnt[45] = 0;  // fringe keys placed
+        tm.cnt[48] = 0;  // rejected keys placed
     }
     __syncthreads();
-    const int base = tm.cnt[46];
-    for (int i = tid; i < k; i += kThreads) {
-        const Key x = srt[i];
-        unext[base + i] = x.tok;
-        if (x.slot < h) fslot[atomicAdd(&tm.cnt[47], 1)] = x.slot;
+    if (tid < S) {
+        const bool rj = !worse(Xk, k0);
+        srt[rj ? f + atomicAdd(&tm.cnt[48], 1) : atomicAdd(&tm.cnt[45], 1)] = k0;
+    }
+    if (tid + kThreads < S) {
+        const bool rj = !worse(Xk, k1);
+        srt[rj ? f + atomicAdd(&tm.cnt[48], 1) : atomicAdd(&tm.cnt[45], 1)] = k1;
     }
     __syncthreads();
-    const int kh = tm.cnt[47];
-    for (int j = tid; j < C - h; j += kThreads) fslot[kh + j] = h + j;
-    if (tid == 0) tm.cnt[45] = 0;
-    __syncthreads();
-    // accepted new bids (above the k-th worst) take the freed slots
-    const bool any_rej = k > 0;
-    const Key Xk = any_rej ? srt[k - 1] : Key{INT64_MIN, INT32_MAX, -2};
-    for (int c = h + tid; c < m; c += kThreads) {
-        const Key x = sk[c];
-        if (!any_rej || worse(Xk, x)) {
-            const int slot = fslot[atomicAdd(&tm.cnt[45], 1)];
-            hb[slot] = x.bid;
-            ht[slot] = x.tok;
-            sk[c].slot = slot;
-        }
+    if (warp_id() == 0) {  // f <= 32: one key per lane
+        const int lane = lane_id();
+        Key x = lane < f ? srt[lane] : pad_key();
+        x = warp_sort(x);
+        __syncwarp();
+        if (lane < f) srt[lane] = x;
     }
     __syncthreads();
-    if (tm.cnt[45] != (h + n - k) - (h - kh) && tid == 0) record_error(1100);
-    // the new fringe: srt[k, k + f) with their final slots
-    for (int i = tid; i < f; i += kThreads) {
-        const Key x = srt[k + i];
-        gfr[i] = Key{x.bid, x.tok, sk[x.slot].slot};
-    }
-    if (nh == C) price = srt[k].bid;
-    h_out = nh;
-    fs_out = f;
-    __syncthreads();
+    finish_cta_resolve(tm, p, cd, sk, hb, ht, unext, ucnt, gfr, srt + f, k, srt, f, Xk, h_out,
+                       fs_out, price);
     return true;
 }
 
