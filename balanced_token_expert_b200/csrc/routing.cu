@@ -93,7 +93,8 @@ __global__ void greedy_kernel(const int32_t* __restrict__ q, int T, int E,
 }
 
 // ---------------------------------------------------------------------------
-// stable counting sort of tokens by expert
+// stable counting sort of tokens by expert (more than kSmallSort tokens; see
+// sort_small_kernel below for the one-CTA version)
 //   chunk = kChunk consecutive tokens handled by one warp, in token order.
 //   1) per-chunk expert histogram  2) scan over chunks and experts
 //   3) per-chunk ranks -> perm, inv (and the permuted gate scores)
@@ -208,6 +209,95 @@ __global__ void chunk_rank_kernel(const int32_t* __restrict__ assign, int T, int
     }
 }
 
+// The same stable counting sort in one CTA for up to kSmallSort tokens (one
+// launch instead of three): warp w takes tokens [w per, (w+1) per) in order;
+// pass 1 counts them per expert, one thread per expert turns the counts into
+// per-warp starting slots (expert-major, warp order), pass 2 ranks each
+// 32-token group with match_any and writes perm, inv and gate.
+constexpr int kSmallSort = 32768;
+
+__global__ void __launch_bounds__(1024) sort_small_kernel(const int32_t* __restrict__ assign,
+                                                          int T, int E, int32_t* __restrict__ perm,
+                                                          int32_t* __restrict__ inv,
+                                                          int32_t* __restrict__ offsets,
+                                                          const float* __restrict__ s,
+                                                          float* __restrict__ gate) {
+    extern __shared__ int32_t sm[];
+    int32_t* cnt = sm;                 // [32][E]: counts, then running slots
+    int32_t* s_warp = sm + 32 * E;     // [32] block-scan partials
+    const int w = warp_id(), lane = lane_id();
+    const unsigned lt = (1u << lane) - 1;
+    const int per = ((T + 31) / 32 + 31) / 32 * 32;  // a multiple of 32 tokens per warp
+    const int t0 = min(T, w * per), t1 = min(T, t0 + per);
+    for (int e = lane; e < E; e += kWarp) cnt[w * E + e] = 0;
+    __syncwarp();
+    for (int b = t0; b < t1; b += kWarp) {
+        const int t = b + lane;
+        int e = t < t1 ? assign[t] : -1;
+        if (t < t1 && (e < 0 || e >= E)) {  // not an expert: recorded, token skipped
+            record_error(2001);
+            e = -1;
+        }
+        const unsigned peers = __match_any_sync(0xffffffffu, e >= 0 ? e : -1 - lane);
+        if (e >= 0 && (peers & lt) == 0) cnt[w * E + e] += __popc(peers);
+        __syncwarp();
+    }
+    __syncthreads();
+    // thread e: exclusive prefix of its column over the warps and its total,
+    // then an exclusive scan of the totals over the experts
+    int run = 0;
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {  // E <= 1024: one pass
+        for (int v = 0; v < 32; ++v) {
+            const int c = cnt[v * E + e];
+            cnt[v * E + e] = run;
+            run += c;
+        }
+    }
+    const int e_me = threadIdx.x;
+    int incl = e_me < E ? run : 0;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int o = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += o;
+    }
+    if (lane == 31) s_warp[w] = incl;
+    __syncthreads();
+    if (w == 0) {
+        const int v = s_warp[lane];
+        int vi = v;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int o = __shfl_up_sync(0xffffffffu, vi, off);
+            if (lane >= off) vi += o;
+        }
+        s_warp[lane] = vi - v;
+    }
+    __syncthreads();
+    if (e_me < E) {
+        const int base = incl - run + s_warp[w];
+        offsets[e_me] = base;
+        if (e_me == E - 1) offsets[E] = base + run;
+        for (int v = 0; v < 32; ++v) cnt[v * E + e_me] += base;
+    }
+    __syncthreads();
+    for (int b = t0; b < t1; b += kWarp) {
+        const int t = b + lane;
+        int e = t < t1 ? assign[t] : -1;
+        if (e >= E) e = -1;
+        const unsigned peers = __match_any_sync(0xffffffffu, e >= 0 ? e : -1 - lane);
+        int slot = 0;
+        if (e >= 0) slot = cnt[w * E + e] + __popc(peers & lt);
+        __syncwarp();
+        if (e >= 0 && (peers & lt) == 0) cnt[w * E + e] += __popc(peers);
+        __syncwarp();
+        if (e >= 0) {
+            perm[slot] = t;
+            inv[t] = slot;
+            if (gate) gate[slot] = s[(size_t)t * E + e];
+        }
+    }
+}
+
 // ---------------------------------------------------------------------------
 // row gather / scatter of bf16 rows with 16-byte vectors:
 //   gather:  dst[r] = src[idx[r]]        scatter: dst[idx[r]] = src[r]
@@ -297,6 +387,15 @@ int launch_sort_by_expert(const int32_t* assign, int T, int E, int32_t* perm, in
                           int32_t* offsets, const float* s, float* gate, void* ws,
                           cudaStream_t stream) {
     using namespace routing;
+    if (T <= kSmallSort) {
+        const size_t sm = sizeof(int32_t) * (32 * (size_t)E + 32);
+        if (cudaFuncSetAttribute(sort_small_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)sm) != cudaSuccess)
+            return BASE_ERR_CUDA;
+        sort_small_kernel<<<1, 1024, sm, stream>>>(assign, T, E, perm, inv, offsets, s, gate);
+        BASE_RETURN_IF_LAUNCH_FAILED();
+        return BASE_OK;
+    }
     const int nchunks = (T + kChunk - 1) / kChunk;
     int32_t* chunk_counts = static_cast<int32_t*>(ws);
     const int blocks = (nchunks + kSortWarps - 1) / kSortWarps;
