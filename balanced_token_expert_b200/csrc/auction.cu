@@ -1884,10 +1884,19 @@ __global__ void __launch_bounds__(kThreads, 1) auction_kernel(const __grid_const
                 if (p.HS) {
                     hbase = reinterpret_cast<int64_t*>(smem + L.hb);
                     htbase = reinterpret_cast<int32_t*>(smem + L.ht);
-                    for (int i = threadIdx.x; i < T; i += kThreads) {
+                    // 16-byte pieces (all bases 16-byte aligned), then the tails
+                    const int4* gb = reinterpret_cast<const int4*>(p.hb);
+                    const int4* gt = reinterpret_cast<const int4*>(p.ht);
+                    int4* sb = reinterpret_cast<int4*>(hbase);
+                    int4* st = reinterpret_cast<int4*>(htbase);
+#pragma unroll 4
+                    for (int i = threadIdx.x; i < T / 2; i += kThreads) sb[i] = __ldcg(gb + i);
+#pragma unroll 4
+                    for (int i = threadIdx.x; i < T / 4; i += kThreads) st[i] = __ldcg(gt + i);
+                    for (int i = (T / 2) * 2 + threadIdx.x; i < T; i += kThreads)
                         hbase[i] = __ldcg(p.hb + i);
+                    for (int i = (T / 4) * 4 + threadIdx.x; i < T; i += kThreads)
                         htbase[i] = __ldcg(p.ht + i);
-                    }
                 }
                 if (threadIdx.x < 5) s_misc[4 + (threadIdx.x < 2 ? threadIdx.x : threadIdx.x + 2)] = 0;
                 __syncthreads();
@@ -2074,8 +2083,12 @@ __global__ void __launch_bounds__(kThreads, 1) auction_kernel(const __grid_const
                 // hand the prices back to the grid; when another phase follows,
                 // reset its state now (the phase start then needs no barrier)
                 const bool again = status == BASE_OK && eps != 1;
-                if (p.HS && !again)  // the last phase: the assignment is read from p.ht
-                    for (int i = threadIdx.x; i < T; i += kThreads) p.ht[i] = htbase[i];
+                if (p.HS && !again) {  // the last phase: the assignment is read from p.ht
+                    const int4* st = reinterpret_cast<const int4*>(htbase);
+                    int4* gt = reinterpret_cast<int4*>(p.ht);
+                    for (int i = threadIdx.x; i < T / 4; i += kThreads) gt[i] = st[i];
+                    for (int i = (T / 4) * 4 + threadIdx.x; i < T; i += kThreads) p.ht[i] = htbase[i];
+                }
                 for (int e = threadIdx.x; e < E; e += kThreads) {
                     p.gprice[e] = s_price[e];
                     p.hcnt[e] = again ? 0 : s_hcnt[e];

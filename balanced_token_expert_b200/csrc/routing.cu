@@ -127,17 +127,24 @@ __global__ void chunk_hist_kernel(const int32_t* __restrict__ assign, int T, int
 }
 
 // one thread per expert walks the chunks; then a block scan over experts
-__global__ void chunk_scan_kernel(int32_t* __restrict__ chunk_counts, int nchunks, int E,
+__global__ void __launch_bounds__(1024) chunk_scan_kernel(int32_t* __restrict__ chunk_counts, int nchunks, int E,
                                   int32_t* __restrict__ offsets) {
     __shared__ int32_t s_tot[1024];
     __shared__ int32_t s_warp[32];
     const int e = threadIdx.x;
     int run = 0;
+    constexpr int kB = 8;  // chunks loaded per batch (their loads in flight together)
     if (e < E) {
-        for (int c = 0; c < nchunks; ++c) {
-            const int v = chunk_counts[(size_t)c * E + e];
-            chunk_counts[(size_t)c * E + e] = run;
-            run += v;
+        for (int c0 = 0; c0 < nchunks; c0 += kB) {
+            int v[kB];
+#pragma unroll
+            for (int i = 0; i < kB; ++i)
+                v[i] = c0 + i < nchunks ? chunk_counts[(size_t)(c0 + i) * E + e] : 0;
+#pragma unroll
+            for (int i = 0; i < kB; ++i) {
+                if (c0 + i < nchunks) chunk_counts[(size_t)(c0 + i) * E + e] = run;
+                run += v[i];
+            }
         }
     }
     // exclusive scan of run over experts (blockDim = 1024)
@@ -169,7 +176,16 @@ __global__ void chunk_scan_kernel(int32_t* __restrict__ chunk_counts, int nchunk
     }
     __syncthreads();
     if (e < E) {
-        for (int c = 0; c < nchunks; ++c) chunk_counts[(size_t)c * E + e] += s_tot[e];
+        const int base = s_tot[e];
+        for (int c0 = 0; c0 < nchunks; c0 += kB) {
+            int v[kB];
+#pragma unroll
+            for (int i = 0; i < kB; ++i)
+                v[i] = c0 + i < nchunks ? chunk_counts[(size_t)(c0 + i) * E + e] : 0;
+#pragma unroll
+            for (int i = 0; i < kB; ++i)
+                if (c0 + i < nchunks) chunk_counts[(size_t)(c0 + i) * E + e] = v[i] + base;
+        }
     }
 }
 
@@ -214,7 +230,7 @@ __global__ void chunk_rank_kernel(const int32_t* __restrict__ assign, int T, int
 // pass 1 counts them per expert, one thread per expert turns the counts into
 // per-warp starting slots (expert-major, warp order), pass 2 ranks each
 // 32-token group with match_any and writes perm, inv and gate.
-constexpr int kSmallSort = 32768;
+constexpr int kSmallSort = 16384;
 
 __global__ void __launch_bounds__(1024) sort_small_kernel(const int32_t* __restrict__ assign,
                                                           int T, int E, int32_t* __restrict__ perm,
@@ -229,18 +245,28 @@ __global__ void __launch_bounds__(1024) sort_small_kernel(const int32_t* __restr
     const unsigned lt = (1u << lane) - 1;
     const int per = ((T + 31) / 32 + 31) / 32 * 32;  // a multiple of 32 tokens per warp
     const int t0 = min(T, w * per), t1 = min(T, t0 + per);
+    const int ni = (t1 - t0 + kWarp - 1) / kWarp;      // <= kSmallSort / 1024 = 32 groups
     for (int e = lane; e < E; e += kWarp) cnt[w * E + e] = 0;
-    __syncwarp();
-    for (int b = t0; b < t1; b += kWarp) {
-        const int t = b + lane;
-        int e = t < t1 ? assign[t] : -1;
-        if (t < t1 && (e < 0 || e >= E)) {  // not an expert: recorded, token skipped
+    // every expert index of the warp's range in registers, loaded at once
+    int ev[kSmallSort / 1024];
+#pragma unroll
+    for (int i = 0; i < kSmallSort / 1024; ++i) {
+        const int t = t0 + i * kWarp + lane;
+        ev[i] = (i < ni && t < t1) ? assign[t] : -1;
+        if (i < ni && t < t1 && (ev[i] < 0 || ev[i] >= E)) {  // not an expert: recorded, skipped
             record_error(2001);
-            e = -1;
+            ev[i] = -1;
         }
-        const unsigned peers = __match_any_sync(0xffffffffu, e >= 0 ? e : -1 - lane);
-        if (e >= 0 && (peers & lt) == 0) cnt[w * E + e] += __popc(peers);
-        __syncwarp();
+    }
+    __syncwarp();
+#pragma unroll
+    for (int i = 0; i < kSmallSort / 1024; ++i) {
+        if (i < ni) {
+            const int e = ev[i];
+            const unsigned peers = __match_any_sync(0xffffffffu, e >= 0 ? e : -1 - lane);
+            if (e >= 0 && (peers & lt) == 0) cnt[w * E + e] += __popc(peers);
+            __syncwarp();
+        }
     }
     __syncthreads();
     // thread e: exclusive prefix of its column over the warps and its total,
@@ -280,20 +306,29 @@ __global__ void __launch_bounds__(1024) sort_small_kernel(const int32_t* __restr
         for (int v = 0; v < 32; ++v) cnt[v * E + e_me] += base;
     }
     __syncthreads();
-    for (int b = t0; b < t1; b += kWarp) {
-        const int t = b + lane;
-        int e = t < t1 ? assign[t] : -1;
-        if (e >= E) e = -1;
-        const unsigned peers = __match_any_sync(0xffffffffu, e >= 0 ? e : -1 - lane);
-        int slot = 0;
-        if (e >= 0) slot = cnt[w * E + e] + __popc(peers & lt);
-        __syncwarp();
-        if (e >= 0 && (peers & lt) == 0) cnt[w * E + e] += __popc(peers);
-        __syncwarp();
-        if (e >= 0) {
-            perm[slot] = t;
-            inv[t] = slot;
-            if (gate) gate[slot] = s[(size_t)t * E + e];
+    // the gate scores of the range, loaded at once
+    float gv[kSmallSort / 1024];
+#pragma unroll
+    for (int i = 0; i < kSmallSort / 1024; ++i) {
+        const int t = t0 + i * kWarp + lane;
+        gv[i] = (gate && i < ni && ev[i] >= 0) ? s[(size_t)t * E + ev[i]] : 0.f;
+    }
+#pragma unroll
+    for (int i = 0; i < kSmallSort / 1024; ++i) {
+        if (i < ni) {
+            const int t = t0 + i * kWarp + lane;
+            const int e = ev[i];
+            const unsigned peers = __match_any_sync(0xffffffffu, e >= 0 ? e : -1 - lane);
+            int slot = 0;
+            if (e >= 0) slot = cnt[w * E + e] + __popc(peers & lt);
+            __syncwarp();
+            if (e >= 0 && (peers & lt) == 0) cnt[w * E + e] += __popc(peers);
+            __syncwarp();
+            if (e >= 0) {
+                perm[slot] = t;
+                inv[t] = slot;
+                if (gate) gate[slot] = gv[i];
+            }
         }
     }
 }
