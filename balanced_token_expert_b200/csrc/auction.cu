@@ -644,7 +644,7 @@ struct Params {
     int32_t* assign;
     int64_t* price_out;
     base_auction_stats* stats;
-    const int32_t* minmax;
+    unsigned* mmenc;  // [2] max over q of enc(q) and of ~enc(q) (enc keeps the signed order)
     Ctrl* ctrl;
     unsigned* bar_flags;  // [gridDim.x] grid-barrier counts
     int64_t* gprice;   // [E]
@@ -1674,13 +1674,60 @@ __global__ void __launch_bounds__(kThreads, 1) auction_kernel(const __grid_const
     Team<kThreads> cta_team{s_hist, s_red, s_cnt};
     Team<32> warp_team{s_hist + warp * kHist, nullptr, nullptr};
 
-    const int64_t qmin = p.minmax[0], qmax = p.minmax[1];
-    const int64_t range = qmax - qmin;
     int status = BASE_OK;
     unsigned bar_gen = 0;  // grid barriers passed (the same in every CTA)
-    if (range > 0 && range > ((int64_t)1 << 58) / scale) status = BASE_ERR_INVALID_ARG;
-    int64_t eps = range * scale / kEpsDivisor;
-    if (eps < 1) eps = 1;
+    int64_t eps = 1;
+    {
+        // the score range for eps0: every CTA reduces a slice of q; the first
+        // phase's grid barrier publishes the result.  enc(x) = x ^ 2^31 as
+        // unsigned keeps the signed order, so two atomicMax on zeroed words
+        // give the max and (through ~enc) the min
+        unsigned mx = 0u, mn = 0u;
+        const size_t n = (size_t)T * E;
+        const bool vec = (reinterpret_cast<uintptr_t>(p.q) & 15) == 0;
+        const size_t n4 = vec ? n / 4 : 0;
+        const int4* q4 = reinterpret_cast<const int4*>(p.q);
+        for (size_t i = (size_t)cta * kThreads + threadIdx.x; i < n4; i += (size_t)ncta * kThreads) {
+            const int4 v = __ldg(q4 + i);
+            const unsigned a = (unsigned)v.x ^ 0x80000000u, b = (unsigned)v.y ^ 0x80000000u;
+            const unsigned c = (unsigned)v.z ^ 0x80000000u, d = (unsigned)v.w ^ 0x80000000u;
+            mx = max(mx, max(max(a, b), max(c, d)));
+            mn = max(mn, max(max(~a, ~b), max(~c, ~d)));
+        }
+        for (size_t i = n4 * 4 + (size_t)cta * kThreads + threadIdx.x; i < n;
+             i += (size_t)ncta * kThreads) {
+            const unsigned a = (unsigned)__ldg(p.q + i) ^ 0x80000000u;
+            mx = max(mx, a);
+            mn = max(mn, ~a);
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+            mn = max(mn, __shfl_xor_sync(0xffffffffu, mn, off));
+        }
+        // one pair of atomics per CTA (thousands on two words serialise)
+        unsigned* s_mm = reinterpret_cast<unsigned*>(s_hist);
+        if (lane == 0) {
+            s_mm[warp] = mx;
+            s_mm[kWarps + warp] = mn;
+        }
+        __syncthreads();
+        if (warp == 0) {
+            mx = lane < kWarps ? s_mm[lane] : 0u;
+            mn = lane < kWarps ? s_mm[kWarps + lane] : 0u;
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) {
+                mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+                mn = max(mn, __shfl_xor_sync(0xffffffffu, mn, off));
+            }
+            if (lane == 0) {
+                atomicMax(&p.mmenc[0], mx);
+                atomicMax(&p.mmenc[1], mn);
+            }
+        }
+        __syncthreads();
+    }
+    bool first_phase = true;
 
     // lanes per bidding token: the smallest power of two >= E, at most 32
     int G = 1;
@@ -1694,7 +1741,6 @@ __global__ void __launch_bounds__(kThreads, 1) auction_kernel(const __grid_const
     int cur = 0;  // which global list holds the bidders
 
     while (status == BASE_OK && ok) {
-        ++phases;
         // ---- phase start: nothing held, prices kept (in p.gprice); after a
         // narrow phase CTA 0 has done this already, before the grid barrier
         if (!reset_done) {
@@ -1706,6 +1752,20 @@ __global__ void __launch_bounds__(kThreads, 1) auction_kernel(const __grid_const
             if (cta == 0 && threadIdx.x < 3) p.ctrl->ucount[threadIdx.x] = 0;
             if (!(ok = grid_sync(p, bar_gen, s_misc))) break;
         }
+        if (first_phase) {
+            // eps0 = (max q - min q)(T+1) / 50, from the range every CTA has reduced
+            first_phase = false;
+            const int64_t qmax = (int32_t)(vload(&p.mmenc[0]) ^ 0x80000000u);
+            const int64_t qmin = (int32_t)((~vload(&p.mmenc[1])) ^ 0x80000000u);
+            const int64_t range = qmax - qmin;
+            if (range > 0 && range > ((int64_t)1 << 58) / scale) {
+                status = BASE_ERR_INVALID_ARG;
+                break;
+            }
+            eps = range * scale / kEpsDivisor;
+            if (eps < 1) eps = 1;
+        }
+        ++phases;
         reset_done = false;
         int U = T;
         bool first = true;
@@ -2146,47 +2206,6 @@ __global__ void __launch_bounds__(kThreads, 1) auction_kernel(const __grid_const
     }
 }
 
-__global__ void minmax_init(int32_t* mm) {
-    mm[0] = INT32_MAX;
-    mm[1] = INT32_MIN;
-}
-
-__global__ void minmax_kernel(const int32_t* __restrict__ q, size_t n, int32_t* mm) {
-    int lo = INT32_MAX, hi = INT32_MIN;
-    const size_t n4 = n / 4;
-    const int4* q4 = reinterpret_cast<const int4*>(q);
-    for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n4;
-         i += (size_t)gridDim.x * blockDim.x) {
-        const int4 v = __ldg(q4 + i);
-        lo = min(min(lo, v.x), min(v.y, min(v.z, v.w)));
-        hi = max(max(hi, v.x), max(v.y, max(v.z, v.w)));
-    }
-    for (size_t i = n4 * 4 + blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n;
-         i += (size_t)gridDim.x * blockDim.x) {
-        lo = min(lo, q[i]);
-        hi = max(hi, q[i]);
-    }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-        lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, off));
-        hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, off));
-    }
-    __shared__ int slo[32], shi[32];
-    if (lane_id() == 0) {
-        slo[warp_id()] = lo;
-        shi[warp_id()] = hi;
-    }
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        for (int w = 1; w < (int)(blockDim.x / 32); ++w) {
-            lo = min(lo, slo[w]);
-            hi = max(hi, shi[w]);
-        }
-        atomicMin(&mm[0], lo);
-        atomicMax(&mm[1], hi);
-    }
-}
-
 // Shared-memory plan: the fringe capacity FK (<= 32), the per-expert bid
 // bucket NB (<= 32) and the staged rows RC (<= 32) as large as 200 KB allows,
 // the fringe first.
@@ -2220,7 +2239,7 @@ static SmemPlan smem_plan(int E, int NM, int T) {
 
 size_t auction_workspace_bytes(int T, int E) {
     const int C = T / E;
-    size_t b = 256;                                         // minmax
+    size_t b = align_up(2 * sizeof(unsigned), 256);         // score range
     b += align_up(sizeof(auction::Ctrl), 256);
     b += align_up(sizeof(unsigned) * auction::kMaxGrid, 256);  // grid-barrier flags
     b += align_up(64, 256);                                 // objective + counters
@@ -2270,9 +2289,8 @@ int launch_auction(const int32_t* q, int T, int E, int32_t* assign, int64_t* pri
     prm.u_trace = u_trace;
     prm.t_trace = t_trace;
     prm.trace_cap = (u_trace || t_trace) ? trace_cap : 0;
-    int32_t* mm = reinterpret_cast<int32_t*>(take(256));
-    prm.minmax = mm;
     unsigned char* zero_begin = w + o;
+    prm.mmenc = reinterpret_cast<unsigned*>(take(2 * sizeof(unsigned)));
     prm.ctrl = reinterpret_cast<Ctrl*>(take(sizeof(Ctrl)));
     prm.bar_flags = reinterpret_cast<unsigned*>(take(sizeof(unsigned) * kMaxGrid));
     prm.obj = reinterpret_cast<unsigned long long*>(take(64));
@@ -2292,12 +2310,7 @@ int launch_auction(const int32_t* q, int T, int E, int32_t* assign, int64_t* pri
 
     // control block, objective, prices (start at 0), counts
     if (cudaMemsetAsync(zero_begin, 0, zero_bytes, stream) != cudaSuccess) return BASE_ERR_CUDA;
-    minmax_init<<<1, 1, 0, stream>>>(mm);
-    BASE_RETURN_IF_LAUNCH_FAILED();
-    const size_t n = (size_t)T * E;
-    const int blocks = (int)std::min<size_t>((n / 4 + 255) / 256 + 1, 148 * 8);
-    minmax_kernel<<<blocks, 256, 0, stream>>>(q, n, mm);
-    BASE_RETURN_IF_LAUNCH_FAILED();
+
 
     if (cudaFuncSetAttribute(auction_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem) != cudaSuccess)
