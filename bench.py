@@ -33,6 +33,17 @@ METRIC = "tokens routed/s (auction) & BASE-layer fwd tokens/s; % of HBM/TC roofl
 UNIT = "tokens/s"
 
 
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per launch of a
+# step component, from one ncu capture of this bench's own command on the
+# named workload at its full size (the component's kernels summed); a
+# component whose kernels changed after their capture has no entry.
+NCU_TRAFFIC = {
+    ("auction", "layer_fwd"): 883200 + 3584,
+    ("scores", "layer_fwd"): 16837632,
+    ("ffn", "layer_fwd"): 151049984 + 39332864 + 222304000 + 11714816,
+}
+
+
 def parse():
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
@@ -384,15 +395,16 @@ def main():
 
         def roof(n):
             bound, work = alg[n]
+            traffic = None if args.tokens else NCU_TRAFFIC.get((n, wl.name))
             sec = comp[n] / 1e3
             if bound == "tensor":
                 a_ = work / sec / 1e12
                 return dict(bound="tensor", achieved=a_, peak=pk["bf16"], unit="TFLOP/s",
-                            frac=a_ / pk["bf16"], traffic=None, kernel=n, ms=comp[n],
+                            frac=a_ / pk["bf16"], traffic=traffic, kernel=n, ms=comp[n],
                             peak_source=pk["source"] + " burst bf16")
             a_ = work / sec / 1e9
             return dict(bound="hbm", achieved=a_, peak=pk["hbm"], unit="GB/s",
-                        frac=a_ / pk["hbm"], traffic=None, kernel=n, ms=comp[n],
+                        frac=a_ / pk["hbm"], traffic=traffic, kernel=n, ms=comp[n],
                         peak_source=pk["source"] + " hbm copy")
 
         res = dict(

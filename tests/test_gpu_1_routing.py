@@ -208,9 +208,12 @@ def test_auction_round_cap_in_the_last_rounds_of_a_phase(orc, name):
 
 
 # ------------------------------------------------------------------ permute / combine
+# up to 16384 tokens the sort by expert is one CTA; above, the three-kernel version
 @pytest.mark.parametrize("T,E,D,kind", [(1536, 4, 64, "balanced"), (1000, 5, 200, "ragged"),
                                         (4096, 128, 128, "ragged"), (333, 7, 8, "ragged"),
-                                        (2048, 2, 1024, "empty-expert")])
+                                        (2048, 2, 1024, "empty-expert"), (16384, 1024, 8, "ragged"),
+                                        (16385, 3, 16, "ragged"), (40000, 64, 64, "ragged"),
+                                        (20000, 5, 8, "empty-expert")])
 def test_permute_and_combine_bit_exact(orc, T, E, D, kind):
     rng = np.random.default_rng(T + D)
     if kind == "balanced":
