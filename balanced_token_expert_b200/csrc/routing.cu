@@ -341,43 +341,28 @@ template <bool kScatter>
 __global__ void __launch_bounds__(256) move_rows_kernel(const uint4* __restrict__ src,
                                                         const int32_t* __restrict__ idx, int T,
                                                         int vec_per_row, uint4* __restrict__ dst) {
+    // one warp per row: the index is read once, the row's 16-byte vectors are
+    // spread over the lanes (coalesced), several loads in flight per lane
     constexpr int kUnroll = 4;
-    const long long total = (long long)T * vec_per_row;
-    const long long stride = (long long)gridDim.x * blockDim.x;
-    long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x;
-    for (; i + (kUnroll - 1) * stride < total; i += kUnroll * stride) {
-        uint4 v[kUnroll];
-        long long o[kUnroll];
-        bool bad = false;
-#pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-            const long long j = i + u * stride;
-            const int r = (int)(j / vec_per_row), c = (int)(j % vec_per_row);
-            int m = __ldg(idx + r);
-            if ((unsigned)m >= (unsigned)T) {  // not a row: recorded, row 0 used instead
-                bad = true;
-                m = 0;
-            }
-            const long long si = kScatter ? j : (long long)m * vec_per_row + c;
-            o[u] = kScatter ? (long long)m * vec_per_row + c : j;
-            v[u] = __ldcs(src + si);
-        }
-        if (bad) {
-            record_error(2002);
-            continue;
-        }
-#pragma unroll
-        for (int u = 0; u < kUnroll; ++u) __stcs(dst + o[u], v[u]);
-    }
-    for (; i < total; i += stride) {
-        const int r = (int)(i / vec_per_row), c = (int)(i % vec_per_row);
+    const int lane = lane_id();
+    const long long nwarps = (long long)gridDim.x * (blockDim.x / kWarp);
+    for (long long r = blockIdx.x * (long long)(blockDim.x / kWarp) + warp_id(); r < T; r += nwarps) {
         const int m = __ldg(idx + r);
-        if ((unsigned)m >= (unsigned)T) {
-            record_error(2002);
+        if ((unsigned)m >= (unsigned)T) {  // not a row: recorded, the row skipped
+            if (lane == 0) record_error(2002);
             continue;
         }
-        if (kScatter) __stcs(dst + (long long)m * vec_per_row + c, __ldcs(src + i));
-        else __stcs(dst + i, __ldcs(src + (long long)m * vec_per_row + c));
+        const uint4* s_row = src + (kScatter ? r : (long long)m) * vec_per_row;
+        uint4* d_row = dst + (kScatter ? (long long)m : r) * vec_per_row;
+        int c = lane;
+        for (; c + (kUnroll - 1) * kWarp < vec_per_row; c += kUnroll * kWarp) {
+            uint4 v[kUnroll];
+#pragma unroll
+            for (int u = 0; u < kUnroll; ++u) v[u] = __ldcs(s_row + c + u * kWarp);
+#pragma unroll
+            for (int u = 0; u < kUnroll; ++u) __stcs(d_row + c + u * kWarp, v[u]);
+        }
+        for (; c < vec_per_row; c += kWarp) __stcs(d_row + c, __ldcs(s_row + c));
     }
 }
 
@@ -448,10 +433,9 @@ int launch_sort_by_expert(const int32_t* assign, int T, int E, int32_t* perm, in
 int launch_move_rows(const void* src, const int32_t* idx, int T, int D, void* dst, bool scatter,
                      cudaStream_t stream) {
     const int vec = D * 2 / 16;
-    const long long total = (long long)T * vec;
-    const int threads = 256;
-    long long blocks = (total + threads - 1) / threads;
-    if (blocks > 148 * 16) blocks = 148 * 16;
+    const int threads = 256;  // eight rows in flight per block, one per warp
+    long long blocks = ((long long)T + threads / kWarp - 1) / (threads / kWarp);
+    if (blocks > 148 * 64) blocks = 148 * 64;
     if (blocks < 1) blocks = 1;
     if (scatter)
         routing::move_rows_kernel<true><<<(int)blocks, threads, 0, stream>>>(

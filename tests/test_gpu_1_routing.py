@@ -242,3 +242,30 @@ def test_permute_and_combine_bit_exact(orc, T, E, D, kind):
     assert torch.equal(xp.cpu(), h[torch.from_numpy(po.astype(np.int64))])
     assert np.array_equal(to_np(gate), s[po, assign[po]])
     assert torch.equal(out.cpu(), h)  # combine undoes the permutation exactly
+
+
+def test_out_of_range_entries_are_recorded_not_followed():
+    # the kernels' own range checks: an expert index outside [0, E) in the
+    # assignment (2001) and a row index outside [0, T) in the permutation
+    # (2002) are recorded in the device error word and skipped
+    T, E, D = 1000, 5, 64
+    B.base_device_error(clear=True)
+    assign = torch.randint(0, E, (T,), dtype=torch.int32, generator=torch.Generator().manual_seed(1))
+    assign[17] = E
+    perm = torch.empty(T, dtype=torch.int32, device="cuda")
+    inv = torch.empty_like(perm)
+    offs = torch.empty(E + 1, dtype=torch.int32, device="cuda")
+    B.base_permute(None, assign.cuda(), E, perm, inv, offs, None, ws=buffers.workspace(T, E, D))
+    torch.cuda.synchronize()
+    assert B.base_device_error(clear=True) == 2001
+    assert int(offs[E].item()) == T - 1  # the bad token is left out
+    y = torch.randn(T, D).to(torch.bfloat16).cuda()
+    bad = torch.arange(T, dtype=torch.int32, device="cuda")
+    bad[3] = T
+    out = torch.zeros(T, D, dtype=torch.bfloat16, device="cuda")
+    B.base_combine(y, bad, out)
+    torch.cuda.synchronize()
+    assert B.base_device_error(clear=True) == 2002
+    keep = torch.ones(T, dtype=torch.bool)
+    keep[3] = False
+    assert torch.equal(out.cpu()[keep], y.cpu()[keep])
