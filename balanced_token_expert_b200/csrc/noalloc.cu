@@ -4,12 +4,13 @@
 // Some callers of this library only ever hold the input and output buffers
 // and a stream: a plugin running inside another runtime that owns all device
 // memory, or a serving loop that must not call cudaMalloc while it runs.
-// They cannot pass base_permute the workspace it needs for its per-chunk
+// They cannot pass base_permute the workspace it needs for its per-slice
 // expert counts.  base_permute_noalloc keeps that scratch in the file-scope
 // array below instead, a fixed 4 MiB reserved in every GPU that loads the
 // library, until the process exits.
 //
-// The scratch holds ceil(T / 256) * E int32 counts, so a call needs
+// The scratch holds the expert counts of at most ceil(T / 256) token slices
+// (ceil(T / 256) * E int32), so a call needs
 // ceil(T / 256) * E <= kNoallocScratchInts (for example T = 131072 tokens
 // with E up to 2048 experts); larger shapes are rejected with
 // BASE_ERR_WORKSPACE before anything is launched.  Every count the kernels

@@ -6,6 +6,8 @@
 //   * the expert-major permutation (fig. 2 sort_by_expert) as a stable
 //     counting sort, and the 16-byte-vector row gather / scatter used by the
 //     permute, the combine (inverse_sort) and the backward.
+#include <algorithm>
+
 #include "common.cuh"
 
 namespace base {
@@ -93,164 +95,58 @@ __global__ void greedy_kernel(const int32_t* __restrict__ q, int T, int E,
 }
 
 // ---------------------------------------------------------------------------
-// stable counting sort of tokens by expert (more than kSmallSort tokens; see
-// sort_small_kernel below for the one-CTA version)
-//   chunk = kChunk consecutive tokens handled by one warp, in token order.
-//   1) per-chunk expert histogram  2) scan over chunks and experts
-//   3) per-chunk ranks -> perm, inv (and the permuted gate scores)
+// stable counting sort of tokens by expert (expert-major slots, ascending
+// token inside an expert): perm, inv, offsets and the permuted gate scores
 // ---------------------------------------------------------------------------
-constexpr int kChunk = 256;
-constexpr int kSortWarps = 4;
+// The sort runs over P slices of consecutive tokens, one CTA
+// per slice, in two launches:
+//   slice_hist_kernel   the expert counts of every slice (shared atomics);
+//   slice_rank_kernel   each CTA sums the counts of the slices before its own
+//                       (its starting slot per expert) and of all slices (the
+//                       expert offsets, an exclusive scan over experts), then
+//                       ranks its tokens in order: warp w takes a contiguous
+//                       part of the slice, counts it per expert, the counts
+//                       become per-warp starting slots, and each 32-token group
+//                       is ranked with match_any (ties in token order).
+constexpr int kSliceMax = 8192;  // tokens per slice: 32 warps x 8 groups of 32
 
-__global__ void chunk_hist_kernel(const int32_t* __restrict__ assign, int T, int E,
-                                  int32_t* __restrict__ chunk_counts) {
-    extern __shared__ int32_t s_cnt[];  // [kSortWarps][E]
-    const int w = warp_id(), lane = lane_id();
-    int32_t* my = s_cnt + w * E;
-    const int chunk = blockIdx.x * kSortWarps + w;
-    const int nchunks = (T + kChunk - 1) / kChunk;
-    for (int e = lane; e < E; e += kWarp) my[e] = 0;
-    __syncwarp();
-    if (chunk < nchunks) {
-        const int t0 = chunk * kChunk, t1 = min(T, t0 + kChunk);
-        for (int t = t0 + lane; t < t1; t += kWarp) {
-            const int e = assign[t];
-            if (e < 0 || e >= E) {  // not an expert: recorded, token skipped
-                record_error(2001);
-                continue;
-            }
-            atomicAdd(&my[e], 1);
-        }
-        __syncwarp();
-        for (int e = lane; e < E; e += kWarp) chunk_counts[(size_t)chunk * E + e] = my[e];
-    }
-}
-
-// one thread per expert walks the chunks; then a block scan over experts
-__global__ void __launch_bounds__(1024) chunk_scan_kernel(int32_t* __restrict__ chunk_counts, int nchunks, int E,
-                                  int32_t* __restrict__ offsets) {
-    __shared__ int32_t s_tot[1024];
-    __shared__ int32_t s_warp[32];
-    const int e = threadIdx.x;
-    int run = 0;
-    constexpr int kB = 8;  // chunks loaded per batch (their loads in flight together)
-    if (e < E) {
-        for (int c0 = 0; c0 < nchunks; c0 += kB) {
-            int v[kB];
-#pragma unroll
-            for (int i = 0; i < kB; ++i)
-                v[i] = c0 + i < nchunks ? chunk_counts[(size_t)(c0 + i) * E + e] : 0;
-#pragma unroll
-            for (int i = 0; i < kB; ++i) {
-                if (c0 + i < nchunks) chunk_counts[(size_t)(c0 + i) * E + e] = run;
-                run += v[i];
-            }
-        }
-    }
-    // exclusive scan of run over experts (blockDim = 1024)
-    const int lane = lane_id(), w = warp_id();
-    int incl = (e < E) ? run : 0;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-        const int o = __shfl_up_sync(0xffffffffu, incl, off);
-        if (lane >= off) incl += o;
-    }
-    if (lane == 31) s_warp[w] = incl;
+__global__ void __launch_bounds__(1024) slice_hist_kernel(const int32_t* __restrict__ assign,
+                                                          int T, int E, int slice,
+                                                          int32_t* __restrict__ cnt) {
+    extern __shared__ int32_t sh[];  // [E]
+    for (int e = threadIdx.x; e < E; e += blockDim.x) sh[e] = 0;
     __syncthreads();
-    if (w == 0) {
-        int v = s_warp[lane];
-        int vi = v;
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-            const int o = __shfl_up_sync(0xffffffffu, vi, off);
-            if (lane >= off) vi += o;
-        }
-        s_warp[lane] = vi - v;
+    const int t0 = blockIdx.x * slice, t1 = min(T, t0 + slice);
+    for (int t = t0 + threadIdx.x; t < t1; t += blockDim.x) {
+        const int e = assign[t];
+        if (e >= 0 && e < E) atomicAdd(&sh[e], 1);
     }
     __syncthreads();
-    const int excl = incl - ((e < E) ? run : 0) + s_warp[w];
-    if (e < E) {
-        s_tot[e] = excl;
-        offsets[e] = excl;
-        if (e == E - 1) offsets[E] = excl + run;
-    }
-    __syncthreads();
-    if (e < E) {
-        const int base = s_tot[e];
-        for (int c0 = 0; c0 < nchunks; c0 += kB) {
-            int v[kB];
-#pragma unroll
-            for (int i = 0; i < kB; ++i)
-                v[i] = c0 + i < nchunks ? chunk_counts[(size_t)(c0 + i) * E + e] : 0;
-#pragma unroll
-            for (int i = 0; i < kB; ++i)
-                if (c0 + i < nchunks) chunk_counts[(size_t)(c0 + i) * E + e] = v[i] + base;
-        }
-    }
+    for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[(size_t)blockIdx.x * E + e] = sh[e];
 }
 
-__global__ void chunk_rank_kernel(const int32_t* __restrict__ assign, int T, int E,
-                                  const int32_t* __restrict__ chunk_base,
-                                  int32_t* __restrict__ perm, int32_t* __restrict__ inv,
-                                  const float* __restrict__ s, float* __restrict__ gate) {
-    extern __shared__ int32_t s_run[];  // [kSortWarps][E]
-    const int w = warp_id(), lane = lane_id();
-    int32_t* run = s_run + w * E;
-    const int chunk = blockIdx.x * kSortWarps + w;
-    const int nchunks = (T + kChunk - 1) / kChunk;
-    if (chunk >= nchunks) return;
-    for (int e = lane; e < E; e += kWarp) run[e] = chunk_base[(size_t)chunk * E + e];
-    __syncwarp();
-    const int t0 = chunk * kChunk, t1 = min(T, t0 + kChunk);
-    for (int b = t0; b < t1; b += kWarp) {
-        const int t = b + lane;
-        bool valid = t < t1;
-        int e = valid ? assign[t] : -1;
-        if (e < 0 || e >= E) {
-            e = -1 - lane;  // distinct dummies never match
-            valid = false;
-        }
-        const unsigned peers = __match_any_sync(0xffffffffu, e);
-        const int rank = __popc(peers & ((1u << lane) - 1));
-        int slot = 0;
-        if (valid) slot = run[e] + rank;
-        __syncwarp();
-        if (valid && lane == 31 - __clz(peers)) run[e] += __popc(peers);
-        __syncwarp();
-        if (valid) {
-            perm[slot] = t;
-            inv[t] = slot;
-            if (gate) gate[slot] = s[(size_t)t * E + e];
-        }
-    }
-}
-
-// The same stable counting sort in one CTA for up to kSmallSort tokens (one
-// launch instead of three): warp w takes tokens [w per, (w+1) per) in order;
-// pass 1 counts them per expert, one thread per expert turns the counts into
-// per-warp starting slots (expert-major, warp order), pass 2 ranks each
-// 32-token group with match_any and writes perm, inv and gate.
-constexpr int kSmallSort = 16384;
-
-__global__ void __launch_bounds__(1024) sort_small_kernel(const int32_t* __restrict__ assign,
-                                                          int T, int E, int32_t* __restrict__ perm,
+__global__ void __launch_bounds__(1024) slice_rank_kernel(const int32_t* __restrict__ assign,
+                                                          int T, int E, int slice,
+                                                          const int32_t* __restrict__ cnt,
+                                                          int32_t* __restrict__ perm,
                                                           int32_t* __restrict__ inv,
                                                           int32_t* __restrict__ offsets,
                                                           const float* __restrict__ s,
                                                           float* __restrict__ gate) {
     extern __shared__ int32_t sm[];
-    int32_t* cnt = sm;                 // [32][E]: counts, then running slots
+    int32_t* wc = sm;                  // [32][E]: per-warp counts, then running slots
     int32_t* s_warp = sm + 32 * E;     // [32] block-scan partials
     const int w = warp_id(), lane = lane_id();
     const unsigned lt = (1u << lane) - 1;
-    const int per = ((T + 31) / 32 + 31) / 32 * 32;  // a multiple of 32 tokens per warp
-    const int t0 = min(T, w * per), t1 = min(T, t0 + per);
-    const int ni = (t1 - t0 + kWarp - 1) / kWarp;      // <= kSmallSort / 1024 = 32 groups
-    for (int e = lane; e < E; e += kWarp) cnt[w * E + e] = 0;
-    // every expert index of the warp's range in registers, loaded at once
-    int ev[kSmallSort / 1024];
+    const int b = blockIdx.x;
+    const int s0 = b * slice, s1 = min(T, s0 + slice);
+    const int per = ((s1 - s0 + 31) / 32 + 31) / 32 * 32;  // tokens per warp (multiple of 32)
+    const int t0 = min(s1, s0 + w * per), t1 = min(s1, t0 + per);
+    const int ni = (t1 - t0 + kWarp - 1) / kWarp;         // <= kSliceMax / 1024 groups
+    for (int e = lane; e < E; e += kWarp) wc[w * E + e] = 0;
+    int ev[kSliceMax / 1024];
 #pragma unroll
-    for (int i = 0; i < kSmallSort / 1024; ++i) {
+    for (int i = 0; i < kSliceMax / 1024; ++i) {
         const int t = t0 + i * kWarp + lane;
         ev[i] = (i < ni && t < t1) ? assign[t] : -1;
         if (i < ni && t < t1 && (ev[i] < 0 || ev[i] >= E)) {  // not an expert: recorded, skipped
@@ -260,27 +156,32 @@ __global__ void __launch_bounds__(1024) sort_small_kernel(const int32_t* __restr
     }
     __syncwarp();
 #pragma unroll
-    for (int i = 0; i < kSmallSort / 1024; ++i) {
+    for (int i = 0; i < kSliceMax / 1024; ++i) {
         if (i < ni) {
             const int e = ev[i];
             const unsigned peers = __match_any_sync(0xffffffffu, e >= 0 ? e : -1 - lane);
-            if (e >= 0 && (peers & lt) == 0) cnt[w * E + e] += __popc(peers);
+            if (e >= 0 && (peers & lt) == 0) wc[w * E + e] += __popc(peers);
             __syncwarp();
         }
     }
     __syncthreads();
-    // thread e: exclusive prefix of its column over the warps and its total,
-    // then an exclusive scan of the totals over the experts
-    int run = 0;
-    for (int e = threadIdx.x; e < E; e += blockDim.x) {  // E <= 1024: one pass
+    // thread e: the slices before this one and all slices, then this slice's
+    // warps; an exclusive scan of the totals over the experts
+    const int e_me = threadIdx.x;  // E <= 1024 = blockDim
+    int before = 0, total = 0, run = 0;
+    if (e_me < E) {
+        for (int bb = 0; bb < (int)gridDim.x; ++bb) {
+            const int c = cnt[(size_t)bb * E + e_me];
+            before += bb < b ? c : 0;
+            total += c;
+        }
         for (int v = 0; v < 32; ++v) {
-            const int c = cnt[v * E + e];
-            cnt[v * E + e] = run;
+            const int c = wc[v * E + e_me];
+            wc[v * E + e_me] = run;
             run += c;
         }
     }
-    const int e_me = threadIdx.x;
-    int incl = e_me < E ? run : 0;
+    int incl = e_me < E ? total : 0;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
         const int o = __shfl_up_sync(0xffffffffu, incl, off);
@@ -300,29 +201,31 @@ __global__ void __launch_bounds__(1024) sort_small_kernel(const int32_t* __restr
     }
     __syncthreads();
     if (e_me < E) {
-        const int base = incl - run + s_warp[w];
-        offsets[e_me] = base;
-        if (e_me == E - 1) offsets[E] = base + run;
-        for (int v = 0; v < 32; ++v) cnt[v * E + e_me] += base;
+        const int off_e = incl - total + s_warp[w];  // expert e's first slot
+        if (b == 0) {
+            offsets[e_me] = off_e;
+            if (e_me == E - 1) offsets[E] = off_e + total;
+        }
+        const int base = off_e + before;
+        for (int v = 0; v < 32; ++v) wc[v * E + e_me] += base;
     }
     __syncthreads();
-    // the gate scores of the range, loaded at once
-    float gv[kSmallSort / 1024];
+    float gv[kSliceMax / 1024];
 #pragma unroll
-    for (int i = 0; i < kSmallSort / 1024; ++i) {
+    for (int i = 0; i < kSliceMax / 1024; ++i) {
         const int t = t0 + i * kWarp + lane;
         gv[i] = (gate && i < ni && ev[i] >= 0) ? s[(size_t)t * E + ev[i]] : 0.f;
     }
 #pragma unroll
-    for (int i = 0; i < kSmallSort / 1024; ++i) {
+    for (int i = 0; i < kSliceMax / 1024; ++i) {
         if (i < ni) {
             const int t = t0 + i * kWarp + lane;
             const int e = ev[i];
             const unsigned peers = __match_any_sync(0xffffffffu, e >= 0 ? e : -1 - lane);
             int slot = 0;
-            if (e >= 0) slot = cnt[w * E + e] + __popc(peers & lt);
+            if (e >= 0) slot = wc[w * E + e] + __popc(peers & lt);
             __syncwarp();
-            if (e >= 0 && (peers & lt) == 0) cnt[w * E + e] += __popc(peers);
+            if (e >= 0 && (peers & lt) == 0) wc[w * E + e] += __popc(peers);
             __syncwarp();
             if (e >= 0) {
                 perm[slot] = t;
@@ -396,9 +299,10 @@ int launch_greedy(const int32_t* q, int T, int E, int32_t* assign, int32_t* coun
     return BASE_OK;
 }
 
+// the slices' expert counts: at most ceil(T / 256) slices (slices hold >= 512 tokens)
 size_t permute_workspace_bytes(int T, int E) {
-    const size_t nchunks = (size_t)(T + routing::kChunk - 1) / routing::kChunk;
-    return align_up(sizeof(int32_t) * nchunks * E, 256) + 256;
+    const size_t nslices = (size_t)(T + 255) / 256;
+    return align_up(sizeof(int32_t) * nslices * E, 256) + 256;
 }
 
 // perm / inv / offsets (+ gate) from an assignment.  An expert index out of
@@ -407,25 +311,19 @@ int launch_sort_by_expert(const int32_t* assign, int T, int E, int32_t* perm, in
                           int32_t* offsets, const float* s, float* gate, void* ws,
                           cudaStream_t stream) {
     using namespace routing;
-    if (T <= kSmallSort) {
-        const size_t sm = sizeof(int32_t) * (32 * (size_t)E + 32);
-        if (cudaFuncSetAttribute(sort_small_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)sm) != cudaSuccess)
-            return BASE_ERR_CUDA;
-        sort_small_kernel<<<1, 1024, sm, stream>>>(assign, T, E, perm, inv, offsets, s, gate);
-        BASE_RETURN_IF_LAUNCH_FAILED();
-        return BASE_OK;
-    }
-    const int nchunks = (T + kChunk - 1) / kChunk;
-    int32_t* chunk_counts = static_cast<int32_t*>(ws);
-    const int blocks = (nchunks + kSortWarps - 1) / kSortWarps;
-    const size_t smem = sizeof(int32_t) * kSortWarps * E;
-    chunk_hist_kernel<<<blocks, kSortWarps * kWarp, smem, stream>>>(assign, T, E, chunk_counts);
+    // slices of at least 512 tokens, at most 128 of them up to 1M tokens (every
+    // CTA reads the counts of all slices)
+    const int slice = std::min(kSliceMax, std::max(512, (T + 127) / 128));
+    const int P = (T + slice - 1) / slice;
+    int32_t* cnt = static_cast<int32_t*>(ws);  // [P][E]
+    slice_hist_kernel<<<P, 1024, sizeof(int32_t) * E, stream>>>(assign, T, E, slice, cnt);
     BASE_RETURN_IF_LAUNCH_FAILED();
-    chunk_scan_kernel<<<1, 1024, 0, stream>>>(chunk_counts, nchunks, E, offsets);
-    BASE_RETURN_IF_LAUNCH_FAILED();
-    chunk_rank_kernel<<<blocks, kSortWarps * kWarp, smem, stream>>>(assign, T, E, chunk_counts, perm,
-                                                                   inv, s, gate);
+    const size_t sm = sizeof(int32_t) * (32 * (size_t)E + 32);
+    if (cudaFuncSetAttribute(slice_rank_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)sm) != cudaSuccess)
+        return BASE_ERR_CUDA;
+    slice_rank_kernel<<<P, 1024, sm, stream>>>(assign, T, E, slice, cnt, perm, inv, offsets, s,
+                                               gate);
     BASE_RETURN_IF_LAUNCH_FAILED();
     return BASE_OK;
 }

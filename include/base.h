@@ -156,9 +156,11 @@ int base_assign_greedy(const int32_t* q, int T, int E, int32_t* assign, int32_t*
  *   assign: T int32 output.  price: E int64 output (final prices).
  *   stats (nullable): device base_auction_stats.
  *   ws: workspace of at least base_workspace_size(T, E, 0, 0) bytes.
- * Runs as one cooperative grid of one 512-thread CTA per SM: rounds with
- * many bidders use every SM, the tail of each phase runs on one CTA with the
- * prices and each expert's worst held bids in shared memory.
+ * Runs as one cooperative grid of one 512-thread CTA per SM (the score range
+ * for eps is reduced inside it): rounds with many bidders use every SM, the
+ * tail of each phase runs on one CTA with the prices and each expert's worst
+ * held bids in shared memory, and once a single bidder is left one warp
+ * finishes the phase.
  */
 int base_assign_balanced(const int32_t* q, int T, int E, int32_t* assign, int64_t* price,
                          base_auction_stats* stats, void* ws, size_t ws_bytes,
@@ -197,8 +199,8 @@ int base_permute(const void* h, const int32_t* assign, int T, int D, int E,
  * inputs, outputs and a stream -- a plugin inside another runtime that owns
  * all device memory, or a serving loop that must not call cudaMalloc -- has
  * no workspace to give base_permute.  This entry point takes the same
- * arguments minus the workspace and keeps the scratch (the per-chunk expert
- * counts, ceil(T/256) * E int32) in a 4 MiB array that the library reserves
+ * arguments minus the workspace and keeps the scratch (the expert counts of
+ * up to ceil(T/256) token slices, int32) in a 4 MiB array that the library reserves
  * in every GPU that loads it, for the life of the process.
  *   Limit: ceil(T/256) * E <= 1048576, else BASE_ERR_WORKSPACE and nothing
  *   is launched.  Allocates nothing.
