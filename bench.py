@@ -337,47 +337,86 @@ def main():
     ms = replicas.max_over_ranks(ms, device=torch.device("cuda"))
     clk = clocks.stop() if clocks else None
 
-    # end to end through the public call: host inputs in, host output back
-    h_host = inp.h.pin_memory()
-    h_dev = torch.empty_like(h)
+    # end to end through the public call: every step copies its tokens in from
+    # pinned host memory and reads its result back.  Measured two ways: step by
+    # step (copy in, compute, copy out, synchronise), and as a serving loop runs
+    # it (one copy stream each way and two device buffers: step i+1's input
+    # copy and step i-1's output copy overlap step i's compute).  Both keep the
+    # L2 flush between steps, on the compute stream inside the timed region.
+    nbuf = 2
+    h_host = [inp.h.pin_memory() for _ in range(nbuf)]
+    h_dev = [torch.empty_like(h) for _ in range(nbuf)]
     if F:
-        out_host = torch.empty(T, D, dtype=torch.bfloat16).pin_memory()
+        res_dev = [torch.empty(T, D, dtype=torch.bfloat16, device="cuda") for _ in range(nbuf)]
+        res_host = [torch.empty(T, D, dtype=torch.bfloat16).pin_memory() for _ in range(nbuf)]
         sv2 = buffers.layer_saved(T, E, D, F, for_backward=False)
 
-        def e2e_step():
-            h_dev.copy_(h_host, non_blocking=True)
-            B.base_layer_fwd(h_dev, w, W1, W2, act, B.BASE_ROUTE_BALANCED, out, sv2, ws)
-            out_host.copy_(out, non_blocking=True)
+        def compute(b):
+            B.base_layer_fwd(h_dev[b], w, W1, W2, act, B.BASE_ROUTE_BALANCED, res_dev[b], sv2, ws,
+                             stream=stream)
         d2h = T * D * 2
     else:
-        out_host = torch.empty(T, dtype=torch.int32).pin_memory()
+        res_dev = [torch.empty(T, dtype=torch.int32, device="cuda") for _ in range(nbuf)]
+        res_host = [torch.empty(T, dtype=torch.int32).pin_memory() for _ in range(nbuf)]
 
-        def e2e_step():
-            h_dev.copy_(h_host, non_blocking=True)
-            B.base_scores(h_dev, w, sv["s"], sv["q"])
+        def compute(b):
+            B.base_scores(h_dev[b], w, sv["s"], sv["q"], stream=stream)
             if q_bump is not None:
                 comps[1][1]()
-            B.base_assign_balanced(sv["q"], sv["assign"], sv["price"], sv["stats"], ws)
-            B.base_permute(h_dev, sv["assign"], E, sv["perm"], sv["inv"], sv["offsets"],
-                           sv["x_perm"], sv["s"], sv["gate"], ws)
-            out_host.copy_(sv["assign"], non_blocking=True)
+            B.base_assign_balanced(sv["q"], res_dev[b], sv["price"], sv["stats"], ws, stream=stream)
+            B.base_permute(h_dev[b], res_dev[b], E, sv["perm"], sv["inv"], sv["offsets"],
+                           sv["x_perm"], sv["s"], sv["gate"], ws, stream=stream)
         d2h = T * 4
 
-    for _ in range(3):
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    ev_in = [torch.cuda.Event() for _ in range(nbuf)]
+    ev_done = [torch.cuda.Event() for _ in range(nbuf)]
+    ev_out = [torch.cuda.Event() for _ in range(nbuf)]
+
+    def pipelined(K):
+        for i in range(K):
+            b = i % nbuf
+            with torch.cuda.stream(s_in):
+                if i >= nbuf:  # step i-2's compute has read h_dev[b]
+                    s_in.wait_event(ev_done[b])
+                h_dev[b].copy_(h_host[b], non_blocking=True)
+                ev_in[b].record(s_in)
+            stream.wait_event(ev_in[b])
+            if i >= nbuf:  # step i-2's output copy has read res_dev[b]
+                stream.wait_event(ev_out[b])
+            flush.zero_()
+            compute(b)
+            ev_done[b].record(stream)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(ev_done[b])
+                res_host[b].copy_(res_dev[b], non_blocking=True)
+                ev_out[b].record(s_out)
+
+    def serial_step():
         flush.zero_()
-        e2e_step()
-    torch.cuda.synchronize()
-    e2e_ms = []
-    for _ in range(args.steps):
-        flush.zero_()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
-        e2e_step()
-        b.record(stream)
-        b.synchronize()
-        e2e_ms.append(a.elapsed_time(b))
-    e2e = statistics.mean(e2e_ms)
+        h_dev[0].copy_(h_host[0], non_blocking=True)
+        compute(0)
+        res_host[0].copy_(res_dev[0], non_blocking=True)
+        b_.record(stream)
+        b_.synchronize()
+        return a.elapsed_time(b_)
+
+    for _ in range(3):
+        serial_step()
+    e2e_serial = statistics.mean([serial_step() for _ in range(args.steps)])
+    pipelined(3)
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(s_in)
+    pipelined(args.steps)
+    s_out.wait_stream(stream)
+    t1.record(s_out)
+    t1.synchronize()
+    e2e = t0.elapsed_time(t1) / args.steps
     e2e = replicas.max_over_ranks(e2e, device=torch.device("cuda"))
+    e2e_serial = replicas.max_over_ranks(e2e_serial, device=torch.device("cuda"))
 
     if rank == 0:
         pk = peaks()
@@ -419,6 +458,9 @@ def main():
                          phases=st["phases"], bids=bids, status=st["status"],
                          us_per_round=1e3 * comp["auction"] / max(1, st["rounds"])),
             e2e=dict(value=replicas.job_tokens_per_s(T, world, e2e), unit=UNIT,
+                     mode="pipelined: copy streams each way, two device buffers",
+                     serial_value=replicas.job_tokens_per_s(T, world, e2e_serial),
+                     serial_ms_per_step=e2e_serial,
                      h2d_bytes_per_step=T * D * 2,
                      d2h_bytes_per_step=d2h, ms_per_step=e2e),
             gpu_launches=kernels_per_step * args.steps,
