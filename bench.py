@@ -258,14 +258,16 @@ def main():
     if q_bump is not None:
         comps.append(("bump", lambda: sv["q"][:, 0].index_add_(
             0, q_bump[0], torch.full_like(q_bump[0], q_bump[1], dtype=torch.int32)), 0))
+    # third field: our kernels the call launches (the auction: one cooperative
+    # kernel; the permute: two sort launches and the row gather)
     comps.append(("auction", lambda: B.base_assign_balanced(sv["q"], sv["assign"], sv["price"],
-                                                             sv["stats"], ws), 3))
+                                                             sv["stats"], ws), 1))
     if not F:
         comps.append(("greedy", lambda: B.base_assign_greedy(sv["q"], greedy_assign,
                                                               greedy_counts), 1))
     comps.append(("permute", lambda: B.base_permute(h, sv["assign"], E, sv["perm"], sv["inv"],
                                                      sv["offsets"], sv["x_perm"], sv["s"],
-                                                     sv["gate"], ws), 4))
+                                                     sv["gate"], ws), 3))
     if F:
         comps.append(("ffn", lambda: B.base_expert_ffn(sv["x_perm"], sv["offsets"], W1, W2, act,
                                                        sv["gate"], sv["y_perm"], sv["h1"],
