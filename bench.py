@@ -339,8 +339,9 @@ def main():
     ms = replicas.max_over_ranks(ms, device=torch.device("cuda"))
     clk = clocks.stop() if clocks else None
 
-    # end to end through the public call: every step copies its tokens in from
-    # pinned host memory and reads its result back.  Measured two ways: step by
+    # end to end through the public call: every step copies its inputs in from
+    # pinned host memory (the tokens; for a training step also the upstream
+    # gradient) and reads its result back.  Measured two ways: step by
     # step (copy in, compute, copy out, synchronise), and as a serving loop runs
     # it (one copy stream each way and two device buffers: step i+1's input
     # copy and step i-1's output copy overlap step i's compute).  Both keep the
@@ -348,14 +349,30 @@ def main():
     nbuf = 2
     h_host = [inp.h.pin_memory() for _ in range(nbuf)]
     h_dev = [torch.empty_like(h) for _ in range(nbuf)]
+    ins = [[(h_dev[b], h_host[b])] for b in range(nbuf)]  # (device, pinned host) per input
     if F:
         res_dev = [torch.empty(T, D, dtype=torch.bfloat16, device="cuda") for _ in range(nbuf)]
         res_host = [torch.empty(T, D, dtype=torch.bfloat16).pin_memory() for _ in range(nbuf)]
-        sv2 = buffers.layer_saved(T, E, D, F, for_backward=False)
+        if wl.backward:
+            # a training step: forward (saving what the backward reads), then
+            # the backward; its inputs are h and the upstream gradient dout,
+            # the result read back is dh, the weight gradients stay on the
+            # device for an optimizer there
+            dout_dev = [torch.empty_like(dout) for _ in range(nbuf)]
+            for b in range(nbuf):
+                ins[b].append((dout_dev[b], inp.dout.pin_memory()))
 
-        def compute(b):
-            B.base_layer_fwd(h_dev[b], w, W1, W2, act, B.BASE_ROUTE_BALANCED, res_dev[b], sv2, ws,
-                             stream=stream)
+            def compute(b):
+                B.base_layer_fwd(h_dev[b], w, W1, W2, act, B.BASE_ROUTE_BALANCED, out, sv, ws,
+                                 stream=stream)
+                B.base_layer_bwd(h_dev[b], w, W1, W2, act, sv, dout_dev[b], res_dev[b], dw, dW1,
+                                 dW2, ws, stream=stream)
+        else:
+            sv2 = buffers.layer_saved(T, E, D, F, for_backward=False)
+
+            def compute(b):
+                B.base_layer_fwd(h_dev[b], w, W1, W2, act, B.BASE_ROUTE_BALANCED, res_dev[b], sv2,
+                                 ws, stream=stream)
         d2h = T * D * 2
     else:
         res_dev = [torch.empty(T, dtype=torch.int32, device="cuda") for _ in range(nbuf)]
@@ -381,7 +398,8 @@ def main():
             with torch.cuda.stream(s_in):
                 if i >= nbuf:  # step i-2's compute has read h_dev[b]
                     s_in.wait_event(ev_done[b])
-                h_dev[b].copy_(h_host[b], non_blocking=True)
+                for dst, src in ins[b]:
+                    dst.copy_(src, non_blocking=True)
                 ev_in[b].record(s_in)
             stream.wait_event(ev_in[b])
             if i >= nbuf:  # step i-2's output copy has read res_dev[b]
@@ -398,7 +416,8 @@ def main():
         flush.zero_()
         a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
-        h_dev[0].copy_(h_host[0], non_blocking=True)
+        for dst, src in ins[0]:
+            dst.copy_(src, non_blocking=True)
         compute(0)
         res_host[0].copy_(res_dev[0], non_blocking=True)
         b_.record(stream)
@@ -463,7 +482,7 @@ def main():
                      mode="pipelined: copy streams each way, two device buffers",
                      serial_value=replicas.job_tokens_per_s(T, world, e2e_serial),
                      serial_ms_per_step=e2e_serial,
-                     h2d_bytes_per_step=T * D * 2,
+                     h2d_bytes_per_step=sum(d.numel() * d.element_size() for d, _ in ins[0]),
                      d2h_bytes_per_step=d2h, ms_per_step=e2e),
             gpu_launches=kernels_per_step * args.steps,
             clocks=clk, device_error=err, wall_s=wall,
