@@ -41,6 +41,9 @@ NCU_TRAFFIC = {
     ("auction", "layer_fwd"): 883200 + 3584,
     ("scores", "layer_fwd"): 16837632,
     ("ffn", "layer_fwd"): 151049984 + 39332864 + 222304000 + 11714816,
+    # slice histogram + slice rank + row gather; the rows' writes stay in L2
+    ("permute", "layer_fwd"): 36608 + 588032 + 16819968,
+    ("combine", "layer_fwd"): 16815616,
 }
 
 
