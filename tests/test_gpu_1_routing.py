@@ -208,17 +208,24 @@ def test_auction_round_cap_in_the_last_rounds_of_a_phase(orc, name):
 
 
 # ------------------------------------------------------------------ permute / combine
-# up to 16384 tokens the sort by expert is one CTA; above, the three-kernel version
+# the sort by expert splits the tokens into up to 128 slices of 512..8192
+# consecutive tokens: one slice (T <= 512), a ragged last slice, the 8192-token
+# cap, and the three full workload shapes (balanced counts, shuffled experts)
 @pytest.mark.parametrize("T,E,D,kind", [(1536, 4, 64, "balanced"), (1000, 5, 200, "ragged"),
                                         (4096, 128, 128, "ragged"), (333, 7, 8, "ragged"),
                                         (2048, 2, 1024, "empty-expert"), (16384, 1024, 8, "ragged"),
                                         (16385, 3, 16, "ragged"), (40000, 64, 64, "ragged"),
-                                        (20000, 5, 8, "empty-expert")])
+                                        (20000, 5, 8, "empty-expert"),
+                                        (8192, 16, 1024, "shuffled-balanced"),
+                                        (32768, 32, 2048, "shuffled-balanced"),
+                                        (131072, 128, 2048, "shuffled-balanced")])
 def test_permute_and_combine_bit_exact(orc, T, E, D, kind):
     rng = np.random.default_rng(T + D)
     if kind == "balanced":
         q = rng.integers(-100000, 100000, size=(T, E)).astype(np.int32)
         assign = orc.auction(q)[0]
+    elif kind == "shuffled-balanced":
+        assign = rng.permutation(np.repeat(np.arange(E, dtype=np.int32), T // E))
     elif kind == "empty-expert":
         assign = np.zeros(T, dtype=np.int32)
     else:
