@@ -22,7 +22,8 @@ __all__ = [
     "base_status_string", "base_version", "base_workspace_size", "base_device_error",
     "base_scores", "base_assign_greedy", "base_assign_balanced", "base_assign_balanced_ex",
     "base_permute", "base_permute_noalloc", "base_expert_ffn", "base_combine", "base_layer_fwd",
-    "base_layer_bwd", "EXPORTED",
+    "base_layer_bwd", "base_test_inject", "BASE_TEST_WAIT_LIMIT_NS",
+    "BASE_TEST_AUCTION_ABSENT_CTA", "BASE_TEST_GEMM_DROP_FIRST_LOAD", "EXPORTED",
 ]
 
 BASE_OK = 0
@@ -30,13 +31,14 @@ BASE_F32, BASE_BF16 = 0, 1
 BASE_RELU, BASE_GELU = 0, 1
 BASE_ROUTE_BALANCED, BASE_ROUTE_GREEDY = 0, 1
 QSCALE = 65536.0
+BASE_TEST_WAIT_LIMIT_NS, BASE_TEST_AUCTION_ABSENT_CTA, BASE_TEST_GEMM_DROP_FIRST_LOAD = 0, 1, 2
 
 # every symbol include/base.h declares
 EXPORTED = (
     "base_status_string", "base_device_error", "base_version", "base_workspace_size",
     "base_scores", "base_assign_greedy", "base_assign_balanced", "base_assign_balanced_ex",
     "base_permute", "base_permute_noalloc", "base_expert_ffn", "base_combine", "base_layer_fwd",
-    "base_layer_bwd",
+    "base_layer_bwd", "base_test_inject",
 )
 
 
@@ -72,6 +74,7 @@ _SIGS = {
     "base_version": (ctypes.c_char_p, []),
     "base_device_error": (_i, [ctypes.POINTER(ctypes.c_int64), _i]),
     "base_workspace_size": (_sz, [_i, _i, _i, _i]),
+    "base_test_inject": (_i, [_i, ctypes.c_longlong]),
     "base_scores": (_i, [_vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp]),
     "base_assign_greedy": (_i, [_vp, _i, _i, _vp, _vp, _vp]),
     "base_assign_balanced": (_i, [_vp, _i, _i, _vp, _vp, _vp, _vp, _sz, _vp]),
@@ -138,6 +141,12 @@ def base_device_error(clear: bool = True) -> int:
     v = ctypes.c_int64(0)
     _check("base_device_error", lib().base_device_error(ctypes.byref(v), 1 if clear else 0))
     return int(v.value)
+
+
+def base_test_inject(hook: int, value: int) -> None:
+    """Test hooks of the bounded waits (include/base.h): a shorter wait limit,
+    an auction CTA that never arrives, a GEMM load that is never issued."""
+    _check("base_test_inject", lib().base_test_inject(int(hook), int(value)))
 
 
 def _dtype_code(t: torch.Tensor) -> int:

@@ -86,6 +86,25 @@ int base_device_error(int64_t* code, int clear) {
     return BASE_OK;
 }
 
+int base_test_inject(int hook, long long value) {
+    switch (hook) {
+        case BASE_TEST_WAIT_LIMIT_NS:
+            if (value < 0) return BASE_ERR_INVALID_ARG;
+            g_test_hooks.wait_ns = value;
+            return BASE_OK;
+        case BASE_TEST_AUCTION_ABSENT_CTA:
+            if (value < -1 || value > 1 << 20) return BASE_ERR_INVALID_ARG;
+            g_test_hooks.auction_absent_cta = (int)value;
+            return BASE_OK;
+        case BASE_TEST_GEMM_DROP_FIRST_LOAD:
+            if (value != 0 && value != 1) return BASE_ERR_INVALID_ARG;
+            g_test_hooks.gemm_drop_first_load = (int)value;
+            return BASE_OK;
+        default:
+            return BASE_ERR_INVALID_ARG;
+    }
+}
+
 int base_scores(const void* h, const void* w, int dtype, int T, int D, int E, float* s,
                 int32_t* q, cudaStream_t stream) {
     if (!h || !w || (!s && !q) || !shapes_ok(T, E) || D < 1) return BASE_ERR_INVALID_ARG;

@@ -663,6 +663,8 @@ struct Params {
     int32_t* u_trace;  // nullable: bidders of round r
     int64_t* t_trace;  // nullable: globaltimer (ns) at the start of round r
     long long trace_cap;
+    unsigned long long wait_ns;  // limit of every grid-barrier wait
+    int absent_cta;              // test hook: this CTA returns at once (-1: none)
 };
 
 __device__ __forceinline__ uint64_t globaltimer();
@@ -755,7 +757,7 @@ __device__ bool grid_sync(const Params& p, unsigned& gen, int* s_flag) {
                 if (lane == 0) {
                     if (*reinterpret_cast<volatile int*>(&p.ctrl->abort)) {
                         stop = 1;
-                    } else if (globaltimer() - t0 > kWaitNs || it > (1ll << 30)) {
+                    } else if (globaltimer() - t0 > p.wait_ns || it > (1ll << 30)) {
                         atomicExch(&p.ctrl->abort, 1);
                         record_error(5001);
                         stop = 1;
@@ -1670,6 +1672,7 @@ __global__ void __launch_bounds__(kThreads, 1) auction_kernel(const __grid_const
     const int64_t scale = (int64_t)T + 1;
     const int lane = lane_id(), warp = warp_id();
     const int cta = blockIdx.x, ncta = gridDim.x;
+    if (cta == p.absent_cta) return;  // test hook: the others' first grid barrier gives up
 
     Team<kThreads> cta_team{s_hist, s_red, s_cnt};
     Team<32> warp_team{s_hist + warp * kHist, nullptr, nullptr};
@@ -2177,7 +2180,10 @@ __global__ void __launch_bounds__(kThreads, 1) auction_kernel(const __grid_const
         eps /= kEpsFactor;
         if (eps < 1) eps = 1;
     }
-    if (!ok) return;
+    if (!ok) {
+        if (cta == 0 && threadIdx.x == 0 && p.stats) p.stats->status = BASE_ERR_TIMEOUT;
+        return;
+    }
 
     // results: every CTA writes its experts' tokens
     unsigned long long part = 0;
@@ -2195,7 +2201,10 @@ __global__ void __launch_bounds__(kThreads, 1) auction_kernel(const __grid_const
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
     if (lane == 0 && part) atomicAdd(p.obj, part);
-    if (!grid_sync(p, bar_gen, s_misc)) return;
+    if (!grid_sync(p, bar_gen, s_misc)) {
+        if (cta == 0 && threadIdx.x == 0 && p.stats) p.stats->status = BASE_ERR_TIMEOUT;
+        return;
+    }
     if (cta == 0 && threadIdx.x == 0 && p.stats) {
         p.stats->status = status;
         p.stats->phases = phases;
@@ -2289,6 +2298,8 @@ int launch_auction(const int32_t* q, int T, int E, int32_t* assign, int64_t* pri
     prm.u_trace = u_trace;
     prm.t_trace = t_trace;
     prm.trace_cap = (u_trace || t_trace) ? trace_cap : 0;
+    prm.wait_ns = g_test_hooks.wait_ns > 0 ? (unsigned long long)g_test_hooks.wait_ns : kWaitNs;
+    prm.absent_cta = g_test_hooks.auction_absent_cta;
     unsigned char* zero_begin = w + o;
     prm.mmenc = reinterpret_cast<unsigned*>(take(2 * sizeof(unsigned)));
     prm.ctrl = reinterpret_cast<Ctrl*>(take(sizeof(Ctrl)));

@@ -120,7 +120,7 @@ int launch_layer_bwd(const void* h, const void* w, const void* W1, const void* W
     {
         const int threads = 256;
         long long blocks = ((long long)T * kWarp + threads - 1) / threads;
-        if (blocks > 148 * 16) blocks = 148 * 16;
+        if (blocks > num_sms() * 16) blocks = num_sms() * 16;
         bwd::gate_grad_kernel<<<(int)blocks, threads, 0, stream>>>(
             dy, static_cast<const __nv_bfloat16*>(sv->f), sv->gate, T, D, dF, ds, sv->offsets, E, C);
         BASE_RETURN_IF_LAUNCH_FAILED();

@@ -30,10 +30,37 @@ __device__ __forceinline__ bool device_error_set() {
     return *reinterpret_cast<volatile int64_t*>(&g_device_error) != 0;
 }
 
+// Test hooks, set by base_test_inject (host side, process-wide; the
+// launchers copy them into the kernels' parameters).  With every field at its
+// default nothing changes.  They exist so that a test can watch a bounded wait
+// give up: a shorter wait limit, and an arrival that never comes (one auction
+// CTA that leaves before its first grid barrier, or one single-CTA GEMM CTA
+// that never issues its first TMA load).  No hook makes a kernel fault.
+struct TestHooks {
+    long long wait_ns;          // > 0: limit of every bounded wait, in ns
+    int auction_absent_cta;     // >= 0: this auction CTA returns at once
+    int gemm_drop_first_load;   // 1: CTA 0 of a one-CTA GEMM skips its first load
+};
+static TestHooks g_test_hooks = {0, -1, 0};
+
 // Iteration limit for every spin-wait in the library (try_wait already
 // suspends the thread for a while per attempt, so this is well above any
 // legitimate wait and far below a hung GPU).
 constexpr long long kSpinLimit = 1ll << 26;
+
+// SM count of the current device (host side, cached per device ordinal)
+static inline int num_sms() {
+    static int cache[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) dev = 0;
+    int* slot = dev < 64 ? &cache[dev] : nullptr;
+    if (slot && *slot > 0) return *slot;
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+        n = 148;
+    if (slot) *slot = n;
+    return n;
+}
 
 __device__ __forceinline__ int lane_id() { return threadIdx.x & 31; }
 __device__ __forceinline__ int warp_id() { return threadIdx.x >> 5; }

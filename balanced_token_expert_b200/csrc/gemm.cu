@@ -73,6 +73,8 @@ struct Args {
     int kgroup;                  // 1: groups split K (weight gradients), M and N fixed
     int m_tiles;                 // K-grouped mode: tiles along M per group
     int staged;                  // set by the launcher: output tensor maps are valid
+    unsigned long long wait_ns;  // set by the launcher: limit of every bounded wait
+    int drop_first_load;         // set by the launcher: test hook (one-CTA kernels only)
 };
 
 struct TileInfo {
@@ -423,9 +425,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             const TileInfo ti = decode_tile(args, tile, BN, BMP);
             const int a_row = ti.a_row + BM * (int)rank;
             for (int kb = 0; kb < ti.kblocks; ++kb) {
-                if (!tc::mbar_wait(&empty[stage], phase ^ 1, 3001)) {
+                if (!tc::mbar_wait(&empty[stage], phase ^ 1, 3001, args.wait_ns)) {
                     ok = false;
                     break;
+                }
+                if constexpr (CG == 1) {
+                    // test hook: CTA 0's first load is never issued, so the MMA
+                    // warp's wait for it runs out (the other copies still land)
+                    if (args.drop_first_load && blockIdx.x == 0 && tile == unit && kb == 0) {
+                        issued[stage] = false;
+                        if (++stage == STAGES) {
+                            stage = 0;
+                            phase ^= 1;
+                        }
+                        continue;
+                    }
                 }
                 uint32_t fbar;
                 if constexpr (CG == 2) {
@@ -493,14 +507,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t acc_phase = 0;
         bool ok = true;
         for (int tile = unit; tile < total && ok; tile += nunits) {
-            if (!tc::mbar_wait(&tempty[acc], acc_phase ^ 1, 3002)) break;
+            if (!tc::mbar_wait(&tempty[acc], acc_phase ^ 1, 3002, args.wait_ns)) break;
             tc::tc_fence_after();
             const uint32_t d_tmem = tmem_base + acc * BN;
             // only K-grouped tiles differ in depth (and need the tile's group)
             const int kblocks = args.kgroup ? decode_tile(args, tile, BN, BMP).kblocks
                                             : (args.K + BK - 1) / BK;
             for (int kb = 0; kb < kblocks; ++kb) {
-                if (!tc::mbar_wait(&full[stage], phase, 3003)) {
+                if (!tc::mbar_wait(&full[stage], phase, 3003, args.wait_ns)) {
                     ok = false;
                     break;
                 }
@@ -536,7 +550,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // every MMA issued by this thread has finished once `done` flips
         if constexpr (CG == 2) tc::umma_commit_cg2_mc(done, 0x1);
         else tc::umma_commit(done);
-        tc::mbar_wait(done, 0, 3004);
+        tc::mbar_wait(done, 0, 3004, args.wait_ns);
     } else if (warp >= 4) {
         // ---------------- epilogue ----------------
         const int ew = (warp - 4) & 3;                   // lane quadrant
@@ -552,7 +566,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t tempty_leader1 = (CG == 2) ? tc::map_to_rank(&tempty[1], 0) : 0u;
         for (int tile = unit; tile < total; tile += nunits) {
             const TileInfo ti = decode_tile(args, tile, BN, BMP);
-            const bool ok = tc::mbar_wait(&tfull[acc], acc_phase, 3005);
+            const bool ok = tc::mbar_wait(&tfull[acc], acc_phase, 3005, 2 * args.wait_ns);
             if (!__all_sync(0xffffffffu, ok)) break;  // the whole warp leaves together
             tc::tc_fence_after();
             const int r = BM * (int)rank + ew * 32 + lane;
@@ -709,16 +723,6 @@ static bool make_tmap_out(CUtensorMap* m, const void* base, uint64_t rows, uint6
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-static int num_sms() {
-    static int n = 0;
-    if (n == 0) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
-            n = 148;
-    }
-    return n;
-}
 
 // A: a_rows x a_cols row-major (K-major: a_cols = K; MN-major: a_rows = K)
 // B: b_rows x b_cols row-major (likewise).  CG = 2 launches clusters of two
@@ -733,6 +737,9 @@ static int launch(const void* A, uint64_t a_rows, uint64_t a_cols, const void* B
     memset(&to1, 0, sizeof(to1));
     Args a = args;
     a.staged = 0;
+    a.wait_ns = g_test_hooks.wait_ns > 0 ? (unsigned long long)g_test_hooks.wait_ns
+                                         : (unsigned long long)tc::kWaitNs;
+    a.drop_first_load = (CG == 1) ? g_test_hooks.gemm_drop_first_load : 0;
     // whole 128-byte row pieces and 16-byte aligned rows
     const bool stageable = EPI == EPI_F32 ? (args.N % 32 == 0) : (args.N % 64 == 0 && args.ld % 8 == 0);
     if (kStagedEpi<EPI> && stageable) {

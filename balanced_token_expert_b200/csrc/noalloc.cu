@@ -37,7 +37,9 @@ constexpr int kMaxDevices = 64;
 
 static __device__ __align__(256) int32_t g_permute_scratch[kNoallocScratchInts];
 
-// device address of g_permute_scratch, looked up once per device
+// device address of g_permute_scratch, looked up once per device ordinal and
+// kept for the life of the process (stale after cudaDeviceReset or in another
+// driver context on the same device: such callers use base_permute)
 static void* g_scratch_addr[kMaxDevices];
 static std::mutex g_scratch_mutex;
 

@@ -276,7 +276,7 @@ int launch_scores_f32(const float* h, const float* w, int T, int D, int E, float
     const long long items = (long long)T * E;
     const int threads = 256;
     long long blocks = (items * kWarp + threads - 1) / threads;
-    if (blocks > 148 * 16) blocks = 148 * 16;
+    if (blocks > num_sms() * 16) blocks = num_sms() * 16;
     routing::scores_f32_kernel<<<(int)blocks, threads, 0, stream>>>(h, w, T, D, E, s, q);
     BASE_RETURN_IF_LAUNCH_FAILED();
     return BASE_OK;
@@ -291,7 +291,7 @@ int launch_greedy(const int32_t* q, int T, int E, int32_t* assign, int32_t* coun
     while (G < E && G < kWarp) G <<= 1;
     const long long warps_needed = ((long long)T * G + kWarp - 1) / kWarp;
     long long blocks = (warps_needed * kWarp + threads - 1) / threads;
-    if (blocks > 148 * 8) blocks = 148 * 8;
+    if (blocks > num_sms() * 8) blocks = num_sms() * 8;
     if (blocks < 1) blocks = 1;
     routing::greedy_kernel<<<(int)blocks, threads, sizeof(int32_t) * E, stream>>>(q, T, E, assign,
                                                                                    counts);
@@ -333,7 +333,7 @@ int launch_move_rows(const void* src, const int32_t* idx, int T, int D, void* ds
     const int vec = D * 2 / 16;
     const int threads = 256;  // eight rows in flight per block, one per warp
     long long blocks = ((long long)T + threads / kWarp - 1) / (threads / kWarp);
-    if (blocks > 148 * 64) blocks = 148 * 64;
+    if (blocks > num_sms() * 64) blocks = num_sms() * 64;
     if (blocks < 1) blocks = 1;
     if (scatter)
         routing::move_rows_kernel<true><<<(int)blocks, threads, 0, stream>>>(

@@ -52,7 +52,8 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 // Waits for the phase with the given parity.  Returns false (and records
 // `code` in the device error word) when the wait gives up, or when another
 // part of the kernel already gave up.
-__device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int64_t code) {
+__device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int64_t code,
+                                       uint64_t limit_ns = kWaitNs) {
     const uint32_t a = smem_u32(bar);
     if (mbar_try_wait(a, parity)) return true;
     const uint64_t t0 = globaltimer();
@@ -60,7 +61,7 @@ __device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int64_t c
         if (mbar_try_wait(a, parity)) return true;
         if ((i & 127) == 0) {
             if (device_error_set()) return false;
-            if (globaltimer() - t0 > kWaitNs) break;
+            if (globaltimer() - t0 > limit_ns) break;
         }
     }
     record_error(code);

@@ -10,6 +10,12 @@ h ~ N(0,1), w ~ N(0, 1/D)).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
+The same run then times the other workloads a few steps each (--extra-steps)
+and reports them under "workloads": the skewed-affinity auction stress
+(T=32768, E=64), large routing (T=131072, E=128: scores, auction, greedy,
+permute) and the training step (T=32768, E=32, D=2048, FFN 8192 GELU,
+forward + backward).  --workload NAME --only times one workload alone.
+
 With N > 1 (torchrun, one rank per GPU) every rank runs its own independent
 problem (the balanced assignment decomposes per worker, so no collective is
 on the data path); the time is the max over ranks.  Rank 0 prints one JSON
@@ -56,6 +62,10 @@ def parse():
     p.add_argument("--workload", default="layer_fwd")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--flush-mb", type=int, default=256)
+    p.add_argument("--only", action="store_true",
+                   help="time the chosen workload alone (no other workloads in the same run)")
+    p.add_argument("--extra-steps", type=int, default=5,
+                   help="timed steps of each of the other workloads")
     p.add_argument("--tokens", type=int, default=0,
                    help="run the workload with this many tokens instead (profiling a small case)")
     return p.parse_args()
@@ -210,33 +220,17 @@ def _config(wl, args):
                 parallelism="independent replica per GPU")
 
 
-def main():
-    args = parse()
-    from balanced_token_expert_b200 import synth
-    wl = synth.WORKLOADS[args.workload]
-    if args.tokens:
-        wl = wl.scaled(T=args.tokens)
-    from balanced_token_expert_b200 import replicas
-    rank, world, local_rank = replicas.rank_env()
-    if args.impl == "reference":
-        run_reference(args, wl, rank, world)
-        return
+EXTRA_WORKLOADS = ("skewed", "large_routing", "layer_fwd_bwd")
 
+
+def measure(args, wl, steps, warmup, rank, world, local_rank):
+    """Times one workload: every component with CUDA events on the launching
+    stream (L2 flushed between steps, max over ranks), then end to end through
+    the public call with host buffers.  Returns the result dict (rank 0) or
+    None (other ranks); every rank takes the same collective steps."""
     import torch
-    import torch.distributed as dist
-    torch.cuda.set_device(local_rank)
-    if world > 1:
-        from datetime import timedelta
-        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
-                                device_id=torch.device("cuda", local_rank))
-    from balanced_token_expert_b200 import _build
     from balanced_token_expert_b200 import binding as B
-    from balanced_token_expert_b200 import buffers
-    if rank == 0 or world == 1:
-        _build.build()
-    if world > 1:
-        dist.barrier()
-    B.lib()
+    from balanced_token_expert_b200 import buffers, replicas, synth
 
     T, E, D, F = wl.T, wl.E, wl.D, wl.F
     inp = synth.make_inputs(wl, seed=replicas.rank_seed(rank))
@@ -309,20 +303,21 @@ def main():
     clocks = Clocks(phys) if rank == 0 else None
     kernels_per_step = sum(k for _, _, k in comps)
     mk = lambda: [torch.cuda.Event(enable_timing=True) for _ in range(2 * len(names))]  # noqa: E731
-    for _ in range(max(3, args.warmup)):
+    for _ in range(max(3, warmup)):
         flush.zero_()
         step(mk())
     torch.cuda.synchronize()
     B.base_device_error(clear=True)
 
-    evs = [mk() for _ in range(args.steps)]
+    evs = [mk() for _ in range(steps)]
     if world > 1:
+        import torch.distributed as dist
         dist.barrier()
     torch.cuda.synchronize()
     if clocks:
         clocks.mark_start()
     wall0 = time.perf_counter()
-    for i in range(args.steps):
+    for i in range(steps):
         flush.zero_()
         step(evs[i])
     torch.cuda.synchronize()
@@ -335,12 +330,23 @@ def main():
     for ev in evs:
         for j, n in enumerate(names):
             per[n].append(ev[2 * j].elapsed_time(ev[2 * j + 1]))
-    step_ms = [sum(per[n][i] for n in names) for i in range(args.steps)]
+    step_ms = [sum(per[n][i] for n in names) for i in range(steps)]
     ms = statistics.mean(step_ms)
     st = buffers.stats_dict(sv["stats"])
     err = B.base_device_error(clear=True)
     ms = replicas.max_over_ranks(ms, device=torch.device("cuda"))
     clk = clocks.stop() if clocks else None
+
+    # the auction's rounds by kind (an untimed traced run of the same call):
+    # time per round grouped by the number of bidders, from the GPU timer
+    trace_cap = st["rounds"] + 1
+    u_tr = torch.zeros(trace_cap, dtype=torch.int32, device="cuda")
+    t_tr = torch.zeros(trace_cap, dtype=torch.int64, device="cuda")
+    B.base_assign_balanced_ex(sv["q"], sv["assign"], sv["price"], sv["stats"], ws, 1000000,
+                              u_trace=u_tr, t_trace=t_tr)
+    torch.cuda.synchronize()
+    rounds_by_kind = _rounds_by_kind(u_tr.cpu().tolist(), t_tr.cpu().tolist(), st["rounds"],
+                                     wl.T)
 
     # end to end through the public call: every step copies its inputs in from
     # pinned host memory (the tokens; for a training step also the upstream
@@ -429,67 +435,135 @@ def main():
 
     for _ in range(3):
         serial_step()
-    e2e_serial = statistics.mean([serial_step() for _ in range(args.steps)])
+    e2e_serial = statistics.mean([serial_step() for _ in range(steps)])
     pipelined(3)
     torch.cuda.synchronize()
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     t0.record(s_in)
-    pipelined(args.steps)
+    pipelined(steps)
     s_out.wait_stream(stream)
     t1.record(s_out)
     t1.synchronize()
-    e2e = t0.elapsed_time(t1) / args.steps
+    e2e = t0.elapsed_time(t1) / steps
     e2e = replicas.max_over_ranks(e2e, device=torch.device("cuda"))
     e2e_serial = replicas.max_over_ranks(e2e_serial, device=torch.device("cuda"))
+    if rank != 0:
+        return None
 
+    pk = peaks()
+    comp = {n: statistics.mean(per[n]) for n in names}
+    dom = max(comp, key=comp.get)
+    bids = st["bids"]
+    alg = dict(  # algorithmic work per launch (bytes or flops)
+        scores=("hbm", 2 * T * D + 2 * E * D + 8 * T * E),
+        auction=("hbm", 4 * E * bids + 4 * T + 8 * E),
+        permute=("hbm", 4 * T * D + 12 * T + 8 * T),
+        ffn=("tensor", 4 * T * D * F),
+        combine=("hbm", 4 * T * D + 4 * T),
+        greedy=("hbm", 4 * T * E + 4 * T),
+        backward=("tensor", 8 * T * D * F))
+
+    def roof(n):
+        bound, work = alg[n]
+        traffic = None if args.tokens else NCU_TRAFFIC.get((n, wl.name))
+        sec = comp[n] / 1e3
+        if bound == "tensor":
+            a_ = work / sec / 1e12
+            return dict(bound="tensor", achieved=a_, peak=pk["bf16"], unit="TFLOP/s",
+                        frac=a_ / pk["bf16"], traffic=traffic, kernel=n, ms=comp[n],
+                        peak_source=pk["source"] + " burst bf16")
+        a_ = work / sec / 1e9
+        return dict(bound="hbm", achieved=a_, peak=pk["hbm"], unit="GB/s",
+                    frac=a_ / pk["hbm"], traffic=traffic, kernel=n, ms=comp[n],
+                    peak_source=pk["source"] + " hbm copy")
+
+    return dict(
+        value=replicas.job_tokens_per_s(T, world, ms), ms_per_step=ms, steps=steps,
+        warmup=warmup, config=_config(wl, args),
+        roofline=roof(dom),
+        per_kernel={n: roof(n) for n in names},
+        auction=dict(tokens_per_s=replicas.job_tokens_per_s(T, world, comp["auction"]),
+                     rounds=st["rounds"],
+                     phases=st["phases"], bids=bids, status=st["status"],
+                     us_per_round=1e3 * comp["auction"] / max(1, st["rounds"]),
+                     rounds_by_kind=rounds_by_kind),
+        e2e=dict(value=replicas.job_tokens_per_s(T, world, e2e), unit=UNIT,
+                 mode="pipelined: copy streams each way, two device buffers",
+                 serial_value=replicas.job_tokens_per_s(T, world, e2e_serial),
+                 serial_ms_per_step=e2e_serial,
+                 h2d_bytes_per_step=sum(d.numel() * d.element_size() for d, _ in ins[0]),
+                 d2h_bytes_per_step=d2h, ms_per_step=e2e),
+        gpu_launches=kernels_per_step * steps,
+        clocks=clk, device_error=err, wall_s=wall,
+    )
+
+
+def _rounds_by_kind(u, t, rounds, T):
+    """Per-round durations of a traced auction run, grouped by how many tokens
+    bid: the whole-grid rounds (every token bids: the phase starts), and the
+    rest by bidder count.  The last round has no successor and is left out."""
+    kinds = [("phase start", lambda x: x == T), ("1 bidder", lambda x: x == 1),
+             ("2-8 bidders", lambda x: 2 <= x <= 8), ("9-128 bidders", lambda x: 9 <= x <= 128),
+             ("129+ bidders", lambda x: 128 < x < T)]
+    groups = {name: [] for name, _ in kinds}
+    n = min(rounds, len(u), len(t))
+    for r in range(n - 1):
+        for name, test in kinds:  # the first kind that matches
+            if test(u[r]):
+                groups[name].append((t[r + 1] - t[r]) / 1e3)
+                break
+    return {name: dict(rounds=len(ds), us_total=sum(ds), us_median=statistics.median(ds))
+            for name, ds in groups.items() if ds}
+
+
+def main():
+    args = parse()
+    from balanced_token_expert_b200 import synth
+    wl = synth.WORKLOADS[args.workload]
+    if args.tokens:
+        wl = wl.scaled(T=args.tokens)
+    from balanced_token_expert_b200 import replicas
+    rank, world, local_rank = replicas.rank_env()
+    if args.impl == "reference":
+        run_reference(args, wl, rank, world)
+        return
+
+    import torch
+    import torch.distributed as dist
+    torch.cuda.set_device(local_rank)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    from balanced_token_expert_b200 import _build
+    from balanced_token_expert_b200 import binding as B
+    if rank == 0 or world == 1:
+        _build.build()
+    if world > 1:
+        dist.barrier()
+    B.lib()
+
+    head = measure(args, wl, args.steps, args.warmup, rank, world, local_rank)
+    torch.cuda.empty_cache()
+    extra = {}
+    if args.workload == "layer_fwd" and not args.tokens and not args.only:
+        # the other workloads on the same run, a few steps each
+        for name in EXTRA_WORKLOADS:
+            r = measure(args, synth.WORKLOADS[name], args.extra_steps, 3, rank, world, local_rank)
+            torch.cuda.empty_cache()
+            if r is not None:
+                extra[name] = r
     if rank == 0:
-        pk = peaks()
-        comp = {n: statistics.mean(per[n]) for n in names}
-        dom = max(comp, key=comp.get)
-        bids = st["bids"]
-        alg = dict(  # algorithmic work per launch (bytes or flops)
-            scores=("hbm", 2 * T * D + 2 * E * D + 8 * T * E),
-            auction=("hbm", 4 * E * bids + 4 * T + 8 * E),
-            permute=("hbm", 4 * T * D + 12 * T + 8 * T),
-            ffn=("tensor", 4 * T * D * F),
-            combine=("hbm", 4 * T * D + 4 * T),
-            greedy=("hbm", 4 * T * E + 4 * T),
-            backward=("tensor", 8 * T * D * F))
-
-        def roof(n):
-            bound, work = alg[n]
-            traffic = None if args.tokens else NCU_TRAFFIC.get((n, wl.name))
-            sec = comp[n] / 1e3
-            if bound == "tensor":
-                a_ = work / sec / 1e12
-                return dict(bound="tensor", achieved=a_, peak=pk["bf16"], unit="TFLOP/s",
-                            frac=a_ / pk["bf16"], traffic=traffic, kernel=n, ms=comp[n],
-                            peak_source=pk["source"] + " burst bf16")
-            a_ = work / sec / 1e9
-            return dict(bound="hbm", achieved=a_, peak=pk["hbm"], unit="GB/s",
-                        frac=a_ / pk["hbm"], traffic=traffic, kernel=n, ms=comp[n],
-                        peak_source=pk["source"] + " hbm copy")
-
         res = dict(
-            metric=METRIC, value=replicas.job_tokens_per_s(T, world, ms), unit=UNIT, n_gpus=world,
-            steps=args.steps, warmup=args.warmup, ms_per_step=ms, higher_is_better=True,
+            metric=METRIC, value=head["value"], unit=UNIT, n_gpus=world, steps=args.steps,
+            warmup=args.warmup, ms_per_step=head["ms_per_step"], higher_is_better=True,
             scaling="weak", vs_baseline=None, dtype="bf16", data="synthetic",
-            config=_config(wl, args),
-            roofline=roof(dom),
-            per_kernel={n: roof(n) for n in names},
-            auction=dict(tokens_per_s=replicas.job_tokens_per_s(T, world, comp["auction"]),
-                         rounds=st["rounds"],
-                         phases=st["phases"], bids=bids, status=st["status"],
-                         us_per_round=1e3 * comp["auction"] / max(1, st["rounds"])),
-            e2e=dict(value=replicas.job_tokens_per_s(T, world, e2e), unit=UNIT,
-                     mode="pipelined: copy streams each way, two device buffers",
-                     serial_value=replicas.job_tokens_per_s(T, world, e2e_serial),
-                     serial_ms_per_step=e2e_serial,
-                     h2d_bytes_per_step=sum(d.numel() * d.element_size() for d, _ in ins[0]),
-                     d2h_bytes_per_step=d2h, ms_per_step=e2e),
-            gpu_launches=kernels_per_step * args.steps,
-            clocks=clk, device_error=err, wall_s=wall,
-        )
+            config=head["config"], roofline=head["roofline"], per_kernel=head["per_kernel"],
+            auction=head["auction"], e2e=head["e2e"],
+            gpu_launches=head["gpu_launches"] + sum(r["gpu_launches"] for r in extra.values()),
+            clocks=head["clocks"], device_error=head["device_error"], wall_s=head["wall_s"])
+        if extra:
+            res["workloads"] = extra
         if world == 1 and not args.no_cpu_baseline:
             res["cpu_baseline"] = cpu_baseline(wl)
         print(json.dumps(res))

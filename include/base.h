@@ -114,6 +114,33 @@ const char* base_status_string(int status);
  */
 int base_device_error(int64_t* code, int clear);
 
+/*
+ * Test hooks (no counterpart in the paper).  Every device-side wait in the
+ * library is bounded: the auction's grid barrier gives up after 20 s (device
+ * error 5001, stats->status = BASE_ERR_TIMEOUT), the tensor-core GEMM
+ * pipeline's waits after 4 s (codes 3001-3005); the kernel then lets its
+ * copies in flight land, frees what it holds and returns, so the context
+ * stays usable.  These hooks let a test watch that happen without any fault:
+ *   BASE_TEST_WAIT_LIMIT_NS        value > 0: every bounded wait gives up
+ *                                  after `value` ns; 0: the defaults above.
+ *   BASE_TEST_AUCTION_ABSENT_CTA   value >= 0: that CTA of the auction's grid
+ *                                  returns at once, so the other CTAs' first
+ *                                  grid barrier runs out; -1: off.
+ *   BASE_TEST_GEMM_DROP_FIRST_LOAD 1: CTA 0 of a one-CTA tensor-core GEMM
+ *                                  (the bf16 score GEMM) never issues its
+ *                                  first TMA load, so its MMA warp's wait for
+ *                                  that stage runs out (3003); 0: off.
+ * The settings are process-wide host state read when a kernel is launched;
+ * they are for tests only and are not safe to change while other threads
+ * launch.  Returns BASE_ERR_INVALID_ARG for an unknown hook or value.
+ */
+typedef enum {
+    BASE_TEST_WAIT_LIMIT_NS = 0,
+    BASE_TEST_AUCTION_ABSENT_CTA = 1,
+    BASE_TEST_GEMM_DROP_FIRST_LOAD = 2
+} base_test_hook;
+int base_test_inject(int hook, long long value);
+
 /* Library version string (static). */
 const char* base_version(void);
 
@@ -205,7 +232,11 @@ int base_permute(const void* h, const int32_t* assign, int T, int D, int E,
  *   Limit: ceil(T/256) * E <= 1048576, else BASE_ERR_WORKSPACE and nothing
  *   is launched.  Allocates nothing.
  *   The first call on a device looks up the array's device address (a CUDA
- *   runtime query); make that first call before any stream capture.
+ *   runtime query); make that first call before any stream capture.  The
+ *   address is kept per device ordinal for the life of the process: after
+ *   cudaDeviceReset, or from a driver context other than the one current at
+ *   that first call, it is stale, so callers that reset the device or switch
+ *   contexts must use base_permute instead.
  *   All calls share the one array, whose contents the next call overwrites
  *   before reading; calls that overlap on the GPU race on it, so the caller
  *   must order them (one stream, or events).

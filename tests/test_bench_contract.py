@@ -23,3 +23,17 @@ def test_reference_arm_prints_one_contract_line(orc):
     assert d["impl"] == "reference" and d["value"] > 0 and d["n_gpus"] == 1
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["cpu_baseline"]["kind"] == "oracle"
     assert d["config"]["T"] == 512
+
+
+def test_rounds_by_kind_groups_traced_rounds():
+    sys.path.insert(0, ROOT)
+    import bench
+    # T = 8: a phase start (8 bidders), two narrow rounds, two one-bidder
+    # rounds, a second phase start, and a last round with no successor
+    u = [8, 3, 2, 1, 1, 8, 1]
+    t = [0, 10000, 13000, 15000, 16000, 17500, 30000]
+    k = bench._rounds_by_kind(u, t, rounds=7, T=8)
+    assert k["phase start"] == dict(rounds=2, us_total=10.0 + 12.5, us_median=11.25)
+    assert k["2-8 bidders"]["rounds"] == 2 and k["2-8 bidders"]["us_total"] == 5.0
+    assert k["1 bidder"] == dict(rounds=2, us_total=2.5, us_median=1.25)
+    assert "9-128 bidders" not in k

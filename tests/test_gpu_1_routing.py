@@ -182,6 +182,43 @@ def test_auction_trajectory_matches_round_by_round(orc, name):
     assert np.array_equal(u, uo)
 
 
+def test_auction_hand_worked_cases():
+    # the tie, price and phase rules on the cases worked through by hand in
+    # test_oracle_auction_hand.py: the GPU must reproduce the paper working
+    from test_oracle_auction_hand import check_result, hand_cases
+    for name, q, exp in hand_cases():
+        a, p, st, u = gpu_auction(q, trace=True)
+        check_result(exp, a, p, st, u)
+
+
+@pytest.mark.parametrize("name", ["skewed", "large_routing"])
+def test_auction_is_deterministic(name):
+    # bidders of a wide round reserve bucket space with atomics, in whatever
+    # order the SMs get there; the result must not depend on that order: five
+    # runs on the same q, reusing the workspace, give the same bits
+    wl = synth.WORKLOADS[name]
+    inp = synth.make_inputs(wl, 1, with_weights=False, with_dout=False)
+    q = torch.empty(wl.T, wl.E, dtype=torch.int32, device="cuda")
+    B.base_scores(dev(inp.h), dev(inp.w), None, q)
+    if inp.bump_tokens is not None:
+        q[inp.bump_tokens.cuda(), 0] += int(round(inp.bump_value * 65536))
+    ws = buffers.workspace(wl.T, wl.E)
+    runs = []
+    for _ in range(5):
+        assign = torch.full((wl.T,), -1, dtype=torch.int32, device="cuda")
+        price = torch.full((wl.E,), -7, dtype=torch.int64, device="cuda")
+        st = buffers.stats()
+        u = torch.full((100000,), -1, dtype=torch.int32, device="cuda")
+        B.base_assign_balanced_ex(q, assign, price, st, ws, 1000000, u_trace=u)
+        torch.cuda.synchronize()
+        runs.append((to_np(assign), to_np(price), buffers.stats_dict(st), to_np(u)))
+    a0, p0, s0, u0 = runs[0]
+    assert s0["status"] == 0
+    for a, p, s, u in runs[1:]:
+        assert s == s0
+        assert np.array_equal(a, a0) and np.array_equal(p, p0) and np.array_equal(u, u0)
+
+
 def test_auction_equal_scores_single_phase(orc):
     q = np.zeros((256, 8), dtype=np.int32)
     _check_auction(orc, q)

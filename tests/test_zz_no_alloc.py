@@ -1,8 +1,12 @@
 """base_permute_noalloc: the permutation for callers that cannot allocate
 device memory (it keeps its scratch in a fixed array inside the library
 instead of a caller workspace).  Its results must equal base_permute's, call
-after call, although every call reuses the same scratch.  This file is
-collected last on purpose."""
+after call, although every call reuses the same scratch.
+
+The file name makes pytest collect it last, so that if it fails, a run that
+stops at the first failure (``-x``) has already run every other test; it
+does not depend on anything the other tests leave behind and passes alone
+in a fresh process too."""
 import numpy as np
 import pytest
 import torch
@@ -50,6 +54,21 @@ def test_noalloc_permute_matches_the_workspace_version_on_consecutive_calls():
         perm = got[0].cpu().numpy()
         a_np = assign.cpu().numpy()
         assert np.array_equal(perm, np.argsort(a_np, kind="stable"))
+    assert B.base_device_error(clear=True) == 0
+
+
+def test_noalloc_permute_without_rows_or_gate():
+    # h = None and s = None: only the slot order (perm, inv, offsets) is made
+    B.base_device_error(clear=True)
+    T, E, D = 20000, 5, 8
+    assign, h, s = _case(T, E, D, 3, False)
+    ref = _outputs(T, E, D)
+    got = _outputs(T, E, D)
+    B.base_permute(None, assign, E, ref[0], ref[1], ref[2], None, ws=buffers.workspace(T, E, D))
+    B.base_permute_noalloc(None, assign, E, got[0], got[1], got[2], None)
+    torch.cuda.synchronize()
+    for a, b in zip(ref[:3], got[:3]):
+        assert torch.equal(a, b)
     assert B.base_device_error(clear=True) == 0
 
 
