@@ -25,6 +25,10 @@ Sparse Models" (wikillm.com summary; section names below are that page's):
 * backward with the assignment held fixed -- "Paper vs code", gradient into
   routing: affinities for assignment carry no gradient, centroids get
   gradient only through the gate.
+* the released code's layer variant -- "Paper vs code", Mixing equation (a
+  convex blend ``alpha f + (1 - alpha) h``) and "Placement and shape" (each
+  expert a stack of sublayers: layer norm, projection up, ReLU, projection
+  back, residual).
 """
 from __future__ import annotations
 
@@ -40,6 +44,7 @@ __all__ = [
     "scores", "quantize", "greedy", "auction", "hungarian", "bruteforce",
     "certificate", "permutation", "gather_rows", "scatter_rows", "act",
     "act_grad", "sigmoid", "expert_ffn", "layer_forward", "layer_backward",
+    "LN_EPS", "layer_norm", "expert_stack", "layer_forward_blend",
 ]
 
 # Spec constants, restated independently of the CUDA library.
@@ -332,3 +337,57 @@ def layer_backward(fw: dict, h, w, W1, W2, kind: str, dout, experts=None):
         dW1 = np.stack([dW1[e] for e in range(E)])
         dW2 = np.stack([dW2[e] for e in range(E)])
     return dict(dh=dh, dw=dw, dW1=dW1, dW2=dW2, ds=ds, dgate=dgate)
+
+
+# --------------------------------------------------------------------------
+# the released code's layer variant
+# --------------------------------------------------------------------------
+LN_EPS = 1e-5  # the pages name no layer-norm epsilon; the common default
+
+
+def layer_norm(x, gamma, beta, eps: float = LN_EPS) -> np.ndarray:
+    """Layer norm of every row: ``(x - mean) / sqrt(var + eps) * gamma + beta``
+    with the biased variance (the mean of squared deviations).  float64."""
+    x = _f64(x)
+    mu = x.mean(axis=-1, keepdims=True)
+    d = x - mu
+    var = (d * d).mean(axis=-1, keepdims=True)
+    return d / np.sqrt(var + eps) * _f64(gamma) + _f64(beta)
+
+
+def expert_stack(x, W1s, W2s, gammas, betas, kind: str = "relu"):
+    """One expert as the released code builds it ("Placement and shape"): S
+    sublayers, each ``x <- x + W2_i act(W1_i LN_i(x))``.  W1s (S, F, D), W2s
+    (S, D, F), gammas / betas (S, D).  float64.  Returns the output."""
+    x = _f64(x)
+    for i in range(len(W1s)):
+        u = layer_norm(x, gammas[i], betas[i])
+        x = x + act(u @ _f64(W1s[i]).T, kind) @ _f64(W2s[i]).T
+    return x
+
+
+def layer_forward_blend(h, w, W1, W2, gamma, beta, kind: str, assign: np.ndarray, experts=None):
+    """The released code's BASE layer with a given assignment ("Paper vs
+    code", Mixing equation): ``out_t = alpha_t E_a(h_t) + (1 - alpha_t) h_t``
+    with ``alpha_t = sigmoid(h_t . w_a)`` and ``E_a`` the expert stack of
+    expert ``a = assign[t]``.  W1 (E, S, F, D), W2 (E, S, D, F), gamma / beta
+    (E, S, D).  ``experts`` limits the work to some experts (the other tokens'
+    outputs are NaN).  Returns dict(out, y_perm, perm, offsets, gate_s)."""
+    h64, w64 = _f64(h), _f64(w)
+    E = w64.shape[0]
+    s = h64 @ w64.T
+    assign = np.asarray(assign, dtype=np.int64)
+    perm, inv, offsets = permutation(assign, E)
+    x = h64[perm]
+    gate_s = s[perm, assign[perm]]
+    alpha = sigmoid(gate_s)[:, None]
+    y = np.full_like(x, np.nan)
+    g64, b64 = _f64(gamma), _f64(beta)
+    for e in (range(E) if experts is None else experts):
+        lo, hi = int(offsets[e]), int(offsets[e + 1])
+        if hi == lo:
+            continue
+        f = expert_stack(x[lo:hi], W1[e], W2[e], g64[e], b64[e], kind)
+        y[lo:hi] = alpha[lo:hi] * f + (1.0 - alpha[lo:hi]) * x[lo:hi]
+    return dict(out=scatter_rows(y, perm), y_perm=y, perm=perm, inv=inv, offsets=offsets,
+                gate_s=gate_s)
