@@ -23,6 +23,7 @@ __all__ = [
     "base_scores", "base_assign_greedy", "base_assign_balanced", "base_assign_balanced_ex",
     "base_permute", "base_permute_noalloc", "base_expert_ffn", "base_combine", "base_layer_fwd",
     "base_layer_bwd", "base_test_inject", "BASE_TEST_WAIT_LIMIT_NS",
+    "base_workspace_size_blend", "base_layer_fwd_blend", "base_expert_stack",
     "BASE_TEST_AUCTION_ABSENT_CTA", "BASE_TEST_GEMM_DROP_FIRST_LOAD", "EXPORTED",
 ]
 
@@ -38,7 +39,8 @@ EXPORTED = (
     "base_status_string", "base_device_error", "base_version", "base_workspace_size",
     "base_scores", "base_assign_greedy", "base_assign_balanced", "base_assign_balanced_ex",
     "base_permute", "base_permute_noalloc", "base_expert_ffn", "base_combine", "base_layer_fwd",
-    "base_layer_bwd", "base_test_inject",
+    "base_layer_bwd", "base_test_inject", "base_workspace_size_blend", "base_layer_fwd_blend",
+    "base_expert_stack",
 )
 
 
@@ -75,6 +77,11 @@ _SIGS = {
     "base_device_error": (_i, [ctypes.POINTER(ctypes.c_int64), _i]),
     "base_workspace_size": (_sz, [_i, _i, _i, _i]),
     "base_test_inject": (_i, [_i, ctypes.c_longlong]),
+    "base_workspace_size_blend": (_sz, [_i, _i, _i, _i]),
+    "base_expert_stack": (_i, [_vp, _vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _i, _vp, _vp, _vp,
+                               _vp, _sz, _vp]),
+    "base_layer_fwd_blend": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp,
+                                  ctypes.POINTER(LayerSaved), _vp, _sz, _vp]),
     "base_scores": (_i, [_vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp]),
     "base_assign_greedy": (_i, [_vp, _i, _i, _vp, _vp, _vp]),
     "base_assign_balanced": (_i, [_vp, _i, _i, _vp, _vp, _vp, _vp, _sz, _vp]),
@@ -240,6 +247,32 @@ def base_layer_fwd(h, w, W1, W2, act: int, routing: int, out, saved: dict, ws, s
     _check("base_layer_fwd", lib().base_layer_fwd(
         _ptr(h), _ptr(w), _ptr(W1), _ptr(W2), int(act), int(routing), T, D, E, F, _ptr(out),
         ctypes.byref(sv), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def base_workspace_size_blend(T: int, E: int, D: int, F: int) -> int:
+    return int(lib().base_workspace_size_blend(T, E, D, F))
+
+
+def base_expert_stack(x_perm, offsets, W1, W2, gamma, beta, act: int, gate, y_perm, h1, ws,
+                      stream=None):
+    T, D = x_perm.shape
+    E, S, F, _ = W1.shape
+    _check("base_expert_stack", lib().base_expert_stack(
+        _ptr(x_perm), _ptr(offsets), T, D, F, E, S, _ptr(W1), _ptr(W2), _ptr(gamma), _ptr(beta),
+        int(act), _ptr(gate), _ptr(y_perm), _ptr(h1), _ptr(ws), ws.numel() * ws.element_size(),
+        _stream(stream)))
+
+
+def base_layer_fwd_blend(h, w, W1, W2, gamma, beta, act: int, routing: int, out, saved: dict, ws,
+                         stream=None):
+    """The released code's variant: W1 (E, S, F, D), W2 (E, S, D, F), gamma / beta (E, S, D)."""
+    T, D = h.shape
+    E, S, F, _ = W1.shape
+    sv = _saved(saved)
+    _check("base_layer_fwd_blend", lib().base_layer_fwd_blend(
+        _ptr(h), _ptr(w), _ptr(W1), _ptr(W2), _ptr(gamma), _ptr(beta), S, int(act), int(routing),
+        T, D, E, F, _ptr(out), ctypes.byref(sv), _ptr(ws), ws.numel() * ws.element_size(),
+        _stream(stream)))
 
 
 def base_layer_bwd(h, w, W1, W2, act: int, saved: dict, dout, dh, dw, dW1, dW2, ws, stream=None):

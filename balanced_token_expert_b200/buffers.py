@@ -15,6 +15,14 @@ def workspace(T: int, E: int, D: int = 0, F: int = 0, device="cuda") -> torch.Te
     return ws[off:off + n]
 
 
+def workspace_blend(T: int, E: int, D: int, F: int, device="cuda") -> torch.Tensor:
+    """A 256-byte-aligned workspace of base_workspace_size_blend(T, E, D, F) bytes."""
+    n = binding.base_workspace_size_blend(T, E, D, F)
+    ws = torch.empty(n + 256, dtype=torch.uint8, device=device)
+    off = (-ws.data_ptr()) % 256
+    return ws[off:off + n]
+
+
 def stats(device="cuda") -> torch.Tensor:
     """Device storage for one base_auction_stats (6 int64)."""
     return torch.zeros(6, dtype=torch.int64, device=device)

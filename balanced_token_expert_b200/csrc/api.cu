@@ -28,6 +28,11 @@ int launch_expert_ffn(const void* x_perm, const int32_t* offsets, int T, int D, 
                       const void* W1, const void* W2, int act, const float* gate, void* y_perm,
                       void* h1, void* a1, void* f, void* ws, cudaStream_t stream);
 size_t backward_workspace_bytes(int T, int E, int D, int F);
+size_t stack_workspace_bytes(int T, int E, int D);
+int launch_expert_stack(const void* x_perm, const int32_t* offsets, int T, int D, int F, int E,
+                        int S, const void* W1, const void* W2, const float* gamma,
+                        const float* beta, int act, const float* gate, void* y_perm, void* h1,
+                        void* ws, cudaStream_t stream);
 int launch_layer_bwd(const void* h, const void* w, const void* W1, const void* W2, int act, int T,
                      int D, int E, int F, const base_layer_saved* sv, const void* dout, void* dh,
                      float* dw, float* dW1, float* dW2, void* ws, size_t ws_bytes,
@@ -224,6 +229,69 @@ int base_layer_fwd(const void* h, const void* w, const void* W1, const void* W2,
     if (st != BASE_OK) return st;
     st = base_expert_ffn(sv->x_perm, sv->offsets, T, D, F, E, W1, W2, act, sv->gate, sv->y_perm,
                          sv->h1, sv->a1, sv->f, ws, ws_bytes, stream);
+    if (st != BASE_OK) return st;
+    return base_combine(sv->y_perm, sv->perm, T, D, out, stream);
+}
+
+size_t base_workspace_size_blend(int T, int E, int D, int F) {
+    if (!shapes_ok(T, E) || D < 8 || F < 8) return 0;
+    const size_t w = base_workspace_size(T, E, D, 0);
+    const size_t st = stack_workspace_bytes(T, E, D);
+    return w > st ? w : st;
+}
+
+int base_expert_stack(const void* x_perm, const int32_t* offsets, int T, int D, int F, int E,
+                      int S, const void* W1, const void* W2, const float* gamma, const float* beta,
+                      int act, const float* gate, void* y_perm, void* h1, void* ws,
+                      size_t ws_bytes, cudaStream_t stream) {
+    if (!x_perm || !offsets || !W1 || !W2 || !gamma || !beta || !gate || !y_perm || !h1 || !ws ||
+        !shapes_ok(T, E))
+        return BASE_ERR_INVALID_ARG;
+    if (S < 1 || D < 8 || D % 8 != 0 || F < 8 || F % 8 != 0) return BASE_ERR_INVALID_ARG;
+    if (act != BASE_RELU && act != BASE_GELU) return BASE_ERR_INVALID_ARG;
+    const void* p16[] = {x_perm, W1, W2, gamma, beta, y_perm, h1};
+    for (const void* p : p16)
+        if (!aligned(p, 16)) return BASE_ERR_INVALID_ARG;
+    if (!aligned(ws, 256)) return BASE_ERR_INVALID_ARG;
+    if (ws_bytes < stack_workspace_bytes(T, E, D)) return BASE_ERR_WORKSPACE;
+    return launch_expert_stack(x_perm, offsets, T, D, F, E, S, W1, W2, gamma, beta, act, gate,
+                               y_perm, h1, ws, stream);
+}
+
+int base_layer_fwd_blend(const void* h, const void* w, const void* W1, const void* W2,
+                         const float* gamma, const float* beta, int S, int act, int routing,
+                         int T, int D, int E, int F, void* out, const base_layer_saved* sv,
+                         void* ws, size_t ws_bytes, cudaStream_t stream) {
+    if (!h || !w || !W1 || !W2 || !gamma || !beta || !out || !sv || !ws || !shapes_ok(T, E))
+        return BASE_ERR_INVALID_ARG;
+    if (S < 1 || D < 8 || D % 8 != 0 || F < 8 || F % 8 != 0) return BASE_ERR_INVALID_ARG;
+    if (act != BASE_RELU && act != BASE_GELU) return BASE_ERR_INVALID_ARG;
+    if (!sv->s || !sv->q || !sv->assign || !sv->perm || !sv->inv || !sv->offsets || !sv->gate ||
+        !sv->x_perm || !sv->h1 || !sv->y_perm)
+        return BASE_ERR_INVALID_ARG;
+    if (routing == BASE_ROUTE_BALANCED) {
+        if (!sv->price || T % E != 0) return BASE_ERR_INVALID_ARG;
+    } else if (routing != BASE_ROUTE_GREEDY) {
+        return BASE_ERR_INVALID_ARG;
+    }
+    const void* p16[] = {h, w, W1, W2, gamma, beta, out, sv->x_perm, sv->h1, sv->y_perm};
+    for (const void* p : p16)
+        if (!aligned(p, 16)) return BASE_ERR_INVALID_ARG;
+    if (!aligned(ws, 256)) return BASE_ERR_INVALID_ARG;
+    if (ws_bytes < base_workspace_size_blend(T, E, D, F)) return BASE_ERR_WORKSPACE;
+    int st = base_scores(h, w, BASE_BF16, T, D, E, sv->s, sv->q, stream);
+    if (st != BASE_OK) return st;
+    if (routing == BASE_ROUTE_BALANCED)
+        st = base_assign_balanced(sv->q, T, E, sv->assign, sv->price, sv->stats, ws, ws_bytes,
+                                  stream);
+    else
+        st = base_assign_greedy(sv->q, T, E, sv->assign, nullptr, stream);
+    if (st != BASE_OK) return st;
+    st = base_permute(h, sv->assign, T, D, E, sv->perm, sv->inv, sv->offsets, sv->x_perm, sv->s,
+                      sv->gate, ws, ws_bytes, stream);
+    if (st != BASE_OK) return st;
+    st = base_expert_stack(sv->x_perm, sv->offsets, T, D, F, E, S, W1, W2, gamma, beta, act,
+                           sv->gate, sv->y_perm, sv->h1, ws, ws_bytes, stream);
     if (st != BASE_OK) return st;
     return base_combine(sv->y_perm, sv->perm, T, D, out, stream);
 }

@@ -663,6 +663,9 @@ struct Params {
     int32_t* u_trace;  // nullable: bidders of round r
     int64_t* t_trace;  // nullable: globaltimer (ns) at the start of round r
     long long trace_cap;
+    int SW;        // 1: wide rounds keep the owned experts' held sets sorted in shared memory
+    int own_max;   // experts a CTA owns at most: ceil(E / grid)
+    int nsc;       // keys of the sorted-resolve scratch (a power of two >= C)
     unsigned long long wait_ns;  // limit of every grid-barrier wait
     int absent_cta;              // test hook: this CTA returns at once (-1: none)
 };
@@ -679,10 +682,16 @@ __device__ __forceinline__ void trace_round(const Params& p, long long r, int U)
 // shared memory of every CTA (narrow-mode arrays are used by CTA 0 only)
 struct SmemLayout {
     size_t price, fr, fsize, hcnt, ncnt, act0, act1, nbk_b, nbk_t, list0, list1, rows, wb, wt, we,
-        wp, hist, red, cnt, misc, hb, ht, scratch, total;
+        wp, hist, red, cnt, misc, swm, hb, ht, scratch, total;
 };
 
 constexpr int kWideChunk = 1024;  // bids a CTA stages before reserving bucket space
+constexpr int kMaxOwn = 16;       // experts per CTA with sorted held sets
+
+// Sorted held sets in the scratch area: for owned expert j and buffer s,
+// bids at sw_bids(j, s) and tokens at sw_toks(j, s); the sort scratch after.
+__host__ __device__ inline size_t sw_set_bytes(int C) { return align_up(12 * (size_t)C, 16); }
+__host__ __device__ inline size_t sw_bytes(int own, int C) { return 2 * (size_t)own * sw_set_bytes(C); }
 constexpr int kMaxGrid = 1024;    // CTAs of the cooperative grid (one per SM)
 
 // NB: new bids per expert kept in shared memory (the rest in the global
@@ -705,7 +714,9 @@ __host__ __device__ inline SmemLayout smem_layout(int E, int FK, int NM, int NB,
     L.red = take(8 * 32);
     L.cnt = take(4 * 64);
     L.misc = take(64);
+    L.swm = take(4 * 2 * kMaxOwn);  // sorted held sets: count and buffer per owned expert
     // narrow rounds (CTA 0) only; in wide rounds the scratch of the resolve
+    // (or, with sorted held sets, those sets and the sort scratch)
     L.scratch = o;
     L.fr = take(sizeof(Key) * (size_t)E * FK);
     L.fsize = take(4 * (size_t)E);
@@ -1228,6 +1239,185 @@ __device__ bool resolve_cta_cached(const Team<kThreads>& tm, const Params& p, co
     return true;
 }
 
+// ---------------------------------------------------------------- sorted held sets
+// Wide rounds can keep held sets sorted.  The CTA that owns expert e (e %
+// grid) holds e's held keys in shared memory in "worse" order (worst first),
+// in two buffers that alternate by round.  A resolve then needs no select:
+// the new bids are sorted, a key's place in the merged order is its index
+// plus its rank in the other list (a binary search; keys are unique), the
+// first k places are rejected and the rest is the new held set.  It goes to
+// the other buffer and through to the global held arrays and the fringe
+// (its first FK keys, slot = index), which the narrow rounds and the final
+// assignment read.
+struct SortedSet {
+    int64_t* b;
+    int32_t* t;
+};
+
+// number of keys of the sorted list (b, t)[0, n) that are worse than x
+__device__ __forceinline__ int rank_sorted(const int64_t* b, const int32_t* t, int n,
+                                           const Key& x) {
+    int lo = 0, hi = n;
+    while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        if (worse(Key{b[mid], t[mid], 0}, x)) lo = mid + 1;
+        else hi = mid;
+    }
+    return lo;
+}
+
+// number of keys of the sorted keys a[0, n) that are worse than x
+__device__ __forceinline__ int rank_keys(const Key* a, int n, const Key& x) {
+    int lo = 0, hi = n;
+    while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        if (worse(a[mid], x)) lo = mid + 1;
+        else hi = mid;
+    }
+    return lo;
+}
+
+constexpr int kSortedSmall = 2048;  // new bids sorted whole up to this many
+
+// Ascending ("worse" order) sort of n keys in shared memory by the whole CTA:
+// every warp sorts runs of 32 keys in registers, then merge levels double
+// the run length; at each level a key's new place is its offset in its run
+// plus its rank in the partner run (a binary search; keys are unique).
+// a and tmp hold n keys each; returns the buffer that holds the result.
+__device__ Key* cta_sort_keys_fast(Key* a, Key* tmp, int n) {
+    const int lane = lane_id(), warp = warp_id();
+    for (int r0 = warp * 32; r0 < n; r0 += kWarps * 32) {
+        Key x = r0 + lane < n ? a[r0 + lane] : pad_key();
+        x = warp_sort(x);
+        if (r0 + lane < n) a[r0 + lane] = x;
+    }
+    __syncthreads();
+    Key* src = a;
+    Key* dst = tmp;
+    for (int R = 32; R < n; R <<= 1) {
+        for (int i0 = threadIdx.x; i0 < n; i0 += 2 * kThreads) {
+            // two keys per thread per pass, their searches interleaved
+            Key x[2];
+            int pos[2], lo[2], hi[2];
+            bool ok[2];
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const int i = i0 + u * kThreads;
+                ok[u] = i < n;
+                pos[u] = 0;
+                lo[u] = hi[u] = 0;
+                if (ok[u]) {
+                    x[u] = src[i];
+                    const int run = i / R;
+                    const int pair0 = (run & ~1) * R;
+                    const int ps = (run ^ 1) * R;  // the partner run
+                    lo[u] = min(ps, n);
+                    hi[u] = min(ps + R, n);
+                    pos[u] = pair0 + (i - run * R) - lo[u];
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                int l = lo[u], h = hi[u];
+                while (l < h) {
+                    const int mid = (l + h) >> 1;
+                    if (worse(src[mid], x[u])) l = mid + 1;
+                    else h = mid;
+                }
+                if (ok[u]) dst[pos[u] + l] = x[u];  // pos + l in [0, n)
+            }
+        }
+        __syncthreads();
+        Key* t = src;
+        src = dst;
+        dst = t;
+    }
+    return src;
+}
+
+// Keeps the C best of the sorted held set cur[0, h) and the n new bids
+// (nb, nt) of one expert.  The new held set (sorted) goes to nxt and to the
+// global hb / ht / fringe gfr; rejected tokens go to unext through ucnt.
+// sk, sk2: scratch of nsc keys each (nsc a power of two >= C).  Returns the new held count;
+// sets price (the smallest held bid) when the expert is full.  Bids beyond
+// kSortedSmall go through a radix select first (then only the accepted ones,
+// at most C, are sorted).
+__device__ int resolve_sorted(const Team<kThreads>& tm, const Params& p, SortedSet cur, int h,
+                              SortedSet nxt, const int64_t* nb, const int32_t* nt, int n,
+                              Key* sk, Key* sk2, int nsc, int64_t* hb, int32_t* ht, Key* gfr,
+                              int32_t* unext, int32_t* ucnt, int64_t& price) {
+    const int C = p.C, FK = p.FK, tid = threadIdx.x;
+    const int m = h + n, k = max(0, m - C), nh = m - k;
+    if (tid == 0) {
+        tm.cnt[56] = k > 0 ? atomicAdd(ucnt, k) : 0;
+        tm.cnt[57] = 0;  // new keys accepted (large case)
+        tm.cnt[58] = 0;  // new keys rejected (large case)
+    }
+    __syncthreads();
+    const int base = tm.cnt[56];
+    auto keep = [&](int r, const Key& x) {
+        if (r < 0 || r >= C) return;  // (only an inconsistent select could get here)
+        nxt.b[r] = x.bid;
+        nxt.t[r] = x.tok;
+        hb[r] = x.bid;
+        ht[r] = x.tok;
+        if (r < FK) gfr[r] = Key{x.bid, x.tok, r};
+    };
+    if (n <= kSortedSmall && n <= nsc) {
+        for (int i = tid; i < n; i += kThreads) sk[i] = Key{nb[i], nt[i], -1};
+        __syncthreads();
+        const Key* srt = cta_sort_keys_fast(sk, sk2, n);
+        for (int i = tid; i < h; i += kThreads) {
+            const Key x{cur.b[i], cur.t[i], 0};
+            const int pos = i + rank_keys(srt, n, x);
+            if (pos < k) unext[base + pos] = x.tok;
+            else keep(pos - k, x);
+        }
+        for (int j = tid; j < n; j += kThreads) {
+            const Key x = srt[j];
+            const int pos = j + rank_sorted(cur.b, cur.t, h, x);
+            if (pos < k) unext[base + pos] = x.tok;
+            else keep(pos - k, x);
+        }
+    } else {
+        // k >= 1 here: n > min(kSortedSmall, nsc) >= C.  X = the k-th worst
+        // of held + new; held keys up to X are a prefix cur[0, a0)
+        auto visit = [&](auto fn) {
+            for (int i = tid; i < h; i += kThreads) fn(Key{cur.b[i], cur.t[i], 0});
+            for (int j = tid; j < n; j += kThreads) fn(Key{nb[j], nt[j], -1});
+        };
+        const Key X = kth_worst_v<kThreads>(tm, visit, k, p.T - 1);
+        const int r = rank_sorted(cur.b, cur.t, h, X);
+        const int a0 = r + ((r < h && cur.b[r] == X.bid && cur.t[r] == X.tok) ? 1 : 0);
+        for (int i = tid; i < min(a0, k); i += kThreads) unext[base + i] = cur.t[i];
+        for (int j = tid; j < n; j += kThreads) {
+            const Key x{nb[j], nt[j], -1};
+            if (!worse(X, x)) {
+                const int at = a0 + atomicAdd(&tm.cnt[58], 1);
+                if (at < k) unext[base + at] = x.tok;
+            } else {
+                const int at = atomicAdd(&tm.cnt[57], 1);
+                if (at < nsc) sk[at] = x;
+            }
+        }
+        __syncthreads();
+        const int nacc = min(tm.cnt[57], nsc);
+        if (tid == 0 && (tm.cnt[57] + (h - a0) != nh || a0 + tm.cnt[58] != k)) record_error(1200);
+        const Key* srt = cta_sort_keys_fast(sk, sk2, nacc);
+        for (int i = a0 + tid; i < h; i += kThreads) {
+            const Key x{cur.b[i], cur.t[i], 0};
+            keep(i - a0 + rank_keys(srt, nacc, x), x);
+        }
+        for (int j = tid; j < nacc; j += kThreads) {
+            const Key x = srt[j];
+            keep(j + rank_sorted(cur.b + a0, cur.t + a0, h - a0, x), x);
+        }
+    }
+    __syncthreads();
+    if (nh == C) price = nxt.b[0];
+    return nh;
+}
+
 template <int TEAM>
 __device__ int build_fringe_radix(const Team<TEAM>& tm, const int64_t* hb, const int32_t* ht,
                                   int C, int FK, int tmax, Key* fr) {
@@ -1667,6 +1857,16 @@ __global__ void __launch_bounds__(kThreads, 1) auction_kernel(const __grid_const
     int32_t* s_misc = reinterpret_cast<int32_t*>(smem + L.misc);
     Key* s_scratch = reinterpret_cast<Key*>(smem + L.scratch);  // wide rounds only
     const int scratch_cap = (int)((L.total - L.scratch) / sizeof(Key));
+    // sorted held sets (p.SW): counts [0, kMaxOwn) and buffer selectors
+    // [kMaxOwn, 2 kMaxOwn) of the owned experts; the sets and the sort
+    // scratch (two buffers of nsc keys) in the scratch area
+    int32_t* s_swm = reinterpret_cast<int32_t*>(smem + L.swm);
+    unsigned char* s_sw = smem + L.scratch;
+    Key* s_swk = reinterpret_cast<Key*>(s_sw + sw_bytes(p.own_max, p.C));
+    auto sw_set = [&](int j, int sel) {
+        unsigned char* b = s_sw + (size_t)(2 * j + (sel & 1)) * sw_set_bytes(p.C);
+        return SortedSet{reinterpret_cast<int64_t*>(b), reinterpret_cast<int32_t*>(b + 8 * (size_t)p.C)};
+    };
 
     const int T = p.T, E = p.E, C = p.C, FK = p.FK;
     const int64_t scale = (int64_t)T + 1;
@@ -1770,6 +1970,9 @@ __global__ void __launch_bounds__(kThreads, 1) auction_kernel(const __grid_const
         }
         ++phases;
         reset_done = false;
+        // owned sorted held sets start empty in buffer 0 (read after the wide
+        // round's first barrier)
+        if (p.SW && threadIdx.x < 2 * kMaxOwn) s_swm[threadIdx.x] = 0;
         int U = T;
         bool first = true;
         bool narrow = false;
@@ -1844,7 +2047,32 @@ __global__ void __launch_bounds__(kThreads, 1) auction_kernel(const __grid_const
                 }
             }
             if (!(ok = grid_sync(p, bar_gen, s_misc))) break;
-            for (int e = cta; e < E; e += ncta) {
+            if (p.SW) {
+                // every owned expert with new bids: a merge with its sorted held set
+                int j = 0;
+                for (int e = cta; e < E; e += ncta, ++j) {
+                    const int n = vload(p.bcnt + e);
+                    if (n == 0) continue;
+                    __syncthreads();
+                    const int sel = s_swm[kMaxOwn + j];
+                    const int h0 = s_swm[j];
+                    int64_t price = INT64_MIN;
+                    const int nh = resolve_sorted(
+                        cta_team, p, sw_set(j, sel), h0, sw_set(j, sel ^ 1), p.bb + (size_t)e * T,
+                        p.bt + (size_t)e * T, n, s_swk, s_swk + p.nsc, p.nsc, p.hb + (size_t)e * C,
+                        p.ht + (size_t)e * C, p.gfr + (size_t)e * FK, unext, ucnt, price);
+                    if (threadIdx.x == 0) {
+                        s_swm[j] = nh;
+                        s_swm[kMaxOwn + j] = sel ^ 1;
+                        p.hcnt[e] = nh;
+                        p.bcnt[e] = 0;
+                        p.gfs[e] = min(FK, nh);
+                        if (nh == C) p.gprice[e] = price;
+                    }
+                    __syncthreads();
+                }
+            }
+            for (int e = cta; e < E && !p.SW; e += ncta) {
                 const int n = vload(p.bcnt + e);
                 if (n == 0) continue;
                 __syncthreads();
@@ -2223,6 +2451,8 @@ struct SmemPlan {
     size_t bytes;
 };
 
+constexpr size_t kSmemMax = 227 * 1024;  // dynamic shared memory of one CTA
+
 static SmemPlan smem_plan(int E, int NM, int T) {
     constexpr size_t kBudget = 200 * 1024;
     SmemPlan pl{0, 0, 0, 0, 0};
@@ -2276,7 +2506,7 @@ int launch_auction(const int32_t* q, int T, int E, int32_t* assign, int64_t* pri
     const SmemPlan sp = smem_plan(E, NM, T);
     if (sp.FK == 0) return BASE_ERR_UNSUPPORTED;
     const int FK = sp.FK;
-    const size_t smem = sp.bytes;
+    size_t smem = sp.bytes;
 
     unsigned char* w = static_cast<unsigned char*>(ws);
     size_t o = 0;
@@ -2323,12 +2553,32 @@ int launch_auction(const int32_t* q, int T, int E, int32_t* assign, int64_t* pri
     if (cudaMemsetAsync(zero_begin, 0, zero_bytes, stream) != cudaSuccess) return BASE_ERR_CUDA;
 
 
-    if (cudaFuncSetAttribute(auction_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem) != cudaSuccess)
-        return BASE_ERR_CUDA;
     int dev = 0, nsm = 0, per_sm = 0;
     cudaGetDevice(&dev);
     if (cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return BASE_ERR_CUDA;
+    // sorted held sets in the wide rounds when the owned experts' sets (two
+    // buffers each) and the sort scratch (a power of two >= C keys, 2048 at
+    // least when it fits) fit next to the narrow plan
+    {
+        const int own = (E + nsm - 1) / nsm;
+        const size_t scratch_off = smem_layout(E, FK, NM, sp.NB, sp.RC, T, sp.HS).scratch;
+        int nmin = 64;
+        while (nmin < C) nmin <<= 1;
+        prm.SW = 0;
+        for (int nsc = std::max(nmin, kSortedSmall); nsc >= nmin && own <= kMaxOwn; nsc >>= 1) {
+            const size_t need = scratch_off + sw_bytes(own, C) + 2 * sizeof(Key) * (size_t)nsc;
+            if (need <= kSmemMax) {
+                prm.SW = 1;
+                prm.own_max = own;
+                prm.nsc = nsc;
+                smem = std::max(smem, need);
+                break;
+            }
+        }
+    }
+    if (cudaFuncSetAttribute(auction_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem) != cudaSuccess)
         return BASE_ERR_CUDA;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, auction_kernel, kThreads, smem) !=
             cudaSuccess ||

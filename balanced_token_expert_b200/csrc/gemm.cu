@@ -45,7 +45,9 @@ constexpr int kThreads = 128 + 32 * kEpiWarps;
 enum Epi : int {
     EPI_SCORES = 0,  // s (fp32) and q = rint(s 2^16) (int32)
     EPI_ACT = 1,     // h1 = act(acc) bf16, a1 = acc bf16 (optional)
-    EPI_GATE = 2,    // y = sigmoid(gate[row]) acc + x[row] bf16, f = acc bf16 (optional)
+    EPI_GATE = 2,    // y = sigmoid(gate[row]) acc + x[row] bf16, f = acc bf16 (optional);
+                     // mix 1: y = acc + x[row]; mix 2: y = x0 + a (acc + x[row] - x0),
+                     // a = sigmoid(gate[row]), x0 = side2[row]
     EPI_DACT = 3,    // dA1 = acc * act'(a1[row]) bf16
     EPI_DX = 4,      // dh[idx[row]] = acc + dy[row] + ds[row] w_g  bf16
     EPI_F32 = 5,     // out_f32[g][row][col] = acc (K-grouped weight gradients)
@@ -72,6 +74,7 @@ struct Args {
     const int32_t* idx;          // destination rows (EPI_DX)
     int kgroup;                  // 1: groups split K (weight gradients), M and N fixed
     int m_tiles;                 // K-grouped mode: tiles along M per group
+    int mix;                     // EPI_GATE: 0 eq. 1, 1 residual only, 2 residual then blend
     int staged;                  // set by the launcher: output tensor maps are valid
     unsigned long long wait_ns;  // set by the launcher: limit of every bounded wait
     int drop_first_load;         // set by the launcher: test hook (one-CTA kernels only)
@@ -222,20 +225,33 @@ __device__ __forceinline__ void epilogue16(const Args& a, const TileInfo& ti, in
             }
         }
     } else if constexpr (EPI == EPI_GATE) {
-        const float g = __ldg(a.gate + row);
-        const float sg = 1.f / (1.f + expf(-g));
+        const float sg = a.mix == 1 ? 1.f : 1.f / (1.f + expf(-__ldg(a.gate + row)));
         if (col + 16 <= a.N) {
             if (a.out1) store_bf16x16(a.out1 + base, f);
             float x[16];
             load_bf16x16(a.side + base, x);
+            if (a.mix == 2) {
+                float x0[16];
+                load_bf16x16(a.side2 + base, x0);
 #pragma unroll
-            for (int i = 0; i < 16; ++i) x[i] = fmaf(sg, f[i], x[i]);
+                for (int i = 0; i < 16; ++i) x[i] = fmaf(sg, (f[i] + x[i]) - x0[i], x0[i]);
+            } else {
+#pragma unroll
+                for (int i = 0; i < 16; ++i) x[i] = fmaf(sg, f[i], x[i]);
+            }
             store_bf16x16(a.out0 + base, x);
         } else {
             for (int i = 0; i < a.N - col; ++i) {
                 if (a.out1) a.out1[base + i] = __float2bfloat16_rn(f[i]);
                 const float x = __bfloat162float(a.side[base + i]);
-                a.out0[base + i] = __float2bfloat16_rn(fmaf(sg, f[i], x));
+                float y;
+                if (a.mix == 2) {
+                    const float x0 = __bfloat162float(a.side2[base + i]);
+                    y = fmaf(sg, (f[i] + x) - x0, x0);
+                } else {
+                    y = fmaf(sg, f[i], x);
+                }
+                a.out0[base + i] = __float2bfloat16_rn(y);
             }
         }
     } else if constexpr (EPI == EPI_DACT) {
@@ -304,12 +320,18 @@ __device__ __forceinline__ void epi_values16(const Args& a, int row, int col, in
 #pragma unroll
         for (int i = 0; i < 16; ++i) o[i] = act_fwd(o[i], a.act);
     } else if constexpr (EPI == EPI_GATE) {
-        const float g = __ldg(a.gate + row);
-        const float sg = 1.f / (1.f + expf(-g));
+        const float sg = a.mix == 1 ? 1.f : 1.f / (1.f + expf(-__ldg(a.gate + row)));
         float x[16];
         load_bf16x16(a.side + base, x);
+        if (a.mix == 2) {
+            float x0[16];
+            load_bf16x16(a.side2 + base, x0);
 #pragma unroll
-        for (int i = 0; i < 16; ++i) o[i] = fmaf(sg, o[i], x[i]);
+            for (int i = 0; i < 16; ++i) o[i] = fmaf(sg, (o[i] + x[i]) - x0[i], x0[i]);
+        } else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) o[i] = fmaf(sg, o[i], x[i]);
+        }
     } else if constexpr (EPI == EPI_DACT) {
         float x[16];
         load_bf16x16(a.side + base, x);
@@ -864,6 +886,83 @@ int launch_expert_ffn(const void* x_perm, const int32_t* offsets, int T, int D, 
     g2.side = static_cast<const __nv_bfloat16*>(x_perm);
     return launch<256, 5, EPI_GATE, false, false, 2>(h1, T, F, W2, (uint64_t)E * D, F, g2,
                                                      max_mt * g2.n_tiles, stream);
+}
+
+int launch_layer_norm_rows(const void* x, const int32_t* offsets, int T, int D, int E,
+                           const float* gamma, const float* beta, int stride, void* y,
+                           cudaStream_t stream);
+
+// The released code's expert: S sublayers x <- x + W2_i act(W1_i LN_i(x)) on
+// every expert segment, then the blend y = x0 + a (x_S - x0), a =
+// sigmoid(gate), x0 = x_perm, in the last GEMM's epilogue.  W1 (E, S, F, D),
+// W2 (E, S, D, F), gamma / beta (E, S, D) fp32.  Scratch: the tile prefix,
+// then ln and one more T x D bf16 buffer (sublayer outputs alternate between
+// it and y_perm, the last one in y_perm).
+size_t stack_workspace_bytes(int T, int E, int D) {
+    return ffn_workspace_bytes(E) + 2 * align_up((size_t)T * D * 2, 256);
+}
+
+int launch_expert_stack(const void* x_perm, const int32_t* offsets, int T, int D, int F, int E,
+                        int S, const void* W1, const void* W2, const float* gamma,
+                        const float* beta, int act, const float* gate, void* y_perm, void* h1,
+                        void* ws, cudaStream_t stream) {
+    using namespace gemm;
+    constexpr int BMP = 2 * BM;
+    uint8_t* w8 = static_cast<uint8_t*>(ws);
+    int32_t* tile_start = reinterpret_cast<int32_t*>(w8);
+    void* ln = w8 + ffn_workspace_bytes(E);
+    void* xb = w8 + ffn_workspace_bytes(E) + align_up((size_t)T * D * 2, 256);
+    tile_prefix_kernel<<<1, 1024, 0, stream>>>(offsets, E, BMP, tile_start);
+    BASE_RETURN_IF_LAUNCH_FAILED();
+    const int max_mt = (T + BMP - 1) / BMP + E;
+    const __nv_bfloat16* W1b = static_cast<const __nv_bfloat16*>(W1);
+    const __nv_bfloat16* W2b = static_cast<const __nv_bfloat16*>(W2);
+    const void* cur = x_perm;
+    for (int i = 0; i < S; ++i) {
+        int st = launch_layer_norm_rows(cur, offsets, T, D, E, gamma + (size_t)i * D,
+                                        beta + (size_t)i * D, S * D, ln, stream);
+        if (st != BASE_OK) return st;
+        Args g1{};
+        g1.M = T;
+        g1.N = F;
+        g1.K = D;
+        g1.groups = E;
+        g1.offsets = offsets;
+        g1.tile_start = tile_start;
+        g1.b_rows_per_group = S * F;  // expert e's sublayer i: rows (e S + i) F of W1
+        g1.n_tiles = (F + 255) / 256;
+        g1.ld = F;
+        g1.act = act;
+        g1.out0 = static_cast<__nv_bfloat16*>(h1);
+        st = launch<256, 5, EPI_ACT, false, false, 2>(ln, T, D, W1b + (size_t)i * F * D,
+                                                      (uint64_t)(E * S - i) * F, D, g1,
+                                                      max_mt * g1.n_tiles, stream);
+        if (st != BASE_OK) return st;
+        const bool last = i == S - 1;
+        // outputs alternate so that the last one lands in y_perm
+        void* out = ((S - 1 - i) % 2 == 0) ? y_perm : xb;
+        Args g2{};
+        g2.M = T;
+        g2.N = D;
+        g2.K = F;
+        g2.groups = E;
+        g2.offsets = offsets;
+        g2.tile_start = tile_start;
+        g2.b_rows_per_group = S * D;
+        g2.n_tiles = (D + 255) / 256;
+        g2.ld = D;
+        g2.out0 = static_cast<__nv_bfloat16*>(out);
+        g2.gate = gate;
+        g2.mix = last ? 2 : 1;
+        g2.side = static_cast<const __nv_bfloat16*>(cur);
+        g2.side2 = static_cast<const __nv_bfloat16*>(x_perm);
+        st = launch<256, 5, EPI_GATE, false, false, 2>(h1, T, F, W2b + (size_t)i * D * F,
+                                                       (uint64_t)(E * S - i) * D, F, g2,
+                                                       max_mt * g2.n_tiles, stream);
+        if (st != BASE_OK) return st;
+        cur = out;
+    }
+    return BASE_OK;
 }
 
 }  // namespace base

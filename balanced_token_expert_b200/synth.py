@@ -19,6 +19,9 @@ of width D, E expert centroids w_e, expert FFNs D -> F -> D):
   the caller applies it to the quantised scores).
 * ``large_routing``: T=131072, E=128, D=2048, bf16.
 * ``layer_fwd_bwd``: T=32768, E=32, D=2048, F=8192 GELU, bf16, plus dout ~ N(0,1).
+* ``layer_fwd_blend``: the layer_fwd shape through the released code's variant
+  (one sublayer per expert; ``make_stack_params`` adds layer-norm gains and
+  biases and the weights of further sublayers).
 """
 from __future__ import annotations
 
@@ -28,7 +31,7 @@ from typing import Optional
 
 import torch
 
-__all__ = ["Workload", "WORKLOADS", "make_inputs", "Inputs"]
+__all__ = ["Workload", "WORKLOADS", "make_inputs", "make_stack_params", "Inputs"]
 
 
 @dataclass(frozen=True)
@@ -42,6 +45,7 @@ class Workload:
     dtype: str = "bf16"        # "f32" | "bf16"
     kind: str = "normal"       # "normal" | "mixture"
     backward: bool = False
+    S: int = 0                 # > 0: the released code's variant with S sublayers per expert
 
     def scaled(self, **kw) -> "Workload":
         d = dict(self.__dict__)
@@ -56,6 +60,9 @@ WORKLOADS = {
     "large_routing": Workload("large_routing", T=131072, E=128, D=2048),
     "layer_fwd_bwd": Workload("layer_fwd_bwd", T=32768, E=32, D=2048, F=8192, act="gelu",
                               backward=True),
+    # the layer_fwd shape through the released code's variant (one sublayer
+    # per expert, the code's default, and the convex blend)
+    "layer_fwd_blend": Workload("layer_fwd_blend", T=8192, E=16, D=1024, F=4096, act="relu", S=1),
 }
 
 
@@ -107,3 +114,21 @@ def make_inputs(wl: Workload, seed: int = 0, with_weights: bool = True,
     if with_dout:
         inp.dout = _cast(torch.randn(T, D, generator=g), "bf16")
     return inp
+
+
+def make_stack_params(wl: Workload, S: int, seed: int = 0) -> dict:
+    """Parameters of the released code's expert stacks (S sublayers per
+    expert): the weights of sublayers 1 .. S-1 (sublayer 0 uses the
+    workload's W1 / W2), W ~ N(0, 0.02^2) bf16, and every sublayer's layer
+    norm gain ~ 1 + 0.1 N(0,1) and bias ~ 0.1 N(0,1), fp32.  From a generator
+    seeded with seed + 1000, so the workload's own draws are unchanged."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(int(seed) + 1000)
+    E, D, F = wl.E, wl.D, wl.F
+    out = {}
+    if S > 1:
+        out["W1"] = _cast(torch.randn(E, S - 1, F, D, generator=g) * 0.02, "bf16")
+        out["W2"] = _cast(torch.randn(E, S - 1, D, F, generator=g) * 0.02, "bf16")
+    out["gamma"] = (1.0 + 0.1 * torch.randn(E, S, D, generator=g)).contiguous()
+    out["beta"] = (0.1 * torch.randn(E, S, D, generator=g)).contiguous()
+    return out

@@ -13,8 +13,9 @@ h ~ N(0,1), w ~ N(0, 1/D)).
 The same run then times the other workloads a few steps each (--extra-steps)
 and reports them under "workloads": the skewed-affinity auction stress
 (T=32768, E=64), large routing (T=131072, E=128: scores, auction, greedy,
-permute) and the training step (T=32768, E=32, D=2048, FFN 8192 GELU,
-forward + backward).  --workload NAME --only times one workload alone.
+permute), the training step (T=32768, E=32, D=2048, FFN 8192 GELU, forward +
+backward) and the released code's layer variant on the default shape (layer
+norm + FFN + residual expert, convex blend).  --workload NAME --only times one workload alone.
 
 With N > 1 (torchrun, one rank per GPU) every rank runs its own independent
 problem (the balanced assignment decomposes per worker, so no collective is
@@ -204,7 +205,12 @@ def run_reference(args, wl, rank, world):
 
 
 def _config(wl, args):
-    if wl.F:
+    if wl.S:
+        desc = ("%s: the released code's BASE layer variant, T=%d tokens, E=%d experts, D=%d, "
+                "experts of %d sublayer(s) layer norm + FFN %d->%d->%d %s + residual, convex "
+                "blend, balanced auction routing, bf16" % (wl.name, wl.T, wl.E, wl.D, wl.S, wl.D,
+                                                          wl.F, wl.D, wl.act))
+    elif wl.F:
         desc = ("%s: BASE layer %s, T=%d tokens, E=%d experts, D=%d, FFN %d->%d->%d %s, "
                 "balanced auction routing, bf16" % (wl.name, "forward+backward" if wl.backward
                                                      else "forward", wl.T, wl.E, wl.D, wl.D, wl.F,
@@ -220,7 +226,7 @@ def _config(wl, args):
                 parallelism="independent replica per GPU")
 
 
-EXTRA_WORKLOADS = ("skewed", "large_routing", "layer_fwd_bwd")
+EXTRA_WORKLOADS = ("skewed", "large_routing", "layer_fwd_bwd", "layer_fwd_blend")
 
 
 def measure(args, wl, steps, warmup, rank, world, local_rank):
@@ -241,7 +247,12 @@ def measure(args, wl, steps, warmup, rank, world, local_rank):
     act = B.BASE_RELU if wl.act == "relu" else B.BASE_GELU
     sv = buffers.layer_saved(T, E, D, max(F, 8), for_backward=wl.backward)
     out = torch.empty(T, D, dtype=torch.bfloat16, device="cuda")
-    ws = buffers.workspace(T, E, D, F)
+    ws = buffers.workspace_blend(T, E, D, F) if wl.S else buffers.workspace(T, E, D, F)
+    if wl.S:  # the released code's variant: S sublayers per expert
+        extra = synth.make_stack_params(wl, wl.S, seed=replicas.rank_seed(rank))
+        W1 = torch.cat([inp.W1[:, None]] + ([extra["W1"]] if wl.S > 1 else []), 1).cuda()
+        W2 = torch.cat([inp.W2[:, None]] + ([extra["W2"]] if wl.S > 1 else []), 1).cuda()
+        gam, bet = extra["gamma"].cuda(), extra["beta"].cuda()
     flush = torch.empty(args.flush_mb * (1 << 20), dtype=torch.uint8, device="cuda")
     stream = torch.cuda.current_stream()
 
@@ -265,7 +276,12 @@ def measure(args, wl, steps, warmup, rank, world, local_rank):
     comps.append(("permute", lambda: B.base_permute(h, sv["assign"], E, sv["perm"], sv["inv"],
                                                      sv["offsets"], sv["x_perm"], sv["s"],
                                                      sv["gate"], ws), 3))
-    if F:
+    if F and wl.S:
+        comps.append(("stack", lambda: B.base_expert_stack(sv["x_perm"], sv["offsets"], W1, W2,
+                                                           gam, bet, act, sv["gate"], sv["y_perm"],
+                                                           sv["h1"], ws), 1 + 3 * wl.S))
+        comps.append(("combine", lambda: B.base_combine(sv["y_perm"], sv["perm"], out), 1))
+    elif F:
         comps.append(("ffn", lambda: B.base_expert_ffn(sv["x_perm"], sv["offsets"], W1, W2, act,
                                                        sv["gate"], sv["y_perm"], sv["h1"],
                                                        sv.get("a1"), sv.get("f"), ws), 3))
@@ -376,6 +392,12 @@ def measure(args, wl, steps, warmup, rank, world, local_rank):
                                  stream=stream)
                 B.base_layer_bwd(h_dev[b], w, W1, W2, act, sv, dout_dev[b], res_dev[b], dw, dW1,
                                  dW2, ws, stream=stream)
+        elif wl.S:
+            sv2 = buffers.layer_saved(T, E, D, F, for_backward=False)
+
+            def compute(b):
+                B.base_layer_fwd_blend(h_dev[b], w, W1, W2, gam, bet, act, B.BASE_ROUTE_BALANCED,
+                                       res_dev[b], sv2, ws, stream=stream)
         else:
             sv2 = buffers.layer_saved(T, E, D, F, for_backward=False)
 
@@ -459,6 +481,7 @@ def measure(args, wl, steps, warmup, rank, world, local_rank):
         auction=("hbm", 4 * E * bids + 4 * T + 8 * E),
         permute=("hbm", 4 * T * D + 12 * T + 8 * T),
         ffn=("tensor", 4 * T * D * F),
+        stack=("tensor", 4 * T * D * F * max(1, wl.S)),
         combine=("hbm", 4 * T * D + 4 * T),
         greedy=("hbm", 4 * T * E + 4 * T),
         backward=("tensor", 8 * T * D * F))

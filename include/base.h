@@ -278,6 +278,38 @@ int base_layer_fwd(const void* h, const void* w, const void* W1, const void* W2,
                    const base_layer_saved* sv, void* ws, size_t ws_bytes, cudaStream_t stream);
 
 /*
+ * The released code's layer variant (the wikillm.com summary's "Paper vs
+ * code", Mixing equation, and "Placement and shape"): the same routing and
+ * permutation, but every expert is a stack of S sublayers
+ *   x <- x + W2[e][i] act(W1[e][i] LN_i(x)),   i = 0 .. S-1,
+ * with LN_i the layer norm of the row (biased variance, eps 1e-5) scaled by
+ * gamma[e][i] and shifted by beta[e][i], and the token leaves the layer as
+ * the convex blend  alpha_t x_S + (1 - alpha_t) h_t,  alpha_t =
+ * sigmoid(h_t . w_{a_t})  (instead of eq. 1's sigmoid(.) f + h).
+ *   W1: E*S*F*D bf16, W2: E*S*D*F bf16 (expert-major, then sublayer);
+ *   gamma, beta: E*S*D fp32; S >= 1; the other arguments as base_layer_fwd.
+ *   sv: s, q, assign, price, stats, perm, inv, offsets, gate, x_perm, h1 and
+ *   y_perm are written (a1 and f are not used); ws: at least
+ *   base_workspace_size_blend(T, E, D, F) bytes.  Forward only.
+ */
+size_t base_workspace_size_blend(int T, int E, int D, int F);
+/*
+ * The variant's expert step alone (its counterpart of base_expert_ffn): for
+ * every expert e and slot r in [offsets[e], offsets[e+1]), starting from
+ * x = x_perm[r], the S sublayers above, then
+ *   y_perm[r] = x_perm[r] + sigmoid(gate[r]) (x_S - x_perm[r]).
+ *   h1: T*F bf16 scratch of the sublayers; ws: base_workspace_size_blend bytes.
+ */
+int base_expert_stack(const void* x_perm, const int32_t* offsets, int T, int D, int F, int E,
+                      int S, const void* W1, const void* W2, const float* gamma, const float* beta,
+                      int act, const float* gate, void* y_perm, void* h1, void* ws,
+                      size_t ws_bytes, cudaStream_t stream);
+int base_layer_fwd_blend(const void* h, const void* w, const void* W1, const void* W2,
+                         const float* gamma, const float* beta, int S, int act, int routing,
+                         int T, int D, int E, int F, void* out, const base_layer_saved* sv,
+                         void* ws, size_t ws_bytes, cudaStream_t stream);
+
+/*
  * a9: the layer backward with the assignment held fixed (the released code
  * computes the routing affinities without gradient; the centroids receive
  * gradient only through the gate, "Paper vs code").  Given dout (T*D bf16):

@@ -285,3 +285,45 @@ def test_layer_bwd_rejects_unbalanced_shapes():
                          z(E, D, device="cuda"), z(E, F, D, device="cuda"),
                          z(E, D, F, device="cuda"), buffers.workspace(T, E, D, F))
     assert ei.value.status == 6  # C = 24 is not a multiple of 64
+
+
+# ------------------------------------------------------------------ the released code's variant
+def _blend_inputs(wl, S, seed):
+    """The workload's inputs plus S sublayers of weights per expert (the
+    first sublayer's are the workload's own W1 / W2) and layer-norm gains and
+    biases near (1, 0)."""
+    inp = synth.make_inputs(wl, seed)
+    extra = synth.make_stack_params(wl, S, seed)
+    W1 = torch.cat([inp.W1[:, None], extra["W1"]], dim=1) if S > 1 else inp.W1[:, None]
+    W2 = torch.cat([inp.W2[:, None], extra["W2"]], dim=1) if S > 1 else inp.W2[:, None]
+    return inp, W1.contiguous(), W2.contiguous(), extra["gamma"], extra["beta"]
+
+
+def _blend_check(orc, wl, S, seed, routing, experts=None):
+    inp, W1, W2, gam, bet = _blend_inputs(wl, S, seed)
+    T, E, D, F = wl.T, wl.E, wl.D, wl.F
+    sv = buffers.layer_saved(T, E, D, F, for_backward=False)
+    out = torch.empty(T, D, dtype=torch.bfloat16, device="cuda")
+    ws = buffers.workspace_blend(T, E, D, F)
+    B.base_layer_fwd_blend(dev(inp.h), dev(inp.w), dev(W1), dev(W2), dev(gam), dev(bet),
+                           ACT[wl.act],
+                           B.BASE_ROUTE_BALANCED if routing == "balanced" else B.BASE_ROUTE_GREEDY,
+                           out, sv, ws)
+    torch.cuda.synchronize()
+    a_g = _check_routing_of_fwd(orc, inp, sv, routing)
+    r = orc.layer_forward_blend(inp.h, inp.w, W1, W2, gam, bet, wl.act, a_g, experts=experts)
+    keep = np.ones(T, dtype=bool) if experts is None else np.isin(a_g, experts)
+    ok, worst = close_rel_rms(to_np(out)[keep], r["out"][keep], FWD_TOL)
+    assert ok, worst
+
+
+@pytest.mark.parametrize("S,routing,act", [(1, "balanced", "relu"), (2, "balanced", "relu"),
+                                           (3, "greedy", "gelu")])
+def test_blend_variant_small(orc, S, routing, act):
+    wl = synth.WORKLOADS["layer_fwd"].scaled(T=1536, E=6, D=256, F=1024, act=act)
+    _blend_check(orc, wl, S, 6, routing)
+
+
+def test_blend_variant_full_layer_fwd_workload_sampled(orc):
+    # the benchmarked shape (T=8192, E=16, D=1024, F=4096) with two sublayers
+    _blend_check(orc, synth.WORKLOADS["layer_fwd"], 2, 0, "balanced", experts=[0, 9])
