@@ -44,7 +44,7 @@ __all__ = [
     "scores", "quantize", "greedy", "auction", "hungarian", "bruteforce",
     "certificate", "permutation", "gather_rows", "scatter_rows", "act",
     "act_grad", "sigmoid", "expert_ffn", "layer_forward", "layer_backward",
-    "LN_EPS", "layer_norm", "expert_stack", "layer_forward_blend",
+    "LN_EPS", "layer_norm", "expert_stack", "layer_forward_blend", "sanitize_scores",
 ]
 
 # Spec constants, restated independently of the CUDA library.
@@ -116,6 +116,19 @@ def quantize(s) -> np.ndarray:
     s32 = np.asarray(s, dtype=np.float64).astype(np.float32)
     x = np.rint(s32 * np.float32(QSCALE)).astype(np.float64)
     return np.clip(x, -2147483647.0, 2147483647.0).astype(np.int32)
+
+
+def sanitize_scores(s) -> np.ndarray:
+    """Non-finite affinities replaced by the smallest finite one ("Paper vs
+    code", Non-finite scores: the released code does this before solving).
+    When no score is finite the pages leave the value open; this reading uses
+    0.  Returns a float32 copy (the scores are fp32)."""
+    s32 = np.array(s, dtype=np.float32, copy=True)
+    bad = ~np.isfinite(s32)
+    if bad.any():
+        good = s32[~bad]
+        s32[bad] = good.min() if good.size else np.float32(0.0)
+    return s32
 
 
 def greedy(q: np.ndarray):

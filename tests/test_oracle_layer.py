@@ -172,3 +172,19 @@ def test_synth_is_deterministic_and_shaped():
     f = synth.make_inputs(synth.WORKLOADS["layer_fwd"].scaled(T=64, E=4, D=16, F=32), 0)
     assert f.W1.shape == (4, 32, 16) and f.W2.shape == (4, 16, 32)
     assert f.W1.dtype == torch.bfloat16
+
+
+def test_sanitize_replaces_non_finite_scores_by_the_smallest_finite_one(orc):
+    # "Paper vs code", Non-finite scores: NaN and +-Inf become the minimum finite score
+    s = np.array([[0.5, np.nan, -2.0], [np.inf, 3.0, -np.inf], [1.0, 0.25, -1.5]], dtype=np.float32)
+    out = orc.sanitize_scores(s)
+    assert out.tolist() == [[0.5, -2.0, -2.0], [-2.0, 3.0, -2.0], [1.0, 0.25, -1.5]]
+    assert np.isnan(s[0, 1])  # the input is left alone
+    # finite scores pass unchanged; no finite score at all gives zeros (a reading)
+    f = np.arange(6, dtype=np.float32).reshape(2, 3)
+    assert np.array_equal(orc.sanitize_scores(f), f)
+    assert orc.sanitize_scores(np.full((2, 2), np.nan, dtype=np.float32)).tolist() == [[0, 0], [0, 0]]
+    # sanitised, the quantised scores are those of the minimum: every
+    # replaced entry quantises to the smallest quantised finite entry
+    q = orc.quantize(out)
+    assert q[0, 1] == q[1, 0] == q[1, 2] == q[0, 2] == orc.quantize(np.array([[-2.0]]))[0, 0]
