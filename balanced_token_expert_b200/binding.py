@@ -24,6 +24,7 @@ __all__ = [
     "base_permute", "base_permute_noalloc", "base_expert_ffn", "base_combine", "base_layer_fwd",
     "base_layer_bwd", "base_test_inject", "BASE_TEST_WAIT_LIMIT_NS",
     "base_workspace_size_blend", "base_layer_fwd_blend", "base_expert_stack",
+    "base_sanitize_scores", "BASE_ROUTE_SANITIZE",
     "BASE_TEST_AUCTION_ABSENT_CTA", "BASE_TEST_GEMM_DROP_FIRST_LOAD", "EXPORTED",
 ]
 
@@ -31,6 +32,7 @@ BASE_OK = 0
 BASE_F32, BASE_BF16 = 0, 1
 BASE_RELU, BASE_GELU = 0, 1
 BASE_ROUTE_BALANCED, BASE_ROUTE_GREEDY = 0, 1
+BASE_ROUTE_SANITIZE = 0x100
 QSCALE = 65536.0
 BASE_TEST_WAIT_LIMIT_NS, BASE_TEST_AUCTION_ABSENT_CTA, BASE_TEST_GEMM_DROP_FIRST_LOAD = 0, 1, 2
 
@@ -40,7 +42,7 @@ EXPORTED = (
     "base_scores", "base_assign_greedy", "base_assign_balanced", "base_assign_balanced_ex",
     "base_permute", "base_permute_noalloc", "base_expert_ffn", "base_combine", "base_layer_fwd",
     "base_layer_bwd", "base_test_inject", "base_workspace_size_blend", "base_layer_fwd_blend",
-    "base_expert_stack",
+    "base_expert_stack", "base_sanitize_scores",
 )
 
 
@@ -78,6 +80,7 @@ _SIGS = {
     "base_workspace_size": (_sz, [_i, _i, _i, _i]),
     "base_test_inject": (_i, [_i, ctypes.c_longlong]),
     "base_workspace_size_blend": (_sz, [_i, _i, _i, _i]),
+    "base_sanitize_scores": (_i, [_vp, _vp, _i, _i, _vp, _sz, _vp]),
     "base_expert_stack": (_i, [_vp, _vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _i, _vp, _vp, _vp,
                                _vp, _sz, _vp]),
     "base_layer_fwd_blend": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp,
@@ -169,6 +172,12 @@ def base_scores(h, w, s=None, q=None, stream=None):
     E = w.shape[0]
     _check("base_scores", lib().base_scores(_ptr(h), _ptr(w), _dtype_code(h), T, D, E, _ptr(s),
                                             _ptr(q), _stream(stream)))
+
+
+def base_sanitize_scores(s, q, ws, stream=None):
+    T, E = s.shape
+    _check("base_sanitize_scores", lib().base_sanitize_scores(
+        _ptr(s), _ptr(q), T, E, _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)))
 
 
 def base_assign_greedy(q, assign, counts=None, stream=None):

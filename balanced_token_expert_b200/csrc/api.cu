@@ -29,6 +29,8 @@ int launch_expert_ffn(const void* x_perm, const int32_t* offsets, int T, int D, 
                       void* h1, void* a1, void* f, void* ws, cudaStream_t stream);
 size_t backward_workspace_bytes(int T, int E, int D, int F);
 size_t stack_workspace_bytes(int T, int E, int D);
+size_t sanitize_workspace_bytes();
+int launch_sanitize_scores(float* s, int32_t* q, int T, int E, void* ws, cudaStream_t stream);
 int launch_expert_stack(const void* x_perm, const int32_t* offsets, int T, int D, int F, int E,
                         int S, const void* W1, const void* W2, const float* gamma,
                         const float* beta, int act, const float* gate, void* y_perm, void* h1,
@@ -68,6 +70,7 @@ const char* base_version(void) { return "libbase 0.1 (sm_100a)"; }
 size_t base_workspace_size(int T, int E, int D, int F) {
     if (!shapes_ok(T, E) || D < 0 || F < 0) return 0;
     size_t w = auction_workspace_bytes(T, E);
+    if (sanitize_workspace_bytes() > w) w = sanitize_workspace_bytes();
     const size_t p = permute_workspace_bytes(T, E);
     if (p > w) w = p;
     const size_t f = ffn_workspace_bytes(E);
@@ -122,6 +125,14 @@ int base_scores(const void* h, const void* w, int dtype, int T, int D, int E, fl
     if (dtype != BASE_BF16) return BASE_ERR_INVALID_ARG;
     if (D % 8 != 0 || !aligned(h, 16) || !aligned(w, 16)) return BASE_ERR_INVALID_ARG;
     return launch_scores_bf16(h, w, T, D, E, s, q, stream);
+}
+
+int base_sanitize_scores(float* s, int32_t* q, int T, int E, void* ws, size_t ws_bytes,
+                         cudaStream_t stream) {
+    if (!s || !ws || !shapes_ok(T, E)) return BASE_ERR_INVALID_ARG;
+    if (!aligned(s, 4) || (q && !aligned(q, 4)) || !aligned(ws, 256)) return BASE_ERR_INVALID_ARG;
+    if (ws_bytes < sanitize_workspace_bytes()) return BASE_ERR_WORKSPACE;
+    return launch_sanitize_scores(s, q, T, E, ws, stream);
 }
 
 int base_assign_greedy(const int32_t* q, int T, int E, int32_t* assign, int32_t* counts,
@@ -210,6 +221,8 @@ int base_layer_fwd(const void* h, const void* w, const void* W1, const void* W2,
     if (!sv->s || !sv->q || !sv->assign || !sv->perm || !sv->inv || !sv->offsets || !sv->gate ||
         !sv->x_perm || !sv->h1 || !sv->y_perm)
         return BASE_ERR_INVALID_ARG;
+    const bool sanitize = (routing & BASE_ROUTE_SANITIZE) != 0;
+    routing &= ~BASE_ROUTE_SANITIZE;
     if (routing == BASE_ROUTE_BALANCED) {
         if (!sv->price || T % E != 0) return BASE_ERR_INVALID_ARG;
     } else if (routing != BASE_ROUTE_GREEDY) {
@@ -218,6 +231,10 @@ int base_layer_fwd(const void* h, const void* w, const void* W1, const void* W2,
     if (ws_bytes < base_workspace_size(T, E, D, 0)) return BASE_ERR_WORKSPACE;
     int st = base_scores(h, w, BASE_BF16, T, D, E, sv->s, sv->q, stream);
     if (st != BASE_OK) return st;
+    if (sanitize) {
+        st = base_sanitize_scores(sv->s, sv->q, T, E, ws, ws_bytes, stream);
+        if (st != BASE_OK) return st;
+    }
     if (routing == BASE_ROUTE_BALANCED)
         st = base_assign_balanced(sv->q, T, E, sv->assign, sv->price, sv->stats, ws, ws_bytes,
                                   stream);
@@ -269,6 +286,8 @@ int base_layer_fwd_blend(const void* h, const void* w, const void* W1, const voi
     if (!sv->s || !sv->q || !sv->assign || !sv->perm || !sv->inv || !sv->offsets || !sv->gate ||
         !sv->x_perm || !sv->h1 || !sv->y_perm)
         return BASE_ERR_INVALID_ARG;
+    const bool sanitize = (routing & BASE_ROUTE_SANITIZE) != 0;
+    routing &= ~BASE_ROUTE_SANITIZE;
     if (routing == BASE_ROUTE_BALANCED) {
         if (!sv->price || T % E != 0) return BASE_ERR_INVALID_ARG;
     } else if (routing != BASE_ROUTE_GREEDY) {
@@ -281,6 +300,10 @@ int base_layer_fwd_blend(const void* h, const void* w, const void* W1, const voi
     if (ws_bytes < base_workspace_size_blend(T, E, D, F)) return BASE_ERR_WORKSPACE;
     int st = base_scores(h, w, BASE_BF16, T, D, E, sv->s, sv->q, stream);
     if (st != BASE_OK) return st;
+    if (sanitize) {
+        st = base_sanitize_scores(sv->s, sv->q, T, E, ws, ws_bytes, stream);
+        if (st != BASE_OK) return st;
+    }
     if (routing == BASE_ROUTE_BALANCED)
         st = base_assign_balanced(sv->q, T, E, sv->assign, sv->price, sv->stats, ws, ws_bytes,
                                   stream);

@@ -346,3 +346,119 @@ int launch_move_rows(const void* src, const int32_t* idx, int T, int D, void* ds
 }
 
 }  // namespace base
+
+// ---------------------------------------------------------------------------
+// Non-finite scores ("Paper vs code", Non-finite scores: the released code
+// replaces NaN and infinite affinities with the minimum finite score before
+// solving).  Pass 1: per-block minimum of the finite scores and count of the
+// others; pass 2: every block reduces the partials and, when something is not
+// finite, rewrites those entries of s and q (q = rint(min 2^16), the
+// quantisation of the minimum).  With no finite score at all the minimum is
+// taken as 0.
+// ---------------------------------------------------------------------------
+namespace base {
+namespace routing {
+
+constexpr int kSanThreads = 256;
+constexpr int kSanMaxBlocks = 1024;
+
+__device__ __forceinline__ void block_min_count(float& m, int& c, float* s_m, int* s_c) {
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+        m = fminf(m, __shfl_xor_sync(0xffffffffu, m, off));
+        c += __shfl_xor_sync(0xffffffffu, c, off);
+    }
+    if (lane_id() == 0) {
+        s_m[warp_id()] = m;
+        s_c[warp_id()] = c;
+    }
+    __syncthreads();
+    if (warp_id() == 0) {
+        const int nw = blockDim.x / kWarp;
+        m = lane_id() < nw ? s_m[lane_id()] : INFINITY;
+        c = lane_id() < nw ? s_c[lane_id()] : 0;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            m = fminf(m, __shfl_xor_sync(0xffffffffu, m, off));
+            c += __shfl_xor_sync(0xffffffffu, c, off);
+        }
+        if (lane_id() == 0) {
+            s_m[0] = m;
+            s_c[0] = c;
+        }
+    }
+    __syncthreads();
+    m = s_m[0];
+    c = s_c[0];
+}
+
+__global__ void __launch_bounds__(kSanThreads) sanitize_reduce_kernel(const float* __restrict__ s,
+                                                                      long long n,
+                                                                      float* __restrict__ pmin,
+                                                                      int* __restrict__ pcnt) {
+    __shared__ float s_m[32];
+    __shared__ int s_c[32];
+    float m = INFINITY;
+    int c = 0;
+    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n;
+         i += (long long)gridDim.x * blockDim.x) {
+        const float v = __ldg(s + i);
+        if (isfinite(v)) m = fminf(m, v);
+        else ++c;
+    }
+    block_min_count(m, c, s_m, s_c);
+    if (threadIdx.x == 0) {
+        pmin[blockIdx.x] = m;
+        pcnt[blockIdx.x] = c;
+    }
+}
+
+__global__ void __launch_bounds__(kSanThreads) sanitize_fix_kernel(float* __restrict__ s,
+                                                                   int32_t* __restrict__ q,
+                                                                   long long n, int nparts,
+                                                                   const float* __restrict__ pmin,
+                                                                   const int* __restrict__ pcnt) {
+    __shared__ float s_m[32];
+    __shared__ int s_c[32];
+    float m = INFINITY;
+    int c = 0;
+    for (int i = threadIdx.x; i < nparts; i += blockDim.x) {
+        m = fminf(m, pmin[i]);
+        c += pcnt[i];
+    }
+    block_min_count(m, c, s_m, s_c);
+    if (c == 0) return;
+    if (!isfinite(m)) m = 0.f;  // nothing finite
+    const int32_t qm = quantize_score(m);
+    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n;
+         i += (long long)gridDim.x * blockDim.x) {
+        if (!isfinite(s[i])) {
+            s[i] = m;
+            if (q) q[i] = qm;
+        }
+    }
+}
+
+}  // namespace routing
+
+size_t sanitize_workspace_bytes() {
+    return align_up(2 * sizeof(float) * routing::kSanMaxBlocks, 256);
+}
+
+int launch_sanitize_scores(float* s, int32_t* q, int T, int E, void* ws, cudaStream_t stream) {
+    using namespace routing;
+    const long long n = (long long)T * E;
+    long long blocks = (n + kSanThreads * 4 - 1) / (kSanThreads * 4);
+    if (blocks > num_sms() * 4) blocks = num_sms() * 4;
+    if (blocks > kSanMaxBlocks) blocks = kSanMaxBlocks;
+    if (blocks < 1) blocks = 1;
+    float* pmin = static_cast<float*>(ws);
+    int* pcnt = reinterpret_cast<int*>(pmin + kSanMaxBlocks);
+    sanitize_reduce_kernel<<<(int)blocks, kSanThreads, 0, stream>>>(s, n, pmin, pcnt);
+    BASE_RETURN_IF_LAUNCH_FAILED();
+    sanitize_fix_kernel<<<(int)blocks, kSanThreads, 0, stream>>>(s, q, n, (int)blocks, pmin, pcnt);
+    BASE_RETURN_IF_LAUNCH_FAILED();
+    return BASE_OK;
+}
+
+}  // namespace base

@@ -55,7 +55,13 @@ typedef enum {
 
 typedef enum { BASE_F32 = 0, BASE_BF16 = 1 } base_dtype;
 typedef enum { BASE_RELU = 0, BASE_GELU = 1 } base_act;
-typedef enum { BASE_ROUTE_BALANCED = 0, BASE_ROUTE_GREEDY = 1 } base_routing;
+/* Routing of the layer forward; BASE_ROUTE_SANITIZE may be OR'ed in to
+ * replace non-finite scores first (see base_sanitize_scores). */
+typedef enum {
+    BASE_ROUTE_BALANCED = 0,
+    BASE_ROUTE_GREEDY = 1,
+    BASE_ROUTE_SANITIZE = 0x100
+} base_routing;
 
 /* Quantisation scale of the affinity scores: q = rint(s * 2^16). */
 #define BASE_QSCALE 65536.0f
@@ -161,6 +167,18 @@ size_t base_workspace_size(int T, int E, int D, int F);
  */
 int base_scores(const void* h, const void* w, int dtype, int T, int D, int E,
                 float* s, int32_t* q, cudaStream_t stream);
+
+/*
+ * Non-finite scores (the wikillm.com summary's "Paper vs code", Non-finite
+ * scores: the released code replaces NaN and infinite affinities with the
+ * minimum finite score before solving).  Every entry of s (T*E fp32) that is
+ * NaN or +-Inf becomes the smallest finite entry m (0 when none is finite),
+ * and the same entries of q (nullable) become rint(m * 65536), the
+ * quantisation of m.  Finite entries are not touched.  ws: at least
+ * base_workspace_size(T, E, 0, 0) bytes.  Two launches, no host sync.
+ */
+int base_sanitize_scores(float* s, int32_t* q, int T, int E, void* ws, size_t ws_bytes,
+                         cudaStream_t stream);
 
 /*
  * a3: greedy test-time routing (Method, "Test time": each token to its

@@ -45,6 +45,7 @@ __all__ = [
     "certificate", "permutation", "gather_rows", "scatter_rows", "act",
     "act_grad", "sigmoid", "expert_ffn", "layer_forward", "layer_backward",
     "LN_EPS", "layer_norm", "expert_stack", "layer_forward_blend", "sanitize_scores",
+    "fig9_auction", "FIG9_MAX_ITERATIONS",
 ]
 
 # Spec constants, restated independently of the CUDA library.
@@ -80,6 +81,9 @@ def lib():
                                   i64p, i32p, ctypes.c_int64]
         L.orc_hungarian.restype = ctypes.c_int64
         L.orc_hungarian.argtypes = [i32p, ctypes.c_int, ctypes.c_int, i32p]
+        L.orc_fig9.restype = ctypes.c_int
+        L.orc_fig9.argtypes = [i32p, ctypes.c_int, ctypes.c_int, ctypes.c_int64, ctypes.c_int64,
+                               i32p, i64p, i64p]
         L.orc_bruteforce.restype = ctypes.c_int64
         L.orc_bruteforce.argtypes = [i32p, ctypes.c_int, ctypes.c_int, i32p, i64p, i64p]
         _lib = L
@@ -162,6 +166,26 @@ def auction(q: np.ndarray, max_rounds: int = MAX_ROUNDS, trace: bool = False):
     if trace:
         return assign, price, stats, tr[: min(stats["rounds"], cap)].copy()
     return assign, price, stats
+
+
+FIG9_MAX_ITERATIONS = 100  # the listing's default iteration cap
+
+
+def fig9_auction(q: np.ndarray, max_iterations: int = FIG9_MAX_ITERATIONS,
+                 max_rounds: int = MAX_ROUNDS):
+    """The page's fig. 9 solver (experts bid for tokens, prices per token)
+    with the released code's rules, as ``orc_fig9`` in ``base_oracle.c``
+    states them.  Returns ``(assign int32[T], token price int64[T], stats)``
+    with stats status, rounds, eps and objective."""
+    q = np.ascontiguousarray(q, dtype=np.int32)
+    T, E = q.shape
+    assign = np.full(T, -1, dtype=np.int32)
+    price = np.zeros(T, dtype=np.int64)
+    st = np.zeros(4, dtype=np.int64)
+    rc = lib().orc_fig9(_p32(q), T, E, int(max_iterations), int(max_rounds), _p32(assign),
+                        _p64(price), _p64(st))
+    return assign, price, dict(status=int(rc), rounds=int(st[1]), eps=int(st[2]),
+                               objective=int(st[3]))
 
 
 def hungarian(q: np.ndarray):

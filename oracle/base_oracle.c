@@ -354,3 +354,143 @@ int64_t orc_bruteforce(const int32_t* q, int T, int E, int32_t* best_assign,
     if (n_opt) *n_opt = st.n_opt;
     return st.best;
 }
+
+/*
+ * The page's fig. 9 listing ("Solver"): an auction in which EXPERTS bid for
+ * TOKENS and prices live per token, with the released code's rules where the
+ * page says the code differs ("Paper vs code": eps = range / 50, winners kept
+ * in their holder's list at the largest score rather than infinity, and after
+ * the iteration cap the update rule changes while the loop goes on until
+ * every token has a bid -- no greedy fallback).  Integer version on the
+ * quantised scores S[e][t] = q[t][e] (int64):
+ *   eps = max(1, floor((max q - min q) / 50));  RETAIN = max q + 1;
+ *   price[t] = 0; adjusted = S; nobody has won.
+ *   round r (while some token has not won):
+ *     every expert takes its C + 1 largest adjusted values (ties: smaller
+ *     token first) and bids raise = v_j - v_C + eps on its top C tokens;
+ *     if 0 < r < max_iterations, every token won in the last round gets the
+ *     bid eps from its holder instead (overwriting that holder's own bid);
+ *     each token goes to its largest bid (smaller expert on ties); it is won
+ *     when that bid is > 0; price[t] += that bid;
+ *     adjusted[e][t] = S[e][t] - price[t], and for every won token, in its
+ *     holder's row: RETAIN if r < max_iterations, else S[holder][t].
+ *   The result is the last round's top-C lists (a partition of the tokens
+ *   once every token has won).
+ * RETAIN is the largest score plus one: with the largest score itself a kept
+ * token ties with an untouched token of that score, and the tie rule could
+ * push it out of its holder's list.
+ * stats_out (nullable) int64[4]: status, rounds, eps, objective.
+ * price_out (nullable): T int64 final token prices.
+ */
+typedef struct {
+    int64_t v;
+    int32_t t;
+} orc_vt;
+
+/* larger value first, then smaller token */
+static int orc_vt_cmp(const void* pa, const void* pb) {
+    const orc_vt* a = (const orc_vt*)pa;
+    const orc_vt* b = (const orc_vt*)pb;
+    if (a->v != b->v) return (a->v > b->v) ? -1 : 1;
+    return (a->t < b->t) ? -1 : (a->t > b->t);
+}
+
+int orc_fig9(const int32_t* q, int T, int E, int64_t max_iterations, int64_t max_rounds,
+             int32_t* assign, int64_t* price_out, int64_t* stats_out) {
+    if (!q || !assign || T <= 0 || E < 2 || T % E != 0 || max_rounds <= 0 || max_iterations < 0)
+        return ORC_ERR_INVALID_ARG;
+    const int C = T / E;
+    if (C + 1 > T) return ORC_ERR_INVALID_ARG;
+    int64_t qmin = INT64_MAX, qmax = INT64_MIN;
+    for (int64_t i = 0; i < (int64_t)T * E; ++i) {
+        if (q[i] < qmin) qmin = q[i];
+        if (q[i] > qmax) qmax = q[i];
+    }
+    int64_t eps = (qmax - qmin) / 50;
+    if (eps < 1) eps = 1;
+    const int64_t RETAIN = qmax + 1;
+    int64_t* adj = (int64_t*)malloc(sizeof(int64_t) * (size_t)E * T);
+    int64_t* bids = (int64_t*)malloc(sizeof(int64_t) * (size_t)E * T);
+    int64_t* price = (int64_t*)calloc((size_t)T, sizeof(int64_t));
+    char* won = (char*)calloc((size_t)T, 1);
+    int32_t* holder = (int32_t*)malloc(sizeof(int32_t) * (size_t)T);
+    int32_t* best_ids = (int32_t*)malloc(sizeof(int32_t) * (size_t)E * (C + 1));
+    int64_t* best_vals = (int64_t*)malloc(sizeof(int64_t) * (size_t)E * (C + 1));
+    orc_vt* work = (orc_vt*)malloc(sizeof(orc_vt) * (size_t)E * T);
+    if (!adj || !bids || !price || !won || !holder || !best_ids || !best_vals || !work) {
+        free(adj); free(bids); free(price); free(won); free(holder); free(best_ids);
+        free(best_vals); free(work);
+        return ORC_ERR_INVALID_ARG;
+    }
+    for (int e = 0; e < E; ++e)
+        for (int t = 0; t < T; ++t) adj[(int64_t)e * T + t] = q[(int64_t)t * E + e];
+    for (int t = 0; t < T; ++t) holder[t] = -1;
+    int status = ORC_OK;
+    int64_t round = 0;
+    for (;;) {
+        int all = 1;
+        for (int t = 0; t < T; ++t) all &= won[t];
+        if (all && round > 0) break;
+        if (round >= max_rounds) { status = ORC_ERR_NOT_CONVERGED; break; }
+        /* each expert's C + 1 largest adjusted values */
+        #pragma omp parallel for schedule(static)
+        for (int e = 0; e < E; ++e) {
+            orc_vt* w = work + (int64_t)e * T;
+            for (int t = 0; t < T; ++t) { w[t].v = adj[(int64_t)e * T + t]; w[t].t = t; }
+            qsort(w, (size_t)T, sizeof(orc_vt), orc_vt_cmp);
+            for (int j = 0; j <= C; ++j) {
+                best_ids[(int64_t)e * (C + 1) + j] = w[j].t;
+                best_vals[(int64_t)e * (C + 1) + j] = w[j].v;
+            }
+        }
+        memset(bids, 0, sizeof(int64_t) * (size_t)E * T);
+        for (int e = 0; e < E; ++e) {
+            const int64_t vc = best_vals[(int64_t)e * (C + 1) + C];
+            for (int j = 0; j < C; ++j) {
+                const int t = best_ids[(int64_t)e * (C + 1) + j];
+                bids[(int64_t)e * T + t] = best_vals[(int64_t)e * (C + 1) + j] - vc + eps;
+            }
+        }
+        if (round > 0 && round < max_iterations)
+            for (int t = 0; t < T; ++t)
+                if (won[t]) bids[(int64_t)holder[t] * T + t] = eps;
+        for (int t = 0; t < T; ++t) {
+            int64_t best = bids[t];
+            int arg = 0;
+            for (int e = 1; e < E; ++e)
+                if (bids[(int64_t)e * T + t] > best) { best = bids[(int64_t)e * T + t]; arg = e; }
+            won[t] = best > 0;
+            holder[t] = won[t] ? arg : -1;
+            price[t] += best;
+        }
+        for (int e = 0; e < E; ++e)
+            for (int t = 0; t < T; ++t) adj[(int64_t)e * T + t] = (int64_t)q[(int64_t)t * E + e] - price[t];
+        for (int t = 0; t < T; ++t)
+            if (won[t])
+                adj[(int64_t)holder[t] * T + t] =
+                    (round < max_iterations) ? RETAIN : (int64_t)q[(int64_t)t * E + holder[t]];
+        ++round;
+    }
+    int64_t objective = 0;
+    if (status == ORC_OK) {
+        for (int t = 0; t < T; ++t) assign[t] = -1;
+        for (int e = 0; e < E && status == ORC_OK; ++e)
+            for (int j = 0; j < C; ++j) {
+                const int t = best_ids[(int64_t)e * (C + 1) + j];
+                if (assign[t] != -1) { status = ORC_ERR_NOT_CONVERGED; break; }
+                assign[t] = e;
+            }
+        if (status == ORC_OK)
+            for (int t = 0; t < T; ++t) objective += q[(int64_t)t * E + assign[t]];
+    }
+    if (price_out) for (int t = 0; t < T; ++t) price_out[t] = price[t];
+    if (stats_out) {
+        stats_out[0] = status;
+        stats_out[1] = round;
+        stats_out[2] = eps;
+        stats_out[3] = objective;
+    }
+    free(adj); free(bids); free(price); free(won); free(holder); free(best_ids);
+    free(best_vals); free(work);
+    return status;
+}

@@ -313,3 +313,69 @@ def test_out_of_range_entries_are_recorded_not_followed():
     keep = torch.ones(T, dtype=torch.bool)
     keep[3] = False
     assert torch.equal(out.cpu()[keep], y.cpu()[keep])
+
+
+# ------------------------------------------------------------------ non-finite scores
+def test_sanitize_scores_bit_exact(orc):
+    rng = np.random.default_rng(8)
+    T, E = 1000, 7
+    s = rng.standard_normal((T, E)).astype(np.float32)
+    bad = rng.choice(T * E, size=40, replace=False)
+    s.flat[bad] = [(np.nan, np.inf, -np.inf)[i % 3] for i in range(40)]
+    ws = buffers.workspace(T, E)
+    sg = dev(s)
+    q = torch.zeros(T, E, dtype=torch.int32, device="cuda")
+    B.base_sanitize_scores(sg, q, ws)
+    torch.cuda.synchronize()
+    so = orc.sanitize_scores(s)
+    assert np.array_equal(to_np(sg), so)
+    qn = to_np(q)
+    assert np.array_equal(qn.flat[bad], orc.quantize(so).flat[bad])
+    keep = np.ones(T * E, dtype=bool)
+    keep[bad] = False
+    assert np.all(qn.flat[keep] == 0)  # only the replaced entries are written
+    # all finite: nothing changes; nothing finite: zeros
+    f = rng.standard_normal((T, E)).astype(np.float32)
+    fg = dev(f)
+    B.base_sanitize_scores(fg, None, ws)
+    n = dev(np.full((64, 4), np.nan, dtype=np.float32))
+    nq = torch.full((64, 4), 5, dtype=torch.int32, device="cuda")
+    B.base_sanitize_scores(n, nq, ws)
+    torch.cuda.synchronize()
+    assert np.array_equal(to_np(fg), f)
+    assert np.all(to_np(n) == 0.0) and np.all(to_np(nq) == 0)
+
+
+def test_layer_fwd_sanitizes_non_finite_scores(orc):
+    # tokens whose features hold NaN or Inf have non-finite affinities; with
+    # BASE_ROUTE_SANITIZE the layer gives them the smallest finite score and
+    # routes every token exactly as the oracle's auction does on those scores
+    from _util import close_rel_rms
+    wl = synth.WORKLOADS["layer_fwd"].scaled(T=2048, E=8, D=256, F=512)
+    inp = synth.make_inputs(wl, 5)
+    h = inp.h.clone()
+    h[3] = float("nan")
+    h[100, 7] = float("inf")
+    h[2047, :5] = float("-inf")
+    badrows = [3, 100, 2047]
+    T, E, D, F = wl.T, wl.E, wl.D, wl.F
+    sv = buffers.layer_saved(T, E, D, F, for_backward=False)
+    out = torch.empty(T, D, dtype=torch.bfloat16, device="cuda")
+    ws = buffers.workspace(T, E, D, F)
+    B.base_layer_fwd(dev(h), dev(inp.w), dev(inp.W1), dev(inp.W2), B.BASE_RELU,
+                     B.BASE_ROUTE_BALANCED | B.BASE_ROUTE_SANITIZE, out, sv, ws)
+    torch.cuda.synchronize()
+    s_g, q_g = to_np(sv["s"]), to_np(sv["q"])
+    assert np.all(np.isfinite(s_g))
+    assert np.all(s_g[badrows] == s_g.min())
+    good = np.setdiff1d(np.arange(T), badrows)
+    ok, worst = close_scores(s_g[good], orc.scores(h[good], inp.w), 1e-5)
+    assert ok, worst
+    assert np.array_equal(q_g, np.rint(s_g * np.float32(65536)).astype(np.int32))
+    a_g = to_np(sv["assign"])
+    ao, po, so = orc.auction(q_g)
+    assert buffers.stats_dict(sv["stats"]) == so
+    assert np.array_equal(a_g, ao) and np.array_equal(to_np(sv["price"]), po)
+    fw = orc.layer_forward(h, inp.w, inp.W1, inp.W2, "relu", a_g)
+    ok, worst = close_rel_rms(to_np(out)[good], fw["out"][good], 2e-2)
+    assert ok, worst
