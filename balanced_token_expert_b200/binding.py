@@ -24,7 +24,7 @@ __all__ = [
     "base_permute", "base_permute_noalloc", "base_expert_ffn", "base_combine", "base_layer_fwd",
     "base_layer_bwd", "base_test_inject", "BASE_TEST_WAIT_LIMIT_NS",
     "base_workspace_size_blend", "base_layer_fwd_blend", "base_expert_stack",
-    "base_sanitize_scores", "BASE_ROUTE_SANITIZE",
+    "base_sanitize_scores", "BASE_ROUTE_SANITIZE", "base_workspace_size_fig9", "base_assign_fig9",
     "BASE_TEST_AUCTION_ABSENT_CTA", "BASE_TEST_GEMM_DROP_FIRST_LOAD", "EXPORTED",
 ]
 
@@ -42,7 +42,7 @@ EXPORTED = (
     "base_scores", "base_assign_greedy", "base_assign_balanced", "base_assign_balanced_ex",
     "base_permute", "base_permute_noalloc", "base_expert_ffn", "base_combine", "base_layer_fwd",
     "base_layer_bwd", "base_test_inject", "base_workspace_size_blend", "base_layer_fwd_blend",
-    "base_expert_stack", "base_sanitize_scores",
+    "base_expert_stack", "base_sanitize_scores", "base_workspace_size_fig9", "base_assign_fig9",
 )
 
 
@@ -81,6 +81,8 @@ _SIGS = {
     "base_test_inject": (_i, [_i, ctypes.c_longlong]),
     "base_workspace_size_blend": (_sz, [_i, _i, _i, _i]),
     "base_sanitize_scores": (_i, [_vp, _vp, _i, _i, _vp, _sz, _vp]),
+    "base_workspace_size_fig9": (_sz, [_i, _i]),
+    "base_assign_fig9": (_i, [_vp, _i, _i, _vp, _vp, _vp, ctypes.c_longlong, _vp, _sz, _vp]),
     "base_expert_stack": (_i, [_vp, _vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _i, _vp, _vp, _vp,
                                _vp, _sz, _vp]),
     "base_layer_fwd_blend": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp,
@@ -203,6 +205,18 @@ def base_assign_balanced_ex(q, assign, price, stats, ws, max_rounds: int = 10000
     _check("base_assign_balanced_ex", lib().base_assign_balanced_ex(
         _ptr(q), T, E, _ptr(assign), _ptr(price), _ptr(stats), int(max_rounds), _ptr(u_trace),
         _ptr(t_trace), cap, _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def base_workspace_size_fig9(T: int, E: int) -> int:
+    return int(lib().base_workspace_size_fig9(T, E))
+
+
+def base_assign_fig9(q, assign, price, stats, ws, max_iterations: int = 100, stream=None):
+    """The fig. 9 solver; price: T int64 token prices; stats: 4 int64 (device)."""
+    T, E = q.shape
+    _check("base_assign_fig9", lib().base_assign_fig9(
+        _ptr(q), T, E, _ptr(assign), _ptr(price), _ptr(stats), int(max_iterations), _ptr(ws),
+        ws.numel() * ws.element_size(), _stream(stream)))
 
 
 def base_permute(h, assign, E, perm, inv, offsets, x_perm, s=None, gate=None, ws=None,

@@ -23,6 +23,14 @@ def workspace_blend(T: int, E: int, D: int, F: int, device="cuda") -> torch.Tens
     return ws[off:off + n]
 
 
+def workspace_fig9(T: int, E: int, device="cuda") -> torch.Tensor:
+    """A 256-byte-aligned workspace of base_workspace_size_fig9(T, E) bytes."""
+    n = binding.base_workspace_size_fig9(T, E)
+    ws = torch.empty(n + 256, dtype=torch.uint8, device=device)
+    off = (-ws.data_ptr()) % 256
+    return ws[off:off + n]
+
+
 def stats(device="cuda") -> torch.Tensor:
     """Device storage for one base_auction_stats (6 int64)."""
     return torch.zeros(6, dtype=torch.int64, device=device)

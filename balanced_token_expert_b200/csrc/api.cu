@@ -17,6 +17,10 @@ size_t auction_workspace_bytes(int T, int E);
 int launch_auction(const int32_t* q, int T, int E, int32_t* assign, int64_t* price,
                    base_auction_stats* stats, void* ws, size_t ws_bytes, long long max_rounds,
                    int32_t* u_trace, int64_t* t_trace, long long trace_cap, cudaStream_t stream);
+size_t fig9_workspace_bytes(int T, int E);
+int launch_fig9(const int32_t* q, int T, int E, int32_t* assign, int64_t* price, int64_t* stats,
+                long long max_iterations, long long max_rounds, void* ws, size_t ws_bytes,
+                cudaStream_t stream);
 size_t permute_workspace_bytes(int T, int E);
 int launch_sort_by_expert(const int32_t* assign, int T, int E, int32_t* perm, int32_t* inv,
                           int32_t* offsets, const float* s, float* gate, void* ws,
@@ -172,6 +176,24 @@ int base_assign_balanced_ex(const int32_t* q, int T, int E, int32_t* assign, int
     if (ws_bytes < auction_workspace_bytes(T, E)) return BASE_ERR_WORKSPACE;
     return launch_auction(q, T, E, assign, price, stats, ws, ws_bytes, max_rounds, u_trace, t_trace,
                           trace_cap, stream);
+}
+
+size_t base_workspace_size_fig9(int T, int E) {
+    if (!shapes_ok(T, E)) return 0;
+    return fig9_workspace_bytes(T, E);
+}
+
+int base_assign_fig9(const int32_t* q, int T, int E, int32_t* assign, int64_t* price,
+                     int64_t* stats, long long max_iterations, void* ws, size_t ws_bytes,
+                     cudaStream_t stream) {
+    if (!q || !assign || !price || !ws || !shapes_ok(T, E) || T % E != 0 || max_iterations < 0)
+        return BASE_ERR_INVALID_ARG;
+    if (!aligned(q, 4) || !aligned(assign, 4) || !aligned(price, 8) || !aligned(ws, 256) ||
+        (stats && !aligned(stats, 8)))
+        return BASE_ERR_INVALID_ARG;
+    if (ws_bytes < fig9_workspace_bytes(T, E)) return BASE_ERR_WORKSPACE;
+    return launch_fig9(q, T, E, assign, price, stats, max_iterations, BASE_AUCTION_MAX_ROUNDS, ws,
+                       ws_bytes, stream);
 }
 
 int base_permute(const void* h, const int32_t* assign, int T, int D, int E, int32_t* perm,

@@ -744,7 +744,8 @@ __device__ __forceinline__ uint64_t globaltimer() {
 // warp 0 polls all flags.  Every CTA calls it the same number of times, so
 // the counts agree.  Returns false when the wait gave up or another CTA gave
 // up.
-__device__ bool grid_sync(const Params& p, unsigned& gen, int* s_flag) {
+template <class P>
+__device__ bool grid_sync(const P& p, unsigned& gen, int* s_flag) {
     __syncthreads();
     ++gen;
     if (warp_id() == 0) {
@@ -2451,6 +2452,216 @@ struct SmemPlan {
     size_t bytes;
 };
 
+// ---------------------------------------------------------------- fig. 9
+// The page's fig. 9 listing ("Solver"): experts bid for tokens and prices are
+// per token, with the released code's rules where "Paper vs code" says the
+// code differs (eps = range / 50, a won token kept in its holder's list at
+// the largest score -- here that score plus one, strictly above every other
+// value -- and after the iteration cap the listing's update without the
+// holders' minimal bids, looping until every token has a bid).  Integer
+// version on the quantised scores, the same steps as the CPU oracle's
+// orc_fig9.  One cooperative grid; a round is
+//   A: the CTA of expert e (e mod grid) finds e's (C+1)-th best adjusted
+//      value X by a radix select over its T tokens (values in shared memory
+//      when they fit) and bids raise = v - X + eps on its top C tokens (eps
+//      for tokens it won last round while under the cap) with an atomic
+//      max per token;
+//   B: each token's largest bid is matched to the smallest expert that made
+//      it (atomic min);
+//   C: every token: won when its largest bid is > 0, price += that bid;
+// with a grid barrier after each step.
+struct Fig9Params {
+    const int32_t* q;
+    int T, E, C;
+    long long max_iterations, max_rounds;
+    int keys_in_smem;  // 1: an expert's T keys fit in shared memory
+    int32_t* assign;
+    int64_t* price_out;  // [T] final token prices
+    int64_t* stats;      // [4] status, rounds, eps, objective (device)
+    unsigned* mmenc;     // [2] score range (enc keeps the signed order)
+    Ctrl* ctrl;          // abort flag; not-won counts by round mod 3
+    unsigned* bar_flags;
+    unsigned long long* bmax;  // [T] largest bid of the round
+    int32_t* barg;             // [T] smallest expert with it
+    int32_t* holder;           // [T] -1: not won
+    int64_t* price;            // [T]
+    int32_t* cnt;              // [E] tokens per expert at the end
+    unsigned long long* obj;   // [1]
+    unsigned long long wait_ns;
+};
+
+__global__ void __launch_bounds__(kThreads, 1) fig9_kernel(const __grid_constant__ Fig9Params p) {
+    extern __shared__ __align__(16) unsigned char smem[];
+    int32_t* s_hist = reinterpret_cast<int32_t*>(smem);               // kWarps * kHist
+    int64_t* s_red = reinterpret_cast<int64_t*>(s_hist + kWarps * kHist);  // 32
+    int32_t* s_cnt = reinterpret_cast<int32_t*>(s_red + 32);              // 64
+    int32_t* s_misc = s_cnt + 64;                                         // 16
+    int64_t* s_xb = reinterpret_cast<int64_t*>(s_misc + 16);              // 8: X of the owned experts
+    int32_t* s_xt = reinterpret_cast<int32_t*>(s_xb + 8);                 // 8
+    Key* s_keys = reinterpret_cast<Key*>(s_xt + 8);                       // T (keys_in_smem)
+    const Team<kThreads> tm{s_hist, s_red, s_cnt};
+    const int T = p.T, E = p.E, C = p.C;
+    const int cta = blockIdx.x, ncta = gridDim.x, tid = threadIdx.x;
+    unsigned bar_gen = 0;
+    bool ok = true;
+    // the score range, and the per-token state
+    {
+        unsigned mx = 0u, mn = 0u;
+        for (long long i = (long long)cta * kThreads + tid; i < (long long)T * E;
+             i += (long long)ncta * kThreads) {
+            const unsigned a = (unsigned)__ldg(p.q + i) ^ 0x80000000u;
+            mx = max(mx, a);
+            mn = max(mn, ~a);
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+            mn = max(mn, __shfl_xor_sync(0xffffffffu, mn, off));
+        }
+        if (lane_id() == 0) {
+            atomicMax(&p.mmenc[0], mx);
+            atomicMax(&p.mmenc[1], mn);
+        }
+        for (int t = cta * kThreads + tid; t < T; t += ncta * kThreads) {
+            p.holder[t] = -1;
+            p.price[t] = 0;
+            p.bmax[t] = 0ull;
+            p.barg[t] = INT32_MAX;
+        }
+    }
+    if (!(ok = grid_sync(p, bar_gen, s_misc))) return;
+    const int64_t qmax = (int32_t)(vload(&p.mmenc[0]) ^ 0x80000000u);
+    const int64_t qmin = (int32_t)((~vload(&p.mmenc[1])) ^ 0x80000000u);
+    int64_t eps = (qmax - qmin) / 50;
+    if (eps < 1) eps = 1;
+    const int64_t RETAIN = qmax + 1;
+    int status = BASE_OK;
+    long long r = 0;
+    int notwon = T;
+    for (;; ++r) {
+        if (r > 0 && notwon == 0) break;
+        if (r >= p.max_rounds) {
+            status = BASE_ERR_NOT_CONVERGED;
+            break;
+        }
+        const bool retain_bids = r > 0 && r < p.max_iterations;  // holders bid eps
+        const bool retain_top = r > 0 && r - 1 < p.max_iterations;  // won tokens at RETAIN
+        // the counter round r + 1 fills: last read after round r - 2
+        if (cta == 0 && tid == 0) p.ctrl->ucount[(int)((r + 1) % 3)] = 0;
+        // ---- A: the experts' lists and bids
+        for (int e = cta; e < E; e += ncta) {
+            auto key_of = [&](int t) {  // holder / price come from other CTAs: read past L1
+                const int h = __ldcg(p.holder + t);
+                const int64_t qv = __ldg(p.q + (size_t)t * E + e);
+                int64_t v;
+                if (h == e && retain_top) v = RETAIN;
+                else if (h == e) v = qv;
+                else v = qv - (int64_t)__ldcg(reinterpret_cast<const long long*>(p.price) + t);
+                return Key{v, t, 0};
+            };
+            if (p.keys_in_smem) {
+                for (int t = tid; t < T; t += kThreads) s_keys[t] = key_of(t);
+                __syncthreads();
+            }
+            auto visit = [&](auto fn) {
+                if (p.keys_in_smem)
+                    for (int t = tid; t < T; t += kThreads) fn(s_keys[t]);
+                else
+                    for (int t = tid; t < T; t += kThreads) fn(key_of(t));
+            };
+            // X: the (C+1)-th best = the (T-C)-th worst
+            const Key X = kth_worst_cta(tm, visit, T - C, T - 1);
+            for (int t = tid; t < T; t += kThreads) {
+                const Key x = p.keys_in_smem ? s_keys[t] : key_of(t);
+                if (!worse(X, x)) continue;  // not in the top C
+                const int64_t bid =
+                    (retain_bids && __ldcg(p.holder + t) == e) ? eps : x.bid - X.bid + eps;
+                atomicMax(p.bmax + t, (unsigned long long)bid);
+            }
+            // keep X for step B (at most 8 owned experts: E <= 1024 < 8 grid)
+            if (tid == 0) {
+                s_xb[(e / ncta) & 7] = X.bid;
+                s_xt[(e / ncta) & 7] = X.tok;
+            }
+            __syncthreads();
+        }
+        if (!(ok = grid_sync(p, bar_gen, s_misc))) break;
+        // ---- B: the smallest expert with each token's largest bid
+        for (int e = cta; e < E; e += ncta) {
+            const Key X{s_xb[(e / ncta) & 7], s_xt[(e / ncta) & 7], 0};
+            auto key_of = [&](int t) {  // holder / price come from other CTAs: read past L1
+                const int h = __ldcg(p.holder + t);
+                const int64_t qv = __ldg(p.q + (size_t)t * E + e);
+                int64_t v;
+                if (h == e && retain_top) v = RETAIN;
+                else if (h == e) v = qv;
+                else v = qv - (int64_t)__ldcg(reinterpret_cast<const long long*>(p.price) + t);
+                return Key{v, t, 0};
+            };
+            for (int t = tid; t < T; t += kThreads) {
+                const Key x = key_of(t);
+                if (!worse(X, x)) continue;
+                const int64_t bid =
+                    (retain_bids && __ldcg(p.holder + t) == e) ? eps : x.bid - X.bid + eps;
+                if ((unsigned long long)bid == __ldcg(p.bmax + t)) atomicMin(p.barg + t, e);
+            }
+        }
+        if (!(ok = grid_sync(p, bar_gen, s_misc))) break;
+        // ---- C: every token
+        int nw = 0;
+        for (int t = cta * kThreads + tid; t < T; t += ncta * kThreads) {
+            const unsigned long long b = __ldcg(p.bmax + t);  // atomics of other CTAs
+            if (b > 0ull) {
+                p.holder[t] = __ldcg(p.barg + t);
+            } else {
+                p.holder[t] = -1;
+                ++nw;
+            }
+            p.price[t] += (int64_t)b;
+            p.bmax[t] = 0ull;
+            p.barg[t] = INT32_MAX;
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) nw += __shfl_xor_sync(0xffffffffu, nw, off);
+        if (lane_id() == 0 && nw) atomicAdd(&p.ctrl->ucount[(int)(r % 3)], nw);
+        if (!(ok = grid_sync(p, bar_gen, s_misc))) break;
+        notwon = vload(&p.ctrl->ucount[(int)(r % 3)]);
+    }
+    if (!ok) {
+        if (cta == 0 && tid == 0 && p.stats) p.stats[0] = BASE_ERR_TIMEOUT;
+        return;
+    }
+    // the result: every token to its holder; balance checked
+    unsigned long long part = 0;
+    for (int t = cta * kThreads + tid; t < T; t += ncta * kThreads) {
+        const int h = p.holder[t];
+        p.price_out[t] = p.price[t];
+        if (status == BASE_OK && h >= 0 && h < E) {
+            p.assign[t] = h;
+            atomicAdd(p.cnt + h, 1);
+            part += (unsigned long long)(int64_t)__ldg(p.q + (size_t)t * E + h);
+        }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
+    if (lane_id() == 0 && part) atomicAdd(p.obj, part);
+    if (!grid_sync(p, bar_gen, s_misc)) {
+        if (cta == 0 && tid == 0 && p.stats) p.stats[0] = BASE_ERR_TIMEOUT;
+        return;
+    }
+    if (cta == 0 && tid == 0) {
+        if (status == BASE_OK)
+            for (int e = 0; e < E; ++e)
+                if (__ldcg(p.cnt + e) != C) status = BASE_ERR_NOT_CONVERGED;  // not a partition
+        if (p.stats) {
+            p.stats[0] = status;
+            p.stats[1] = r;
+            p.stats[2] = eps;
+            p.stats[3] = status == BASE_OK ? (int64_t)__ldcg(p.obj) : 0;
+        }
+    }
+}
+
 constexpr size_t kSmemMax = 227 * 1024;  // dynamic shared memory of one CTA
 
 static SmemPlan smem_plan(int E, int NM, int T) {
@@ -2475,6 +2686,73 @@ static SmemPlan smem_plan(int E, int NM, int T) {
 }
 
 }  // namespace auction
+
+size_t fig9_workspace_bytes(int T, int E) {
+    size_t b = align_up(2 * sizeof(unsigned), 256);
+    b += align_up(sizeof(auction::Ctrl), 256);
+    b += align_up(sizeof(unsigned) * auction::kMaxGrid, 256);
+    b += align_up(sizeof(unsigned long long) * (size_t)T, 256);  // bmax
+    b += align_up(sizeof(int32_t) * (size_t)T, 256);             // barg
+    b += align_up(sizeof(int32_t) * (size_t)T, 256);             // holder
+    b += align_up(sizeof(int64_t) * (size_t)T, 256);             // price
+    b += align_up(sizeof(int32_t) * (size_t)E, 256);             // counts
+    b += align_up(64, 256);                                      // objective
+    return b;
+}
+
+int launch_fig9(const int32_t* q, int T, int E, int32_t* assign, int64_t* price, int64_t* stats,
+                long long max_iterations, long long max_rounds, void* ws, size_t ws_bytes,
+                cudaStream_t stream) {
+    using namespace auction;
+    if (ws_bytes < fig9_workspace_bytes(T, E)) return BASE_ERR_WORKSPACE;
+    unsigned char* w = static_cast<unsigned char*>(ws);
+    size_t o = 0;
+    auto take = [&](size_t bytes) { unsigned char* r = w + o; o += align_up(bytes, 256); return r; };
+    Fig9Params prm{};
+    prm.q = q;
+    prm.T = T;
+    prm.E = E;
+    prm.C = T / E;
+    prm.max_iterations = max_iterations;
+    prm.max_rounds = max_rounds;
+    prm.assign = assign;
+    prm.price_out = price;
+    prm.stats = stats;
+    prm.wait_ns = g_test_hooks.wait_ns > 0 ? (unsigned long long)g_test_hooks.wait_ns : kWaitNs;
+    unsigned char* zero0 = w;
+    prm.mmenc = reinterpret_cast<unsigned*>(take(2 * sizeof(unsigned)));
+    prm.ctrl = reinterpret_cast<Ctrl*>(take(sizeof(Ctrl)));
+    prm.bar_flags = reinterpret_cast<unsigned*>(take(sizeof(unsigned) * kMaxGrid));
+    const size_t zero_a = o;
+    prm.bmax = reinterpret_cast<unsigned long long*>(take(sizeof(unsigned long long) * (size_t)T));
+    prm.barg = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * (size_t)T));
+    prm.holder = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * (size_t)T));
+    prm.price = reinterpret_cast<int64_t*>(take(sizeof(int64_t) * (size_t)T));
+    unsigned char* zero1 = w + o;
+    prm.cnt = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * (size_t)E));
+    prm.obj = reinterpret_cast<unsigned long long*>(take(64));
+    if (cudaMemsetAsync(zero0, 0, zero_a, stream) != cudaSuccess) return BASE_ERR_CUDA;
+    if (cudaMemsetAsync(zero1, 0, (size_t)((w + o) - zero1), stream) != cudaSuccess)
+        return BASE_ERR_CUDA;
+    const size_t base_smem = sizeof(int32_t) * kWarps * kHist + 8 * 32 + 4 * 64 + 4 * 16 + 8 * 8 + 4 * 8;
+    const size_t keys = sizeof(Key) * (size_t)T;
+    prm.keys_in_smem = base_smem + keys <= kSmemMax ? 1 : 0;
+    const size_t smem = base_smem + (prm.keys_in_smem ? keys : 0);
+    if (cudaFuncSetAttribute(fig9_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem) != cudaSuccess)
+        return BASE_ERR_CUDA;
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fig9_kernel, kThreads, smem) !=
+            cudaSuccess ||
+        per_sm < 1)
+        return BASE_ERR_UNSUPPORTED;
+    const int grid = std::min(num_sms(), kMaxGrid);
+    void* args[] = {&prm};
+    if (cudaLaunchCooperativeKernel(reinterpret_cast<void*>(fig9_kernel), dim3(grid),
+                                    dim3(kThreads), args, smem, stream) != cudaSuccess)
+        return BASE_ERR_CUDA;
+    return BASE_OK;
+}
 
 size_t auction_workspace_bytes(int T, int E) {
     const int C = T / E;

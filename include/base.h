@@ -226,6 +226,32 @@ int base_assign_balanced_ex(const int32_t* q, int T, int E, int32_t* assign, int
                             cudaStream_t stream);
 
 /*
+ * The page's fig. 9 solver (the wikillm.com summary's "Solver": experts bid
+ * for tokens and prices are per token), with the released code's rules that
+ * "Paper vs code" describes: eps = max(1, (max q - min q) / 50) on the
+ * quantised scores; a token won in a round stays in its holder's list at the
+ * largest score plus one (the listing's "infinity", kept finite and strictly
+ * above every other value); while the round number is below max_iterations
+ * (the listing's cap, 100) the holder bids eps on it; after the cap the
+ * listing's other update runs and rounds go on until every token has a bid.
+ * Every round, each expert bids raise = v_j - v_{C+1} + eps on the tokens of
+ * its C best adjusted values (ties: smaller token first); a token goes to its
+ * largest bid (smaller expert on ties), is won when that bid is > 0, and its
+ * price grows by it.  The result is balanced; it is not the exact optimum of
+ * eq. 2 (the eps of one phase bounds the loss), and base_assign_balanced
+ * remains the training solver.
+ *   q: T*E int32; assign: T int32; price: T int64 token prices;
+ *   stats (nullable): 4 int64 of device memory -- status, rounds, eps,
+ *   objective (sum_t q[t][assign[t]]); status BASE_ERR_NOT_CONVERGED when
+ *   BASE_AUCTION_MAX_ROUNDS pass.
+ *   ws: at least base_workspace_size_fig9(T, E) bytes.  One cooperative grid.
+ */
+size_t base_workspace_size_fig9(int T, int E);
+int base_assign_fig9(const int32_t* q, int T, int E, int32_t* assign, int64_t* price,
+                     int64_t* stats, long long max_iterations, void* ws, size_t ws_bytes,
+                     cudaStream_t stream);
+
+/*
  * a5: permutation into expert-contiguous slots (fig. 2 sort_by_expert).
  * Slot order is expert-major and ascending token index inside an expert.
  *   h: T*D bf16; assign: T int32 in [0, E).

@@ -379,3 +379,43 @@ def test_layer_fwd_sanitizes_non_finite_scores(orc):
     fw = orc.layer_forward(h, inp.w, inp.W1, inp.W2, "relu", a_g)
     ok, worst = close_rel_rms(to_np(out)[good], fw["out"][good], 2e-2)
     assert ok, worst
+
+
+# ------------------------------------------------------------------ fig. 9 solver
+def gpu_fig9(q_np, max_iterations=100):
+    T, E = q_np.shape
+    assign = torch.full((T,), -1, dtype=torch.int32, device="cuda")
+    price = torch.zeros(T, dtype=torch.int64, device="cuda")
+    st = torch.zeros(4, dtype=torch.int64, device="cuda")
+    B.base_assign_fig9(dev(q_np), assign, price, st, buffers.workspace_fig9(T, E), max_iterations)
+    torch.cuda.synchronize()
+    s = st.tolist()
+    return to_np(assign), to_np(price), dict(status=s[0], rounds=s[1], eps=s[2], objective=s[3])
+
+
+def test_fig9_hand_worked_cases():
+    from test_oracle_fig9 import check_fig9, fig9_hand_cases
+    for name, q, cap, exp in fig9_hand_cases():
+        check_fig9(exp, *gpu_fig9(q, cap))
+
+
+@pytest.mark.parametrize("T,E,small,cap", [(12, 3, True, 100), (512, 8, False, 100),
+                                           (1000, 8, True, 100), (4096, 16, False, 2),
+                                           (2048, 64, False, 100), (1536, 1536 // 16, True, 100)])
+def test_fig9_bit_exact(orc, T, E, small, cap):
+    rng = np.random.default_rng(T + 3 * E)
+    q = (rng.integers(0, 4, size=(T, E)) if small else
+         rng.integers(-300000, 300000, size=(T, E))).astype(np.int32)
+    a, p, st = gpu_fig9(q, cap)
+    ao, po, so = orc.fig9_auction(q, max_iterations=cap)
+    assert st == so, (st, so)
+    assert np.array_equal(a, ao) and np.array_equal(p, po)
+
+
+@pytest.mark.parametrize("name", ["routing_ref", "layer_fwd"])
+def test_fig9_workloads_bit_exact(orc, name):
+    _, _, q = oracle_q(orc, synth.WORKLOADS[name])
+    a, p, st = gpu_fig9(q)
+    ao, po, so = orc.fig9_auction(q)
+    assert st == so and np.array_equal(a, ao) and np.array_equal(p, po)
+    assert st["objective"] <= orc.auction(q)[2]["objective"]  # never above the optimum
