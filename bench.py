@@ -45,7 +45,6 @@ UNIT = "tokens/s"
 # named workload at its full size (the component's kernels summed); a
 # component whose kernels changed after their capture has no entry.
 NCU_TRAFFIC = {
-    ("auction", "layer_fwd"): 883200 + 3584,
     ("scores", "layer_fwd"): 16837632,
     ("ffn", "layer_fwd"): 151049984 + 39332864 + 222304000 + 11714816,
     # slice histogram + slice rank + row gather; the rows' writes stay in L2
