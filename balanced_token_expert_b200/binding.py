@@ -25,6 +25,7 @@ __all__ = [
     "base_layer_bwd", "base_test_inject", "BASE_TEST_WAIT_LIMIT_NS",
     "base_workspace_size_blend", "base_layer_fwd_blend", "base_expert_stack",
     "base_sanitize_scores", "BASE_ROUTE_SANITIZE", "base_workspace_size_fig9", "base_assign_fig9",
+    "base_probe_workspace_size", "base_measure_latency",
     "BASE_TEST_AUCTION_ABSENT_CTA", "BASE_TEST_GEMM_DROP_FIRST_LOAD", "EXPORTED",
 ]
 
@@ -43,6 +44,7 @@ EXPORTED = (
     "base_permute", "base_permute_noalloc", "base_expert_ffn", "base_combine", "base_layer_fwd",
     "base_layer_bwd", "base_test_inject", "base_workspace_size_blend", "base_layer_fwd_blend",
     "base_expert_stack", "base_sanitize_scores", "base_workspace_size_fig9", "base_assign_fig9",
+    "base_probe_workspace_size", "base_measure_latency",
 )
 
 
@@ -82,6 +84,8 @@ _SIGS = {
     "base_workspace_size_blend": (_sz, [_i, _i, _i, _i]),
     "base_sanitize_scores": (_i, [_vp, _vp, _i, _i, _vp, _sz, _vp]),
     "base_workspace_size_fig9": (_sz, [_i, _i]),
+    "base_probe_workspace_size": (_sz, []),
+    "base_measure_latency": (_i, [_vp, _vp, _sz, _vp]),
     "base_assign_fig9": (_i, [_vp, _i, _i, _vp, _vp, _vp, ctypes.c_longlong, _vp, _sz, _vp]),
     "base_expert_stack": (_i, [_vp, _vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _i, _vp, _vp, _vp,
                                _vp, _sz, _vp]),
@@ -205,6 +209,16 @@ def base_assign_balanced_ex(q, assign, price, stats, ws, max_rounds: int = 10000
     _check("base_assign_balanced_ex", lib().base_assign_balanced_ex(
         _ptr(q), T, E, _ptr(assign), _ptr(price), _ptr(stats), int(max_rounds), _ptr(u_trace),
         _ptr(t_trace), cap, _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def base_probe_workspace_size() -> int:
+    return int(lib().base_probe_workspace_size())
+
+
+def base_measure_latency(out, ws, stream=None):
+    """out: 4 float64 on the device (ns: grid barrier, block barrier, L2 load, shared load)."""
+    _check("base_measure_latency", lib().base_measure_latency(
+        _ptr(out), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)))
 
 
 def base_workspace_size_fig9(T: int, E: int) -> int:

@@ -17,6 +17,8 @@ size_t auction_workspace_bytes(int T, int E);
 int launch_auction(const int32_t* q, int T, int E, int32_t* assign, int64_t* price,
                    base_auction_stats* stats, void* ws, size_t ws_bytes, long long max_rounds,
                    int32_t* u_trace, int64_t* t_trace, long long trace_cap, cudaStream_t stream);
+size_t probe_workspace_bytes();
+int launch_latency_probe(double* out, void* ws, cudaStream_t stream);
 size_t fig9_workspace_bytes(int T, int E);
 int launch_fig9(const int32_t* q, int T, int E, int32_t* assign, int64_t* price, int64_t* stats,
                 long long max_iterations, long long max_rounds, void* ws, size_t ws_bytes,
@@ -176,6 +178,14 @@ int base_assign_balanced_ex(const int32_t* q, int T, int E, int32_t* assign, int
     if (ws_bytes < auction_workspace_bytes(T, E)) return BASE_ERR_WORKSPACE;
     return launch_auction(q, T, E, assign, price, stats, ws, ws_bytes, max_rounds, u_trace, t_trace,
                           trace_cap, stream);
+}
+
+size_t base_probe_workspace_size(void) { return probe_workspace_bytes(); }
+
+int base_measure_latency(double* out, void* ws, size_t ws_bytes, cudaStream_t stream) {
+    if (!out || !ws || !aligned(out, 8) || !aligned(ws, 256)) return BASE_ERR_INVALID_ARG;
+    if (ws_bytes < probe_workspace_bytes()) return BASE_ERR_WORKSPACE;
+    return launch_latency_probe(out, ws, stream);
 }
 
 size_t base_workspace_size_fig9(int T, int E) {

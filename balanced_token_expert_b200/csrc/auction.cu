@@ -746,43 +746,45 @@ __device__ __forceinline__ uint64_t globaltimer() {
 // up.
 template <class P>
 __device__ bool grid_sync(const P& p, unsigned& gen, int* s_flag) {
+    // A counter barrier: every CTA adds one to an arrival count that only
+    // grows (it reaches gen * grid at barrier gen); the CTA that brings it
+    // there publishes gen in a release word, which the others poll -- one
+    // word per poll instead of every CTA's flag.  The counter and the
+    // release word sit 128 bytes apart in bar_flags (zeroed per launch).
     __syncthreads();
     ++gen;
-    if (warp_id() == 0) {
-        const int lane = lane_id();
-        if (lane == 0) {
-            __threadfence();
-            *reinterpret_cast<volatile unsigned*>(p.bar_flags + blockIdx.x) = gen;
-        }
+    if (threadIdx.x == 0) {
+        unsigned* count = p.bar_flags;
+        unsigned* release = p.bar_flags + 32;
         int ok = 1;
-        const uint64_t t0 = globaltimer();
-        for (long long it = 1;; ++it) {
-            bool mine = true;
-            for (int c = lane; c < (int)gridDim.x; c += 32)
-                mine &= (int)(vload(p.bar_flags + c) - gen) >= 0;
-            if (__all_sync(0xffffffffu, mine)) break;
-            // short naps while the barrier is young, longer ones in a long
-            // wait (the narrow rounds of CTA 0) to spare the L2
-            __nanosleep(it < 64 ? 20 : 200);
-            if ((it & 31) == 0) {
-                int stop = 0;
-                if (lane == 0) {
+        __threadfence();  // this CTA's writes before its arrival
+        const unsigned old = atomicAdd(count, 1u);
+        if (old + 1u == gen * gridDim.x) {
+            __threadfence();
+            *reinterpret_cast<volatile unsigned*>(release) = gen;
+        } else {
+            const uint64_t t0 = globaltimer();
+            for (long long it = 1;; ++it) {
+                if ((int)(vload(release) - gen) >= 0) break;
+                // short naps while the barrier is young, longer ones in a long
+                // wait (the narrow rounds of CTA 0) to spare the L2
+                __nanosleep(it < 256 ? 20 : 200);
+                if ((it & 63) == 0) {
                     if (*reinterpret_cast<volatile int*>(&p.ctrl->abort)) {
-                        stop = 1;
-                    } else if (globaltimer() - t0 > p.wait_ns || it > (1ll << 30)) {
+                        ok = 0;
+                        break;
+                    }
+                    if (globaltimer() - t0 > p.wait_ns || it > (1ll << 30)) {
                         atomicExch(&p.ctrl->abort, 1);
                         record_error(5001);
-                        stop = 1;
+                        ok = 0;
+                        break;
                     }
-                }
-                if (__shfl_sync(0xffffffffu, stop, 0)) {
-                    ok = 0;
-                    break;
                 }
             }
         }
         __threadfence();
-        if (lane == 0) *s_flag = ok;
+        *s_flag = ok;
     }
     __syncthreads();
     return *s_flag != 0;

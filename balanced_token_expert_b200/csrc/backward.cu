@@ -11,6 +11,8 @@
 // The four contractions run on the tcgen05 GEMM: dH1 and dx read the
 // weights as MN-major operands (no transposed copy), dW1 / dW2 read the
 // activations as MN-major operands and reduce over each expert's slot range.
+#include <algorithm>
+
 #include "common.cuh"
 
 namespace base {
@@ -70,21 +72,54 @@ __global__ void gate_grad_kernel(const __nv_bfloat16* __restrict__ dy,
     }
 }
 
-// dw[e][d] = sum_{r in segment e} ds[r] x_perm[r][d]; a block per (expert, 256 columns,
-// row split); partial sums are added atomically into the zeroed dw
-__global__ void centroid_grad_kernel(const __nv_bfloat16* __restrict__ x, const float* __restrict__ ds,
-                                     const int32_t* __restrict__ offsets, int D, int splits,
-                                     float* __restrict__ dw) {
-    const int e = blockIdx.y;
-    const int d = blockIdx.x * blockDim.x + threadIdx.x;
-    const int r0 = offsets[e], r1 = offsets[e + 1];
-    const int len = r1 - r0;
-    const int per = (len + splits - 1) / splits;
-    const int a = r0 + blockIdx.z * per, b = min(r1, a + per);
-    if (d >= D) return;
-    float acc = 0.f;
-    for (int r = a; r < b; ++r) acc = fmaf(__ldg(ds + r), __bfloat162float(x[(size_t)r * D + d]), acc);
-    if (b > a) atomicAdd(dw + (size_t)e * D + d, acc);
+// dw[e][d] = sum_{r in segment e} ds[r] x_perm[r][d], in two deterministic
+// steps.  Partials: a block per (2048 columns, expert, row split), every
+// thread 8 consecutive columns read as one 16-byte vector per row; the
+// partial sums go to part[z][e][d].  Then every (e, d) adds its splits in
+// order.  HBM-bound: the T x D bf16 rows are read once.
+__global__ void __launch_bounds__(256) centroid_grad_partial_kernel(
+    const __nv_bfloat16* __restrict__ x, const float* __restrict__ ds,
+    const int32_t* __restrict__ offsets, int D, int E, int splits, float* __restrict__ part) {
+    const int e = blockIdx.y, z = blockIdx.z;
+    const int d0 = (blockIdx.x * blockDim.x + threadIdx.x) * 8;
+    const int r0 = __ldg(offsets + e), r1 = __ldg(offsets + e + 1);
+    const int per = (r1 - r0 + splits - 1) / splits;
+    const int a = r0 + z * per, b = min(r1, a + per);
+    if (d0 >= D) return;
+    float acc[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+#pragma unroll 4
+    for (int r = a; r < b; ++r) {
+        const uint4 v = __ldg(reinterpret_cast<const uint4*>(x + (size_t)r * D + d0));
+        const float sv = __ldg(ds + r);
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            acc[2 * i] = fmaf(sv, __uint_as_float(w[i] << 16), acc[2 * i]);
+            acc[2 * i + 1] = fmaf(sv, __uint_as_float(w[i] & 0xFFFF0000u), acc[2 * i + 1]);
+        }
+    }
+    float4* o = reinterpret_cast<float4*>(part + ((size_t)z * E + e) * D + d0);
+    o[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+    o[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+}
+
+__global__ void centroid_grad_reduce_kernel(const float* __restrict__ part, int splits, long long n,
+                                            float* __restrict__ dw) {
+    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n;
+         i += (long long)gridDim.x * blockDim.x) {
+        float acc = 0.f;
+        for (int z = 0; z < splits; ++z) acc += __ldg(part + (size_t)z * n + i);
+        dw[i] = acc;
+    }
+}
+
+static int centroid_splits(int E, int D, int C) {
+    const int bxy = ((D / 8 + 255) / 256) * E;
+    int splits = (8 * num_sms() + bxy - 1) / bxy;
+    splits = std::min(splits, std::max(1, C / 16));
+    return std::max(1, std::min(splits, 64));
 }
 
 }  // namespace bwd
@@ -96,6 +131,7 @@ size_t backward_workspace_bytes(int T, int E, int D, int F) {
     b += align_up((size_t)T * 4, 256);      // ds
     b += align_up((size_t)T * F * 2, 256);  // dA1
     b += align_up((size_t)(E + 1) * 4, 256);
+    b += align_up(sizeof(float) * 64 * (size_t)E * D, 256);  // centroid-gradient partials
     return b;
 }
 
@@ -113,6 +149,7 @@ int launch_layer_bwd(const void* h, const void* w, const void* W1, const void* W
     float* ds = reinterpret_cast<float*>(p + o); o += align_up((size_t)T * 4, 256);
     __nv_bfloat16* dA1 = reinterpret_cast<__nv_bfloat16*>(p + o); o += align_up((size_t)T * F * 2, 256);
     int32_t* tile_start = reinterpret_cast<int32_t*>(p + o); o += align_up((size_t)(E + 1) * 4, 256);
+    float* dw_part = reinterpret_cast<float*>(p + o); o += align_up(sizeof(float) * 64 * (size_t)E * D, 256);
     if (o > ws_bytes) return BASE_ERR_WORKSPACE;
 
     int st = launch_move_rows(dout, sv->perm, T, D, dy, false, stream);
@@ -125,13 +162,16 @@ int launch_layer_bwd(const void* h, const void* w, const void* W1, const void* W
             dy, static_cast<const __nv_bfloat16*>(sv->f), sv->gate, T, D, dF, ds, sv->offsets, E, C);
         BASE_RETURN_IF_LAUNCH_FAILED();
     }
-    if (cudaMemsetAsync(dw, 0, sizeof(float) * (size_t)E * D, stream) != cudaSuccess)
-        return BASE_ERR_CUDA;
     {
-        const int splits = (C + 127) / 128;
-        dim3 grid((D + 255) / 256, E, splits);
-        bwd::centroid_grad_kernel<<<grid, 256, 0, stream>>>(
-            static_cast<const __nv_bfloat16*>(sv->x_perm), ds, sv->offsets, D, splits, dw);
+        const int splits = bwd::centroid_splits(E, D, C);
+        dim3 grid((D / 8 + 255) / 256, E, splits);
+        bwd::centroid_grad_partial_kernel<<<grid, 256, 0, stream>>>(
+            static_cast<const __nv_bfloat16*>(sv->x_perm), ds, sv->offsets, D, E, splits, dw_part);
+        BASE_RETURN_IF_LAUNCH_FAILED();
+        const long long n = (long long)E * D;
+        long long blocks = (n + 255) / 256;
+        if (blocks > num_sms() * 8) blocks = num_sms() * 8;
+        bwd::centroid_grad_reduce_kernel<<<(int)blocks, 256, 0, stream>>>(dw_part, splits, n, dw);
         BASE_RETURN_IF_LAUNCH_FAILED();
     }
     return launch_bwd_gemms(dF, nullptr, dA1, sv->a1, sv->h1, sv->x_perm, dy, ds, w, sv->perm,

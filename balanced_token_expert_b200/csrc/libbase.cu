@@ -2,6 +2,7 @@
 // device error word and the kernels in one module without relocatable code).
 #include "routing.cu"
 #include "auction.cu"
+#include "probe.cu"
 #include "variant.cu"
 #include "gemm.cu"
 #include "backward.cu"

@@ -292,7 +292,7 @@ def measure(args, wl, steps, warmup, rank, world, local_rank):
         dW1 = torch.empty(E, F, D, device="cuda")
         dW2 = torch.empty(E, D, F, device="cuda")
         comps.append(("backward", lambda: B.base_layer_bwd(h, w, W1, W2, act, sv, dout, dh, dw,
-                                                           dW1, dW2, ws), 8))
+                                                           dW1, dW2, ws), 9))
     names = [n for n, _, _ in comps if n != "bump"]
 
     def step(ev):
@@ -360,8 +360,8 @@ def measure(args, wl, steps, warmup, rank, world, local_rank):
     B.base_assign_balanced_ex(sv["q"], sv["assign"], sv["price"], sv["stats"], ws, 1000000,
                               u_trace=u_tr, t_trace=t_tr)
     torch.cuda.synchronize()
-    rounds_by_kind = _rounds_by_kind(u_tr.cpu().tolist(), t_tr.cpu().tolist(), st["rounds"],
-                                     wl.T)
+    u_list = u_tr.cpu().tolist()
+    rounds_by_kind = _rounds_by_kind(u_list, t_tr.cpu().tolist(), st["rounds"], wl.T)
 
     # the fig. 9 solver on the same scores: the alternative the pages print,
     # compared on rounds, time and objective (it is not the exact optimum)
@@ -520,6 +520,7 @@ def measure(args, wl, steps, warmup, rank, world, local_rank):
                     frac=a_ / pk["hbm"], traffic=traffic, kernel=n, ms=comp[n],
                     peak_source=pk["source"] + " hbm copy")
 
+    lat = latency_roofline(u_list[:st["rounds"]], T, E, comp["auction"], args._floors, pk["hbm"])
     return dict(
         value=replicas.job_tokens_per_s(T, world, ms), ms_per_step=ms, steps=steps,
         warmup=warmup, config=_config(wl, args),
@@ -529,7 +530,8 @@ def measure(args, wl, steps, warmup, rank, world, local_rank):
                      rounds=st["rounds"],
                      phases=st["phases"], bids=bids, status=st["status"],
                      us_per_round=1e3 * comp["auction"] / max(1, st["rounds"]),
-                     rounds_by_kind=rounds_by_kind, objective=st["objective"], fig9=fig9),
+                     rounds_by_kind=rounds_by_kind, objective=st["objective"], fig9=fig9,
+                     latency_roofline=lat),
         e2e=dict(value=replicas.job_tokens_per_s(T, world, e2e), unit=UNIT,
                  mode="pipelined: copy streams each way, two device buffers",
                  serial_value=replicas.job_tokens_per_s(T, world, e2e_serial),
@@ -539,6 +541,49 @@ def measure(args, wl, steps, warmup, rank, world, local_rank):
         gpu_launches=kernels_per_step * steps,
         clocks=clk, device_error=err, wall_s=wall,
     )
+
+
+def measure_floors():
+    """Latency floors (ns) of the auction's steps on this GPU, from the
+    library's probe: grid barrier, block barrier, L2 load, shared load."""
+    import torch
+    from balanced_token_expert_b200 import binding as B
+    out = torch.zeros(4, dtype=torch.float64, device="cuda")
+    ws = torch.empty(B.base_probe_workspace_size() + 256, dtype=torch.uint8, device="cuda")
+    off = (-ws.data_ptr()) % 256
+    B.base_measure_latency(out, ws[off:])
+    torch.cuda.synchronize()
+    g, c, l2, sm = out.tolist()
+    return dict(grid_barrier_ns=g, block_barrier_ns=c, l2_load_ns=l2, smem_load_ns=sm)
+
+
+def latency_roofline(u, T, E, auction_ms, fl, hbm_gbs):
+    """The auction against its latency floor: every round costs at least its
+    synchronisation chain -- a grid-wide round two grid barriers and two
+    dependent L2 loads (bids in, resolves out), a one-CTA round two block
+    barriers and one L2 load (the rejected token's score row), a one-bidder
+    round one L2 load -- and a phase start no less than reading q from HBM.
+    Which mode a round runs in follows the kernel's rule: one bidder -> one
+    warp; up to 256 bidders (E <= 16) or 32 (else) -> one CTA; more -> grid."""
+    narrow_max = 256 if E <= 16 else 32
+    wide = 2 * fl["grid_barrier_ns"] + 2 * fl["l2_load_ns"]
+    narrow = 2 * fl["block_barrier_ns"] + fl["l2_load_ns"]
+    chain = fl["l2_load_ns"]
+    q_ns = 4.0 * T * E / hbm_gbs  # bytes / (GB/s) = ns
+    floor_ns = 0.0
+    for x in u:
+        if x == T:
+            floor_ns += max(wide, q_ns)
+        elif x == 1 and E <= 128:
+            floor_ns += chain
+        elif x <= narrow_max:
+            floor_ns += narrow
+        else:
+            floor_ns += wide
+    return dict(floor_ms=floor_ns / 1e6, frac=floor_ns / 1e6 / auction_ms, floors_ns=fl,
+                model="rounds x floor of their kind: grid round 2 grid barriers + 2 L2 loads, "
+                      "one-CTA round 2 block barriers + 1 L2 load, one-bidder round 1 L2 load, "
+                      "phase start at least q read from HBM")
 
 
 def _rounds_by_kind(u, t, rounds, T):
@@ -586,6 +631,7 @@ def main():
         dist.barrier()
     B.lib()
 
+    args._floors = measure_floors()
     head = measure(args, wl, args.steps, args.warmup, rank, world, local_rank)
     torch.cuda.empty_cache()
     extra = {}
@@ -601,7 +647,10 @@ def main():
             metric=METRIC, value=head["value"], unit=UNIT, n_gpus=world, steps=args.steps,
             warmup=args.warmup, ms_per_step=head["ms_per_step"], higher_is_better=True,
             scaling="weak", vs_baseline=None, dtype="bf16", data="synthetic",
-            config=head["config"], roofline=head["roofline"], per_kernel=head["per_kernel"],
+            config=head["config"], roofline=dict(head["roofline"], **(
+                {"latency": head["auction"]["latency_roofline"]}
+                if head["roofline"]["kernel"] == "auction" else {})),
+            per_kernel=head["per_kernel"],
             auction=head["auction"], e2e=head["e2e"],
             gpu_launches=head["gpu_launches"] + sum(r["gpu_launches"] for r in extra.values()),
             clocks=head["clocks"], device_error=head["device_error"], wall_s=head["wall_s"])

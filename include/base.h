@@ -147,6 +147,20 @@ typedef enum {
 } base_test_hook;
 int base_test_inject(int hook, long long value);
 
+/*
+ * Latency floors for the auction's latency roofline (no counterpart in the
+ * paper: a measurement aid).  One cooperative grid of the auction's shape
+ * writes to out (4 doubles of DEVICE memory) the nanoseconds of
+ *   [0] one grid barrier of the auction's kind over all SMs,
+ *   [1] one block barrier of 512 threads,
+ *   [2] one dependent load that hits L2,
+ *   [3] one dependent shared-memory load.
+ * ws: at least base_probe_workspace_size() bytes.  Read out after
+ * synchronising the stream.
+ */
+size_t base_probe_workspace_size(void);
+int base_measure_latency(double* out, void* ws, size_t ws_bytes, cudaStream_t stream);
+
 /* Library version string (static). */
 const char* base_version(void);
 

@@ -37,3 +37,20 @@ def test_rounds_by_kind_groups_traced_rounds():
     assert k["2-8 bidders"]["rounds"] == 2 and k["2-8 bidders"]["us_total"] == 5.0
     assert k["1 bidder"] == dict(rounds=2, us_total=2.5, us_median=1.25)
     assert "9-128 bidders" not in k
+
+
+def test_latency_roofline_model():
+    sys.path.insert(0, ROOT)
+    import bench
+    fl = dict(grid_barrier_ns=1000.0, block_barrier_ns=50.0, l2_load_ns=400.0, smem_load_ns=30.0)
+    # T = 8192, E = 16: a phase start, a 300-bidder grid round, a 20-bidder
+    # one-CTA round and two one-bidder rounds
+    u = [8192, 300, 20, 1, 1]
+    r = bench.latency_roofline(u, 8192, 16, auction_ms=0.01, fl=fl, hbm_gbs=6500.0)
+    q_ns = 4.0 * 8192 * 16 / 6500.0
+    expect = max(2800.0, q_ns) + 2800.0 + 500.0 + 400.0 + 400.0
+    assert abs(r["floor_ms"] - expect / 1e6) < 1e-12
+    assert abs(r["frac"] - expect / 1e6 / 0.01) < 1e-9
+    # with E = 64 the one-CTA limit is 32 bidders: 40 bidders run grid-wide
+    r2 = bench.latency_roofline([40], 8192, 64, auction_ms=1.0, fl=fl, hbm_gbs=6500.0)
+    assert abs(r2["floor_ms"] - 2800.0 / 1e6) < 1e-12
