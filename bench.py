@@ -45,10 +45,12 @@ UNIT = "tokens/s"
 # named workload at its full size (the component's kernels summed); a
 # component whose kernels changed after their capture has no entry.
 NCU_TRAFFIC = {
-    ("scores", "layer_fwd"): 16837632,
-    ("ffn", "layer_fwd"): 151049984 + 39332864 + 222304000 + 11714816,
+    ("scores", "layer_fwd"): 16840448 + 768,
+    ("auction", "layer_fwd"): 801792,
     # slice histogram + slice rank + row gather; the rows' writes stay in L2
-    ("permute", "layer_fwd"): 36608 + 588032 + 16819968,
+    ("permute", "layer_fwd"): 36096 + 588032 + 16815872,
+    # tile prefix + GEMM1 (h1 written, partly kept in L2) + GEMM2
+    ("ffn", "layer_fwd"): 4864 + 151050496 + 35908096 + 222283008 + 6628096,
     ("combine", "layer_fwd"): 16815616,
 }
 
