@@ -25,7 +25,7 @@ __all__ = [
     "base_layer_bwd", "base_test_inject", "BASE_TEST_WAIT_LIMIT_NS",
     "base_workspace_size_blend", "base_layer_fwd_blend", "base_expert_stack",
     "base_sanitize_scores", "BASE_ROUTE_SANITIZE", "base_workspace_size_fig9", "base_assign_fig9",
-    "base_probe_workspace_size", "base_measure_latency",
+    "base_probe_workspace_size", "base_measure_latency", "base_scores_greedy",
     "BASE_TEST_AUCTION_ABSENT_CTA", "BASE_TEST_GEMM_DROP_FIRST_LOAD", "EXPORTED",
 ]
 
@@ -44,7 +44,7 @@ EXPORTED = (
     "base_permute", "base_permute_noalloc", "base_expert_ffn", "base_combine", "base_layer_fwd",
     "base_layer_bwd", "base_test_inject", "base_workspace_size_blend", "base_layer_fwd_blend",
     "base_expert_stack", "base_sanitize_scores", "base_workspace_size_fig9", "base_assign_fig9",
-    "base_probe_workspace_size", "base_measure_latency",
+    "base_probe_workspace_size", "base_measure_latency", "base_scores_greedy",
 )
 
 
@@ -83,6 +83,7 @@ _SIGS = {
     "base_test_inject": (_i, [_i, ctypes.c_longlong]),
     "base_workspace_size_blend": (_sz, [_i, _i, _i, _i]),
     "base_sanitize_scores": (_i, [_vp, _vp, _i, _i, _vp, _sz, _vp]),
+    "base_scores_greedy": (_i, [_vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp]),
     "base_workspace_size_fig9": (_sz, [_i, _i]),
     "base_probe_workspace_size": (_sz, []),
     "base_measure_latency": (_i, [_vp, _vp, _sz, _vp]),
@@ -178,6 +179,14 @@ def base_scores(h, w, s=None, q=None, stream=None):
     E = w.shape[0]
     _check("base_scores", lib().base_scores(_ptr(h), _ptr(w), _dtype_code(h), T, D, E, _ptr(s),
                                             _ptr(q), _stream(stream)))
+
+
+def base_scores_greedy(h, w, s, q, assign, counts=None, stream=None):
+    T, D = h.shape
+    E = w.shape[0]
+    _check("base_scores_greedy", lib().base_scores_greedy(
+        _ptr(h), _ptr(w), _dtype_code(h), T, D, E, _ptr(s), _ptr(q), _ptr(assign), _ptr(counts),
+        _stream(stream)))
 
 
 def base_sanitize_scores(s, q, ws, stream=None):

@@ -10,7 +10,7 @@ namespace base {
 int launch_scores_f32(const float* h, const float* w, int T, int D, int E, float* s, int32_t* q,
                       cudaStream_t stream);
 int launch_scores_bf16(const void* h, const void* w, int T, int D, int E, float* s, int32_t* q,
-                       cudaStream_t stream);
+                       cudaStream_t stream, int32_t* assign = nullptr, int32_t* counts = nullptr);
 int launch_greedy(const int32_t* q, int T, int E, int32_t* assign, int32_t* counts,
                   cudaStream_t stream);
 size_t auction_workspace_bytes(int T, int E);
@@ -131,6 +131,23 @@ int base_scores(const void* h, const void* w, int dtype, int T, int D, int E, fl
     if (dtype != BASE_BF16) return BASE_ERR_INVALID_ARG;
     if (D % 8 != 0 || !aligned(h, 16) || !aligned(w, 16)) return BASE_ERR_INVALID_ARG;
     return launch_scores_bf16(h, w, T, D, E, s, q, stream);
+}
+
+int base_scores_greedy(const void* h, const void* w, int dtype, int T, int D, int E, float* s,
+                       int32_t* q, int32_t* assign, int32_t* counts, cudaStream_t stream) {
+    if (!h || !w || !q || !assign || !shapes_ok(T, E) || D < 1) return BASE_ERR_INVALID_ARG;
+    if ((s && !aligned(s, 16)) || !aligned(q, 16) || !aligned(assign, 4) ||
+        (counts && !aligned(counts, 4)))
+        return BASE_ERR_INVALID_ARG;
+    if (dtype == BASE_BF16 && E <= 256) {
+        if (D % 8 != 0 || !aligned(h, 16) || !aligned(w, 16)) return BASE_ERR_INVALID_ARG;
+        if (counts && cudaMemsetAsync(counts, 0, sizeof(int32_t) * (size_t)E, stream) != cudaSuccess)
+            return BASE_ERR_CUDA;
+        return launch_scores_bf16(h, w, T, D, E, s, q, stream, assign, counts);
+    }
+    const int st = base_scores(h, w, dtype, T, D, E, s, q, stream);
+    if (st != BASE_OK) return st;
+    return base_assign_greedy(q, T, E, assign, counts, stream);
 }
 
 int base_sanitize_scores(float* s, int32_t* q, int T, int E, void* ws, size_t ws_bytes,
@@ -261,18 +278,26 @@ int base_layer_fwd(const void* h, const void* w, const void* W1, const void* W2,
         return BASE_ERR_INVALID_ARG;
     }
     if (ws_bytes < base_workspace_size(T, E, D, 0)) return BASE_ERR_WORKSPACE;
-    int st = base_scores(h, w, BASE_BF16, T, D, E, sv->s, sv->q, stream);
-    if (st != BASE_OK) return st;
-    if (sanitize) {
-        st = base_sanitize_scores(sv->s, sv->q, T, E, ws, ws_bytes, stream);
+    int st;
+    if (routing == BASE_ROUTE_GREEDY && !sanitize) {
+        // test-time routing: the argmax comes out of the score GEMM's epilogue
+        st = base_scores_greedy(h, w, BASE_BF16, T, D, E, sv->s, sv->q, sv->assign, nullptr,
+                                stream);
+        if (st != BASE_OK) return st;
+    } else {
+        st = base_scores(h, w, BASE_BF16, T, D, E, sv->s, sv->q, stream);
+        if (st != BASE_OK) return st;
+        if (sanitize) {
+            st = base_sanitize_scores(sv->s, sv->q, T, E, ws, ws_bytes, stream);
+            if (st != BASE_OK) return st;
+        }
+        if (routing == BASE_ROUTE_BALANCED)
+            st = base_assign_balanced(sv->q, T, E, sv->assign, sv->price, sv->stats, ws, ws_bytes,
+                                      stream);
+        else
+            st = base_assign_greedy(sv->q, T, E, sv->assign, nullptr, stream);
         if (st != BASE_OK) return st;
     }
-    if (routing == BASE_ROUTE_BALANCED)
-        st = base_assign_balanced(sv->q, T, E, sv->assign, sv->price, sv->stats, ws, ws_bytes,
-                                  stream);
-    else
-        st = base_assign_greedy(sv->q, T, E, sv->assign, nullptr, stream);
-    if (st != BASE_OK) return st;
     st = base_permute(h, sv->assign, T, D, E, sv->perm, sv->inv, sv->offsets, sv->x_perm, sv->s,
                       sv->gate, ws, ws_bytes, stream);
     if (st != BASE_OK) return st;
@@ -330,18 +355,26 @@ int base_layer_fwd_blend(const void* h, const void* w, const void* W1, const voi
         if (!aligned(p, 16)) return BASE_ERR_INVALID_ARG;
     if (!aligned(ws, 256)) return BASE_ERR_INVALID_ARG;
     if (ws_bytes < base_workspace_size_blend(T, E, D, F)) return BASE_ERR_WORKSPACE;
-    int st = base_scores(h, w, BASE_BF16, T, D, E, sv->s, sv->q, stream);
-    if (st != BASE_OK) return st;
-    if (sanitize) {
-        st = base_sanitize_scores(sv->s, sv->q, T, E, ws, ws_bytes, stream);
+    int st;
+    if (routing == BASE_ROUTE_GREEDY && !sanitize) {
+        // test-time routing: the argmax comes out of the score GEMM's epilogue
+        st = base_scores_greedy(h, w, BASE_BF16, T, D, E, sv->s, sv->q, sv->assign, nullptr,
+                                stream);
+        if (st != BASE_OK) return st;
+    } else {
+        st = base_scores(h, w, BASE_BF16, T, D, E, sv->s, sv->q, stream);
+        if (st != BASE_OK) return st;
+        if (sanitize) {
+            st = base_sanitize_scores(sv->s, sv->q, T, E, ws, ws_bytes, stream);
+            if (st != BASE_OK) return st;
+        }
+        if (routing == BASE_ROUTE_BALANCED)
+            st = base_assign_balanced(sv->q, T, E, sv->assign, sv->price, sv->stats, ws, ws_bytes,
+                                      stream);
+        else
+            st = base_assign_greedy(sv->q, T, E, sv->assign, nullptr, stream);
         if (st != BASE_OK) return st;
     }
-    if (routing == BASE_ROUTE_BALANCED)
-        st = base_assign_balanced(sv->q, T, E, sv->assign, sv->price, sv->stats, ws, ws_bytes,
-                                  stream);
-    else
-        st = base_assign_greedy(sv->q, T, E, sv->assign, nullptr, stream);
-    if (st != BASE_OK) return st;
     st = base_permute(h, sv->assign, T, D, E, sv->perm, sv->inv, sv->offsets, sv->x_perm, sv->s,
                       sv->gate, ws, ws_bytes, stream);
     if (st != BASE_OK) return st;

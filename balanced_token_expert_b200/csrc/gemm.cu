@@ -75,6 +75,8 @@ struct Args {
     int kgroup;                  // 1: groups split K (weight gradients), M and N fixed
     int m_tiles;                 // K-grouped mode: tiles along M per group
     int mix;                     // EPI_GATE: 0 eq. 1, 1 residual only, 2 residual then blend
+    int32_t* out_assign;         // EPI_SCORES, one N tile: greedy argmax of q per row (nullable)
+    int32_t* out_counts;         // with out_assign: tokens per expert, added to (zeroed by the host)
     int staged;                  // set by the launcher: output tensor maps are valid
     unsigned long long wait_ns;  // set by the launcher: limit of every bounded wait
     int drop_first_load;         // set by the launcher: test hook (one-CTA kernels only)
@@ -393,8 +395,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t* tempty = tfull + 2;
     uint64_t* done = tempty + 2;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+    // EPI_SCORES with greedy routing: the CTA's tokens per expert (after the 256
+    // bytes of barriers)
+    int32_t* s_ghist = reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(full) + 256);
+    constexpr bool kGreedy = EPI == EPI_SCORES;
+    const bool greedy = kGreedy && args.out_assign != nullptr;
 
     const int warp = warp_id(), lane = lane_id();
+    if (greedy)
+        for (int e = threadIdx.x; e < args.N; e += blockDim.x) s_ghist[e] = 0;
     const uint32_t rank = (CG == 2) ? tc::cluster_ctarank() : 0u;
     const bool leader = rank == 0;
     const int unit = (CG == 2) ? (int)(blockIdx.x / 2) : (int)blockIdx.x;
@@ -633,6 +642,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
             } else {
+                int gbest = INT32_MIN, garg = -1;  // greedy: this half's best q, lowest column
 #pragma unroll 1
                 for (int c0 = c_begin; c0 < c_end; c0 += 16) {
                     uint32_t v[16];
@@ -643,6 +653,46 @@ __global__ void __launch_bounds__(kThreads, 1)
                         for (int i = 0; i < 16; ++i) v[i] = 0u;
                     }
                     if (valid && ti.n0 + c0 < args.N) epilogue16<EPI>(args, ti, row, ti.n0 + c0, v);
+                    if constexpr (kGreedy) {
+                        if (greedy && half == 0) {
+#pragma unroll
+                            for (int i = 0; i < 16; ++i) {
+                                const int col = ti.n0 + c0 + i;
+                                const int32_t qv = quantize_score(__uint_as_float(v[i]));
+                                if (col < args.N && qv > gbest) {
+                                    gbest = qv;
+                                    garg = col;
+                                }
+                            }
+                        }
+                    }
+                }
+                if constexpr (kGreedy) {
+                    if (greedy && half == 0) {
+                        // the first half also scans the other half's columns (the
+                        // same TMEM lanes; nobody frees this accumulator before every
+                        // epilogue warp has arrived), lowest column first on ties
+#pragma unroll 1
+                        for (int c0 = c_end; c0 < 16 * kChunks; c0 += 16) {
+                            uint32_t v[16];
+                            tc::tmem_ld16(tbase + c0, v);
+                            tc::tmem_wait_ld();
+#pragma unroll
+                            for (int i = 0; i < 16; ++i) {
+                                const int col = ti.n0 + c0 + i;
+                                const int32_t qv = quantize_score(
+                                    ti.kblocks == 0 ? 0.f : __uint_as_float(v[i]));
+                                if (col < args.N && qv > gbest) {
+                                    gbest = qv;
+                                    garg = col;
+                                }
+                            }
+                        }
+                        if (valid && garg >= 0) {
+                            args.out_assign[row] = garg;
+                            atomicAdd(&s_ghist[garg], 1);
+                        }
+                    }
                 }
             }
             tc::tc_fence_before();
@@ -656,6 +706,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         // the staged stores have landed before the CTA (and its shared memory) goes
         if (kStaged && lane == 0) tc::bulk_wait_all();
+        if constexpr (kGreedy) {
+            if (greedy) {  // the CTA's tokens per expert, one atomic per expert
+                asm volatile("bar.sync 12, %0;" ::"r"(32 * kEpiWarps) : "memory");
+                for (int e = threadIdx.x - 128; e < args.N && args.out_counts; e += 32 * kEpiWarps)
+                    if (s_ghist[e]) atomicAdd(args.out_counts + e, s_ghist[e]);
+            }
+        }
     }
     tc::tc_fence_before();
     __syncthreads();
@@ -778,7 +835,8 @@ static int launch(const void* A, uint64_t a_rows, uint64_t a_cols, const void* B
         }
     }
     constexpr size_t smem = STAGES * (size_t)(BM * BK * 2 + (BN / CG) * BK * 2) +
-                            (kStagedEpi<EPI> ? kEpiWarps * kStageSlots * kStageBuf : 0) + 1024 + 256;
+                            (kStagedEpi<EPI> ? kEpiWarps * kStageSlots * kStageBuf : 0) + 1024 + 256 +
+                            (EPI == EPI_SCORES ? 4 * 256 : 0);
     static_assert(smem <= 227 * 1024, "shared memory");
     static_assert(!B_MN || (BN / CG) % 64 == 0, "MN-major B needs 64-wide blocks");
     auto kern = gemm_kernel<BN, STAGES, EPI, A_MN, B_MN, CG>;
@@ -814,9 +872,13 @@ static int launch(const void* A, uint64_t a_rows, uint64_t a_cols, const void* B
 
 // s = h w^T (+ q) for bf16 h (T x D) and w (E x D) on the tensor cores
 int launch_scores_bf16(const void* h, const void* w, int T, int D, int E, float* s, int32_t* q,
-                       cudaStream_t stream) {
+                       cudaStream_t stream, int32_t* assign, int32_t* counts) {
     using namespace gemm;
     Args a{};
+    if (assign && E <= 256) {  // greedy routing in the epilogue: every row in one N tile
+        a.out_assign = assign;
+        a.out_counts = counts;
+    }
     a.M = T;
     a.N = E;
     a.K = D;

@@ -263,7 +263,13 @@ def measure(args, wl, steps, warmup, rank, world, local_rank):
     greedy_assign = torch.empty(T, dtype=torch.int32, device="cuda")
     greedy_counts = torch.empty(E, dtype=torch.int32, device="cuda")
 
-    comps = [("scores", lambda: B.base_scores(h, w, sv["s"], sv["q"]), 1)]
+    fused_greedy = not F and inp.bump_tokens is None and E <= 256
+    if fused_greedy:
+        # the routing step's test-time argmax comes out of the score GEMM's epilogue
+        comps = [("scores_greedy", lambda: B.base_scores_greedy(h, w, sv["s"], sv["q"],
+                                                                 greedy_assign, greedy_counts), 1)]
+    else:
+        comps = [("scores", lambda: B.base_scores(h, w, sv["s"], sv["q"]), 1)]
     if q_bump is not None:
         comps.append(("bump", lambda: sv["q"][:, 0].index_add_(
             0, q_bump[0], torch.full_like(q_bump[0], q_bump[1], dtype=torch.int32)), 0))
@@ -271,7 +277,7 @@ def measure(args, wl, steps, warmup, rank, world, local_rank):
     # kernel; the permute: two sort launches and the row gather)
     comps.append(("auction", lambda: B.base_assign_balanced(sv["q"], sv["assign"], sv["price"],
                                                              sv["stats"], ws), 1))
-    if not F:
+    if not F and not fused_greedy:
         comps.append(("greedy", lambda: B.base_assign_greedy(sv["q"], greedy_assign,
                                                               greedy_counts), 1))
     comps.append(("permute", lambda: B.base_permute(h, sv["assign"], E, sv["perm"], sv["inv"],
@@ -500,6 +506,7 @@ def measure(args, wl, steps, warmup, rank, world, local_rank):
     bids = st["bids"]
     alg = dict(  # algorithmic work per launch (bytes or flops)
         scores=("hbm", 2 * T * D + 2 * E * D + 8 * T * E),
+        scores_greedy=("hbm", 2 * T * D + 2 * E * D + 8 * T * E + 4 * T + 4 * E),
         auction=("hbm", 4 * E * bids + 4 * T + 8 * E),
         permute=("hbm", 4 * T * D + 12 * T + 8 * T),
         ffn=("tensor", 4 * T * D * F),

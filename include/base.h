@@ -183,6 +183,18 @@ int base_scores(const void* h, const void* w, int dtype, int T, int D, int E,
                 float* s, int32_t* q, cudaStream_t stream);
 
 /*
+ * a1 + a2 + a3 in one pass: the scores and their quantisation as base_scores,
+ * and the greedy test-time routing of base_assign_greedy on that q (argmax,
+ * lowest e on ties), computed in the score GEMM's epilogue when the inputs
+ * are bf16 and E <= 256 (every row's experts in one tile); otherwise
+ * base_scores then base_assign_greedy.  q, assign: required; s, counts:
+ * nullable (counts: E int32, tokens per expert).  base_layer_fwd's greedy
+ * routing goes through this call.
+ */
+int base_scores_greedy(const void* h, const void* w, int dtype, int T, int D, int E, float* s,
+                       int32_t* q, int32_t* assign, int32_t* counts, cudaStream_t stream);
+
+/*
  * Non-finite scores (the wikillm.com summary's "Paper vs code", Non-finite
  * scores: the released code replaces NaN and infinite affinities with the
  * minimum finite score before solving).  Every entry of s (T*E fp32) that is

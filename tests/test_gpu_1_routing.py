@@ -419,3 +419,44 @@ def test_fig9_workloads_bit_exact(orc, name):
     ao, po, so = orc.fig9_auction(q)
     assert st == so and np.array_equal(a, ao) and np.array_equal(p, po)
     assert st["objective"] <= orc.auction(q)[2]["objective"]  # never above the optimum
+
+
+# ------------------------------------------------------------------ scores + greedy in one pass
+@pytest.mark.parametrize("T,E,D", [(1000, 16, 200), (4099, 32, 256), (777, 100, 64),
+                                   (8192, 128, 512), (640, 256, 128), (513, 300, 64),
+                                   (2048, 2, 64)])
+def test_scores_greedy_fused(orc, T, E, D):
+    wl = synth.WORKLOADS["layer_fwd"].scaled(T=T, E=E, D=D, F=0)
+    inp = synth.make_inputs(wl, 11)
+    s = torch.empty(T, E, device="cuda")
+    q = torch.empty(T, E, dtype=torch.int32, device="cuda")
+    a = torch.full((T,), -1, dtype=torch.int32, device="cuda")
+    c = torch.full((E,), 123, dtype=torch.int32, device="cuda")
+    B.base_scores_greedy(dev(inp.h), dev(inp.w), s, q, a, c)
+    torch.cuda.synchronize()
+    sg, qg = to_np(s), to_np(q)
+    ok, worst = close_scores(sg, orc.scores(inp.h, inp.w), 1e-5)
+    assert ok, worst
+    assert np.array_equal(qg, np.rint(sg * np.float32(65536)).astype(np.int32))
+    ao, co = orc.greedy(qg)
+    assert np.array_equal(to_np(a), ao)
+    assert np.array_equal(to_np(c), co)
+
+
+def test_scores_greedy_fused_with_ties(orc):
+    # equal scores in a row: the lowest expert wins, across the two column
+    # halves of the epilogue too (E = 64: columns 0-31 and 32-63)
+    T, E, D = 512, 64, 64
+    h = torch.zeros(T, D)
+    h[:, 0] = 1.0
+    w = torch.zeros(E, D)
+    w[[5, 40, 63], 0] = 0.5   # three experts tie on every row
+    h[::2, 1] = 1.0
+    w[40, 1] = 0.25            # even rows prefer expert 40
+    hb, wb = h.to(torch.bfloat16), w.to(torch.bfloat16)
+    q = torch.empty(T, E, dtype=torch.int32, device="cuda")
+    a = torch.empty(T, dtype=torch.int32, device="cuda")
+    B.base_scores_greedy(dev(hb), dev(wb), None, q, a)
+    torch.cuda.synchronize()
+    assert np.array_equal(to_np(a), orc.greedy(to_np(q))[0])
+    assert set(to_np(a)[1::2].tolist()) == {5} and set(to_np(a)[::2].tolist()) == {40}
