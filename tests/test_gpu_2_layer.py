@@ -327,3 +327,31 @@ def test_blend_variant_small(orc, S, routing, act):
 def test_blend_variant_full_layer_fwd_workload_sampled(orc):
     # the benchmarked shape (T=8192, E=16, D=1024, F=4096) with two sublayers
     _blend_check(orc, synth.WORKLOADS["layer_fwd"], 2, 0, "balanced", experts=[0, 9])
+
+
+# ------------------------------------------------------------------ expert parallelism, one worker
+def test_expert_parallel_layer_one_worker(orc):
+    # one worker holds every expert: the shuffle, the layer on the shuffled
+    # tokens with the library's kernels and the undoing of the shuffle
+    from balanced_token_expert_b200 import expert_parallel as ep
+    wl = synth.WORKLOADS["layer_fwd"].scaled(T=2048, E=8, D=256, F=512)
+    inp = synth.make_inputs(wl, 9)
+    T, E, D, F = wl.T, wl.E, wl.D, wl.F
+    plan = ep.EPPlan(T=T, E=E, G=1)
+    be = ep.CudaBackend(T, E, D, F)
+    y, shuffled, assign = ep.ep_layer_fwd(dev(inp.h), dev(inp.w), dev(inp.W1), dev(inp.W2),
+                                          B.BASE_RELU, plan, seed=77, backend=be,
+                                          return_route=True)
+    torch.cuda.synchronize()
+    perm = ep.shuffle_permutation(T, 77)
+    assert torch.equal(shuffled.cpu(), inp.h[perm])
+    q = torch.empty(T, E, dtype=torch.int32, device="cuda")
+    B.base_scores(shuffled, dev(inp.w), None, q)
+    torch.cuda.synchronize()
+    a_g = to_np(assign)
+    assert np.array_equal(a_g, orc.auction(to_np(q))[0])
+    ysh = orc.layer_forward(inp.h[perm], inp.w, inp.W1, inp.W2, "relu", a_g)["out"]
+    expect = np.empty_like(ysh)
+    expect[perm.numpy()] = ysh
+    ok, worst = close_rel_rms(to_np(y), expect, FWD_TOL)
+    assert ok, worst
