@@ -40,6 +40,7 @@ constexpr int BK = 64;
 // warp 0: TMA, warp 1: MMA, warps 2-3: idle, warps 4..: epilogue, two per
 // TMEM lane quadrant (warp w reads lanes 32 (w % 4) ..), each half the columns
 constexpr int kEpiWarps = 8;
+constexpr int kTsSmem = 384;  // groups + 1 whose tile prefix a grouped GEMM computes itself
 constexpr int kThreads = 128 + 32 * kEpiWarps;
 
 enum Epi : int {
@@ -88,7 +89,10 @@ struct TileInfo {
 };
 
 // bm: rows of A per tile (128, or 256 for a CTA pair)
-__device__ __forceinline__ TileInfo decode_tile(const Args& a, int tile, int bn, int bm = BM) {
+// ts: the groups' tile prefix (shared memory when the kernel computed it,
+// else a.tile_start); read with plain loads
+__device__ __forceinline__ TileInfo decode_tile(const Args& a, int tile, int bn, int bm,
+                                                const int32_t* ts_) {
     TileInfo ti;
     ti.k0 = 0;
     ti.kblocks = (a.K + BK - 1) / BK;
@@ -122,11 +126,11 @@ __device__ __forceinline__ TileInfo decode_tile(const Args& a, int tile, int bn,
     int lo = 0, hi = a.groups;  // find the last g with tile_start[g] * n_tiles <= tile
     while (hi - lo > 1) {
         const int mid = (lo + hi) >> 1;
-        if (__ldg(a.tile_start + mid) * a.n_tiles <= tile) lo = mid; else hi = mid;
+        if (ts_[mid] * a.n_tiles <= tile) lo = mid; else hi = mid;
     }
     const int g = lo;
-    const int ts = __ldg(a.tile_start + g);
-    const int mtg = __ldg(a.tile_start + g + 1) - ts;
+    const int ts = ts_[g];
+    const int mtg = ts_[g + 1] - ts;
     const int local = tile - ts * a.n_tiles;
     const int nt = local / mtg, m = local % mtg;
     const int r0 = __ldg(a.offsets + g);
@@ -369,7 +373,9 @@ __device__ __forceinline__ void stage16(uint8_t* buf, int lane, int c, const flo
 // of B (the TMA completions of both land on the leader's barrier), the leader
 // issues the MMAs, each CTA's TMEM holds its 128 rows x BN accumulator and its
 // epilogue writes them.
-template <int BN, int STAGES, int EPI, bool A_MN, bool B_MN, int CG = 1>
+// SLOTS: staging buffers of 32 x 128 bytes per epilogue warp (one frees shared
+// memory for a sixth pipeline stage)
+template <int BN, int STAGES, int EPI, bool A_MN, bool B_MN, int CG = 1, int SLOTS = kStageSlots>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const __grid_constant__ CUtensorMap tmO0, const __grid_constant__ CUtensorMap tmO1,
@@ -385,7 +391,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~uintptr_t(1023));
     constexpr bool kStaged = kStagedEpi<EPI>;
-    constexpr uint32_t STAGE_AREA = kStaged ? kEpiWarps * kStageSlots * kStageBuf : 0;
+    constexpr uint32_t STAGE_AREA = kStaged ? kEpiWarps * SLOTS * kStageBuf : 0;
     uint8_t* sA = smem;
     uint8_t* sB = smem + STAGES * A_BYTES;
     uint8_t* sOut = smem + STAGES * (A_BYTES + B_BYTES);  // 1024-byte aligned
@@ -433,14 +439,42 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc::tma_prefetch_desc(&tmA);
         tc::tma_prefetch_desc(&tmB);
     }
+    // launched behind another kernel (programmatic dependent launch): the set-up
+    // above overlapped its tail; nothing it writes is read before this point
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    // grouped tiles: the groups' tile prefix (a group of r rows has ceil(r / BMP)
+    // row tiles) computed here by the idle warp 3 when the launcher passed none
+    int32_t* s_ts = reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(full) + 256);
+    const bool ts_smem = args.offsets != nullptr && !args.kgroup && args.tile_start == nullptr;
+    if (ts_smem && warp == 3) {
+        int run = 0;
+        for (int base = 0; base <= args.groups; base += 32) {
+            const int g = base + lane;
+            const int v = g < args.groups
+                              ? (__ldg(args.offsets + g + 1) - __ldg(args.offsets + g) + BMP - 1) / BMP
+                              : 0;
+            int incl = v;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const int o = __shfl_up_sync(0xffffffffu, incl, off);
+                if (lane >= off) incl += o;
+            }
+            if (g <= args.groups) s_ts[g] = run + incl - v;
+            run += __shfl_sync(0xffffffffu, incl, 31);
+        }
+    }
     tc::tc_fence_before();
     __syncthreads();
+    // every CTA of this grid is resident (one per SM, persistent): the next
+    // kernel may start its own set-up on SMs as they free up
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    const int32_t* tsp = ts_smem ? s_ts : args.tile_start;
     if constexpr (CG == 2) tc::cluster_sync_all();  // both CTAs' barriers and TMEM are ready
     tc::tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
 
     const int mtiles = args.kgroup ? args.m_tiles * args.groups
-                       : args.offsets ? __ldg(args.tile_start + args.groups)
+                       : args.offsets ? tsp[args.groups]
                                       : (args.M + BMP - 1) / BMP;
     const int total = mtiles * args.n_tiles;
 
@@ -453,7 +487,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool issued[STAGES];
         for (int s = 0; s < STAGES; ++s) issued[s] = false;
         for (int tile = unit; tile < total && ok; tile += nunits) {
-            const TileInfo ti = decode_tile(args, tile, BN, BMP);
+            const TileInfo ti = decode_tile(args, tile, BN, BMP, tsp);
             const int a_row = ti.a_row + BM * (int)rank;
             for (int kb = 0; kb < ti.kblocks; ++kb) {
                 if (!tc::mbar_wait(&empty[stage], phase ^ 1, 3001, args.wait_ns)) {
@@ -542,7 +576,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc::tc_fence_after();
             const uint32_t d_tmem = tmem_base + acc * BN;
             // only K-grouped tiles differ in depth (and need the tile's group)
-            const int kblocks = args.kgroup ? decode_tile(args, tile, BN, BMP).kblocks
+            const int kblocks = args.kgroup ? decode_tile(args, tile, BN, BMP, tsp).kblocks
                                             : (args.K + BK - 1) / BK;
             for (int kb = 0; kb < kblocks; ++kb) {
                 if (!tc::mbar_wait(&full[stage], phase, 3003, args.wait_ns)) {
@@ -596,7 +630,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t tempty_leader0 = (CG == 2) ? tc::map_to_rank(&tempty[0], 0) : 0u;
         const uint32_t tempty_leader1 = (CG == 2) ? tc::map_to_rank(&tempty[1], 0) : 0u;
         for (int tile = unit; tile < total; tile += nunits) {
-            const TileInfo ti = decode_tile(args, tile, BN, BMP);
+            const TileInfo ti = decode_tile(args, tile, BN, BMP, tsp);
             const bool ok = tc::mbar_wait(&tfull[acc], acc_phase, 3005, 2 * args.wait_ns);
             if (!__all_sync(0xffffffffu, ok)) break;  // the whole warp leaves together
             tc::tc_fence_after();
@@ -615,9 +649,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int gc = c_begin; gc < c_end && ti.n0 + gc < args.N; gc += GC) {
 #pragma unroll 1
                     for (int pass = 0; pass < npass; ++pass) {
-                        uint8_t* buf = sOut + ((warp - 4) * kStageSlots + slot) * kStageBuf;
+                        uint8_t* buf = sOut + ((warp - 4) * SLOTS + slot) * kStageBuf;
                         // the store issued from this slot two pieces ago has read it
-                        if (lane == 0) tc::bulk_wait_read<kStageSlots - 1>();
+                        if (lane == 0) tc::bulk_wait_read<SLOTS - 1>();
                         __syncwarp();
 #pragma unroll 1
                         for (int c = 0; c < GC; c += 16) {
@@ -638,7 +672,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                             tc::tma_store_2d(pass ? &tmO1 : &tmO0, buf, ti.n0 + gc, orow);
                             tc::bulk_commit();
                         }
-                        slot = (slot + 1) % kStageSlots;
+                        slot = (slot + 1) % SLOTS;
                     }
                 }
             } else {
@@ -806,7 +840,8 @@ static bool make_tmap_out(CUtensorMap* m, const void* base, uint64_t rows, uint6
 // A: a_rows x a_cols row-major (K-major: a_cols = K; MN-major: a_rows = K)
 // B: b_rows x b_cols row-major (likewise).  CG = 2 launches clusters of two
 // CTAs (pair tiles of 256 rows).
-template <int BN, int STAGES, int EPI, bool A_MN = false, bool B_MN = false, int CG = 1>
+template <int BN, int STAGES, int EPI, bool A_MN = false, bool B_MN = false, int CG = 1,
+          int SLOTS = kStageSlots>
 static int launch(const void* A, uint64_t a_rows, uint64_t a_cols, const void* B, uint64_t b_rows,
                   uint64_t b_cols, const Args& args, int max_tiles, cudaStream_t stream) {
     CUtensorMap ta, tb, to0, to1;
@@ -835,37 +870,39 @@ static int launch(const void* A, uint64_t a_rows, uint64_t a_cols, const void* B
         }
     }
     constexpr size_t smem = STAGES * (size_t)(BM * BK * 2 + (BN / CG) * BK * 2) +
-                            (kStagedEpi<EPI> ? kEpiWarps * kStageSlots * kStageBuf : 0) + 1024 + 256 +
-                            (EPI == EPI_SCORES ? 4 * 256 : 0);
+                            (kStagedEpi<EPI> ? kEpiWarps * SLOTS * kStageBuf : 0) + 1024 + 256 +
+                            (EPI == EPI_SCORES ? 4 * 256 : 4 * kTsSmem);
     static_assert(smem <= 227 * 1024, "shared memory");
     static_assert(!B_MN || (BN / CG) % 64 == 0, "MN-major B needs 64-wide blocks");
-    auto kern = gemm_kernel<BN, STAGES, EPI, A_MN, B_MN, CG>;
+    auto kern = gemm_kernel<BN, STAGES, EPI, A_MN, B_MN, CG, SLOTS>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
         cudaSuccess)
         return BASE_ERR_CUDA;
-    if constexpr (CG == 1) {
-        const int grid = std::min(num_sms(), std::max(1, max_tiles));
-        kern<<<grid, kThreads, smem, stream>>>(ta, tb, to0, to1, a);
-        BASE_RETURN_IF_LAUNCH_FAILED();
-        return BASE_OK;
-    } else {
-        const int grid = 2 * std::min(num_sms() / 2, std::max(1, max_tiles));
-        cudaLaunchConfig_t cfg = {};
-        cudaLaunchAttribute attr[1];
-        attr[0].id = cudaLaunchAttributeClusterDimension;
-        attr[0].val.clusterDim.x = 2;
-        attr[0].val.clusterDim.y = 1;
-        attr[0].val.clusterDim.z = 1;
-        cfg.gridDim = dim3(grid, 1, 1);
-        cfg.blockDim = dim3(kThreads, 1, 1);
-        cfg.dynamicSmemBytes = smem;
-        cfg.stream = stream;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
-        if (cudaLaunchKernelEx(&cfg, kern, ta, tb, to0, to1, a) != cudaSuccess)
-            return BASE_ERR_CUDA;
-        return BASE_OK;
+    // programmatic dependent launch: the set-up (barriers, TMEM, descriptors)
+    // overlaps the previous kernel's tail; the kernel waits for it before reading
+    const int grid = (CG == 1) ? std::min(num_sms(), std::max(1, max_tiles))
+                               : 2 * std::min(num_sms() / 2, std::max(1, max_tiles));
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[2];
+    int nattr = 0;
+    attr[nattr].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[nattr].val.programmaticStreamSerializationAllowed = 1;
+    ++nattr;
+    if constexpr (CG == 2) {
+        attr[nattr].id = cudaLaunchAttributeClusterDimension;
+        attr[nattr].val.clusterDim.x = 2;
+        attr[nattr].val.clusterDim.y = 1;
+        attr[nattr].val.clusterDim.z = 1;
+        ++nattr;
     }
+    cfg.gridDim = dim3(grid, 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = nattr;
+    if (cudaLaunchKernelEx(&cfg, kern, ta, tb, to0, to1, a) != cudaSuccess) return BASE_ERR_CUDA;
+    return BASE_OK;
 }
 
 }  // namespace gemm
@@ -913,8 +950,13 @@ int launch_expert_ffn(const void* x_perm, const int32_t* offsets, int T, int D, 
     using namespace gemm;
     constexpr int BMP = 2 * BM;  // CTA-pair tiles
     int32_t* tile_start = static_cast<int32_t*>(ws);
-    tile_prefix_kernel<<<1, 1024, 0, stream>>>(offsets, E, BMP, tile_start);
-    BASE_RETURN_IF_LAUNCH_FAILED();
+    // the grouped GEMMs compute the tile prefix themselves when it fits their shared memory
+    if (E + 1 > kTsSmem) {
+        tile_prefix_kernel<<<1, 1024, 0, stream>>>(offsets, E, BMP, tile_start);
+        BASE_RETURN_IF_LAUNCH_FAILED();
+    } else {
+        tile_start = nullptr;
+    }
     const int max_mt = (T + BMP - 1) / BMP + E;
     Args g1{};
     g1.M = T;
@@ -929,8 +971,13 @@ int launch_expert_ffn(const void* x_perm, const int32_t* offsets, int T, int D, 
     g1.act = act;
     g1.out0 = static_cast<__nv_bfloat16*>(h1);
     g1.out1 = static_cast<__nv_bfloat16*>(a1);
-    int st = launch<256, 5, EPI_ACT, false, false, 2>(x_perm, T, D, W1, (uint64_t)E * F, D, g1,
-                                                      max_mt * g1.n_tiles, stream);
+    // few tiles per SM pair (T <= 16384): a sixth pipeline stage, one staging
+    // slot per epilogue warp (measured faster there, slower on larger problems)
+    const bool six = T <= 16384;
+    int st = six ? launch<256, 6, EPI_ACT, false, false, 2, 1>(x_perm, T, D, W1, (uint64_t)E * F, D,
+                                                               g1, max_mt * g1.n_tiles, stream)
+                 : launch<256, 5, EPI_ACT, false, false, 2>(x_perm, T, D, W1, (uint64_t)E * F, D,
+                                                            g1, max_mt * g1.n_tiles, stream);
     if (st != BASE_OK) return st;
     Args g2{};
     g2.M = T;
@@ -946,8 +993,10 @@ int launch_expert_ffn(const void* x_perm, const int32_t* offsets, int T, int D, 
     g2.out1 = static_cast<__nv_bfloat16*>(f);
     g2.gate = gate;
     g2.side = static_cast<const __nv_bfloat16*>(x_perm);
-    return launch<256, 5, EPI_GATE, false, false, 2>(h1, T, F, W2, (uint64_t)E * D, F, g2,
-                                                     max_mt * g2.n_tiles, stream);
+    return six ? launch<256, 6, EPI_GATE, false, false, 2, 1>(h1, T, F, W2, (uint64_t)E * D, F, g2,
+                                                              max_mt * g2.n_tiles, stream)
+               : launch<256, 5, EPI_GATE, false, false, 2>(h1, T, F, W2, (uint64_t)E * D, F, g2,
+                                                           max_mt * g2.n_tiles, stream);
 }
 
 int launch_layer_norm_rows(const void* x, const int32_t* offsets, int T, int D, int E,
@@ -974,8 +1023,13 @@ int launch_expert_stack(const void* x_perm, const int32_t* offsets, int T, int D
     int32_t* tile_start = reinterpret_cast<int32_t*>(w8);
     void* ln = w8 + ffn_workspace_bytes(E);
     void* xb = w8 + ffn_workspace_bytes(E) + align_up((size_t)T * D * 2, 256);
-    tile_prefix_kernel<<<1, 1024, 0, stream>>>(offsets, E, BMP, tile_start);
-    BASE_RETURN_IF_LAUNCH_FAILED();
+    // the grouped GEMMs compute the tile prefix themselves when it fits their shared memory
+    if (E + 1 > kTsSmem) {
+        tile_prefix_kernel<<<1, 1024, 0, stream>>>(offsets, E, BMP, tile_start);
+        BASE_RETURN_IF_LAUNCH_FAILED();
+    } else {
+        tile_start = nullptr;
+    }
     const int max_mt = (T + BMP - 1) / BMP + E;
     const __nv_bfloat16* W1b = static_cast<const __nv_bfloat16*>(W1);
     const __nv_bfloat16* W2b = static_cast<const __nv_bfloat16*>(W2);
@@ -1039,8 +1093,13 @@ int launch_bwd_gemms(const void* dF, const void* /*unused*/, void* dA1, const vo
                      int E, int F, void* dh, float* dW1, float* dW2, cudaStream_t stream) {
     using namespace gemm;
     constexpr int BMP = 2 * BM;
-    tile_prefix_kernel<<<1, 1024, 0, stream>>>(offsets, E, BMP, tile_start);
-    BASE_RETURN_IF_LAUNCH_FAILED();
+    // the grouped GEMMs compute the tile prefix themselves when it fits their shared memory
+    if (E + 1 > kTsSmem) {
+        tile_prefix_kernel<<<1, 1024, 0, stream>>>(offsets, E, BMP, tile_start);
+        BASE_RETURN_IF_LAUNCH_FAILED();
+    } else {
+        tile_start = nullptr;
+    }
     const int max_mt = (T + BMP - 1) / BMP + E;
     // dH1 = dF W2_e (B = W2_e stored D x F: MN-major), dA1 = dH1 * act'(A1)
     Args g{};

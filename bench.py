@@ -286,12 +286,12 @@ def measure(args, wl, steps, warmup, rank, world, local_rank):
     if F and wl.S:
         comps.append(("stack", lambda: B.base_expert_stack(sv["x_perm"], sv["offsets"], W1, W2,
                                                            gam, bet, act, sv["gate"], sv["y_perm"],
-                                                           sv["h1"], ws), 1 + 3 * wl.S))
+                                                           sv["h1"], ws), 3 * wl.S))
         comps.append(("combine", lambda: B.base_combine(sv["y_perm"], sv["perm"], out), 1))
     elif F:
         comps.append(("ffn", lambda: B.base_expert_ffn(sv["x_perm"], sv["offsets"], W1, W2, act,
                                                        sv["gate"], sv["y_perm"], sv["h1"],
-                                                       sv.get("a1"), sv.get("f"), ws), 3))
+                                                       sv.get("a1"), sv.get("f"), ws), 2))
         comps.append(("combine", lambda: B.base_combine(sv["y_perm"], sv["perm"], out), 1))
     if wl.backward:
         dout = inp.dout.cuda()
@@ -300,7 +300,7 @@ def measure(args, wl, steps, warmup, rank, world, local_rank):
         dW1 = torch.empty(E, F, D, device="cuda")
         dW2 = torch.empty(E, D, F, device="cuda")
         comps.append(("backward", lambda: B.base_layer_bwd(h, w, W1, W2, act, sv, dout, dh, dw,
-                                                           dW1, dW2, ws), 9))
+                                                           dW1, dW2, ws), 8))
     names = [n for n, _, _ in comps if n != "bump"]
 
     def step(ev):
