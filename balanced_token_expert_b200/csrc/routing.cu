@@ -115,6 +115,8 @@ __global__ void __launch_bounds__(1024) slice_hist_kernel(const int32_t* __restr
                                                           int32_t* __restrict__ cnt) {
     extern __shared__ int32_t sh[];  // [E]
     for (int e = threadIdx.x; e < E; e += blockDim.x) sh[e] = 0;
+    pdl_wait();
+    pdl_trigger();
     __syncthreads();
     const int t0 = blockIdx.x * slice, t1 = min(T, t0 + slice);
     for (int t = t0 + threadIdx.x; t < t1; t += blockDim.x) {
@@ -137,6 +139,8 @@ __global__ void __launch_bounds__(1024) slice_rank_kernel(const int32_t* __restr
     int32_t* wc = sm;                  // [32][E]: per-warp counts, then running slots
     int32_t* s_warp = sm + 32 * E;     // [32] block-scan partials
     const int w = warp_id(), lane = lane_id();
+    pdl_wait();
+    pdl_trigger();
     const unsigned lt = (1u << lane) - 1;
     const int b = blockIdx.x;
     const int s0 = b * slice, s1 = min(T, s0 + slice);
@@ -249,6 +253,8 @@ __global__ void __launch_bounds__(256) move_rows_kernel(const uint4* __restrict_
     constexpr int kUnroll = 4;
     const int lane = lane_id();
     const long long nwarps = (long long)gridDim.x * (blockDim.x / kWarp);
+    pdl_wait();
+    pdl_trigger();
     for (long long r = blockIdx.x * (long long)(blockDim.x / kWarp) + warp_id(); r < T; r += nwarps) {
         const int m = __ldg(idx + r);
         if ((unsigned)m >= (unsigned)T) {  // not a row: recorded, the row skipped
@@ -316,15 +322,16 @@ int launch_sort_by_expert(const int32_t* assign, int T, int E, int32_t* perm, in
     const int slice = std::min(kSliceMax, std::max(512, (T + 127) / 128));
     const int P = (T + slice - 1) / slice;
     int32_t* cnt = static_cast<int32_t*>(ws);  // [P][E]
-    slice_hist_kernel<<<P, 1024, sizeof(int32_t) * E, stream>>>(assign, T, E, slice, cnt);
-    BASE_RETURN_IF_LAUNCH_FAILED();
+    if (launch_pdl(slice_hist_kernel, dim3(P), dim3(1024), sizeof(int32_t) * E, stream, assign, T,
+                   E, slice, cnt) != cudaSuccess)
+        return BASE_ERR_CUDA;
     const size_t sm = sizeof(int32_t) * (32 * (size_t)E + 32);
     if (cudaFuncSetAttribute(slice_rank_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)sm) != cudaSuccess)
         return BASE_ERR_CUDA;
-    slice_rank_kernel<<<P, 1024, sm, stream>>>(assign, T, E, slice, cnt, perm, inv, offsets, s,
-                                               gate);
-    BASE_RETURN_IF_LAUNCH_FAILED();
+    if (launch_pdl(slice_rank_kernel, dim3(P), dim3(1024), sm, stream, assign, T, E, slice,
+                   (const int32_t*)cnt, perm, inv, offsets, s, gate) != cudaSuccess)
+        return BASE_ERR_CUDA;
     return BASE_OK;
 }
 
@@ -335,13 +342,14 @@ int launch_move_rows(const void* src, const int32_t* idx, int T, int D, void* ds
     long long blocks = ((long long)T + threads / kWarp - 1) / (threads / kWarp);
     if (blocks > num_sms() * 64) blocks = num_sms() * 64;
     if (blocks < 1) blocks = 1;
-    if (scatter)
-        routing::move_rows_kernel<true><<<(int)blocks, threads, 0, stream>>>(
-            static_cast<const uint4*>(src), idx, T, vec, static_cast<uint4*>(dst));
-    else
-        routing::move_rows_kernel<false><<<(int)blocks, threads, 0, stream>>>(
-            static_cast<const uint4*>(src), idx, T, vec, static_cast<uint4*>(dst));
-    BASE_RETURN_IF_LAUNCH_FAILED();
+    const cudaError_t err =
+        scatter ? launch_pdl(routing::move_rows_kernel<true>, dim3((int)blocks), dim3(threads), 0,
+                             stream, static_cast<const uint4*>(src), idx, T, vec,
+                             static_cast<uint4*>(dst))
+                : launch_pdl(routing::move_rows_kernel<false>, dim3((int)blocks), dim3(threads), 0,
+                             stream, static_cast<const uint4*>(src), idx, T, vec,
+                             static_cast<uint4*>(dst));
+    if (err != cudaSuccess) return BASE_ERR_CUDA;
     return BASE_OK;
 }
 
