@@ -57,9 +57,21 @@ struct Key {
 };
 
 // "worse" order: smaller bid first, then larger token first; an expert keeps
-// the C best keys.
+// the C best keys.  Written without short-circuit operators, and the key
+// selects below with conditional moves per field: a short-circuit compare
+// becomes divergent branches, which cost a single warp ~5x more per compare
+// (measured: a 32-key warp sort 2.9 k -> 0.9 k cycles).
 __device__ __forceinline__ bool worse(const Key& a, const Key& b) {
-    return a.bid < b.bid || (a.bid == b.bid && a.tok > b.tok);
+    return (a.bid < b.bid) | ((a.bid == b.bid) & (a.tok > b.tok));
+}
+
+// c ? a : b, field by field
+__device__ __forceinline__ Key sel_key(bool c, const Key& a, const Key& b) {
+    Key r;
+    r.bid = c ? a.bid : b.bid;
+    r.tok = c ? a.tok : b.tok;
+    r.slot = c ? a.slot : b.slot;
+    return r;
 }
 
 __device__ __forceinline__ Key pad_key() { return Key{INT64_MAX, -1, -2}; }
@@ -84,7 +96,7 @@ __device__ __forceinline__ Key warp_min_key(Key k) {
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) {
         const Key o = shfl_xor_key(k, off);
-        if (worse(o, k)) k = o;
+        k = sel_key(worse(o, k), o, k);
     }
     return k;
 }
@@ -93,7 +105,7 @@ __device__ __forceinline__ Key warp_max_key(Key k) {
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) {
         const Key o = shfl_xor_key(k, off);
-        if (worse(k, o)) k = o;
+        k = sel_key(worse(k, o), o, k);
     }
     return k;
 }
@@ -108,7 +120,7 @@ __device__ __forceinline__ Key warp_sort(Key x) {
             const Key o = shfl_xor_key(x, j);
             const bool up = (lane & k) == 0;
             const bool lower = (lane & j) == 0;
-            if (lower == up ? worse(o, x) : worse(x, o)) x = o;
+            x = sel_key(lower == up ? worse(o, x) : worse(x, o), o, x);
         }
     }
     return x;
@@ -121,7 +133,7 @@ __device__ __forceinline__ Key warp_bitonic_merge(Key x) {
     for (int j = 16; j > 0; j >>= 1) {
         const Key o = shfl_xor_key(x, j);
         const bool lower = (lane & j) == 0;
-        if (lower ? worse(o, x) : worse(x, o)) x = o;
+        x = sel_key(lower ? worse(o, x) : worse(x, o), o, x);
     }
     return x;
 }
@@ -130,13 +142,9 @@ __device__ __forceinline__ Key warp_bitonic_merge(Key x) {
 // (element i of the result is lo in lane i for i < 32, hi in lane i-32 after)
 __device__ __forceinline__ void warp_merge64(Key a, Key b, Key& lo, Key& hi) {
     const Key br = shfl_key(b, 31 - lane_id());
-    if (worse(br, a)) {
-        lo = br;
-        hi = a;
-    } else {
-        lo = a;
-        hi = br;
-    }
+    const bool sw = worse(br, a);
+    lo = sel_key(sw, br, a);
+    hi = sel_key(sw, a, br);
     lo = warp_bitonic_merge(lo);
     hi = warp_bitonic_merge(hi);
 }
@@ -462,7 +470,7 @@ __device__ Key kth_worst_cta(const Team<kThreads>& tm, Visit visit, int k, int t
         // are <= prefix
         const int sh = nbits - pbits;
         visit([&](const Key& x) {
-            if (shr64((uint64_t)(x.bid - lo), sh) <= prefix && worse(best, x)) best = x;
+            best = sel_key((shr64((uint64_t)(x.bid - lo), sh) <= prefix) & worse(best, x), x, best);
         });
     } else {
         // every bid digit fixed: B* = lo + prefix; `need` of the candidates
@@ -494,7 +502,7 @@ __device__ Key kth_worst_cta(const Team<kThreads>& tm, Visit visit, int k, int t
         visit([&](const Key& x) {
             bool rej = x.bid < bstar;
             if (x.bid == bstar) rej = (uint32_t)shr64(tm_max - (uint32_t)x.tok, sh) <= tprefix;
-            if (rej && worse(best, x)) best = x;
+            best = sel_key(rej & worse(best, x), x, best);
         });
     }
     // the best over the CTA: warp maxima, then every warp reduces them
@@ -554,7 +562,7 @@ __device__ Key kth_worst_v(const Team<TEAM>& tm, Visit visit, int k, int tmax) {
         Key best = Key{INT64_MIN, INT32_MAX, -2};
         const int sh = nbits - pbits;
         visit([&](const Key& x) {
-            if (shr64((uint64_t)(x.bid - lo), sh) <= prefix && worse(best, x)) best = x;
+            best = sel_key((shr64((uint64_t)(x.bid - lo), sh) <= prefix) & worse(best, x), x, best);
         });
         return tm.max_key(best);
     }
@@ -589,7 +597,7 @@ __device__ Key kth_worst_v(const Team<TEAM>& tm, Visit visit, int k, int tmax) {
     visit([&](const Key& x) {
         bool rej = x.bid < bstar;
         if (x.bid == bstar) rej = (uint32_t)shr64(tm_max - (uint32_t)x.tok, sh) <= tprefix;
-        if (rej && worse(best, x)) best = x;
+        best = sel_key(rej & worse(best, x), x, best);
     });
     return tm.max_key(best);
 }
@@ -606,7 +614,7 @@ __device__ Key kth_worst(const Team<TEAM>& tm, const Cands& cd, int k, int tmax)
             Key best = pad_key();
             for (int c = tid; c < m; c += TEAM) {
                 const Key x = cd.get(c);
-                if (worse(last, x) && worse(x, best)) best = x;
+                best = sel_key(worse(last, x) & worse(x, best), x, best);
             }
             last = warp_min_key(best);
         }
@@ -800,13 +808,10 @@ __device__ __forceinline__ void group_bid(const int32_t* row, const int64_t* pri
     e1 = INT32_MAX;
     for (int e = gl; e < E; e += G) {
         const int64_t v = (int64_t)row[e] * scale - price[e];
-        if (v > v1) {
-            v2 = v1;
-            v1 = v;
-            e1 = e;
-        } else if (v > v2) {
-            v2 = v;
-        }
+        const bool g1 = v > v1, g2 = v > v2;
+        v2 = g1 ? v1 : (g2 ? v : v2);
+        v1 = g1 ? v : v1;
+        e1 = g1 ? e : e1;
     }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) {
@@ -814,13 +819,10 @@ __device__ __forceinline__ void group_bid(const int32_t* row, const int64_t* pri
         const int64_t ov1 = __shfl_xor_sync(0xffffffffu, v1, off);
         const int64_t ov2 = __shfl_xor_sync(0xffffffffu, v2, off);
         const int oe1 = __shfl_xor_sync(0xffffffffu, e1, off);
-        if (ov1 > v1 || (ov1 == v1 && oe1 < e1)) {
-            v2 = max(v1, ov2);
-            v1 = ov1;
-            e1 = oe1;
-        } else {
-            v2 = max(v2, ov1);
-        }
+        const bool tk = (ov1 > v1) | ((ov1 == v1) & (oe1 < e1));
+        v2 = tk ? max(v1, ov2) : max(v2, ov1);
+        v1 = tk ? ov1 : v1;
+        e1 = tk ? oe1 : e1;
     }
 }
 
@@ -847,13 +849,10 @@ __device__ __forceinline__ void group_bid_multi(const int32_t* __restrict__ q, c
         for (int u = 0; u < NT; ++u) {
             if (!valid[u]) continue;
             const int64_t v = (int64_t)qv[u] * scale - pe;
-            if (v > v1[u]) {
-                v2[u] = v1[u];
-                v1[u] = v;
-                e1[u] = e;
-            } else if (v > v2[u]) {
-                v2[u] = v;
-            }
+            const bool g1 = v > v1[u], g2 = v > v2[u];
+            v2[u] = g1 ? v1[u] : (g2 ? v : v2[u]);
+            v1[u] = g1 ? v : v1[u];
+            e1[u] = g1 ? e : e1[u];
         }
     }
 #pragma unroll
@@ -864,13 +863,10 @@ __device__ __forceinline__ void group_bid_multi(const int32_t* __restrict__ q, c
             const int64_t ov1 = __shfl_xor_sync(0xffffffffu, v1[u], off);
             const int64_t ov2 = __shfl_xor_sync(0xffffffffu, v2[u], off);
             const int oe1 = __shfl_xor_sync(0xffffffffu, e1[u], off);
-            if (ov1 > v1[u] || (ov1 == v1[u] && oe1 < e1[u])) {
-                v2[u] = max(v1[u], ov2);
-                v1[u] = ov1;
-                e1[u] = oe1;
-            } else {
-                v2[u] = max(v2[u], ov1);
-            }
+            const bool tk = (ov1 > v1[u]) | ((ov1 == v1[u]) & (oe1 < e1[u]));
+            v2[u] = tk ? max(v1[u], ov2) : max(v2[u], ov1);
+            v1[u] = tk ? ov1 : v1[u];
+            e1[u] = tk ? oe1 : e1[u];
         }
     }
 }
@@ -897,13 +893,10 @@ __device__ __forceinline__ void group_bid2(const int32_t* r0, const int32_t* r1,
         for (int u = 0; u < 2; ++u) {
             if (!ok[u]) continue;
             const int64_t v = (int64_t)qa[u] * scale - pe;
-            if (v > v1[u]) {
-                v2[u] = v1[u];
-                v1[u] = v;
-                e1[u] = e;
-            } else if (v > v2[u]) {
-                v2[u] = v;
-            }
+            const bool g1 = v > v1[u], g2 = v > v2[u];
+            v2[u] = g1 ? v1[u] : (g2 ? v : v2[u]);
+            v1[u] = g1 ? v : v1[u];
+            e1[u] = g1 ? e : e1[u];
         }
     }
 #pragma unroll
@@ -914,13 +907,10 @@ __device__ __forceinline__ void group_bid2(const int32_t* r0, const int32_t* r1,
             const int64_t ov1 = __shfl_xor_sync(0xffffffffu, v1[u], off);
             const int64_t ov2 = __shfl_xor_sync(0xffffffffu, v2[u], off);
             const int oe1 = __shfl_xor_sync(0xffffffffu, e1[u], off);
-            if (ov1 > v1[u] || (ov1 == v1[u] && oe1 < e1[u])) {
-                v2[u] = max(v1[u], ov2);
-                v1[u] = ov1;
-                e1[u] = oe1;
-            } else {
-                v2[u] = max(v2[u], ov1);
-            }
+            const bool tk = (ov1 > v1[u]) | ((ov1 == v1[u]) & (oe1 < e1[u]));
+            v2[u] = tk ? max(v1[u], ov2) : max(v2[u], ov1);
+            v1[u] = tk ? ov1 : v1[u];
+            e1[u] = tk ? oe1 : e1[u];
         }
     }
 }
@@ -1028,7 +1018,8 @@ __device__ int resolve_general(const Team<TEAM>& tm, const Params& p, int e, con
         Key x = pad_key();
         if (j < n) {
             x = cd.get(h + j);
-            if (worse(kth, x)) acc = true; else rej = true;
+            acc = worse(kth, x);
+            rej = !acc;
         }
         int nrej = 0;
         const int rr = tm.rank(rej, nrej);
@@ -1138,7 +1129,7 @@ __device__ void finish_cta_resolve(const Team<kThreads>& tm, const Params& p, co
     // accepted new bids (above the k-th worst) take the freed slots
     for (int c = h + tid; c < m; c += kThreads) {
         const Key x = sk[c];
-        if (k == 0 || worse(Xk, x)) {
+        if ((k == 0) | worse(Xk, x)) {
             const int slot = fslot[atomicAdd(&tm.cnt[45], 1)];
             hb[slot] = x.bid;
             ht[slot] = x.tok;
@@ -1263,8 +1254,9 @@ __device__ __forceinline__ int rank_sorted(const int64_t* b, const int32_t* t, i
     int lo = 0, hi = n;
     while (lo < hi) {
         const int mid = (lo + hi) >> 1;
-        if (worse(Key{b[mid], t[mid], 0}, x)) lo = mid + 1;
-        else hi = mid;
+        const bool w = worse(Key{b[mid], t[mid], 0}, x);
+        lo = w ? mid + 1 : lo;
+        hi = w ? hi : mid;
     }
     return lo;
 }
@@ -1274,8 +1266,9 @@ __device__ __forceinline__ int rank_keys(const Key* a, int n, const Key& x) {
     int lo = 0, hi = n;
     while (lo < hi) {
         const int mid = (lo + hi) >> 1;
-        if (worse(a[mid], x)) lo = mid + 1;
-        else hi = mid;
+        const bool w = worse(a[mid], x);
+        lo = w ? mid + 1 : lo;
+        hi = w ? hi : mid;
     }
     return lo;
 }
@@ -1324,8 +1317,9 @@ __device__ Key* cta_sort_keys_fast(Key* a, Key* tmp, int n) {
                 int l = lo[u], h = hi[u];
                 while (l < h) {
                     const int mid = (l + h) >> 1;
-                    if (worse(src[mid], x[u])) l = mid + 1;
-                    else h = mid;
+                    const bool w = worse(src[mid], x[u]);
+                    l = w ? mid + 1 : l;
+                    h = w ? h : mid;
                 }
                 if (ok[u]) dst[pos[u] + l] = x[u];  // pos + l in [0, n)
             }
@@ -1474,12 +1468,9 @@ __device__ int build_fringe_warp(const Team<32>& tm, const int64_t* hb, const in
 #pragma unroll 4
         for (int i = lane; i < C; i += 32) {
             const Key x = Key{hb[i], ht[i], i};
-            if (worse(x, a)) {
-                b = a;
-                a = x;
-            } else if (worse(x, b)) {
-                b = x;
-            }
+            const bool wa = worse(x, a), wb = worse(x, b);
+            b = sel_key(wa, a, sel_key(wb, x, b));
+            a = sel_key(wa, x, a);
         }
         warp_merge64(warp_sort(a), warp_sort(b), lo, hi);
         const Key theta = shfl_key(lo, 31);
@@ -1488,7 +1479,7 @@ __device__ int build_fringe_warp(const Team<32>& tm, const int64_t* hb, const in
         for (int i0 = 0; i0 < C; i0 += 32) {  // uniform trip count: the ballot needs all lanes
             const int i = i0 + lane;
             const Key x = i < C ? Key{hb[i], ht[i], i} : pad_key();
-            const bool in = i < C && !worse(theta, x);
+            const bool in = (i < C) & !worse(theta, x);
             const unsigned m = __ballot_sync(0xffffffffu, in);
             const int pos = got + __popc(m & ((1u << lane) - 1));
             if (in && pos < 64) stage[pos] = x;
@@ -1533,8 +1524,8 @@ __device__ __forceinline__ int fringe_take_one(Key* fr, int& fs, int h, int64_t 
     const Key fi = lane < fs ? fr[lane] : pad_key();
     const Key fn = lane + 1 < fs ? fr[lane + 1] : pad_key();
     const Key b = Key{bid, tok, f0.slot};
-    const bool ins = fs == h || !worse(fl, b);
-    const int pos = __popc(__ballot_sync(0xffffffffu, lane + 1 < fs && worse(fn, b)));
+    const bool ins = (fs == h) | !worse(fl, b);
+    const int pos = __popc(__ballot_sync(0xffffffffu, (lane + 1 < fs) & worse(fn, b)));
     Key out = lane < pos ? fn : (lane == pos ? b : fi);
     if (!ins) out = fn;
     const int nfs = ins ? fs : fs - 1;
@@ -1611,8 +1602,8 @@ __device__ bool resolve_warp(const Params& p, Key* fr, int& fs, int& h, const in
         const Key fn = lane + 1 < fs ? fr[lane + 1] : pad_key();
         const Key f0 = shfl_key(fi, 0);
         const Key b = Key{b0.bid, b0.tok, f0.slot};
-        const bool ins = complete || !worse(shfl_key(fi, fs - 1), b);
-        const int pos = __popc(__ballot_sync(0xffffffffu, lane + 1 < fs && worse(fn, b)));
+        const bool ins = complete | !worse(shfl_key(fi, fs - 1), b);
+        const int pos = __popc(__ballot_sync(0xffffffffu, (lane + 1 < fs) & worse(fn, b)));
         Key out = lane < pos ? fn : (lane == pos ? b : fi);
         if (!ins) out = fn;
         const int nfs = ins ? fs : fs - 1;
@@ -1638,7 +1629,7 @@ __device__ bool resolve_warp(const Params& p, Key* fr, int& fs, int& h, const in
     if (n == 1) {
         // one new key: insert it into the sorted fringe
         const Key b = Key{nb[0], nt[0], -1};
-        const int pos = __popc(__ballot_sync(0xffffffffu, lane < fs && worse(f, b)));
+        const int pos = __popc(__ballot_sync(0xffffffffu, (lane < fs) & worse(f, b)));
         const Key prev = shfl_key(f, (lane + 31) & 31);
         const Key top = shfl_key(f, 31);
         lo = lane < pos ? f : (lane == pos ? b : prev);
@@ -1680,8 +1671,8 @@ __device__ bool resolve_warp(const Params& p, Key* fr, int& fs, int& h, const in
         }
     }
     // the new fringe: survivors not above the threshold, in order, at most FK
-    const bool keep_lo = !rej && lo.slot != -2 && !worse(thr, lo);
-    const bool keep_hi = hi.slot != -2 && !worse(thr, hi);
+    const bool keep_lo = !rej & (lo.slot != -2) & !worse(thr, lo);
+    const bool keep_hi = (hi.slot != -2) & !worse(thr, hi);
     const unsigned kl = __ballot_sync(0xffffffffu, keep_lo);
     const unsigned kh = __ballot_sync(0xffffffffu, keep_hi);
     const int nl = __popc(kl);
@@ -1747,13 +1738,10 @@ __device__ __forceinline__ void chain_rounds(const Params& p, int t, int64_t eps
             const int e = lane + 32 * j;
             if (e < E) {
                 const int64_t v = (int64_t)rv[j] * scale - s_price[e];
-                if (v > v1) {
-                    v2 = v1;
-                    v1 = v;
-                    e1 = e;
-                } else if (v > v2) {
-                    v2 = v;
-                }
+                const bool g1 = v > v1, g2 = v > v2;
+                v2 = g1 ? v1 : (g2 ? v : v2);
+                v1 = g1 ? v : v1;
+                e1 = g1 ? e : e1;
             }
         }
 #pragma unroll
@@ -1761,13 +1749,10 @@ __device__ __forceinline__ void chain_rounds(const Params& p, int t, int64_t eps
             const int64_t ov1 = __shfl_xor_sync(0xffffffffu, v1, off);
             const int64_t ov2 = __shfl_xor_sync(0xffffffffu, v2, off);
             const int oe1 = __shfl_xor_sync(0xffffffffu, e1, off);
-            if (ov1 > v1 || (ov1 == v1 && oe1 < e1)) {
-                v2 = max(v1, ov2);
-                v1 = ov1;
-                e1 = oe1;
-            } else {
-                v2 = max(v2, ov1);
-            }
+            const bool tk = (ov1 > v1) | ((ov1 == v1) & (oe1 < e1));
+            v2 = tk ? max(v1, ov2) : max(v2, ov1);
+            v1 = tk ? ov1 : v1;
+            e1 = tk ? oe1 : e1;
         }
         const int e = e1;
         // bid = q[t][e] (T+1) - v2 + eps = price[e] + (v1 - v2) + eps
