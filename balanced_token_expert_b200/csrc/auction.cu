@@ -1448,16 +1448,21 @@ __device__ int build_fringe_radix(const Team<TEAM>& tm, const int64_t* hb, const
 }
 
 // Warp version: a sampled threshold first.  Each lane keeps the two worst
-// keys of its stripe; the 32nd worst of those 64 keys, theta, has at least 32
-// held keys at or below it, and usually not many more: they are collected
-// (at most 64, else the radix build runs) and sorted.  Two passes over the
-// held keys instead of one per radix digit.
+// keys of its stripe (the candidates); sorted, the 32 worst candidates are
+// lo and the 32nd of them, theta, has at least 32 held keys at or below it.
+// Those are lo plus the held keys at or below theta that are not
+// candidates (usually none): collected (at most 32, else the radix build
+// runs), sorted and merged into lo.  Both passes over the held keys issue
+// kLoads loads before they use one (the collect's shared-memory stores would
+// otherwise keep the next loads from starting: the held keys may be in shared
+// memory too).
+constexpr int kLoads = 8;
+
 __device__ int build_fringe_warp(const Team<32>& tm, const int64_t* hb, const int32_t* ht, int C,
                                  int FK, int tmax, Key* fr) {
     const int k = min(FK, C);
     if (k == 0) return 0;
     const int lane = lane_id();
-    Key* stage = reinterpret_cast<Key*>(tm.hist);  // 64 keys
     Key lo, hi;
     if (C <= 64) {
         Key a = lane < C ? Key{hb[lane], ht[lane], lane} : pad_key();
@@ -1465,32 +1470,53 @@ __device__ int build_fringe_warp(const Team<32>& tm, const int64_t* hb, const in
         warp_merge64(warp_sort(a), warp_sort(b), lo, hi);
     } else {
         Key a = pad_key(), b = pad_key();
-#pragma unroll 4
-        for (int i = lane; i < C; i += 32) {
-            const Key x = Key{hb[i], ht[i], i};
-            const bool wa = worse(x, a), wb = worse(x, b);
-            b = sel_key(wa, a, sel_key(wb, x, b));
-            a = sel_key(wa, x, a);
+        for (int i0 = 0; i0 < C; i0 += 32 * kLoads) {
+            Key x[kLoads];
+#pragma unroll
+            for (int u = 0; u < kLoads; ++u) {
+                const int i = i0 + 32 * u + lane;
+                x[u] = i < C ? Key{hb[i], ht[i], i} : pad_key();
+            }
+#pragma unroll
+            for (int u = 0; u < kLoads; ++u) {
+                const bool wa = worse(x[u], a), wb = worse(x[u], b);
+                b = sel_key(wa, a, sel_key(wb, x[u], b));
+                a = sel_key(wa, x[u], a);
+            }
         }
         warp_merge64(warp_sort(a), warp_sort(b), lo, hi);
         const Key theta = shfl_key(lo, 31);
+        Key* stage = reinterpret_cast<Key*>(tm.hist);  // 32 keys
+        const unsigned lt = (1u << lane) - 1;
         int got = 0;
-#pragma unroll 4
-        for (int i0 = 0; i0 < C; i0 += 32) {  // uniform trip count: the ballot needs all lanes
-            const int i = i0 + lane;
-            const Key x = i < C ? Key{hb[i], ht[i], i} : pad_key();
-            const bool in = (i < C) & !worse(theta, x);
-            const unsigned m = __ballot_sync(0xffffffffu, in);
-            const int pos = got + __popc(m & ((1u << lane) - 1));
-            if (in && pos < 64) stage[pos] = x;
-            got += __popc(m);
+        for (int i0 = 0; i0 < C; i0 += 32 * kLoads) {
+            Key x[kLoads];
+#pragma unroll
+            for (int u = 0; u < kLoads; ++u) {
+                const int i = i0 + 32 * u + lane;
+                x[u] = i < C ? Key{hb[i], ht[i], i} : pad_key();
+            }
+            unsigned m[kLoads];
+#pragma unroll
+            for (int u = 0; u < kLoads; ++u) {
+                const int i = i0 + 32 * u + lane;
+                m[u] = __ballot_sync(0xffffffffu, (i < C) & !worse(theta, x[u]) & (i != a.slot) &
+                                                      (i != b.slot));
+            }
+#pragma unroll
+            for (int u = 0; u < kLoads; ++u) {
+                const int pos = got + __popc(m[u] & lt);
+                if (((m[u] >> lane) & 1u) & (pos < 32)) stage[pos] = x[u];
+                got += __popc(m[u]);
+            }
         }
         __syncwarp();
-        if (got > 64) return build_fringe_radix<32>(tm, hb, ht, C, FK, tmax, fr);
-        const Key sa = lane < got ? stage[lane] : pad_key();
-        const Key sb = lane + 32 < got ? stage[lane + 32] : pad_key();
-        __syncwarp();
-        warp_merge64(warp_sort(sa), warp_sort(sb), lo, hi);
+        if (got > 32) return build_fringe_radix<32>(tm, hb, ht, C, FK, tmax, fr);
+        if (got > 0) {
+            const Key x = lane < got ? stage[lane] : pad_key();
+            __syncwarp();
+            warp_merge64(lo, warp_sort(x), lo, hi);
+        }
     }
     if (lane < k) fr[lane] = lo;
     __syncwarp();
