@@ -50,11 +50,14 @@ __host__ __device__ constexpr int narrow_max_for(int E) { return E <= 16 ? 256 :
 constexpr uint64_t kWaitNs = 20000000000ull;  // grid-barrier wait limit (20 s)
 
 // ---------------------------------------------------------------- keys
-struct Key {
+// 16-byte aligned (one 128-bit load or store); every Key array in shared or
+// global memory starts on a 16-byte boundary
+struct __align__(16) Key {
     int64_t bid;
     int32_t tok;
     int32_t slot;  // >= 0: held slot; -1: a new bid; -2: padding
 };
+static_assert(sizeof(Key) == 16, "Key is 16 bytes");
 
 // "worse" order: smaller bid first, then larger token first; an expert keeps
 // the C best keys.  Written without short-circuit operators, and the key
@@ -273,11 +276,10 @@ struct Team {
             int run = incl - sum, fd = -1, fb = 0, fc = 0;
 #pragma unroll
             for (int b = 0; b < 8; ++b) {
-                if (fd < 0 && run < need && run + c8[b] >= need) {
-                    fd = lane * 8 + b;
-                    fb = run;
-                    fc = c8[b];
-                }
+                const bool hit = (fd < 0) & (run < need) & (run + c8[b] >= need);
+                fd = hit ? lane * 8 + b : fd;
+                fb = hit ? run : fb;
+                fc = hit ? c8[b] : fc;
                 run += c8[b];
             }
             const unsigned m = __ballot_sync(0xffffffffu, fd >= 0);
@@ -303,7 +305,7 @@ struct Team {
         if (t < kHist)
             for (int w = 0; w < warp_id(); ++w) wbase += cnt[34 + w];
         const int excl = wbase + incl - c;
-        if (t < nbins && excl < need && excl + c >= need) {
+        if ((t < nbins) & (excl < need) & (excl + c >= need)) {
             cnt[42] = t;
             cnt[43] = excl;
             cnt[44] = c;
@@ -395,7 +397,7 @@ __device__ __forceinline__ void cta_find_digit(int32_t* hist, int nbins, int nee
     int run = incl - sum;
 #pragma unroll
     for (int q = 0; q < 8; ++q) {
-        if (run < need && run + c8[q] >= need) {
+        if ((run < need) & (run + c8[q] >= need)) {
             out[0] = lane * 8 + q;
             out[1] = run;
             out[2] = c8[q];
@@ -1530,9 +1532,20 @@ __device__ int build_fringe(const Team<TEAM>& tm, const int64_t* hb, const int32
     else return build_fringe_radix<TEAM>(tm, hb, ht, C, FK, tmax, fr);
 }
 
+// position of the r-th (from 0) set bit of m, 0 when m has at most r set
+// bits; five branch-free halving steps (a per-lane loop of r steps diverges)
 __device__ __forceinline__ int nth_set_lane(unsigned m, int r) {
-    for (int i = 0; i < r; ++i) m &= m - 1;
-    return m ? __ffs(m) - 1 : 0;
+    const bool found = __popc(m) > r;
+    int pos = 0;
+#pragma unroll
+    for (int w = 16; w >= 1; w >>= 1) {
+        const int c = __popc(m & ((1u << w) - 1));
+        const bool up = r >= c;  // the bit is in the upper half
+        r = up ? r - c : r;
+        m = up ? m >> w : m;
+        pos = up ? pos + w : pos;
+    }
+    return found ? pos : 0;
 }
 
 // One bid to a full expert whose fringe holds at least two keys (the usual
@@ -1667,9 +1680,9 @@ __device__ bool resolve_warp(const Params& p, Key* fr, int& fs, int& h, const in
         warp_merge64(f, x, lo, hi);
     }
     const bool rej = lane < k;  // the first k elements (k <= n < 32: all in lo)
-    const unsigned freed = __ballot_sync(0xffffffffu, rej && lo.slot >= 0);
+    const unsigned freed = __ballot_sync(0xffffffffu, rej & (lo.slot >= 0));
     const int nfreed = __popc(freed);
-    const unsigned acc_lo = __ballot_sync(0xffffffffu, !rej && lo.slot == -1);
+    const unsigned acc_lo = __ballot_sync(0xffffffffu, !rej & (lo.slot == -1));
     const unsigned acc_hi = __ballot_sync(0xffffffffu, hi.slot == -1);
     // the r-th accepted new key takes the r-th freed slot, then h + (r - nfreed)
     const int r_lo = __popc(acc_lo & lt);
@@ -2277,9 +2290,9 @@ __global__ void __launch_bounds__(kThreads, 1) auction_kernel(const __grid_const
                             const int i0 = base + sub, i1 = base + kWarps * tpw + sub;
                             const bool ok0 = i0 < U, ok1 = i1 < U;
                             const int t0 = ok0 ? list[i0] : 0, t1 = ok1 ? list[i1] : 0;
-                            const int32_t* r0 = (staged && i0 < RC) ? rows_cur + (size_t)i0 * E
+                            const int32_t* r0 = (staged & (i0 < RC)) ? rows_cur + (size_t)i0 * E
                                                                     : p.q + (size_t)t0 * E;
-                            const int32_t* r1 = (staged && i1 < RC) ? rows_cur + (size_t)i1 * E
+                            const int32_t* r1 = (staged & (i1 < RC)) ? rows_cur + (size_t)i1 * E
                                                                     : p.q + (size_t)t1 * E;
                             int64_t v1[2], v2[2];
                             int e1[2];
@@ -2294,7 +2307,7 @@ __global__ void __launch_bounds__(kThreads, 1) auction_kernel(const __grid_const
                         if (warp * tpw < U) {
                             const bool valid = i < U;
                             const int t = valid ? list[i] : 0;
-                            const int32_t* row = (staged && i < RC) ? rows_cur + (size_t)i * E
+                            const int32_t* row = (staged & (i < RC)) ? rows_cur + (size_t)i * E
                                                                     : p.q + (size_t)t * E;
                             int64_t v1, v2;
                             int e1;
