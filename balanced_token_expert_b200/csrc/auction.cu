@@ -841,7 +841,7 @@ __device__ __forceinline__ void group_bid_multi(const int32_t* __restrict__ q, c
         v2[u] = INT64_MIN;
         e1[u] = INT32_MAX;
     }
-#pragma unroll 2
+#pragma unroll 4
     for (int e = gl; e < E; e += G) {
         int32_t qv[NT];
 #pragma unroll
@@ -1334,6 +1334,76 @@ __device__ Key* cta_sort_keys_fast(Key* a, Key* tmp, int n) {
     return src;
 }
 
+// The same for distinct 64-bit keys in ascending order (a packed key's order
+// is the "worse" order: see resolve_sorted): half the shared-memory traffic
+// of a 16-byte key per search step and one compare.
+__device__ __forceinline__ uint64_t warp_sort_u64(uint64_t x) {
+    const int lane = lane_id();
+#pragma unroll
+    for (int k = 2; k <= 32; k <<= 1) {
+#pragma unroll
+        for (int j = k >> 1; j > 0; j >>= 1) {
+            const uint64_t o = __shfl_xor_sync(0xffffffffu, x, j);
+            const bool up = (lane & k) == 0;
+            const bool lower = (lane & j) == 0;
+            x = ((lower == up) ? (o < x) : (x < o)) ? o : x;
+        }
+    }
+    return x;
+}
+
+__device__ uint64_t* cta_sort_u64(uint64_t* a, uint64_t* tmp, int n) {
+    const int lane = lane_id(), warp = warp_id();
+    for (int r0 = warp * 32; r0 < n; r0 += kWarps * 32) {
+        uint64_t x = r0 + lane < n ? a[r0 + lane] : ~0ull;
+        x = warp_sort_u64(x);
+        if (r0 + lane < n) a[r0 + lane] = x;
+    }
+    __syncthreads();
+    uint64_t* src = a;
+    uint64_t* dst = tmp;
+    for (int R = 32; R < n; R <<= 1) {
+        for (int i0 = threadIdx.x; i0 < n; i0 += 2 * kThreads) {
+            uint64_t x[2];
+            int pos[2], lo[2], hi[2];
+            bool ok[2];
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const int i = i0 + u * kThreads;
+                ok[u] = i < n;
+                pos[u] = 0;
+                lo[u] = hi[u] = 0;
+                x[u] = 0;
+                if (ok[u]) {
+                    x[u] = src[i];
+                    const int run = i / R;
+                    const int pair0 = (run & ~1) * R;
+                    const int ps = (run ^ 1) * R;  // the partner run
+                    lo[u] = min(ps, n);
+                    hi[u] = min(ps + R, n);
+                    pos[u] = pair0 + (i - run * R) - lo[u];
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                int l = lo[u], h = hi[u];
+                while (l < h) {
+                    const int mid = (l + h) >> 1;
+                    const bool w = src[mid] < x[u];
+                    l = w ? mid + 1 : l;
+                    h = w ? h : mid;
+                }
+                if (ok[u]) dst[pos[u] + l] = x[u];  // pos + l in [0, n)
+            }
+        }
+        __syncthreads();
+        uint64_t* t = src;
+        src = dst;
+        dst = t;
+    }
+    return src;
+}
+
 // Keeps the C best of the sorted held set cur[0, h) and the n new bids
 // (nb, nt) of one expert.  The new held set (sorted) goes to nxt and to the
 // global hb / ht / fringe gfr; rejected tokens go to unext through ucnt.
@@ -1362,6 +1432,37 @@ __device__ int resolve_sorted(const Team<kThreads>& tm, const Params& p, SortedS
         ht[r] = x.tok;
         if (r < FK) gfr[r] = Key{x.bid, x.tok, r};
     };
+    if (n <= kSortedSmall && n <= nsc && h == 0) {
+        // an expert's first bids (every phase start): when the bid range
+        // leaves room for the token, each bid becomes one 64-bit key
+        // ((bid - lo) << tb | (T - 1 - tok)) whose ascending order is the
+        // "worse" order, and the sorted keys are the held set in order
+        int64_t lo = INT64_MAX, hi = INT64_MIN;
+        for (int i = tid; i < n; i += kThreads) {
+            lo = min(lo, nb[i]);
+            hi = max(hi, nb[i]);
+        }
+        tm.minmax_i64(lo, hi);
+        const int tb = max(1, bit_length_u64((uint64_t)(p.T - 1)));
+        if (bit_length_u64((uint64_t)(hi - lo)) + tb <= 64) {
+            uint64_t* pk = reinterpret_cast<uint64_t*>(sk);
+            const uint64_t tmax = (uint64_t)(p.T - 1);
+            const uint64_t tmask = (1ull << tb) - 1;  // tb <= 31
+            for (int i = tid; i < n; i += kThreads)
+                pk[i] = ((uint64_t)(nb[i] - lo) << tb) | (tmax - (uint64_t)(uint32_t)nt[i]);
+            __syncthreads();
+            const uint64_t* sp = cta_sort_u64(pk, reinterpret_cast<uint64_t*>(sk2), n);
+            for (int j = tid; j < n; j += kThreads) {
+                const uint64_t v = sp[j];
+                const Key x{lo + (int64_t)(v >> tb), (int32_t)(tmax - (v & tmask)), 0};
+                if (j < k) unext[base + j] = x.tok;
+                else keep(j - k, x);
+            }
+            __syncthreads();
+            if (nh == C) price = nxt.b[0];
+            return nh;
+        }
+    }
     if (n <= kSortedSmall && n <= nsc) {
         for (int i = tid; i < n; i += kThreads) sk[i] = Key{nb[i], nt[i], -1};
         __syncthreads();
