@@ -45,13 +45,13 @@ UNIT = "tokens/s"
 # named workload at its full size (the component's kernels summed); a
 # component whose kernels changed after their capture has no entry.
 NCU_TRAFFIC = {
-    ("scores", "layer_fwd"): 16840448 + 768,
-    ("auction", "layer_fwd"): 801792,
+    ("scores", "layer_fwd"): 16854528,
+    ("auction", "layer_fwd"): 775936,
     # slice histogram + slice rank + row gather; the rows' writes stay in L2
-    ("permute", "layer_fwd"): 36096 + 588032 + 16815872,
-    # tile prefix + GEMM1 (h1 written, partly kept in L2) + GEMM2
-    ("ffn", "layer_fwd"): 4864 + 151050496 + 35908096 + 222283008 + 6628096,
-    ("combine", "layer_fwd"): 16815616,
+    ("permute", "layer_fwd"): 36864 + 588544 + 16816640,
+    # GEMM1 (h1 written, partly kept in L2) + GEMM2
+    ("ffn", "layer_fwd"): 151063808 + 35196928 + 222300416 + 6546432,
+    ("combine", "layer_fwd"): 16815872,
 }
 
 

@@ -66,8 +66,12 @@ def test_scores_fp32_routing_reference(orc):
         assert np.abs(qg.astype(np.int64) - qo).max() <= 1
 
 
+# token tails (T not a multiple of the 128-row tile), column tails (D not a
+# multiple of the 64-column k-block) and E from 2 to 300 (the 16- to 256-wide
+# N tiles)
 @pytest.mark.parametrize("T,E,D", [(1000, 16, 200), (333, 40, 64), (256, 8, 128), (640, 300, 96),
-                                   (129, 128, 1024)])
+                                   (129, 128, 1024), (1001, 3, 72), (31, 2, 8), (4099, 16, 1032),
+                                   (32767, 16, 256), (40000, 16, 64)])
 def test_scores_bf16_shapes(orc, T, E, D):
     wl = synth.WORKLOADS["layer_fwd"].scaled(T=T, E=E, D=D, F=0)
     inp = synth.make_inputs(wl, 7)
@@ -424,7 +428,7 @@ def test_fig9_workloads_bit_exact(orc, name):
 # ------------------------------------------------------------------ scores + greedy in one pass
 @pytest.mark.parametrize("T,E,D", [(1000, 16, 200), (4099, 32, 256), (777, 100, 64),
                                    (8192, 128, 512), (640, 256, 128), (513, 300, 64),
-                                   (2048, 2, 64)])
+                                   (2048, 2, 64), (1001, 7, 72), (32767, 16, 64), (40000, 16, 64)])
 def test_scores_greedy_fused(orc, T, E, D):
     wl = synth.WORKLOADS["layer_fwd"].scaled(T=T, E=E, D=D, F=0)
     inp = synth.make_inputs(wl, 11)
@@ -441,6 +445,28 @@ def test_scores_greedy_fused(orc, T, E, D):
     ao, co = orc.greedy(qg)
     assert np.array_equal(to_np(a), ao)
     assert np.array_equal(to_np(c), co)
+
+
+def test_scores_greedy_fused_with_ties_few_experts(orc):
+    # E = 16 (the 16-wide N tile): the lowest expert wins ties, also between
+    # columns the two epilogue warps of a lane quadrant scan (3 and 12)
+    T, E, D = 1002, 16, 64
+    h = torch.zeros(T, D)
+    h[:, 0] = 1.0
+    w = torch.zeros(E, D)
+    w[[3, 12, 15], 0] = 0.5
+    h[::3, 1] = 1.0
+    w[12, 1] = 0.25           # every third row prefers expert 12
+    hb, wb = h.to(torch.bfloat16), w.to(torch.bfloat16)
+    q = torch.empty(T, E, dtype=torch.int32, device="cuda")
+    a = torch.empty(T, dtype=torch.int32, device="cuda")
+    c = torch.empty(E, dtype=torch.int32, device="cuda")
+    B.base_scores_greedy(dev(hb), dev(wb), None, q, a, c)
+    torch.cuda.synchronize()
+    ao, co = orc.greedy(to_np(q))
+    assert np.array_equal(to_np(a), ao) and np.array_equal(to_np(c), co)
+    rows = np.arange(T)
+    assert set(to_np(a)[rows % 3 != 0].tolist()) == {3} and set(to_np(a)[::3].tolist()) == {12}
 
 
 def test_scores_greedy_fused_with_ties(orc):
