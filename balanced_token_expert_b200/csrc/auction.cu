@@ -757,43 +757,40 @@ __device__ __forceinline__ uint64_t globaltimer() {
 template <class P>
 __device__ bool grid_sync(const P& p, unsigned& gen, int* s_flag) {
     // A counter barrier: every CTA adds one to an arrival count that only
-    // grows (it reaches gen * grid at barrier gen); the CTA that brings it
-    // there publishes gen in a release word, which the others poll -- one
-    // word per poll instead of every CTA's flag.  The counter and the
-    // release word sit 128 bytes apart in bar_flags (zeroed per launch).
+    // grows (it reaches gen * grid at barrier gen) with a release reduction
+    // (no reply to wait for) and polls the count with acquire loads until it
+    // gets there.  Against a count that the last arriver answers with a
+    // release word, this takes one L2 trip off the barrier's critical path.
+    // The count sits in bar_flags[0] (zeroed per launch).
     __syncthreads();
     ++gen;
     if (threadIdx.x == 0) {
         unsigned* count = p.bar_flags;
-        unsigned* release = p.bar_flags + 32;
+        const unsigned target = gen * gridDim.x;
         int ok = 1;
-        __threadfence();  // this CTA's writes before its arrival
-        const unsigned old = atomicAdd(count, 1u);
-        if (old + 1u == gen * gridDim.x) {
-            __threadfence();
-            *reinterpret_cast<volatile unsigned*>(release) = gen;
-        } else {
-            const uint64_t t0 = globaltimer();
-            for (long long it = 1;; ++it) {
-                if ((int)(vload(release) - gen) >= 0) break;
-                // short naps while the barrier is young, longer ones in a long
-                // wait (the narrow rounds of CTA 0) to spare the L2
-                __nanosleep(it < 256 ? 20 : 200);
-                if ((it & 63) == 0) {
-                    if (*reinterpret_cast<volatile int*>(&p.ctrl->abort)) {
-                        ok = 0;
-                        break;
-                    }
-                    if (globaltimer() - t0 > p.wait_ns || it > (1ll << 30)) {
-                        atomicExch(&p.ctrl->abort, 1);
-                        record_error(5001);
-                        ok = 0;
-                        break;
-                    }
+        // the release orders this CTA's writes before its arrival
+        asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(count) : "memory");
+        const uint64_t t0 = globaltimer();
+        for (long long it = 1;; ++it) {
+            unsigned c;
+            asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(c) : "l"(count) : "memory");
+            if ((int)(c - target) >= 0) break;
+            // short naps while the barrier is young, longer ones in a long
+            // wait (the narrow rounds of CTA 0) to spare the L2
+            __nanosleep(it < 256 ? 20 : 200);
+            if ((it & 63) == 0) {
+                if (*reinterpret_cast<volatile int*>(&p.ctrl->abort)) {
+                    ok = 0;
+                    break;
+                }
+                if (globaltimer() - t0 > p.wait_ns || it > (1ll << 30)) {
+                    atomicExch(&p.ctrl->abort, 1);
+                    record_error(5001);
+                    ok = 0;
+                    break;
                 }
             }
         }
-        __threadfence();
         *s_flag = ok;
     }
     __syncthreads();
