@@ -147,10 +147,14 @@ def test_auction_routing_reference_is_optimal_and_bit_exact(orc, seed):
     assert st["objective"] == orc.hungarian(q)[0]
 
 
+# C = T/E >= ~3000 (the last three) leaves no room for the sorted held sets in
+# shared memory: the wide rounds then resolve with the radix select and the
+# fringe merges instead
 @pytest.mark.parametrize("T,E,small", [(8, 2, False), (12, 3, True), (64, 64, False),
                                        (100, 4, True), (1000, 8, False), (2048, 2, False),
                                        (4096, 1024, False), (6000, 3, True), (8192, 16, True),
-                                       (30000, 40, False)])
+                                       (30000, 40, False), (16384, 2, False), (24000, 3, True),
+                                       (65536, 8, False)])
 def test_auction_shapes_bit_exact(orc, T, E, small):
     rng = np.random.default_rng(T * 7 + E)
     q = (rng.integers(0, 4, size=(T, E)) if small else
