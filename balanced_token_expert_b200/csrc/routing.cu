@@ -46,8 +46,12 @@ __global__ void greedy_kernel(const int32_t* __restrict__ q, int T, int E,
     extern __shared__ int32_t s_hist[];
     for (int e = threadIdx.x; e < E; e += blockDim.x) s_hist[e] = 0;
     __syncthreads();
+    // lanes per token: one per 16-byte piece of the row when E % 4 == 0
+    // (int4 loads), else one per entry
+    const bool vec = (E & 3) == 0;
+    const int words = vec ? E / 4 : E;
     int G = 1;
-    while (G < E && G < kWarp) G <<= 1;
+    while (G < words && G < kWarp) G <<= 1;
     const int lane = lane_id(), sub = lane / G, gl = lane % G;
     const int per_warp = kWarp / G;
     const long long gw = (blockIdx.x * (long long)blockDim.x + threadIdx.x) / kWarp;
@@ -58,20 +62,31 @@ __global__ void greedy_kernel(const int32_t* __restrict__ q, int T, int E,
         int best_v = INT32_MIN, best_e = INT32_MAX;
         if (valid) {
             const int32_t* row = q + (size_t)t * E;
-            if ((E & 3) == 0 && G == kWarp) {
+            if (vec) {
                 const int4* r4 = reinterpret_cast<const int4*>(row);
-                for (int j = gl; j < E / 4; j += kWarp) {
+                for (int j = gl; j < E / 4; j += G) {
                     const int4 v = __ldg(r4 + j);
                     const int e0 = 4 * j;
-                    if (v.x > best_v) { best_v = v.x; best_e = e0; }
-                    if (v.y > best_v) { best_v = v.y; best_e = e0 + 1; }
-                    if (v.z > best_v) { best_v = v.z; best_e = e0 + 2; }
-                    if (v.w > best_v) { best_v = v.w; best_e = e0 + 3; }
+                    // conditional moves, not branches (the first of equal values stays)
+                    bool g = v.x > best_v;
+                    best_e = g ? e0 : best_e;
+                    best_v = g ? v.x : best_v;
+                    g = v.y > best_v;
+                    best_e = g ? e0 + 1 : best_e;
+                    best_v = g ? v.y : best_v;
+                    g = v.z > best_v;
+                    best_e = g ? e0 + 2 : best_e;
+                    best_v = g ? v.z : best_v;
+                    g = v.w > best_v;
+                    best_e = g ? e0 + 3 : best_e;
+                    best_v = g ? v.w : best_v;
                 }
             } else {
                 for (int e = gl; e < E; e += G) {
                     const int v = __ldg(row + e);
-                    if (v > best_v) { best_v = v; best_e = e; }
+                    const bool g = v > best_v;
+                    best_e = g ? e : best_e;
+                    best_v = g ? v : best_v;
                 }
             }
         }
@@ -80,7 +95,9 @@ __global__ void greedy_kernel(const int32_t* __restrict__ q, int T, int E,
             if (off >= G) continue;
             const int ov = __shfl_xor_sync(0xffffffffu, best_v, off);
             const int oe = __shfl_xor_sync(0xffffffffu, best_e, off);
-            if (ov > best_v || (ov == best_v && oe < best_e)) { best_v = ov; best_e = oe; }
+            const bool tk = (ov > best_v) | ((ov == best_v) & (oe < best_e));
+            best_v = tk ? ov : best_v;
+            best_e = tk ? oe : best_e;
         }
         if (valid && gl == 0) {
             assign[t] = best_e;
@@ -293,8 +310,9 @@ int launch_greedy(const int32_t* q, int T, int E, int32_t* assign, int32_t* coun
     if (counts && cudaMemsetAsync(counts, 0, sizeof(int32_t) * E, stream) != cudaSuccess)
         return BASE_ERR_CUDA;
     const int threads = 256;
+    const int words = (E & 3) == 0 ? E / 4 : E;  // the kernel's lanes per token
     int G = 1;
-    while (G < E && G < kWarp) G <<= 1;
+    while (G < words && G < kWarp) G <<= 1;
     const long long warps_needed = ((long long)T * G + kWarp - 1) / kWarp;
     long long blocks = (warps_needed * kWarp + threads - 1) / threads;
     if (blocks > num_sms() * 8) blocks = num_sms() * 8;
