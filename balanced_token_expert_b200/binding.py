@@ -27,6 +27,7 @@ __all__ = [
     "base_sanitize_scores", "BASE_ROUTE_SANITIZE", "base_workspace_size_fig9", "base_assign_fig9",
     "base_probe_workspace_size", "base_measure_latency", "base_scores_greedy",
     "BASE_TEST_AUCTION_ABSENT_CTA", "BASE_TEST_GEMM_DROP_FIRST_LOAD", "EXPORTED",
+    "base_ep_dispatch", "base_ep_combine",
 ]
 
 BASE_OK = 0
@@ -45,6 +46,7 @@ EXPORTED = (
     "base_layer_bwd", "base_test_inject", "base_workspace_size_blend", "base_layer_fwd_blend",
     "base_expert_stack", "base_sanitize_scores", "base_workspace_size_fig9", "base_assign_fig9",
     "base_probe_workspace_size", "base_measure_latency", "base_scores_greedy",
+    "base_ep_dispatch", "base_ep_combine",
 )
 
 
@@ -102,6 +104,8 @@ _SIGS = {
     "base_expert_ffn": (_i, [_vp, _vp, _i, _i, _i, _i, _vp, _vp, _i, _vp, _vp, _vp, _vp, _vp, _vp,
                              _sz, _vp]),
     "base_combine": (_i, [_vp, _vp, _i, _i, _vp, _vp]),
+    "base_ep_dispatch": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp]),
+    "base_ep_combine": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp]),
     "base_layer_fwd": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp,
                             ctypes.POINTER(LayerSaved), _vp, _sz, _vp]),
     "base_layer_bwd": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, ctypes.POINTER(LayerSaved),
@@ -276,6 +280,36 @@ def base_combine(y_perm, perm, out, stream=None):
     T, D = y_perm.shape
     _check("base_combine", lib().base_combine(_ptr(y_perm), _ptr(perm), T, D, _ptr(out),
                                               _stream(stream)))
+
+
+def _ptr_array(ts):
+    """A host array of the tensors' device pointers (None for a missing list)."""
+    if ts is None:
+        return None
+    return (ctypes.c_void_p * len(ts))(*[t.data_ptr() for t in ts])
+
+
+def base_ep_dispatch(h, perm, gate, recv, recv_gate, g0: int, E: int, stream=None):
+    """Sources g0 .. g0 + len(h) - 1 push their rows to every worker's receive
+    buffer, expert-major (include/base.h).  h, perm, gate: lists over the
+    sources; recv, recv_gate: lists over all G workers; gate and recv_gate
+    None or given together."""
+    T, D = h[0].shape
+    G = len(recv)
+    _check("base_ep_dispatch", lib().base_ep_dispatch(
+        _ptr_array(h), _ptr_array(perm), _ptr_array(gate), _ptr_array(recv),
+        _ptr_array(recv_gate), g0, len(h), G, T, D, E, _stream(stream)))
+
+
+def base_ep_combine(y, perm, out, r0: int, E: int, stream=None):
+    """Receivers r0 .. r0 + len(y) - 1 send every expert output row to its
+    token in its source worker's out (include/base.h).  y: list over the
+    receivers; perm, out: lists over all G workers."""
+    T, D = y[0].shape
+    G = len(out)
+    _check("base_ep_combine", lib().base_ep_combine(
+        _ptr_array(y), _ptr_array(perm), _ptr_array(out), r0, len(y), G, T, D, E,
+        _stream(stream)))
 
 
 def _saved(sv: dict) -> LayerSaved:

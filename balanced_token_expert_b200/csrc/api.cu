@@ -24,6 +24,11 @@ int launch_fig9(const int32_t* q, int T, int E, int32_t* assign, int64_t* price,
                 long long max_iterations, long long max_rounds, void* ws, size_t ws_bytes,
                 cudaStream_t stream);
 size_t permute_workspace_bytes(int T, int E);
+int launch_ep_dispatch(const void* const* h, const int32_t* const* perm, const float* const* gate,
+                       void* const* recv, float* const* recv_gate, int g0, int ns, int G, int T,
+                       int D, int E, cudaStream_t stream);
+int launch_ep_combine(const void* const* y, const int32_t* const* perm, void* const* out, int r0,
+                      int nr, int G, int T, int D, int E, cudaStream_t stream);
 int launch_sort_by_expert(const int32_t* assign, int T, int E, int32_t* perm, int32_t* inv,
                           int32_t* offsets, const float* s, float* gate, void* ws,
                           cudaStream_t stream);
@@ -260,6 +265,41 @@ int base_combine(const void* y_perm, const int32_t* perm, int T, int D, void* ou
     if (!y_perm || !perm || !out || T < 1 || D < 8 || D % 8 != 0) return BASE_ERR_INVALID_ARG;
     if (!aligned(y_perm, 16) || !aligned(out, 16)) return BASE_ERR_INVALID_ARG;
     return launch_move_rows(y_perm, perm, T, D, out, true, stream);
+}
+
+// shapes of an expert-parallel exchange: G workers (at most 8), E/G experts
+// each, C = T/E tokens per expert per worker, rows of D bf16 (16-byte pieces)
+static bool ep_shapes_ok(int G, int T, int D, int E) {
+    return G >= 1 && G <= 8 && shapes_ok(T, E) && E % G == 0 && T % E == 0 && D >= 8 &&
+           D % 8 == 0;
+}
+
+int base_ep_dispatch(const void* const* h, const int32_t* const* perm, const float* const* gate,
+                     void* const* recv, float* const* recv_gate, int g0, int ns, int G, int T,
+                     int D, int E, cudaStream_t stream) {
+    if (!h || !perm || !recv || !ep_shapes_ok(G, T, D, E) || g0 < 0 || ns < 1 || g0 + ns > G)
+        return BASE_ERR_INVALID_ARG;
+    if ((gate == nullptr) != (recv_gate == nullptr)) return BASE_ERR_INVALID_ARG;
+    for (int i = 0; i < ns; ++i)
+        if (!h[i] || !aligned(h[i], 16) || !perm[i] || !aligned(perm[i], 4) ||
+            (gate && (!gate[i] || !aligned(gate[i], 4))))
+            return BASE_ERR_INVALID_ARG;
+    for (int r = 0; r < G; ++r)
+        if (!recv[r] || !aligned(recv[r], 16) || (recv_gate && (!recv_gate[r] || !aligned(recv_gate[r], 4))))
+            return BASE_ERR_INVALID_ARG;
+    return launch_ep_dispatch(h, perm, gate, recv, recv_gate, g0, ns, G, T, D, E, stream);
+}
+
+int base_ep_combine(const void* const* y, const int32_t* const* perm, void* const* out, int r0,
+                    int nr, int G, int T, int D, int E, cudaStream_t stream) {
+    if (!y || !perm || !out || !ep_shapes_ok(G, T, D, E) || r0 < 0 || nr < 1 || r0 + nr > G)
+        return BASE_ERR_INVALID_ARG;
+    for (int i = 0; i < nr; ++i)
+        if (!y[i] || !aligned(y[i], 16)) return BASE_ERR_INVALID_ARG;
+    for (int g = 0; g < G; ++g)
+        if (!perm[g] || !aligned(perm[g], 4) || !out[g] || !aligned(out[g], 16))
+            return BASE_ERR_INVALID_ARG;
+    return launch_ep_combine(y, perm, out, r0, nr, G, T, D, E, stream);
 }
 
 int base_layer_fwd(const void* h, const void* w, const void* W1, const void* W2, int act,

@@ -6,5 +6,6 @@
 #include "variant.cu"
 #include "gemm.cu"
 #include "backward.cu"
+#include "ep.cu"
 #include "api.cu"
 #include "noalloc.cu"

@@ -32,7 +32,7 @@ import torch
 import torch.distributed as dist
 
 __all__ = ["EPPlan", "shuffle_permutation", "receive_order", "exchange", "ep_layer_fwd",
-           "CudaBackend"]
+           "CudaBackend", "ep_layer_fwd_fused"]
 
 
 @dataclass(frozen=True)
@@ -186,3 +186,60 @@ class CudaBackend:
         h1 = torch.empty(T, F, dtype=x.dtype, device="cuda")
         self.B.base_expert_ffn(x, offsets, W1, W2, act, gate, y, h1, None, None, self.ws)
         return y
+
+
+def ep_layer_fwd_fused(hs, w, W1s, W2s, act: int, plan: EPPlan, stream=None):
+    """Steps 2-4 of the expert-parallel forward (route, experts, return; the
+    inputs are the already shuffled batches) with the library's fused
+    exchange kernels, for G workers whose buffers are all on this device.
+
+    Each worker scores its tokens against all E centroids, solves its own
+    balanced assignment and sorts its slots by expert (no rows moved); one
+    base_ep_dispatch call then moves every worker's rows straight into the
+    receiving workers' expert-major buffers (the permutation, the route
+    all-to-all and the regrouping in one pass), each worker runs its E/G
+    experts with eq. 1's gate and residual, and one base_ep_combine call sends
+    every output row to its token in its source worker (the return all-to-all
+    and the inverse sort in one pass).  On one GPU this runs the whole
+    exchange; across GPUs each worker would pass its own rank and the peer
+    mappings of the others' buffers.
+
+    hs: G (T, D) bf16 batches; w: (E, D) bf16 centroids; W1s / W2s: per worker
+    (E/G, F, D) and (E/G, D, F) bf16 expert weights.  Returns the G (T, D)
+    outputs in each worker's token order."""
+    from . import binding as B
+    from . import buffers
+    T, E, G = plan.T, plan.E, plan.G
+    D = hs[0].shape[1]
+    F = W1s[0].shape[1]
+    C, El = plan.C, plan.El
+    ws = buffers.workspace(T, E, D, F)
+    perms, gates = [], []
+    for g in range(G):
+        s = torch.empty(T, E, device="cuda")
+        q = torch.empty(T, E, dtype=torch.int32, device="cuda")
+        B.base_scores(hs[g], w, s, q, stream)
+        assign = torch.empty(T, dtype=torch.int32, device="cuda")
+        price = torch.empty(E, dtype=torch.int64, device="cuda")
+        B.base_assign_balanced(q, assign, price, buffers.stats(), ws, stream)
+        perm = torch.empty(T, dtype=torch.int32, device="cuda")
+        inv = torch.empty_like(perm)
+        offsets = torch.empty(E + 1, dtype=torch.int32, device="cuda")
+        gate = torch.empty(T, device="cuda")
+        B.base_permute(None, assign, E, perm, inv, offsets, None, s, gate, ws, stream)
+        perms.append(perm)
+        gates.append(gate)
+    recv = [torch.empty(T, D, dtype=hs[0].dtype, device="cuda") for _ in range(G)]
+    recv_gate = [torch.empty(T, device="cuda") for _ in range(G)]
+    B.base_ep_dispatch(hs, perms, gates, recv, recv_gate, 0, E, stream)
+    offs = (torch.arange(El + 1, dtype=torch.int32) * (G * C)).cuda()
+    ys = []
+    for r in range(G):
+        y = torch.empty(T, D, dtype=hs[0].dtype, device="cuda")
+        h1 = torch.empty(T, F, dtype=hs[0].dtype, device="cuda")
+        B.base_expert_ffn(recv[r], offs, W1s[r], W2s[r], act, recv_gate[r], y, h1, None, None, ws,
+                          stream)
+        ys.append(y)
+    outs = [torch.empty(T, D, dtype=hs[0].dtype, device="cuda") for _ in range(G)]
+    B.base_ep_combine(ys, perms, outs, 0, E, stream)
+    return outs

@@ -337,6 +337,49 @@ int base_combine(const void* y_perm, const int32_t* perm, int T, int D, void* ou
                  cudaStream_t stream);
 
 /*
+ * Expert parallelism (wikillm.com summary, Method: Sharding; fig. 2's forward
+ * pass): G workers (1 <= G <= 8, one node) each hold T tokens and E/G experts
+ * (El = E/G; worker r holds experts r El .. r El + El - 1), and every expert
+ * gets exactly C = T/E of each worker's tokens (balanced routing: E | T, G | E).
+ * These two calls are each a permutation fused with its all-to-all, as plain
+ * 16-byte loads and stores through pointers to every worker's buffers: the
+ * pointers of other workers may be peer mappings (NVLink); on one GPU, one
+ * call over all workers' buffers runs the whole exchange.
+ *
+ * base_ep_dispatch -- sort_by_expert + the route all-to-all + the receive
+ * side's grouping: for each source worker g in [g0, g0 + ns) and slot s of
+ * its expert-major order (perm_g from base_permute, balanced: expert e =
+ * s / C, c = s % C, worker r = e / El, local expert j = e % El):
+ *     recv_r[(j G + g) C + c] = h_g[perm_g[s]]   (rows of D bf16)
+ *     recv_gate_r[(j G + g) C + c] = gate_g[s]   (when the gate pointers are given)
+ * so every worker receives its experts' rows expert-major (local expert j's
+ * G C rows together: the offsets of base_expert_ffn are j G C).
+ *   h, perm, gate: host arrays of ns device pointers (sources g0..g0+ns-1:
+ *   T*D bf16 tokens, T int32 slot -> token, T fp32 gate scores in slot
+ *   order); gate nullable (then recv_gate must be null too).
+ *   recv, recv_gate: host arrays of G device pointers (T*D bf16, T fp32).
+ *   A worker's own call passes g0 = its rank, ns = 1.  The receivers may read
+ *   only after every source has written (a barrier across the workers).
+ *   A slot whose token is out of range is recorded in the device error word
+ *   (2101) and skipped.
+ */
+int base_ep_dispatch(const void* const* h, const int32_t* const* perm, const float* const* gate,
+                     void* const* recv, float* const* recv_gate, int g0, int ns, int G, int T,
+                     int D, int E, cudaStream_t stream);
+
+/*
+ * base_ep_combine -- the return all-to-all + inverse_sort: for each receiver
+ * r in [r0, r0 + nr) and row i = (j G + g) C + c of its expert outputs,
+ *     out_g[perm_g[(r El + j) C + c]] = y_r[i]   (rows of D bf16)
+ * so every output row lands on its token in the source worker's order.
+ *   y: host array of nr device pointers (receivers r0..r0+nr-1, T*D bf16);
+ *   perm, out: host arrays of G device pointers (T int32, T*D bf16).
+ *   Errors as base_ep_dispatch (2102).
+ */
+int base_ep_combine(const void* const* y, const int32_t* const* perm, void* const* out, int r0,
+                    int nr, int G, int T, int D, int E, cudaStream_t stream);
+
+/*
  * The whole layer forward on one stream without host synchronisation:
  * scores -> (balanced auction | greedy) -> permute -> expert FFN + eq. 1 ->
  * combine.  h: T*D bf16, w: E*D bf16, W1: E*F*D, W2: E*D*F bf16; out: T*D bf16.
