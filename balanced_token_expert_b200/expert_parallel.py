@@ -22,6 +22,11 @@ the permutation, the grouped FFN and the row moves), with torch used for
 device memory and ``torch.distributed`` (NCCL on GPUs) for the all-to-alls.
 With one worker the exchanges are identities and the layer is the single-GPU
 path applied to the shuffled tokens.
+
+:func:`ep_layer_fwd_fused` runs the same layer with the library's fused
+exchange kernels instead of all-to-alls (base_ep_dispatch / base_ep_combine:
+each permutation and its exchange in one pass over peer-addressable
+buffers), for workers whose buffers are all on this device.
 """
 from __future__ import annotations
 
@@ -188,10 +193,16 @@ class CudaBackend:
         return y
 
 
-def ep_layer_fwd_fused(hs, w, W1s, W2s, act: int, plan: EPPlan, stream=None):
-    """Steps 2-4 of the expert-parallel forward (route, experts, return; the
-    inputs are the already shuffled batches) with the library's fused
-    exchange kernels, for G workers whose buffers are all on this device.
+def ep_layer_fwd_fused(hs, w, W1s, W2s, act: int, plan: EPPlan, seeds=None, stream=None):
+    """The expert-parallel forward with the library's fused exchange kernels,
+    for G workers whose buffers are all on this device.
+
+    With seeds (one per worker), the shuffle comes first and the unshuffle
+    last, each the same kind of exchange with one destination block per
+    worker: base_ep_dispatch with G "experts" of T/G rows through the
+    worker's shuffle permutation sends block r of its shuffled tokens to
+    worker r, and base_ep_combine undoes it.  Without seeds the inputs are
+    taken as already shuffled.
 
     Each worker scores its tokens against all E centroids, solves its own
     balanced assignment and sorts its slots by expert (no rows moved); one
@@ -214,6 +225,13 @@ def ep_layer_fwd_fused(hs, w, W1s, W2s, act: int, plan: EPPlan, stream=None):
     F = W1s[0].shape[1]
     C, El = plan.C, plan.El
     ws = buffers.workspace(T, E, D, F)
+    sperms = None
+    if seeds is not None:
+        # 1. shuffle: worker g's shuffled block r goes to worker r, position g T/G
+        sperms = [shuffle_permutation(T, sd).to(device="cuda", dtype=torch.int32) for sd in seeds]
+        shuffled = [torch.empty_like(hs[0]) for _ in range(G)]
+        B.base_ep_dispatch(hs, sperms, None, shuffled, None, 0, G, stream)
+        hs = shuffled
     perms, gates = [], []
     for g in range(G):
         s = torch.empty(T, E, device="cuda")
@@ -242,4 +260,9 @@ def ep_layer_fwd_fused(hs, w, W1s, W2s, act: int, plan: EPPlan, stream=None):
         ys.append(y)
     outs = [torch.empty(T, D, dtype=hs[0].dtype, device="cuda") for _ in range(G)]
     B.base_ep_combine(ys, perms, outs, 0, E, stream)
+    if sperms is not None:
+        # 4. unshuffle: every row back to its worker and position
+        back = [torch.empty_like(outs[0]) for _ in range(G)]
+        B.base_ep_combine(outs, sperms, back, 0, G, stream)
+        outs = back
     return outs

@@ -105,6 +105,38 @@ def test_ep_layer_matches_the_single_gpu_layer(orc, G, T, E, D, F):
     assert B.base_device_error(clear=True) == 0
 
 
+@pytest.mark.parametrize("G,T,E,D,F", [(2, 1024, 8, 256, 512), (4, 2048, 16, 128, 256)])
+def test_ep_layer_with_shuffle(G, T, E, D, F):
+    # the four exchanges of fig. 2 as fused kernels: the shuffle and the
+    # unshuffle are the same exchange with one block of T/G rows per worker
+    wl, base, hs = _batches(G, T, E, D, F, 11)
+    w, W1, W2 = dev(base.w), dev(base.W1), dev(base.W2)
+    El = E // G
+    seeds = [100 + g for g in range(G)]
+    plan = ep.EPPlan(T=T, E=E, G=G)
+    outs = ep.ep_layer_fwd_fused(hs, w, [W1[r * El:(r + 1) * El] for r in range(G)],
+                                 [W2[r * El:(r + 1) * El] for r in range(G)], B.BASE_RELU, plan,
+                                 seeds=seeds)
+    torch.cuda.synchronize()
+    # reference: each worker's shuffled batch through the single-GPU layer,
+    # every row then put back where it came from
+    n = T // G
+    sp = [ep.shuffle_permutation(T, sd).cuda() for sd in seeds]
+    expect = [torch.empty(T, D, dtype=torch.bfloat16, device="cuda") for _ in range(G)]
+    ws = buffers.workspace(T, E, D, F)
+    for r in range(G):
+        sh = torch.cat([hs[g][sp[g][r * n:(r + 1) * n]] for g in range(G)])
+        sv = buffers.layer_saved(T, E, D, F, for_backward=False)
+        y = torch.empty(T, D, dtype=torch.bfloat16, device="cuda")
+        B.base_layer_fwd(sh, w, W1, W2, B.BASE_RELU, B.BASE_ROUTE_BALANCED, y, sv, ws)
+        for g in range(G):
+            expect[g][sp[g][r * n:(r + 1) * n]] = y[g * n:(g + 1) * n]
+    torch.cuda.synchronize()
+    for g in range(G):
+        assert torch.equal(outs[g], expect[g])
+    assert B.base_device_error(clear=True) == 0
+
+
 def test_ep_one_call_per_worker_equals_one_call_for_all():
     G, T, E, D = 4, 1024, 8, 128
     wl, base, hs = _batches(G, T, E, D, 0, 7)
