@@ -29,6 +29,23 @@ namespace ep {
 
 constexpr int kMaxWorkers = 8;  // one NVSwitch node
 
+// one row of vec 16-byte pieces by a warp, four loads in flight per lane
+// before their stores (without that, the compiler keeps every load behind
+// the previous store: the row's reads would wait one after another)
+__device__ __forceinline__ void copy_row(const uint4* __restrict__ s, uint4* __restrict__ d,
+                                         int vec, int lane) {
+    int v = lane;
+    for (; v + 3 * kWarp < vec; v += 4 * kWarp) {
+        const uint4 a0 = __ldg(s + v), a1 = __ldg(s + v + kWarp);
+        const uint4 a2 = __ldg(s + v + 2 * kWarp), a3 = __ldg(s + v + 3 * kWarp);
+        d[v] = a0;
+        d[v + kWarp] = a1;
+        d[v + 2 * kWarp] = a2;
+        d[v + 3 * kWarp] = a3;
+    }
+    for (; v < vec; v += kWarp) d[v] = __ldg(s + v);
+}
+
 struct Ptrs {
     const uint4* src[kMaxWorkers];  // dispatch: h_g;  combine: y_r
     uint4* dst[kMaxWorkers];        // dispatch: recv_r;  combine: out_g
@@ -60,9 +77,7 @@ __global__ void __launch_bounds__(256) ep_dispatch_kernel(const __grid_constant_
             if (lane == 0) record_error(2101);
             continue;
         }
-        const uint4* srow = p.src[g] + (long long)t * vec;
-        uint4* drow = p.dst[r] + row * vec;
-        for (int v = lane; v < vec; v += kWarp) drow[v] = __ldg(srow + v);
+        copy_row(p.src[g] + (long long)t * vec, p.dst[r] + row * vec, vec, lane);
         if (lane == 0 && p.gate[g] && p.gate_out[r]) p.gate_out[r][row] = __ldg(p.gate[g] + s);
     }
 }
@@ -90,9 +105,7 @@ __global__ void __launch_bounds__(256) ep_combine_kernel(const __grid_constant__
             if (lane == 0) record_error(2102);
             continue;
         }
-        const uint4* srow = p.src[r] + (long long)i * vec;
-        uint4* drow = p.dst[g] + (long long)t * vec;
-        for (int v = lane; v < vec; v += kWarp) drow[v] = __ldg(srow + v);
+        copy_row(p.src[r] + (long long)i * vec, p.dst[g] + (long long)t * vec, vec, lane);
     }
 }
 

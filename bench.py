@@ -566,6 +566,46 @@ def measure_floors():
     return dict(grid_barrier_ns=g, block_barrier_ns=c, l2_load_ns=l2, smem_load_ns=sm)
 
 
+def measure_ep_exchange(G, T, D, E, steps, hbm_gbs):
+    """The expert-parallel exchange kernels with G workers' buffers on this
+    GPU (the emulation of the peer exchange): CUDA-event time of one
+    base_ep_dispatch (rows only) and one base_ep_combine over all workers,
+    against the HBM roofline of the bytes they move here (every row read once
+    and written once: 2 G T D 2 bytes; the buffers, 3 G T D 2 bytes, exceed
+    L2).  Across GPUs the bound is NVLink instead: (G-1)/G of those rows
+    cross it in each direction."""
+    import torch
+    from balanced_token_expert_b200 import binding as B
+    g = torch.Generator(device="cuda")
+    g.manual_seed(1234)
+    hs = [torch.randn(T, D, device="cuda", generator=g).to(torch.bfloat16) for _ in range(G)]
+    perms = [torch.randperm(T, device="cuda", generator=g).to(torch.int32) for _ in range(G)]
+    recv = [torch.empty(T, D, dtype=torch.bfloat16, device="cuda") for _ in range(G)]
+    outs = [torch.empty(T, D, dtype=torch.bfloat16, device="cuda") for _ in range(G)]
+    ms = {"dispatch": [], "combine": []}
+    for i in range(3 + steps):
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        ev[0].record()
+        B.base_ep_dispatch(hs, perms, None, recv, None, 0, E)
+        ev[1].record()
+        B.base_ep_combine(recv, perms, outs, 0, E)
+        ev[2].record()
+        torch.cuda.synchronize()
+        if i >= 3:
+            ms["dispatch"].append(ev[0].elapsed_time(ev[1]))
+            ms["combine"].append(ev[1].elapsed_time(ev[2]))
+    ok = all(torch.equal(a, b) for a, b in zip(outs, hs))  # the round trip is the identity
+    nbytes = 2.0 * G * T * D * 2
+    res = dict(workers=G, T=T, D=D, E=E, bytes_per_exchange=nbytes, round_trip_identity=ok,
+               note="all workers' buffers on one GPU; across GPUs NVLink bounds it")
+    for k, v in ms.items():
+        m = statistics.mean(v)
+        res[k] = dict(ms=m, achieved_gbs=nbytes / m / 1e6, frac=nbytes / m / 1e6 / hbm_gbs)
+    del hs, perms, recv, outs
+    torch.cuda.empty_cache()
+    return res
+
+
 def latency_roofline(u, T, E, auction_ms, fl, hbm_gbs):
     """The auction against its latency floor: every round costs at least its
     synchronisation chain -- a grid-wide round two grid barriers and two
@@ -665,6 +705,9 @@ def main():
             clocks=head["clocks"], device_error=head["device_error"], wall_s=head["wall_s"])
         if extra:
             res["workloads"] = extra
+        if world == 1 and args.workload == "layer_fwd" and not args.tokens and not args.only:
+            res["ep_exchange"] = measure_ep_exchange(8, wl.T, wl.D, wl.E, args.extra_steps,
+                                                     peaks()["hbm"])
         if world == 1 and not args.no_cpu_baseline:
             res["cpu_baseline"] = cpu_baseline(wl)
         print(json.dumps(res))
