@@ -355,3 +355,27 @@ def test_expert_parallel_layer_one_worker(orc):
     expect[perm.numpy()] = ysh
     ok, worst = close_rel_rms(to_np(y), expect, FWD_TOL)
     assert ok, worst
+
+
+def test_training_step_is_deterministic():
+    # the forward and the backward three times on the same inputs: every
+    # output, saved activation and gradient the same bits each time (no
+    # floating-point atomics: the centroid gradient sums in a fixed order)
+    wl = synth.WORKLOADS["layer_fwd_bwd"].scaled(T=4096, E=16, D=512, F=1024)
+    inp = synth.make_inputs(wl, 21, with_dout=True)
+    T, E, D, F = wl.T, wl.E, wl.D, wl.F
+    runs = []
+    for _ in range(3):
+        out, sv, ws = _run_layer_fwd(wl, inp, "balanced", for_backward=True)
+        dh = torch.empty(T, D, dtype=torch.bfloat16, device="cuda")
+        dw = torch.empty(E, D, dtype=torch.float32, device="cuda")
+        dW1 = torch.empty(E, F, D, dtype=torch.float32, device="cuda")
+        dW2 = torch.empty(E, D, F, dtype=torch.float32, device="cuda")
+        B.base_layer_bwd(dev(inp.h), dev(inp.w), dev(inp.W1), dev(inp.W2), ACT[wl.act], sv,
+                         dev(inp.dout), dh, dw, dW1, dW2, ws)
+        torch.cuda.synchronize()
+        runs.append(dict(out=out, dh=dh, dw=dw, dW1=dW1, dW2=dW2, **{
+            k: sv[k] for k in ("s", "q", "assign", "price", "perm", "a1", "h1", "f", "y_perm")}))
+    for k, v in runs[0].items():
+        for other in runs[1:]:
+            assert torch.equal(v, other[k]), k
