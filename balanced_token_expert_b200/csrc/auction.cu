@@ -2959,6 +2959,17 @@ int launch_auction(const int32_t* q, int T, int E, int32_t* assign, int64_t* pri
     cudaGetDevice(&dev);
     if (cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
         return BASE_ERR_CUDA;
+    // The grid: one CTA per SM at most, and no more than the larger of E (an
+    // owner for every expert) and the CTAs a phase start needs to bid all T
+    // tokens in one pass (4 per lane group, 16 warps): fewer CTAs make every
+    // grid barrier cheaper and leave fewer pollers during the narrow rounds.
+    {
+        int G = 1;
+        while (G < E && G < 32) G <<= 1;
+        const int per_pass = kWarps * (32 / G) * 4;
+        const long long want = std::max<long long>(E, ((long long)T + per_pass - 1) / per_pass);
+        if (want < nsm) nsm = (int)want;
+    }
     // sorted held sets in the wide rounds when the owned experts' sets (two
     // buffers each) and the sort scratch (a power of two >= C keys, 2048 at
     // least when it fits) fit next to the narrow plan
@@ -2986,7 +2997,7 @@ int launch_auction(const int32_t* q, int T, int E, int32_t* assign, int64_t* pri
             cudaSuccess ||
         per_sm < 1)
         return BASE_ERR_UNSUPPORTED;
-    const int grid = nsm;  // one CTA per SM, all co-resident
+    const int grid = nsm;  // at most one CTA per SM (sized above), all co-resident
     if (grid > kMaxGrid) return BASE_ERR_UNSUPPORTED;
     void* args[] = {&prm};
     if (cudaLaunchCooperativeKernel(reinterpret_cast<void*>(auction_kernel), dim3(grid),
