@@ -2596,6 +2596,7 @@ struct SmemPlan {
 // with a grid barrier after each step.
 struct Fig9Params {
     const int32_t* q;
+    int32_t* qT;  // [E][T]: q by expert, written at the start (an expert's values coalesced)
     int T, E, C;
     long long max_iterations, max_rounds;
     int keys_in_smem;  // 1: an expert's T keys fit in shared memory
@@ -2652,6 +2653,30 @@ __global__ void __launch_bounds__(kThreads, 1) fig9_kernel(const __grid_constant
             p.bmax[t] = 0ull;
             p.barg[t] = INT32_MAX;
         }
+        // q by expert: each warp transposes 32 x 32 tiles in registers (lane l
+        // loads expert e0 + l of 32 tokens, then writes them as one 128-byte run)
+        const long long tt = ((long long)T + 31) / 32;
+        const int et = (E + 31) / 32;
+        const int lane = lane_id();
+        for (long long k = (long long)cta * kWarps + warp_id(); k < tt * et;
+             k += (long long)ncta * kWarps) {
+            const long long t0 = (k / et) * 32;
+            const int e = (int)(k % et) * 32 + lane;
+            int32_t v[32];
+#pragma unroll
+            for (int r = 0; r < 32; ++r)
+                v[r] = (e < E && t0 + r < T) ? __ldg(p.q + (size_t)(t0 + r) * E + e) : 0;
+            if (e < E) {
+                int32_t* dst = p.qT + (size_t)e * T + t0;
+                if (t0 + 32 <= T && (reinterpret_cast<uintptr_t>(dst) & 15) == 0) {
+#pragma unroll
+                    for (int r = 0; r < 32; r += 4)
+                        *reinterpret_cast<int4*>(dst + r) = make_int4(v[r], v[r + 1], v[r + 2], v[r + 3]);
+                } else {
+                    for (int r = 0; r < 32 && t0 + r < T; ++r) dst[r] = v[r];
+                }
+            }
+        }
     }
     if (!(ok = grid_sync(p, bar_gen, s_misc))) return;
     const int64_t qmax = (int32_t)(vload(&p.mmenc[0]) ^ 0x80000000u);
@@ -2676,7 +2701,7 @@ __global__ void __launch_bounds__(kThreads, 1) fig9_kernel(const __grid_constant
         for (int e = cta; e < E; e += ncta) {
             auto key_of = [&](int t) {  // holder / price come from other CTAs: read past L1
                 const int h = __ldcg(p.holder + t);
-                const int64_t qv = __ldg(p.q + (size_t)t * E + e);
+                const int64_t qv = __ldcg(p.qT + (size_t)e * T + t);
                 int64_t v;
                 if (h == e && retain_top) v = RETAIN;
                 else if (h == e) v = qv;
@@ -2715,7 +2740,7 @@ __global__ void __launch_bounds__(kThreads, 1) fig9_kernel(const __grid_constant
             const Key X{s_xb[(e / ncta) & 7], s_xt[(e / ncta) & 7], 0};
             auto key_of = [&](int t) {  // holder / price come from other CTAs: read past L1
                 const int h = __ldcg(p.holder + t);
-                const int64_t qv = __ldg(p.q + (size_t)t * E + e);
+                const int64_t qv = __ldcg(p.qT + (size_t)e * T + t);
                 int64_t v;
                 if (h == e && retain_top) v = RETAIN;
                 else if (h == e) v = qv;
@@ -2813,6 +2838,7 @@ static SmemPlan smem_plan(int E, int NM, int T) {
 
 size_t fig9_workspace_bytes(int T, int E) {
     size_t b = align_up(2 * sizeof(unsigned), 256);
+    b += align_up(sizeof(int32_t) * (size_t)T * E, 256);         // q by expert
     b += align_up(sizeof(auction::Ctrl), 256);
     b += align_up(sizeof(unsigned) * auction::kMaxGrid, 256);
     b += align_up(sizeof(unsigned long long) * (size_t)T, 256);  // bmax
@@ -2852,6 +2878,7 @@ int launch_fig9(const int32_t* q, int T, int E, int32_t* assign, int64_t* price,
     prm.barg = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * (size_t)T));
     prm.holder = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * (size_t)T));
     prm.price = reinterpret_cast<int64_t*>(take(sizeof(int64_t) * (size_t)T));
+    prm.qT = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * (size_t)T * E));
     unsigned char* zero1 = w + o;
     prm.cnt = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * (size_t)E));
     prm.obj = reinterpret_cast<unsigned long long*>(take(64));
